@@ -1,0 +1,328 @@
+"""ctypes wrapper around the CPU oracle (oracle/m3_oracle.cpp).
+
+TEST INFRASTRUCTURE ONLY: the test-suite, the package smoke check and the
+benchmark's CPU-baseline leg may import this module; the product path never
+does.  Arrays cross as numpy buffers of raw bits: bf16 / f16 as uint16.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+class OraMat(C.Structure):
+    _fields_ = [("w", C.c_void_p), ("q", C.c_void_p), ("s", C.c_void_p), ("wfmt", C.c_int)]
+
+
+class OraCfg(C.Structure):
+    _fields_ = [("hidden", C.c_int), ("n_layers", C.c_int), ("n_q_heads", C.c_int),
+                ("n_kv_heads", C.c_int), ("head_dim", C.c_int), ("ffn", C.c_int),
+                ("slice_start", C.c_int), ("slice_len", C.c_int), ("rope_theta", C.c_double),
+                ("rms_eps", C.c_float), ("wfmt", C.c_int), ("kv_f16", C.c_int)]
+
+
+class OraLayer(C.Structure):
+    _fields_ = [("attn_norm", C.c_void_p), ("wq", OraMat), ("wk", OraMat), ("wv", OraMat),
+                ("q_norm", C.c_void_p), ("k_norm", C.c_void_p), ("wo", OraMat),
+                ("mlp_norm", C.c_void_p), ("wg", OraMat), ("wu", OraMat), ("wd", OraMat)]
+
+
+class OraDepth(C.Structure):
+    _fields_ = [("hidden", C.c_int), ("n_layers", C.c_int), ("n_heads", C.c_int),
+                ("head_dim", C.c_int), ("ffn", C.c_int), ("codebooks", C.c_int),
+                ("vocab", C.c_int), ("in_hidden", C.c_int), ("rope_theta", C.c_double),
+                ("rms_eps", C.c_float), ("layers", C.POINTER(OraLayer)), ("proj", OraMat),
+                ("emb", C.POINTER(C.c_void_p)), ("final_norm", C.c_void_p),
+                ("heads", C.POINTER(OraMat))]
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = C.CDLL(path)
+        u64, f32, f64, i64, vp = C.c_uint64, C.c_float, C.c_double, C.c_int64, C.c_void_p
+        L.ora_f2bf.restype = C.c_uint16
+        L.ora_f2bf.argtypes = [f32]
+        L.ora_bf2f.restype = f32
+        L.ora_bf2f.argtypes = [C.c_uint16]
+        L.ora_f2h.restype = C.c_uint16
+        L.ora_f2h.argtypes = [f32]
+        L.ora_mix64.restype = u64
+        L.ora_mix64.argtypes = [u64]
+        L.ora_noise_bits.restype = u64
+        L.ora_noise_bits.argtypes = [u64, u64, u64, u64]
+        L.ora_uniform.restype = f64
+        L.ora_uniform.argtypes = [u64]
+        L.ora_ln.restype = f64
+        L.ora_ln.argtypes = [f64]
+        L.ora_gumbel.restype = f32
+        L.ora_gumbel.argtypes = [u64, u64, u64, u64]
+        L.ora_quantize.restype = None
+        L.ora_quantize.argtypes = [vp, i64, i64, i64, vp, vp]
+        L.ora_gemv.restype = None
+        L.ora_gemv.argtypes = [vp, vp, vp, C.c_int, i64, i64, vp, vp]
+        L.ora_rmsnorm.restype = None
+        L.ora_rmsnorm.argtypes = [vp, vp, i64, f32, vp]
+        L.ora_rope.restype = None
+        L.ora_rope.argtypes = [vp, C.c_int, i64, f64]
+        L.ora_attention.restype = None
+        L.ora_attention.argtypes = [vp, vp, vp, i64, C.c_int, vp]
+        L.ora_sample.restype = C.c_int
+        L.ora_sample.argtypes = [C.POINTER(OraCfg), OraMat, C.c_int, vp, u64, u64, f32, f32, vp,
+                                 vp, vp]
+        L.ora_sample_full_masked.restype = C.c_int
+        L.ora_sample_full_masked.argtypes = [C.POINTER(OraCfg), vp, C.c_int, C.c_int, vp, u64,
+                                             u64, f32, f32, vp]
+        L.ora_decode_frame.restype = C.c_int
+        L.ora_decode_frame.argtypes = [C.POINTER(OraCfg), C.POINTER(OraLayer), vp, OraMat,
+                                       C.c_int, i64, vp, vp, vp, u64, u64, vp, f32, f32, vp, vp,
+                                       vp]
+        L.ora_body.restype = C.c_int
+        L.ora_body.argtypes = [C.POINTER(OraCfg), C.POINTER(OraLayer), C.c_int, i64, vp, vp, vp,
+                               vp, vp]
+        L.ora_depth_decode.restype = C.c_int
+        L.ora_depth_decode.argtypes = [C.POINTER(OraDepth), C.c_int, vp, vp, u64, u64, f32, f32,
+                                       vp, vp, vp]
+        L.ora_gumbel_argmax_draws.restype = None
+        L.ora_gumbel_argmax_draws.argtypes = [vp, i64, f32, u64, u64, i64, vp]
+        L.ora_num_threads.restype = C.c_int
+        L.ora_set_num_threads.argtypes = [C.c_int]
+        _lib = L
+    return _lib
+
+
+# ------------------------------------------------------------ helpers -------
+
+def _p(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data_as(C.c_void_p)
+
+
+def bits(t) -> np.ndarray:
+    """A torch bf16/f16 tensor (or uint16 ndarray) as a C-contiguous uint16 ndarray."""
+    if isinstance(t, np.ndarray):
+        return np.ascontiguousarray(t.view(np.uint16) if t.dtype != np.uint16 else t)
+    import torch
+    return np.ascontiguousarray(t.detach().cpu().contiguous().view(torch.int16).numpy()
+                                .view(np.uint16))
+
+
+def bf16_to_f32(u16: np.ndarray) -> np.ndarray:
+    return (u16.astype(np.uint32) << 16).view(np.float32)
+
+
+def f32_to_bf16(x: np.ndarray) -> np.ndarray:
+    L = lib()
+    flat = np.asarray(x, np.float32).ravel()
+    return np.array([L.ora_f2bf(float(v)) for v in flat], np.uint16).reshape(np.shape(x))
+
+
+def quantize(w_bits: np.ndarray, group: int | None = None):
+    """int8 weight-only quantisation; group None = one scale per row."""
+    w_bits = np.ascontiguousarray(w_bits, np.uint16)
+    rows, cols = w_bits.shape
+    g = cols if group is None else group
+    q = np.empty((rows, cols), np.int8)
+    s = np.empty((rows, cols // g), np.float32)
+    lib().ora_quantize(_p(w_bits), rows, cols, g, _p(q), _p(s))
+    return q, (s[:, 0].copy() if group is None else s)
+
+
+def gemv(w=None, q=None, s=None, wfmt=0, x=None):
+    x = np.ascontiguousarray(x, np.float32)
+    ref = w if wfmt == 0 else q
+    rows, cols = ref.shape
+    y = np.empty(rows, np.float32)
+    lib().ora_gemv(_p(w) if w is not None else None, _p(q) if q is not None else None,
+                   _p(s) if s is not None else None, wfmt, rows, cols, _p(x), _p(y))
+    return y
+
+
+def rmsnorm(x: np.ndarray, gamma_bits: np.ndarray, eps: float) -> np.ndarray:
+    x = np.ascontiguousarray(x, np.float32)
+    g = np.ascontiguousarray(gamma_bits, np.uint16)
+    out = np.empty_like(x)
+    lib().ora_rmsnorm(_p(x), _p(g), x.size, eps, _p(out))
+    return out
+
+
+def rope(v: np.ndarray, pos: int, theta: float) -> np.ndarray:
+    v = np.array(v, np.float32, copy=True)
+    lib().ora_rope(_p(v), v.size, pos, theta)
+    return v
+
+
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray) -> np.ndarray:
+    q = np.ascontiguousarray(q, np.float32)
+    k = np.ascontiguousarray(k, np.float32)
+    v = np.ascontiguousarray(v, np.float32)
+    out = np.empty(q.size, np.float32)
+    lib().ora_attention(_p(q), _p(k), _p(v), k.shape[0], q.size, _p(out))
+    return out
+
+
+def gumbel(seed, frame, row, index) -> float:
+    return lib().ora_gumbel(seed, frame, row, index)
+
+
+def gumbel_argmax_draws(logits, temperature, seed, frame0, ndraws) -> np.ndarray:
+    lg = np.ascontiguousarray(logits, np.float32)
+    out = np.empty(ndraws, np.int32)
+    lib().ora_gumbel_argmax_draws(_p(lg), lg.size, temperature, seed, frame0, ndraws, _p(out))
+    return out
+
+
+def set_threads(n: int) -> None:
+    lib().ora_set_num_threads(int(n))
+
+
+def num_threads() -> int:
+    return lib().ora_num_threads()
+
+
+# -------------------------------------------------------- model objects -----
+
+class _Keep:
+    """Holds numpy arrays alive for as long as the ctypes structs point at them."""
+
+    def __init__(self):
+        self.arrs = []
+
+    def __call__(self, a):
+        self.arrs.append(a)
+        return _p(a)
+
+
+def _mat(keep, w_bits, wfmt, group=128):
+    if wfmt == 0:
+        return OraMat(keep(np.ascontiguousarray(w_bits, np.uint16)), None, None, 0)
+    q, s = quantize(w_bits, None if wfmt == 1 else group)
+    return OraMat(None, keep(q), keep(np.ascontiguousarray(s)), wfmt)
+
+
+class Body:
+    """The oracle's copy of a body: weights as raw bits, optionally int8-quantised
+    by the oracle's own quantiser (wfmt 1 = one scale per row)."""
+
+    def __init__(self, shape, layers: list, final_norm, lm_slice, wfmt=0, kv_f16=False):
+        self.shape = shape
+        self.keep = _Keep()
+        k = self.keep
+        self.cfg = OraCfg(shape.hidden, shape.n_layers, shape.n_q_heads, shape.n_kv_heads,
+                          shape.head_dim, shape.ffn, shape.slice_start, shape.slice_len,
+                          shape.rope_theta, shape.rms_eps, wfmt, int(kv_f16))
+        arr = (OraLayer * len(layers))()
+        for i, Lw in enumerate(layers):
+            b = {n: bits(t) for n, t in Lw.items()}
+            arr[i] = OraLayer(k(b["attn_norm"]), _mat(k, b["wq"], wfmt), _mat(k, b["wk"], wfmt),
+                              _mat(k, b["wv"], wfmt), k(b["q_norm"]), k(b["k_norm"]),
+                              _mat(k, b["wo"], wfmt), k(b["mlp_norm"]), _mat(k, b["wg"], wfmt),
+                              _mat(k, b["wu"], wfmt), _mat(k, b["wd"], wfmt))
+        self.layers = arr
+        self.final_norm = bits(final_norm) if final_norm is not None else None
+        self.lm = _mat(k, bits(lm_slice), wfmt) if lm_slice is not None else None
+
+    def new_cache(self, rows: int, max_pos: int):
+        s = self.shape
+        shp = (rows, s.n_layers, max_pos, s.n_kv_heads, s.head_dim)
+        return np.zeros(shp, np.uint16), np.zeros(shp, np.uint16)
+
+    def decode_frame(self, kc, vc, positions, seed, frame, x_in_bits, cfg_scale=0.0,
+                     temperature=1.0):
+        rows = x_in_bits.shape[0]
+        pos = np.ascontiguousarray(positions, np.int32)
+        x = np.ascontiguousarray(x_in_bits, np.uint16)
+        codes = np.empty(rows, np.int32)
+        h = np.empty((rows, self.shape.hidden), np.uint16)
+        lg = np.empty((rows, self.shape.slice_len), np.float32)
+        rc = lib().ora_decode_frame(C.byref(self.cfg), self.layers, _p(self.final_norm), self.lm,
+                                    rows, kc.shape[2], _p(kc), _p(vc), _p(pos), seed, frame,
+                                    _p(x), cfg_scale, temperature, _p(codes), _p(h), _p(lg))
+        if rc != 0:
+            raise RuntimeError(f"ora_decode_frame: {rc}")
+        return codes, h, lg
+
+    def body(self, kc, vc, positions, x_in_bits):
+        rows = x_in_bits.shape[0]
+        pos = np.ascontiguousarray(positions, np.int32)
+        x = np.ascontiguousarray(x_in_bits, np.uint16)
+        out = np.empty_like(x)
+        lib().ora_body(C.byref(self.cfg), self.layers, rows, kc.shape[2], _p(kc), _p(vc),
+                       _p(pos), _p(x), _p(out))
+        return out
+
+    def sample(self, h_bits, seed, frame, cfg_scale=0.0, temperature=1.0, with_margin=False):
+        h = np.ascontiguousarray(h_bits, np.uint16)
+        rows = h.shape[0]
+        codes = np.empty(rows, np.int32)
+        lg = np.empty((rows, self.shape.slice_len), np.float32)
+        mg = np.empty(rows, np.float32)
+        rc = lib().ora_sample(C.byref(self.cfg), self.lm, rows, _p(h), seed, frame, cfg_scale,
+                              temperature, _p(codes), _p(lg), _p(mg) if with_margin else None)
+        if rc != 0:
+            raise RuntimeError(f"ora_sample: {rc}")
+        return (codes, lg, mg) if with_margin else (codes, lg)
+
+    def sample_full_masked(self, lm_full_bits, h_bits, seed, frame, cfg_scale=0.0,
+                           temperature=1.0):
+        h = np.ascontiguousarray(h_bits, np.uint16)
+        W = np.ascontiguousarray(lm_full_bits, np.uint16)
+        rows = h.shape[0]
+        codes = np.empty(rows, np.int32)
+        rc = lib().ora_sample_full_masked(C.byref(self.cfg), _p(W), W.shape[0], rows, _p(h), seed,
+                                          frame, cfg_scale, temperature, _p(codes))
+        if rc != 0:
+            raise RuntimeError(f"ora_sample_full_masked: {rc}")
+        return codes
+
+
+class Depth:
+    """The oracle's depth decoder; weights int8 with one scale per group of 128,
+    quantised by the oracle's quantiser from the bf16 tensors."""
+
+    def __init__(self, shape, w: dict):
+        self.shape = shape
+        self.keep = _Keep()
+        k = self.keep
+        arr = (OraLayer * shape.n_layers)()
+        for i, Lw in enumerate(w["layers"]):
+            b = {n: bits(t) for n, t in Lw.items()}
+            arr[i] = OraLayer(k(b["attn_norm"]), _mat(k, b["wq"], 2), _mat(k, b["wk"], 2),
+                              _mat(k, b["wv"], 2), k(b["q_norm"]), k(b["k_norm"]),
+                              _mat(k, b["wo"], 2), k(b["mlp_norm"]), _mat(k, b["wg"], 2),
+                              _mat(k, b["wu"], 2), _mat(k, b["wd"], 2))
+        self.layers = arr
+        emb = (C.c_void_p * shape.codebooks)()
+        for j, e in enumerate(w["emb"]):
+            emb[j] = k(bits(e)).value
+        self.emb = emb
+        heads = (OraMat * shape.codebooks)()
+        for j, hw in enumerate(w["heads"]):
+            heads[j] = _mat(k, bits(hw), 2)
+        self.heads = heads
+        self.D = OraDepth(shape.hidden, shape.n_layers, shape.n_heads, shape.head_dim, shape.ffn,
+                          shape.codebooks, shape.vocab, shape.in_hidden, shape.rope_theta,
+                          shape.rms_eps, arr, _mat(k, bits(w["proj"]), 2), emb,
+                          k(bits(w["final_norm"])), heads)
+
+    def decode(self, h_frame_bits, code0, seed, frame, cfg_scale=0.0, temperature=1.0,
+               forced=None):
+        h = np.ascontiguousarray(h_frame_bits, np.uint16)
+        rows = h.shape[0]
+        c0 = np.ascontiguousarray(code0, np.int32)
+        codes = np.empty((rows, self.shape.codebooks), np.int32)
+        lg = np.empty((rows, self.shape.codebooks, self.shape.vocab), np.float32)
+        fc = None if forced is None else np.ascontiguousarray(forced, np.int32)
+        rc = lib().ora_depth_decode(C.byref(self.D), rows, _p(h), _p(c0), seed, frame, cfg_scale,
+                                    temperature, _p(fc) if fc is not None else None, _p(codes),
+                                    _p(lg))
+        if rc != 0:
+            raise RuntimeError(f"ora_depth_decode: {rc}")
+        return codes, lg

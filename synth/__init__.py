@@ -1,0 +1,173 @@
+"""Seeded synthetic inputs shared by the CPU oracle and the CUDA library.
+
+This module only draws random numbers and names model shapes; it holds none
+of the decode step's arithmetic.  Every tensor is a pure function of
+(seed, tensor id, shape, device kind): weights N(0, 0.02^2), norm gains
+1 + N(0, 0.01^2), KV prefill N(0, 1), embeddings N(0, 0.02^2), as the
+workload descriptions fix them.  Values are drawn by torch's generators
+(CPU or CUDA) in fp32 and rounded to bf16, so a tensor drawn on the GPU
+is not the same as one drawn on the CPU with the same seed: a test draws
+each input once and hands the same bytes to both sides.
+"""
+from __future__ import annotations
+
+import dataclasses
+import hashlib
+
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class BodyShape:
+    """Shape of the Qwen3-style Global LLM and its sampleable vocab slice."""
+    hidden: int
+    n_layers: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    ffn: int
+    vocab: int
+    slice_start: int
+    slice_len: int
+    rope_theta: float = 1.0e6
+    rms_eps: float = 1.0e-6
+
+
+@dataclasses.dataclass(frozen=True)
+class DepthShape:
+    """Shape of the RVQ depth decoder (MHA: as many KV heads as query heads)."""
+    hidden: int = 1024
+    n_layers: int = 4
+    n_heads: int = 16
+    head_dim: int = 64
+    ffn: int = 2816
+    codebooks: int = 7
+    vocab: int = 1024
+    sem_vocab: int = 16384
+    in_hidden: int = 4096
+    rope_theta: float = 1.0e6
+    rms_eps: float = 1.0e-6
+
+
+# Tiny 1-layer decode checked over 16 consecutive frames.
+TINY = BodyShape(hidden=256, n_layers=1, n_q_heads=4, n_kv_heads=2, head_dim=64, ffn=768,
+                 vocab=2048, slice_start=1024, slice_len=512)
+# One Qwen3-8B decoder layer (GEMV roofline microbench); no lm_head of its own.
+LAYER8B = BodyShape(hidden=4096, n_layers=1, n_q_heads=32, n_kv_heads=8, head_dim=128,
+                    ffn=12288, vocab=200000, slice_start=151675, slice_len=16384)
+# The full 36-layer 8B body with its sliced lm_head.
+FULL8B = BodyShape(hidden=4096, n_layers=36, n_q_heads=32, n_kv_heads=8, head_dim=128,
+                   ffn=12288, vocab=200000, slice_start=151675, slice_len=16384)
+DEPTH = DepthShape()
+
+LAYER_TENSORS = ("attn_norm", "wq", "wk", "wv", "q_norm", "k_norm", "wo", "mlp_norm",
+                 "wg", "wu", "wd")
+NORM_TENSORS = ("attn_norm", "q_norm", "k_norm", "mlp_norm")
+
+
+def _stream_seed(seed: int, name: str) -> int:
+    h = hashlib.sha256(f"{int(seed)}/{name}".encode()).digest()
+    return int.from_bytes(h[:8], "little") & ((1 << 63) - 1)
+
+
+def _gen(seed: int, name: str, device) -> torch.Generator:
+    dev = torch.device(device)
+    g = torch.Generator(device=dev.type if dev.type != "cuda" else dev)
+    g.manual_seed(_stream_seed(seed, name))
+    return g
+
+
+def normal(shape, seed: int, name: str, std: float = 1.0, mean: float = 0.0,
+           device="cpu", dtype=torch.bfloat16) -> torch.Tensor:
+    """N(mean, std^2) drawn in fp32 from the stream (seed, name), cast to dtype."""
+    g = _gen(seed, name, device)
+    t = torch.randn(tuple(shape), generator=g, device=device, dtype=torch.float32)
+    if std != 1.0:
+        t.mul_(std)
+    if mean != 0.0:
+        t.add_(mean)
+    return t.to(dtype)
+
+
+def layer_shapes(s) -> dict:
+    H, d = s.hidden, s.head_dim
+    hq = s.n_q_heads if isinstance(s, BodyShape) else s.n_heads
+    hkv = s.n_kv_heads if isinstance(s, BodyShape) else s.n_heads
+    return {
+        "attn_norm": (H,), "wq": (hq * d, H), "wk": (hkv * d, H), "wv": (hkv * d, H),
+        "q_norm": (d,), "k_norm": (d,), "wo": (H, hq * d), "mlp_norm": (H,),
+        "wg": (s.ffn, H), "wu": (s.ffn, H), "wd": (H, s.ffn),
+    }
+
+
+def layer_weights(s, seed: int, layer: int, device="cpu", prefix: str = "body") -> dict:
+    """One decoder layer's bf16 tensors (weights N(0,.02^2), gains 1+N(0,.01^2))."""
+    out = {}
+    for name, shape in layer_shapes(s).items():
+        tag = f"{prefix}/L{layer}/{name}"
+        if name in NORM_TENSORS:
+            out[name] = normal(shape, seed, tag, std=0.01, mean=1.0, device=device)
+        else:
+            out[name] = normal(shape, seed, tag, std=0.02, device=device)
+    return out
+
+
+def final_norm(s, seed: int, device="cpu", prefix: str = "body") -> torch.Tensor:
+    return normal((s.hidden,), seed, f"{prefix}/final_norm", std=0.01, mean=1.0, device=device)
+
+
+def lm_head_rows(s: BodyShape, seed: int, row0: int, nrows: int, device="cpu") -> torch.Tensor:
+    """Rows [row0, row0+nrows) of the full [vocab, hidden] lm_head, drawn in
+    blocks of 1024 vocab rows so that any slice equals the same rows of the
+    full matrix."""
+    blocks = []
+    b0, b1 = row0 // 1024, (row0 + nrows - 1) // 1024
+    for b in range(b0, b1 + 1):
+        n = min(1024, s.vocab - b * 1024)
+        blocks.append(normal((n, s.hidden), seed, f"lm_head/block{b}", std=0.02, device=device))
+    full = torch.cat(blocks, 0)
+    off = row0 - b0 * 1024
+    return full[off:off + nrows].contiguous()
+
+
+def lm_head_slice(s: BodyShape, seed: int, device="cpu") -> torch.Tensor:
+    return lm_head_rows(s, seed, s.slice_start, s.slice_len, device)
+
+
+def lm_head_full(s: BodyShape, seed: int, device="cpu") -> torch.Tensor:
+    return lm_head_rows(s, seed, 0, s.vocab, device)
+
+
+def embedding(s: BodyShape, seed: int, device="cpu") -> torch.Tensor:
+    """Token-embedding table [vocab, hidden] used to feed a drawn code back."""
+    return normal((s.vocab, s.hidden), seed, "embed_tokens", std=0.02, device=device)
+
+
+def kv_prefill(s, rows: int, n_pos: int, seed: int, device="cpu"):
+    """Per-row prefilled cache contents N(0,1), layout [rows, layers, n_pos, Hkv, d]
+    for K and for V (the prefill stands for already-rotated keys)."""
+    hkv = s.n_kv_heads if isinstance(s, BodyShape) else s.n_heads
+    ks, vs = [], []
+    for r in range(rows):
+        ks.append(normal((s.n_layers, n_pos, hkv, s.head_dim), seed + 1000 + r, "kv/K",
+                         device=device))
+        vs.append(normal((s.n_layers, n_pos, hkv, s.head_dim), seed + 1000 + r, "kv/V",
+                         device=device))
+    return torch.stack(ks, 0), torch.stack(vs, 0)
+
+
+def frame_input(s, rows: int, seed: int, frame: int, device="cpu") -> torch.Tensor:
+    """A frame's input embedding per row, N(0, 0.02^2) like the embedding tables."""
+    return normal((rows, s.hidden), seed, f"x_in/frame{frame}", std=0.02, device=device)
+
+
+def depth_weights(d: DepthShape, seed: int, device="cpu") -> dict:
+    """Depth decoder bf16 tensors: layers, proj, embedding tables, final norm, heads."""
+    out = {"layers": [layer_weights(d, seed, l, device, prefix="depth") for l in range(d.n_layers)]}
+    out["proj"] = normal((d.hidden, d.in_hidden), seed, "depth/proj", std=0.02, device=device)
+    out["emb"] = [normal((d.sem_vocab if j == 0 else d.vocab, d.hidden), seed, f"depth/emb{j}",
+                         std=0.02, device=device) for j in range(d.codebooks)]
+    out["final_norm"] = final_norm(d, seed, device, prefix="depth")
+    out["heads"] = [normal((d.vocab, d.hidden), seed, f"depth/head{j}", std=0.02, device=device)
+                    for j in range(d.codebooks)]
+    return out
