@@ -1,0 +1,493 @@
+// gemv.cuh -- weight-streaming GEMV for the decode step (1..4 activation rows).
+//
+// The decode step reads every weight once per frame ("MiniMax Music 3
+// modular pipeline", finding 4: the AR stage is memory-bandwidth bound), so
+// each projection is a GEMV whose speed is the HBM stream of W:
+//   * one CTA per SM, each owning a contiguous block of output rows;
+//   * a producer warp streams that block through a 3-stage ring of 32 KB
+//     shared-memory stages with non-multicast bulk copies (TMA engine,
+//     mbarrier transaction counts, L2 evict-first), starting before the
+//     previous kernel has finished (programmatic dependent launch: weights
+//     do not depend on it);
+//   * 8 consumer warps own fixed K positions, keep the (normalised)
+//     activation in registers, and FMA 16 weights per row per thread; a
+//     butterfly shuffle + one named barrier per stage reduces over K;
+//   * the consumer of a norm computes RMSNorm itself (no separate pass):
+//     "MiniMax Music 3 on Metal", section "Next steps", suggests folding the
+//     RMS norms into the GEMVs that read them;
+//   * epilogues: store bf16 (QKV), residual add (O, down), SwiGLU on
+//     interleaved gate/up rows, or the fused lm_head sampler (fp32 logits,
+//     CFG over row pairs, Gumbel noise, block argmax, last-CTA reduction).
+// Weight formats: bf16, int8 + fp32 scale per row, int8 + fp32 scale per
+// group of 128 inputs ("MiniMax Music 3 on Metal", section "Precision").
+#pragma once
+
+#include "common.cuh"
+#include "noise.cuh"
+
+namespace m3 {
+
+enum : int { EPI_STORE = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_SAMPLE = 3 };
+enum : int { WF_BF16 = 0, WF_I8ROW = 1, WF_I8G128 = 2 };
+
+constexpr int kConsumers = 256;
+constexpr int kGemvThreads = kConsumers + 32;
+constexpr int kStageBytes = 32768;
+constexpr int kStages = 3;
+constexpr int kMaxRows = 16;
+
+// Per-frame scalars, written once per frame by set_frame_params before the
+// frame's first kernel.
+struct FrameParams {
+  int rows;
+  int cfg_on;
+  float cfg_scale;
+  float temperature;
+  unsigned long long seed;
+  unsigned long long frame;
+  int pos[kMaxRows];
+};
+
+struct SampleArgs {
+  float* logits;              // [rows][logits_ld] fp32 at column n; nullable
+  int logits_ld;
+  int* codes;                 // code of batch row r at codes[r * code_stride]
+  int code_stride;
+  int* prev;                  // nullable: fed-forward code per row [rows]
+  const int* forced;          // nullable: forced[r * forced_stride] replaces prev
+  int forced_stride;
+  unsigned long long index_base;  // noise index of output row n is index_base + n
+  float* part_z;              // [grid][kMaxRows] scratch
+  int* part_i;                // [grid][kMaxRows] scratch
+  unsigned int* counter;      // zero at rest; the last CTA resets it
+  __nv_bfloat16* h_out;       // nullable: normalised input [rows][K] (CTA 0 writes)
+};
+
+struct GemvArgs {
+  const void* w;              // [N][K] row-major, bf16 or int8
+  const float* scales;        // int8: [N] or [N][K/128]
+  int N, K;
+  int row0;                   // first batch row of this launch
+  int mr;                     // batch rows of this launch (<= MR)
+  const __nv_bfloat16* x;     // [rows][ldx] input activations (row0-relative rows)
+  int ldx;
+  const __nv_bfloat16* gamma; // RMSNorm gain over K, nullable = no norm
+  float eps;
+  __nv_bfloat16* out;         // STORE/RESID: [rows][ldo] at column n; SWIGLU: column n/2
+  int ldo;
+  const FrameParams* fp;
+  SampleArgs smp;
+  int* err;
+};
+
+template <int TPR, int ESZ>
+struct GemvShape {
+  static constexpr int KC = TPR * 16;                 // K elements per segment
+  static constexpr int G = kConsumers / TPR;          // rows in flight per pass
+  static constexpr int R = kStageBytes / (KC * ESZ);  // rows (segments) per stage
+  static constexpr int P = R / G;                     // passes per stage
+  static constexpr int W = TPR < 32 ? TPR : 32;       // shuffle width
+  static constexpr int SLOTS = kConsumers / W;        // partial sums per row
+  static_assert(R % G == 0 && R % 2 == 0, "stage geometry");
+};
+
+// Dynamic shared memory of one CTA (the host sizes it with the same formula).
+template <int MR, int TPR, int ESZ>
+__host__ __device__ constexpr size_t gemv_smem_bytes(int rows_cta_max) {
+  using S = GemvShape<TPR, ESZ>;
+  return (size_t)kStages * kStageBytes + 2 * kStages * sizeof(uint64_t) +
+         sizeof(float) * (2 * S::SLOTS * S::P * MR + 9 * MR + (size_t)rows_cta_max * MR) +
+         (sizeof(float) + sizeof(int)) * S::R * MR + 64;
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
+
+template <int MR, int WF, int EPI, int TPR>
+__global__ void __launch_bounds__(kGemvThreads, MR <= 2 ? 2 : 1) gemv_kernel(const GemvArgs a) {
+  constexpr int ESZ = WF == WF_BF16 ? 2 : 1;
+  using S = GemvShape<TPR, ESZ>;
+  constexpr int KC = S::KC, G = S::G, R = S::R, P = S::P, W = S::W, SLOTS = S::SLOTS;
+  constexpr int UNIT = EPI == EPI_SWIGLU ? 2 : 1;
+
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* ring = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  float* part = reinterpret_cast<float*>(empty + kStages);  // [2][SLOTS][P][MR]
+  float* nrm = part + 2 * SLOTS * P * MR;                    // [8][MR] + [MR]
+  float* accr = nrm + 9 * MR;                                 // [rows_cta][MR]
+
+  const int tid = threadIdx.x;
+  const int K = a.K;
+  const int nkc = (K + KC - 1) / KC;
+  const int U = a.N / UNIT;
+  const int u0 = (int)((long long)U * blockIdx.x / gridDim.x);
+  const int u1 = (int)((long long)U * (blockIdx.x + 1) / gridDim.x);
+  const int r_begin = u0 * UNIT, r_end = u1 * UNIT;
+  const int nrows = r_end - r_begin;
+  const int spk = (nrows + R - 1) / R;
+  const int nstages = spk * nkc;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumers / 32);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  pdl_launch_dependents();
+
+  // ------------------------------------------------------------ producer --
+  if (tid >= kConsumers) {
+    if (tid == kConsumers) {
+      const uint64_t pol = policy_evict_first();
+      const uint8_t* wb = static_cast<const uint8_t*>(a.w);
+      for (int s = 0; s < nstages; ++s) {
+        const int slot = s % kStages;
+        if (s >= kStages && !mbar_wait(&empty[slot], ((s / kStages) - 1) & 1, a.err)) break;
+        const int kc = s / spk, sr = s % spk;
+        const int rs = r_begin + sr * R, re = min(rs + R, r_end);
+        const int kel = min(KC, K - kc * KC);
+        const uint32_t segb = (uint32_t)(kel * ESZ);
+        mbar_arrive_expect_tx(&full[slot], segb * (uint32_t)(re - rs));
+        uint8_t* dst = ring + slot * kStageBytes;
+        for (int r = rs; r < re; ++r)
+          bulk_g2s(dst + (size_t)(r - rs) * KC * ESZ,
+                   wb + ((size_t)r * K + (size_t)kc * KC) * ESZ, segb, &full[slot], pol);
+      }
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------ consumers --
+  const int g = tid / TPR, t = tid % TPR;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int mr = a.mr;
+  const __nv_bfloat16* __restrict__ x = a.x;
+
+  pdl_wait();  // the activations come from the previous kernel
+
+  float inv[MR];
+#pragma unroll
+  for (int m = 0; m < MR; ++m) inv[m] = 1.0f;
+  if (a.gamma) {
+    float ss[MR];
+#pragma unroll
+    for (int m = 0; m < MR; ++m) ss[m] = 0.0f;
+    for (int k = tid; k < K; k += kConsumers) {
+#pragma unroll
+      for (int m = 0; m < MR; ++m)
+        if (m < mr) {
+          const float v = __bfloat162float(x[(size_t)m * a.ldx + k]);
+          ss[m] = fmaf(v, v, ss[m]);
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < MR; ++m) {
+      float v = ss[m];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0) nrm[warp * MR + m] = v;
+    }
+    named_bar_sync(1, kConsumers);
+#pragma unroll
+    for (int m = 0; m < MR; ++m) {
+      float tot = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kConsumers / 32; ++w) tot += nrm[w * MR + m];
+      inv[m] = 1.0f / sqrtf(tot / (float)K + a.eps);
+    }
+  }
+
+  // x in registers: this thread's 16 K positions of the current chunk.
+  float xr[MR][16];
+  auto elem_k = [&](int kc, int e) -> int {
+    if (ESZ == 2) return kc * KC + (e < 8 ? 8 * t + e : 8 * (t + TPR) + (e - 8));
+    return kc * KC + 16 * t + e;
+  };
+  auto load_x = [&](int kc) {
+    const bool write_h = (EPI == EPI_SAMPLE) && a.smp.h_out && blockIdx.x == 0 && g == 0;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const int k = elem_k(kc, e);
+      const bool ok = k < K;
+      const float gm = (a.gamma && ok) ? __bfloat162float(a.gamma[k]) : 1.0f;
+#pragma unroll
+      for (int m = 0; m < MR; ++m) {
+        float v = (ok && m < mr) ? __bfloat162float(x[(size_t)m * a.ldx + k]) : 0.0f;
+        if (a.gamma) v = round_bf16(gm * round_bf16(v * inv[m]));
+        xr[m][e] = v;
+        if (write_h && ok && m < mr)
+          a.smp.h_out[(size_t)(a.row0 + m) * K + k] = __float2bfloat16_rn(v);
+      }
+    }
+  };
+
+  // sampler state: this thread's role (row-in-stage, key) is fixed
+  constexpr int NPMAX = MR;
+  float best_z = -INFINITY;
+  int best_i = 0x7fffffff;
+  const int np = (EPI == EPI_SAMPLE) ? (a.fp->cfg_on ? mr / 2 : mr) : 0;
+
+  int s = 0, buf = 0;
+  for (int kc = 0; kc < nkc; ++kc) {
+    load_x(kc);
+    const int kel = min(KC, K - kc * KC);
+    for (int sr = 0; sr < spk; ++sr, ++s) {
+      const int slot = s % kStages;
+      // On a timeout the error word is set and the stage is consumed as is, so
+      // that every consumer still reaches the same named barriers.
+      mbar_wait(&full[slot], (s / kStages) & 1, a.err);
+      const int rs = r_begin + sr * R;
+      const int nr = min(R, r_end - rs);
+      const uint8_t* st = ring + slot * kStageBytes;
+      float acc[P][MR];
+#pragma unroll
+      for (int p = 0; p < P; ++p)
+#pragma unroll
+        for (int m = 0; m < MR; ++m) acc[p][m] = 0.0f;
+
+#pragma unroll
+      for (int p = 0; p < P; ++p) {
+        const int rl = p * G + g;
+        if (rl < nr) {
+          const uint8_t* seg = st + (size_t)rl * KC * ESZ;
+          if constexpr (ESZ == 2) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int c = t + h * TPR;  // 16-byte chunk index in the segment
+              if (8 * c < kel) {
+                const uint4 wv = *reinterpret_cast<const uint4*>(seg + 16 * c);
+                const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  float lo, hi;
+                  bf16x2_to_f32(ww[j], lo, hi);
+#pragma unroll
+                  for (int m = 0; m < MR; ++m) {
+                    acc[p][m] = fmaf(lo, xr[m][8 * h + 2 * j], acc[p][m]);
+                    acc[p][m] = fmaf(hi, xr[m][8 * h + 2 * j + 1], acc[p][m]);
+                  }
+                }
+              }
+            }
+          } else {
+            if (16 * t < kel) {
+              const uint4 wv = *reinterpret_cast<const uint4*>(seg + 16 * t);
+              const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+              float part_m[MR];
+#pragma unroll
+              for (int m = 0; m < MR; ++m) part_m[m] = 0.0f;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                float f[4];
+                s8x4_to_f32(ww[j], f);
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+#pragma unroll
+                  for (int m = 0; m < MR; ++m) part_m[m] = fmaf(f[q], xr[m][4 * j + q], part_m[m]);
+              }
+              if constexpr (WF == WF_I8G128) {
+                const int n = rs + rl;
+                const int kabs = kc * KC + 16 * t;
+                const float sc = __ldg(a.scales + (size_t)n * (K / 128) + kabs / 128);
+#pragma unroll
+                for (int m = 0; m < MR; ++m) acc[p][m] = fmaf(sc, part_m[m], acc[p][m]);
+              } else {
+#pragma unroll
+                for (int m = 0; m < MR; ++m) acc[p][m] += part_m[m];
+              }
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+
+      // reduce over the TPR threads of each row: shuffles, then partial slots
+#pragma unroll
+      for (int p = 0; p < P; ++p)
+#pragma unroll
+        for (int m = 0; m < MR; ++m) {
+          float v = acc[p][m];
+#pragma unroll
+          for (int o = W / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o, W);
+          acc[p][m] = v;
+        }
+      float* pb = part + buf * SLOTS * P * MR;
+      if ((tid % W) == 0) {
+        const int sl = tid / W;
+#pragma unroll
+        for (int p = 0; p < P; ++p)
+#pragma unroll
+          for (int m = 0; m < MR; ++m) pb[(sl * P + p) * MR + m] = acc[p][m];
+      }
+      named_bar_sync(1, kConsumers);
+
+      // full sum of (row-in-stage rl, batch row m) for this stage
+      auto row_sum = [&](int rl, int m) -> float {
+        const int gg = rl % G, pp = rl / G;
+        constexpr int SPG = TPR / W;  // slots per row group
+        float y = 0.0f;
+#pragma unroll
+        for (int q = 0; q < SPG; ++q) y += pb[((gg * SPG + q) * P + pp) * MR + m];
+        return y;
+      };
+      const bool last_kc = (kc == nkc - 1);
+
+      if constexpr (EPI == EPI_STORE || EPI == EPI_RESID) {
+        for (int c = tid; c < R * MR; c += kConsumers) {
+          const int rl = c / MR, m = c % MR;
+          if (rl >= nr || m >= mr) continue;
+          float y = row_sum(rl, m);
+          if (nkc > 1) {
+            float* ar = accr + (size_t)(sr * R + rl) * MR + m;
+            if (kc > 0) y += *ar;
+            if (!last_kc) {
+              *ar = y;
+              continue;
+            }
+          }
+          const int n = rs + rl;
+          if constexpr (WF == WF_I8ROW) y *= __ldg(a.scales + n);
+          __nv_bfloat16* o = a.out + (size_t)m * a.ldo + n;
+          if constexpr (EPI == EPI_STORE) {
+            *o = __float2bfloat16_rn(y);
+          } else {
+            *o = __float2bfloat16_rn(__bfloat162float(*o) + round_bf16(y));
+          }
+        }
+      } else if constexpr (EPI == EPI_SWIGLU) {
+        for (int c = tid; c < (R / 2) * MR; c += kConsumers) {
+          const int j = c / MR, m = c % MR;
+          if (2 * j >= nr || m >= mr) continue;
+          float yg = row_sum(2 * j, m), yu = row_sum(2 * j + 1, m);
+          if (nkc > 1) {
+            float* ag = accr + (size_t)(sr * R + 2 * j) * MR + m;
+            float* au = accr + (size_t)(sr * R + 2 * j + 1) * MR + m;
+            if (kc > 0) {
+              yg += *ag;
+              yu += *au;
+            }
+            if (!last_kc) {
+              *ag = yg;
+              *au = yu;
+              continue;
+            }
+          }
+          const int n = rs + 2 * j;
+          if constexpr (WF == WF_I8ROW) {
+            yg *= __ldg(a.scales + n);
+            yu *= __ldg(a.scales + n + 1);
+          }
+          const float gb = round_bf16(yg), ub = round_bf16(yu);
+          const float act = round_bf16(round_bf16(silu_f(gb)) * ub);
+          a.out[(size_t)m * a.ldo + n / 2] = __float2bfloat16_rn(act);
+        }
+      } else {  // EPI_SAMPLE: one role per thread
+        const int c = tid;
+        const int rl = c / NPMAX, p = c % NPMAX;
+        if (rl < nr && p < np && (nkc == 1 || last_kc)) {
+          const int n = rs + rl;
+          const bool cfg = a.fp->cfg_on != 0;
+          const int m0 = cfg ? 2 * p : p;
+          float y0 = row_sum(rl, m0);
+          float y1 = cfg ? row_sum(rl, m0 + 1) : 0.0f;
+          if (nkc > 1) {
+            y0 += accr[(size_t)(sr * R + rl) * MR + m0];
+            if (cfg) y1 += accr[(size_t)(sr * R + rl) * MR + m0 + 1];
+          }
+          if constexpr (WF == WF_I8ROW) {
+            const float sc = __ldg(a.scales + n);
+            y0 *= sc;
+            y1 *= sc;
+          }
+          if (a.smp.logits) {
+            a.smp.logits[(size_t)(a.row0 + m0) * a.smp.logits_ld + n] = y0;
+            if (cfg) a.smp.logits[(size_t)(a.row0 + m0 + 1) * a.smp.logits_ld + n] = y1;
+          }
+          float gl = y0;
+          if (cfg) gl = __fadd_rn(y1, __fmul_rn(a.fp->cfg_scale, __fsub_rn(y0, y1)));
+          const unsigned long long key = cfg ? (unsigned long long)(a.row0 / 2 + p)
+                                             : (unsigned long long)(a.row0 + p);
+          const float gn = gumbel_noise(a.fp->seed, a.fp->frame, key,
+                                        a.smp.index_base + (unsigned long long)n);
+          const float z = __fadd_rn(__fdiv_rn(gl, a.fp->temperature), gn);
+          if (z > best_z || (z == best_z && n < best_i)) {
+            best_z = z;
+            best_i = n;
+          }
+        } else if (nkc > 1 && !last_kc && rl < nr && p < np) {
+          // accumulate the K-chunk partials of the rows this role reads
+          const bool cfg = a.fp->cfg_on != 0;
+          const int m0 = cfg ? 2 * p : p;
+          float* a0 = accr + (size_t)(sr * R + rl) * MR + m0;
+          *a0 = (kc > 0 ? *a0 : 0.0f) + row_sum(rl, m0);
+          if (cfg) a0[1] = (kc > 0 ? a0[1] : 0.0f) + row_sum(rl, m0 + 1);
+        }
+      }
+      buf ^= 1;
+    }
+  }
+
+  if constexpr (EPI == EPI_SAMPLE) {
+    // CTA-level argmax per key, then the last CTA reduces over CTAs.
+    float* sz = accr + (size_t)spk * R * MR;
+    int* si = reinterpret_cast<int*>(sz + R * MR);
+    __shared__ int s_last;
+    if (tid < R * NPMAX) {
+      sz[tid] = best_z;
+      si[tid] = best_i;
+    }
+    named_bar_sync(1, kConsumers);
+    if (tid < np) {
+      float bz = -INFINITY;
+      int bi = 0x7fffffff;
+      for (int rl = 0; rl < R; ++rl) {
+        const float z = sz[rl * NPMAX + tid];
+        const int i = si[rl * NPMAX + tid];
+        if (z > bz || (z == bz && i < bi)) {
+          bz = z;
+          bi = i;
+        }
+      }
+      a.smp.part_z[blockIdx.x * kMaxRows + tid] = bz;
+      a.smp.part_i[blockIdx.x * kMaxRows + tid] = bi;
+      __threadfence();
+    }
+    named_bar_sync(1, kConsumers);
+    if (tid == 0) {
+      __threadfence();
+      const unsigned old = atomicAdd(a.smp.counter, 1u);
+      s_last = (old == gridDim.x - 1);
+    }
+    named_bar_sync(1, kConsumers);
+    if (s_last) {
+      __threadfence();
+      if (tid < np) {
+        float bz = -INFINITY;
+        int bi = 0x7fffffff;
+        for (int b = 0; b < (int)gridDim.x; ++b) {
+          const float z = __ldcg(a.smp.part_z + b * kMaxRows + tid);
+          const int i = __ldcg(a.smp.part_i + b * kMaxRows + tid);
+          if (z > bz || (z == bz && i < bi)) {
+            bz = z;
+            bi = i;
+          }
+        }
+        const bool cfg = a.fp->cfg_on != 0;
+        const int nm = cfg ? 2 : 1;
+        for (int q = 0; q < nm; ++q) {
+          const int r = a.row0 + (cfg ? 2 * tid + q : tid);
+          a.smp.codes[(size_t)r * a.smp.code_stride] = bi;
+          if (a.smp.prev)
+            a.smp.prev[r] = a.smp.forced ? a.smp.forced[(size_t)r * a.smp.forced_stride] : bi;
+        }
+      }
+      if (tid == 0) *a.smp.counter = 0u;
+    }
+  }
+}
+
+}  // namespace m3

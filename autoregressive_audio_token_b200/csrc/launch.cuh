@@ -1,0 +1,55 @@
+// launch.cuh -- host-side launchers of the decode kernels (one definition per
+// weight format lives in gemv_<format>.cu so they compile in parallel).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "attention.cuh"
+#include "gemv.cuh"
+
+namespace m3 {
+
+// Launch `kernel` with cudaLaunchKernelEx; with pdl the launch may begin
+// while the previous kernel in the stream is still running
+// (programmatic stream serialization); the kernel orders itself with
+// griddepcontrol.wait before touching that kernel's outputs.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t st, bool pdl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl ? attr : nullptr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Threads per output row for a GEMV over K inputs (16 inputs per thread per
+// segment); K > 1024 streams in segments of 4096.
+inline int gemv_tpr(int K) { return K <= 256 ? 16 : (K <= 1024 ? 64 : 256); }
+
+inline int gemv_rows_per_stage(int K, int esz) {
+  const int kc = gemv_tpr(K) * 16;
+  return kStageBytes / (kc * esz);
+}
+
+cudaError_t launch_gemv_bf16(const GemvArgs& a, int epi, cudaStream_t st, bool pdl, int nsm);
+cudaError_t launch_gemv_i8row(const GemvArgs& a, int epi, cudaStream_t st, bool pdl, int nsm);
+cudaError_t launch_gemv_i8g128(const GemvArgs& a, int epi, cudaStream_t st, bool pdl, int nsm);
+
+inline cudaError_t launch_gemv(const GemvArgs& a, int wf, int epi, cudaStream_t st, bool pdl,
+                               int nsm) {
+  if (wf == WF_BF16) return launch_gemv_bf16(a, epi, st, pdl, nsm);
+  if (wf == WF_I8ROW) return launch_gemv_i8row(a, epi, st, pdl, nsm);
+  return launch_gemv_i8g128(a, epi, st, pdl, nsm);
+}
+
+cudaError_t launch_attn(const AttnArgs& a, int D, int kv_f16, int splits, int rows,
+                        cudaStream_t st, bool pdl);
+
+}  // namespace m3

@@ -1,0 +1,883 @@
+// m3.cu -- host runtime behind the C ABI of include/m3.h: context, weight
+// store (upload, GPU quantisation, gate/up interleave), paged KV cache with
+// bucketed growth, one CUDA graph per (rows, KV bucket count) for the frame
+// and per (rows, teacher forcing) for the depth decoder, error plumbing.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <string>
+#include <tuple>
+#include <vector>
+
+#include "m3.h"
+#include "launch.cuh"
+#include "misc.cuh"
+
+using namespace m3;
+typedef __nv_bfloat16 bf16;
+
+// ------------------------------------------------------------------ errors --
+static thread_local std::string g_err;
+
+static int fail(int code, const std::string& msg) {
+  g_err = msg;
+  return code;
+}
+
+#define CK(call)                                                                        \
+  do {                                                                                  \
+    cudaError_t e_ = (call);                                                            \
+    if (e_ != cudaSuccess)                                                              \
+      return fail(e_ == cudaErrorMemoryAllocation ? M3_ENOMEM : M3_ECUDA,               \
+                  std::string(#call) + ": " + cudaGetErrorString(e_));                  \
+  } while (0)
+
+#define CKR(expr)             \
+  do {                        \
+    int r_ = (expr);          \
+    if (r_ != M3_OK) return r_; \
+  } while (0)
+
+// ------------------------------------------------------------------- state --
+struct DMat {
+  void* w = nullptr;   // [N][K] bf16 or int8
+  float* s = nullptr;  // int8 scales
+  int N = 0, K = 0, wf = WF_BF16;
+};
+
+struct DLayer {
+  DMat qkv, o, gu, d;
+  bf16 *attn_norm = nullptr, *mlp_norm = nullptr, *q_norm = nullptr, *k_norm = nullptr;
+};
+
+struct Acts {  // activation buffers of one stack (body or depth)
+  bf16 *x = nullptr, *qkv = nullptr, *o = nullptr, *act = nullptr;
+  float* apart = nullptr;
+  unsigned* acnt = nullptr;
+};
+
+struct m3_ctx {
+  m3_config cfg{};
+  cudaStream_t user_st = nullptr;  // caller's stream
+  cudaStream_t st = nullptr;       // internal stream (capturable)
+  cudaEvent_t ev_in = nullptr, ev_out = nullptr;
+  int dev = 0, nsm = 148;
+  bool use_graphs = true;
+  std::vector<void*> allocs;
+
+  // body
+  int wdtype = -1;
+  std::vector<DLayer> L;
+  std::vector<char> loaded;
+  bf16* final_norm = nullptr;
+  DMat lm;
+  bool head_loaded = false;
+  double* inv_freq = nullptr;
+
+  // depth decoder
+  bool depth_loaded = false;
+  std::vector<DLayer> DL;
+  DMat dproj;
+  std::vector<bf16*> demb;
+  std::vector<int> demb_rows;
+  std::vector<DMat> dheads;
+  bf16* dfinal = nullptr;
+  double* dinv_freq = nullptr;
+
+  // KV cache
+  int kv_rows = 0, kv_max_pos = 0, kv_f16 = 0, bucket = 256, max_pages = 0, n_buckets = 0;
+  std::vector<void*> buckets;
+  unsigned long long* d_pages = nullptr;
+  std::vector<unsigned long long> h_pages;
+  size_t bucket_bytes = 0;
+
+  // per-frame buffers
+  Acts A, DA;
+  bf16* h = nullptr;
+  float* logits = nullptr;
+  int* codes = nullptr;
+  float* spz = nullptr;
+  int* spi = nullptr;
+  unsigned* scnt = nullptr;
+  FrameParams* fp = nullptr;
+  int* err = nullptr;
+  int max_splits = 64;
+  // depth buffers
+  bf16* dh = nullptr;
+  int* dcodes = nullptr;
+  int* dprev = nullptr;
+  int* dforced = nullptr;
+  float* dlogits = nullptr;
+  unsigned long long* d_dpages = nullptr;
+  void* dkv = nullptr;
+
+  std::map<std::pair<int, int>, cudaGraphExec_t> graphs;
+  std::map<std::pair<int, int>, cudaGraphExec_t> dgraphs;
+};
+
+template <typename T>
+static int dalloc(m3_ctx* c, T** p, size_t bytes) {
+  void* q = nullptr;
+  CK(cudaMalloc(&q, bytes < 256 ? 256 : bytes));
+  c->allocs.push_back(q);
+  *p = static_cast<T*>(q);
+  return M3_OK;
+}
+
+static int dzalloc(m3_ctx* c, void** p, size_t bytes) {
+  CKR(dalloc(c, p, bytes));
+  CK(cudaMemset(*p, 0, bytes < 256 ? 256 : bytes));
+  return M3_OK;
+}
+
+// Order the internal stream after the caller's stream, and back.
+static int enter(m3_ctx* c) {
+  CK(cudaSetDevice(c->dev));
+  CK(cudaEventRecord(c->ev_in, c->user_st));
+  CK(cudaStreamWaitEvent(c->st, c->ev_in, 0));
+  return M3_OK;
+}
+
+static int leave(m3_ctx* c) {
+  CK(cudaEventRecord(c->ev_out, c->st));
+  CK(cudaStreamWaitEvent(c->user_st, c->ev_out, 0));
+  return M3_OK;
+}
+
+static void drop_graphs(m3_ctx* c) {
+  for (auto& kv : c->graphs) cudaGraphExecDestroy(kv.second);
+  c->graphs.clear();
+  for (auto& kv : c->dgraphs) cudaGraphExecDestroy(kv.second);
+  c->dgraphs.clear();
+}
+
+static double* make_inv_freq(m3_ctx* c, int d, double theta, int* rc) {
+  std::vector<double> h(d / 2);
+  for (int i = 0; i < d / 2; ++i) h[i] = std::pow(theta, -2.0 * (double)i / (double)d);
+  double* p = nullptr;
+  *rc = dalloc(c, &p, sizeof(double) * h.size());
+  if (*rc != M3_OK) return nullptr;
+  if (cudaMemcpy(p, h.data(), sizeof(double) * h.size(), cudaMemcpyHostToDevice) != cudaSuccess)
+    *rc = fail(M3_ECUDA, "inv_freq upload");
+  return p;
+}
+
+static int alloc_acts(m3_ctx* c, Acts& A, int rows, int H, int Hq, int Hkv, int d, int ffn,
+                      int splits) {
+  CKR(dalloc(c, &A.x, sizeof(bf16) * rows * H));
+  CKR(dalloc(c, &A.qkv, sizeof(bf16) * rows * (Hq + 2 * Hkv) * d));
+  CKR(dalloc(c, &A.o, sizeof(bf16) * rows * Hq * d));
+  CKR(dalloc(c, &A.act, sizeof(bf16) * rows * ffn));
+  CKR(dalloc(c, &A.apart, sizeof(float) * rows * Hq * splits * (d + 2)));
+  void* cnt = nullptr;
+  CKR(dzalloc(c, &cnt, sizeof(unsigned) * rows * Hkv));
+  A.acnt = static_cast<unsigned*>(cnt);
+  return M3_OK;
+}
+
+// ------------------------------------------------------------- validation --
+static bool valid_cfg(const m3_config* g, std::string& why) {
+  if (g->hidden <= 0 || g->n_layers <= 0 || g->n_q_heads <= 0 || g->n_kv_heads <= 0 ||
+      g->ffn <= 0) { why = "non-positive dimension"; return false; }
+  if (g->head_dim != 64 && g->head_dim != 128) { why = "head_dim must be 64 or 128"; return false; }
+  if (g->n_q_heads % g->n_kv_heads || g->n_q_heads / g->n_kv_heads > kAttnWarps) {
+    why = "n_q_heads / n_kv_heads must be an integer <= 4"; return false; }
+  if (g->hidden % 16 || g->ffn % 16 || (g->n_q_heads * g->head_dim) % 16) {
+    why = "hidden, ffn and n_q_heads*head_dim must be multiples of 16"; return false; }
+  if (g->max_rows < 1 || g->max_rows > kMaxRows) { why = "max_rows must be in 1..16"; return false; }
+  if (g->slice_len <= 0 || g->slice_start < 0) { why = "bad vocab slice"; return false; }
+  if (g->depth_layers > 0) {
+    if (g->depth_head_dim != 64 && g->depth_head_dim != 128) { why = "depth_head_dim"; return false; }
+    if (g->depth_hidden % 128 || g->depth_ffn % 128 || g->hidden % 128 ||
+        (g->depth_heads * g->depth_head_dim) % 128) {
+      why = "depth dimensions (and hidden) must be multiples of 128 (int8 groups)"; return false; }
+    if (g->depth_codebooks < 1 || g->depth_codebooks > 31 || g->depth_codebooks + 1 > 32) {
+      why = "depth_codebooks must be in 1..31"; return false; }
+    if (g->depth_vocab <= 0) { why = "depth_vocab"; return false; }
+  }
+  return true;
+}
+
+// ------------------------------------------------------------------ create --
+extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) {
+  if (!cfg || !out) return fail(M3_EINVAL, "null argument");
+  std::string why;
+  if (!valid_cfg(cfg, why)) return fail(M3_EINVAL, "m3_config: " + why);
+  m3_ctx* c = new m3_ctx();
+  c->cfg = *cfg;
+  c->user_st = static_cast<cudaStream_t>(cuda_stream);
+  auto bail = [&](int rc) { m3_destroy(c); return rc; };
+  if (cudaGetDevice(&c->dev) != cudaSuccess) return bail(fail(M3_ECUDA, "cudaGetDevice"));
+  if (cudaDeviceGetAttribute(&c->nsm, cudaDevAttrMultiProcessorCount, c->dev) != cudaSuccess)
+    return bail(fail(M3_ECUDA, "SM count"));
+  if (const char* e = getenv("M3_NO_GRAPH")) c->use_graphs = (e[0] == '0');
+  if (cudaStreamCreateWithFlags(&c->st, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&c->ev_in, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&c->ev_out, cudaEventDisableTiming) != cudaSuccess)
+    return bail(fail(M3_ECUDA, "stream/event creation"));
+  const m3_config& g = c->cfg;
+  const int R = g.max_rows;
+  c->L.resize(g.n_layers);
+  c->loaded.assign(g.n_layers, 0);
+  int rc = M3_OK;
+  c->inv_freq = make_inv_freq(c, g.head_dim, g.rope_theta, &rc);
+  if (rc) return bail(rc);
+  if ((rc = alloc_acts(c, c->A, R, g.hidden, g.n_q_heads, g.n_kv_heads, g.head_dim, g.ffn,
+                       c->max_splits)))
+    return bail(rc);
+  void* p = nullptr;
+  if ((rc = dalloc(c, &c->h, sizeof(bf16) * R * g.hidden)) ||
+      (rc = dalloc(c, &c->logits, sizeof(float) * R * g.slice_len)) ||
+      (rc = dalloc(c, &c->codes, sizeof(int) * R)) ||
+      (rc = dalloc(c, &c->spz, sizeof(float) * 1024 * kMaxRows)) ||
+      (rc = dalloc(c, &c->spi, sizeof(int) * 1024 * kMaxRows)) ||
+      (rc = dzalloc(c, &p, sizeof(unsigned) * 64)) )
+    return bail(rc);
+  c->scnt = static_cast<unsigned*>(p);
+  if ((rc = dzalloc(c, &p, sizeof(FrameParams)))) return bail(rc);
+  c->fp = static_cast<FrameParams*>(p);
+  if ((rc = dzalloc(c, &p, sizeof(int)))) return bail(rc);
+  c->err = static_cast<int*>(p);
+  if (g.depth_layers > 0) {
+    const int Dh = g.depth_hidden, NC = g.depth_codebooks;
+    c->DL.resize(g.depth_layers);
+    c->dinv_freq = make_inv_freq(c, g.depth_head_dim, g.depth_rope_theta, &rc);
+    if (rc) return bail(rc);
+    if ((rc = alloc_acts(c, c->DA, R, Dh, g.depth_heads, g.depth_heads, g.depth_head_dim,
+                         g.depth_ffn, 1)) ||
+        (rc = dalloc(c, &c->dh, sizeof(bf16) * R * g.hidden)) ||
+        (rc = dalloc(c, &c->dcodes, sizeof(int) * R * NC)) ||
+        (rc = dalloc(c, &c->dprev, sizeof(int) * R)) ||
+        (rc = dalloc(c, &c->dforced, sizeof(int) * R * NC)) ||
+        (rc = dalloc(c, &c->dlogits, sizeof(float) * R * NC * g.depth_vocab)))
+      return bail(rc);
+    // depth KV: one 32-position page per (row, layer), bf16
+    const size_t page = (size_t)2 * g.depth_heads * 32 * g.depth_head_dim * 2;
+    if ((rc = dzalloc(c, &c->dkv, page * R * g.depth_layers))) return bail(rc);
+    std::vector<unsigned long long> hp((size_t)R * g.depth_layers);
+    for (size_t i = 0; i < hp.size(); ++i)
+      hp[i] = (unsigned long long)(static_cast<char*>(c->dkv) + i * page);
+    if ((rc = dalloc(c, &c->d_dpages, sizeof(unsigned long long) * hp.size()))) return bail(rc);
+    if (cudaMemcpy(c->d_dpages, hp.data(), sizeof(unsigned long long) * hp.size(),
+                   cudaMemcpyHostToDevice) != cudaSuccess)
+      return bail(fail(M3_ECUDA, "depth page table"));
+  }
+  *out = c;
+  return M3_OK;
+}
+
+extern "C" void m3_destroy(m3_ctx* c) {
+  if (!c) return;
+  cudaSetDevice(c->dev);
+  if (c->st) cudaStreamSynchronize(c->st);
+  drop_graphs(c);
+  for (void* p : c->buckets) cudaFree(p);
+  for (void* p : c->allocs) cudaFree(p);
+  if (c->ev_in) cudaEventDestroy(c->ev_in);
+  if (c->ev_out) cudaEventDestroy(c->ev_out);
+  if (c->st) cudaStreamDestroy(c->st);
+  delete c;
+}
+
+extern "C" const char* m3_last_error(void) { return g_err.c_str(); }
+
+// ----------------------------------------------------------------- weights --
+// Copy a bf16 [rows, cols] source into device staging memory (or use it as is).
+static int stage_src(m3_ctx* c, const void* src, size_t bytes, int mem, const void** dev,
+                     void** owned) {
+  *owned = nullptr;
+  if (mem == M3_MEM_DEVICE) {
+    *dev = src;
+    return M3_OK;
+  }
+  CK(cudaMallocAsync(owned, bytes, c->st));
+  CK(cudaMemcpyAsync(*owned, src, bytes, cudaMemcpyHostToDevice, c->st));
+  *dev = *owned;
+  return M3_OK;
+}
+
+// Place a [rows, cols] bf16 source at rows dst_row0, dst_row0 + row_step, ...
+// of matrix M, quantising on the GPU when M is int8.
+static int put_rows(m3_ctx* c, DMat& M, const void* src, int mem, int rows, int dst_row0,
+                    int row_step) {
+  if (!src) return fail(M3_EINVAL, "null weight pointer");
+  const int cols = M.K;
+  const size_t bytes = sizeof(bf16) * (size_t)rows * cols;
+  const void* dsrc = nullptr;
+  void* owned = nullptr;
+  CKR(stage_src(c, src, bytes, mem, &dsrc, &owned));
+  if (M.wf == WF_BF16) {
+    CK(cudaMemcpy2DAsync(static_cast<bf16*>(M.w) + (size_t)dst_row0 * cols,
+                         sizeof(bf16) * cols * row_step, dsrc, sizeof(bf16) * cols,
+                         sizeof(bf16) * cols, rows, cudaMemcpyDeviceToDevice, c->st));
+  } else if (M.wf == WF_I8ROW) {
+    quantize_rows_kernel<<<dim3(1, rows), 256, 0, c->st>>>(
+        static_cast<const bf16*>(dsrc), cols, cols,
+        static_cast<int8_t*>(M.w) + (size_t)dst_row0 * cols, (int64_t)cols * row_step,
+        M.s + dst_row0, row_step);
+    CK(cudaGetLastError());
+  } else {
+    const int ng = cols / 128;
+    const int64_t warps = (int64_t)rows * ng;
+    quantize_g128_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, c->st>>>(
+        static_cast<const bf16*>(dsrc), rows, cols,
+        static_cast<int8_t*>(M.w) + (size_t)dst_row0 * cols, (int64_t)cols * row_step,
+        M.s + (size_t)dst_row0 * ng, (int64_t)ng * row_step);
+    CK(cudaGetLastError());
+  }
+  if (owned) CK(cudaFreeAsync(owned, c->st));
+  return M3_OK;
+}
+
+static int alloc_mat(m3_ctx* c, DMat& M, int N, int K, int wf) {
+  M.N = N;
+  M.K = K;
+  M.wf = wf;
+  const size_t esz = wf == WF_BF16 ? 2 : 1;
+  CKR(dalloc(c, &M.w, esz * (size_t)N * K));
+  if (wf == WF_I8ROW) CKR(dalloc(c, &M.s, sizeof(float) * N));
+  if (wf == WF_I8G128) CKR(dalloc(c, &M.s, sizeof(float) * (size_t)N * (K / 128)));
+  return M3_OK;
+}
+
+static int put_vec(m3_ctx* c, bf16** dst, const void* src, int n, int mem) {
+  if (!src) return fail(M3_EINVAL, "null norm pointer");
+  if (!*dst) CKR(dalloc(c, dst, sizeof(bf16) * n));
+  CK(cudaMemcpyAsync(*dst, src, sizeof(bf16) * n,
+                     mem == M3_MEM_DEVICE ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice,
+                     c->st));
+  return M3_OK;
+}
+
+static int load_layer(m3_ctx* c, DLayer& L, const m3_layer_src& s, int mem, int wf, int H,
+                      int Hq, int Hkv, int d, int ffn) {
+  const int nq = Hq * d, nkv = Hkv * d;
+  if (!L.qkv.w) {
+    CKR(alloc_mat(c, L.qkv, nq + 2 * nkv, H, wf));
+    CKR(alloc_mat(c, L.o, H, nq, wf));
+    CKR(alloc_mat(c, L.gu, 2 * ffn, H, wf));
+    CKR(alloc_mat(c, L.d, H, ffn, wf));
+  }
+  CKR(put_rows(c, L.qkv, s.wq, mem, nq, 0, 1));
+  CKR(put_rows(c, L.qkv, s.wk, mem, nkv, nq, 1));
+  CKR(put_rows(c, L.qkv, s.wv, mem, nkv, nq + nkv, 1));
+  CKR(put_rows(c, L.o, s.wo, mem, H, 0, 1));
+  CKR(put_rows(c, L.gu, s.wg, mem, ffn, 0, 2));  // gate rows at 2j
+  CKR(put_rows(c, L.gu, s.wu, mem, ffn, 1, 2));  // up rows at 2j+1
+  CKR(put_rows(c, L.d, s.wd, mem, ffn == 0 ? 0 : H, 0, 1));
+  CKR(put_vec(c, &L.attn_norm, s.attn_norm, H, mem));
+  CKR(put_vec(c, &L.mlp_norm, s.mlp_norm, H, mem));
+  CKR(put_vec(c, &L.q_norm, s.q_norm, d, mem));
+  CKR(put_vec(c, &L.k_norm, s.k_norm, d, mem));
+  return M3_OK;
+}
+
+extern "C" int m3_load_weights(m3_ctx* c, const m3_weight_src* src, int wdtype) {
+  if (!c || !src) return fail(M3_EINVAL, "null argument");
+  if (wdtype != M3_W_BF16 && wdtype != M3_W_INT8) return fail(M3_EINVAL, "wdtype");
+  if (c->wdtype >= 0 && c->wdtype != wdtype) return fail(M3_ESTATE, "wdtype differs from first load");
+  const m3_config& g = c->cfg;
+  if (src->n_layers < 0 || src->first_layer < 0 || src->first_layer + src->n_layers > g.n_layers)
+    return fail(M3_EINVAL, "layer range");
+  if (src->n_layers > 0 && !src->layers) return fail(M3_EINVAL, "null layers");
+  c->wdtype = wdtype;
+  const int wf = wdtype == M3_W_INT8 ? WF_I8ROW : WF_BF16;
+  CKR(enter(c));
+  for (int i = 0; i < src->n_layers; ++i) {
+    const int l = src->first_layer + i;
+    CKR(load_layer(c, c->L[l], src->layers[i], src->mem, wf, g.hidden, g.n_q_heads, g.n_kv_heads,
+                   g.head_dim, g.ffn));
+    c->loaded[l] = 1;
+  }
+  if (src->final_norm) CKR(put_vec(c, &c->final_norm, src->final_norm, g.hidden, src->mem));
+  if (src->lm_head) {
+    if (!c->lm.w) CKR(alloc_mat(c, c->lm, g.slice_len, g.hidden, wf));
+    CKR(put_rows(c, c->lm, src->lm_head, src->mem, g.slice_len, 0, 1));
+    c->head_loaded = true;
+  }
+  CK(cudaStreamSynchronize(c->st));  // sources may be freed on return
+  return leave(c);
+}
+
+extern "C" int m3_load_depth_weights(m3_ctx* c, const m3_depth_src* src) {
+  if (!c || !src) return fail(M3_EINVAL, "null argument");
+  const m3_config& g = c->cfg;
+  if (g.depth_layers <= 0) return fail(M3_ESTATE, "config has no depth decoder");
+  if (!src->layers || !src->proj || !src->emb || !src->final_norm || !src->heads)
+    return fail(M3_EINVAL, "null depth weight pointer");
+  CKR(enter(c));
+  const int Dh = g.depth_hidden;
+  for (int l = 0; l < g.depth_layers; ++l)
+    CKR(load_layer(c, c->DL[l], src->layers[l], src->mem, WF_I8G128, Dh, g.depth_heads,
+                   g.depth_heads, g.depth_head_dim, g.depth_ffn));
+  if (!c->dproj.w) CKR(alloc_mat(c, c->dproj, Dh, g.hidden, WF_I8G128));
+  CKR(put_rows(c, c->dproj, src->proj, src->mem, Dh, 0, 1));
+  c->demb.resize(g.depth_codebooks, nullptr);
+  c->demb_rows.resize(g.depth_codebooks);
+  c->dheads.resize(g.depth_codebooks);
+  for (int j = 0; j < g.depth_codebooks; ++j) {
+    const int n = j == 0 ? g.slice_len : g.depth_vocab;
+    c->demb_rows[j] = n;
+    if (!src->emb[j] || !src->heads[j]) return fail(M3_EINVAL, "null depth table");
+    if (!c->demb[j]) CKR(dalloc(c, &c->demb[j], sizeof(bf16) * (size_t)n * Dh));
+    CK(cudaMemcpyAsync(c->demb[j], src->emb[j], sizeof(bf16) * (size_t)n * Dh,
+                       src->mem == M3_MEM_DEVICE ? cudaMemcpyDeviceToDevice
+                                                 : cudaMemcpyHostToDevice,
+                       c->st));
+    if (!c->dheads[j].w) CKR(alloc_mat(c, c->dheads[j], g.depth_vocab, Dh, WF_I8G128));
+    CKR(put_rows(c, c->dheads[j], src->heads[j], src->mem, g.depth_vocab, 0, 1));
+  }
+  CKR(put_vec(c, &c->dfinal, src->final_norm, Dh, src->mem));
+  CK(cudaStreamSynchronize(c->st));
+  c->depth_loaded = true;
+  return leave(c);
+}
+
+extern "C" int m3_quantize_int8(const void* w, int64_t rows, int64_t cols, int64_t group,
+                                int8_t* q, float* scales, void* cuda_stream) {
+  if (!w || !q || !scales || rows <= 0 || cols <= 0) return fail(M3_EINVAL, "bad argument");
+  if (group != cols && group != 128) return fail(M3_EINVAL, "group must be cols or 128");
+  if (cols % group) return fail(M3_EINVAL, "cols % group != 0");
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  if (group == cols) {
+    quantize_rows_kernel<<<dim3(1, (unsigned)rows), 256, 0, st>>>(static_cast<const bf16*>(w),
+                                                                  cols, cols, q, cols, scales, 1);
+  } else {
+    const int64_t warps = rows * (cols / 128);
+    quantize_g128_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(
+        static_cast<const bf16*>(w), rows, cols, q, cols, scales, cols / 128);
+  }
+  CK(cudaGetLastError());
+  return M3_OK;
+}
+
+// which: 0 wq 1 wk 2 wv 3 wo 4 wg 5 wu 6 wd 7 lm_head; 8.. the same for depth
+// layers; 16 depth proj; 17 + j depth head j.
+extern "C" int m3_export_weight(m3_ctx* c, int which, int layer, void* q_host, float* s_host) {
+  if (!c || !q_host) return fail(M3_EINVAL, "null argument");
+  const m3_config& g = c->cfg;
+  const DMat* M = nullptr;
+  int row0 = 0, rows = 0, step = 1;
+  const bool depth = which >= 8;
+  const int w = depth && which < 16 ? which - 8 : which;
+  if (which == 16) {
+    M = &c->dproj;
+    rows = M->N;
+  } else if (which >= 17) {
+    if (which - 17 >= (int)c->dheads.size()) return fail(M3_EINVAL, "depth head index");
+    M = &c->dheads[which - 17];
+    rows = M->N;
+  } else if (w == 7) {
+    if (depth) return fail(M3_EINVAL, "which");
+    M = &c->lm;
+    rows = M->N;
+  } else {
+    const std::vector<DLayer>& LL = depth ? c->DL : c->L;
+    if (layer < 0 || layer >= (int)LL.size()) return fail(M3_EINVAL, "layer");
+    const DLayer& L = LL[layer];
+    const int hq = depth ? g.depth_heads : g.n_q_heads, hkv = depth ? g.depth_heads : g.n_kv_heads;
+    const int d = depth ? g.depth_head_dim : g.head_dim;
+    switch (w) {
+      case 0: M = &L.qkv; row0 = 0; rows = hq * d; break;
+      case 1: M = &L.qkv; row0 = hq * d; rows = hkv * d; break;
+      case 2: M = &L.qkv; row0 = (hq + hkv) * d; rows = hkv * d; break;
+      case 3: M = &L.o; rows = M->N; break;
+      case 4: M = &L.gu; row0 = 0; step = 2; rows = M->N / 2; break;
+      case 5: M = &L.gu; row0 = 1; step = 2; rows = M->N / 2; break;
+      case 6: M = &L.d; rows = M->N; break;
+      default: return fail(M3_EINVAL, "which");
+    }
+  }
+  if (!M || !M->w) return fail(M3_ESTATE, "weight not loaded");
+  CK(cudaStreamSynchronize(c->st));
+  const size_t esz = M->wf == WF_BF16 ? 2 : 1;
+  const size_t rb = esz * M->K;
+  CK(cudaMemcpy2D(q_host, rb, static_cast<const char*>(M->w) + (size_t)row0 * rb, rb * step, rb,
+                  rows, cudaMemcpyDeviceToHost));
+  if (M->wf != WF_BF16 && s_host) {
+    const int ns = M->wf == WF_I8ROW ? 1 : M->K / 128;
+    CK(cudaMemcpy2D(s_host, sizeof(float) * ns, M->s + (size_t)row0 * ns,
+                    sizeof(float) * ns * step, sizeof(float) * ns, rows, cudaMemcpyDeviceToHost));
+  }
+  return M3_OK;
+}
+
+// ---------------------------------------------------------------- KV cache --
+extern "C" int m3_kv_alloc(m3_ctx* c, int rows, int max_positions, int kvdtype, int bucket) {
+  if (!c) return fail(M3_EINVAL, "null ctx");
+  if (rows < 1 || rows > c->cfg.max_rows) return fail(M3_EINVAL, "rows out of 1..max_rows");
+  if (max_positions < 1) return fail(M3_EINVAL, "max_positions");
+  if (bucket < 32 || bucket % 32) return fail(M3_EINVAL, "bucket must be a multiple of 32");
+  if (kvdtype != M3_KV_BF16 && kvdtype != M3_KV_F16) return fail(M3_EINVAL, "kvdtype");
+  CKR(enter(c));
+  CK(cudaStreamSynchronize(c->st));
+  drop_graphs(c);
+  for (void* p : c->buckets) cudaFree(p);
+  c->buckets.clear();
+  const m3_config& g = c->cfg;
+  c->kv_rows = rows;
+  c->kv_max_pos = max_positions;
+  c->kv_f16 = kvdtype == M3_KV_F16;
+  c->bucket = bucket;
+  c->max_pages = (max_positions + bucket - 1) / bucket;
+  c->n_buckets = 0;
+  c->bucket_bytes = (size_t)rows * g.n_layers * 2 * g.n_kv_heads * bucket * g.head_dim * 2;
+  c->h_pages.assign((size_t)rows * g.n_layers * c->max_pages, 0ull);
+  if (c->d_pages) {
+    cudaFree(c->d_pages);
+    for (auto it = c->allocs.begin(); it != c->allocs.end(); ++it)
+      if (*it == c->d_pages) { c->allocs.erase(it); break; }
+    c->d_pages = nullptr;
+  }
+  CKR(dalloc(c, &c->d_pages, sizeof(unsigned long long) * c->h_pages.size()));
+  CK(cudaMemset(c->d_pages, 0, sizeof(unsigned long long) * c->h_pages.size()));
+  return leave(c);
+}
+
+// Make sure buckets cover positions [0, npos).  New buckets are zeroed, so a
+// row that skips positions reads zeros there.
+static int ensure_pages(m3_ctx* c, int npos) {
+  const int need = (npos + c->bucket - 1) / c->bucket;
+  if (need <= c->n_buckets) return M3_OK;
+  if (need > c->max_pages) return fail(M3_ECAPACITY, "KV capacity exceeded");
+  CK(cudaStreamSynchronize(c->st));
+  const m3_config& g = c->cfg;
+  const size_t page_bytes = (size_t)2 * g.n_kv_heads * c->bucket * g.head_dim * 2;
+  for (int b = c->n_buckets; b < need; ++b) {
+    void* p = nullptr;
+    CK(cudaMalloc(&p, c->bucket_bytes));
+    CK(cudaMemset(p, 0, c->bucket_bytes));
+    c->buckets.push_back(p);
+    for (int r = 0; r < c->kv_rows; ++r)
+      for (int l = 0; l < g.n_layers; ++l)
+        c->h_pages[((size_t)r * g.n_layers + l) * c->max_pages + b] =
+            (unsigned long long)(static_cast<char*>(p) + ((size_t)r * g.n_layers + l) * page_bytes);
+  }
+  c->n_buckets = need;
+  CK(cudaMemcpy(c->d_pages, c->h_pages.data(), sizeof(unsigned long long) * c->h_pages.size(),
+                cudaMemcpyHostToDevice));
+  CK(cudaDeviceSynchronize());
+  return M3_OK;
+}
+
+extern "C" int m3_kv_set(m3_ctx* c, int row, int n_positions, const void* k, const void* v, int mem) {
+  if (!c || !k || !v) return fail(M3_EINVAL, "null argument");
+  if (!c->d_pages) return fail(M3_ESTATE, "m3_kv_alloc first");
+  if (row < 0 || row >= c->kv_rows) return fail(M3_EINVAL, "row");
+  if (n_positions < 0 || n_positions > c->kv_max_pos) return fail(M3_ECAPACITY, "n_positions");
+  if (n_positions == 0) return M3_OK;
+  CKR(enter(c));
+  CKR(ensure_pages(c, n_positions));
+  const m3_config& g = c->cfg;
+  const size_t bytes = sizeof(bf16) * (size_t)g.n_layers * n_positions * g.n_kv_heads * g.head_dim;
+  const void *dk = nullptr, *dv = nullptr;
+  void *ok = nullptr, *ov = nullptr;
+  CKR(stage_src(c, k, bytes, mem, &dk, &ok));
+  CKR(stage_src(c, v, bytes, mem, &dv, &ov));
+  kv_set_kernel<<<c->nsm * 4, 256, 0, c->st>>>(
+      static_cast<const bf16*>(dk), static_cast<const bf16*>(dv),
+      c->d_pages + (size_t)row * g.n_layers * c->max_pages, g.n_layers, c->max_pages, c->bucket,
+      n_positions, g.n_kv_heads, g.head_dim, c->kv_f16);
+  CK(cudaGetLastError());
+  if (ok) CK(cudaFreeAsync(ok, c->st));
+  if (ov) CK(cudaFreeAsync(ov, c->st));
+  CK(cudaStreamSynchronize(c->st));
+  return leave(c);
+}
+
+extern "C" int m3_kv_get(m3_ctx* c, int row, int n_positions, void* k_host, void* v_host) {
+  if (!c || !k_host || !v_host) return fail(M3_EINVAL, "null argument");
+  if (!c->d_pages) return fail(M3_ESTATE, "m3_kv_alloc first");
+  if (row < 0 || row >= c->kv_rows) return fail(M3_EINVAL, "row");
+  if (n_positions < 0 || n_positions > c->n_buckets * c->bucket)
+    return fail(M3_ECAPACITY, "n_positions beyond the allocated buckets");
+  if (n_positions == 0) return M3_OK;
+  CKR(enter(c));
+  const m3_config& g = c->cfg;
+  const size_t n = (size_t)g.n_layers * n_positions * g.n_kv_heads * g.head_dim;
+  void *dk = nullptr, *dv = nullptr;
+  CK(cudaMallocAsync(&dk, n * 2, c->st));
+  CK(cudaMallocAsync(&dv, n * 2, c->st));
+  kv_get_kernel<<<c->nsm * 4, 256, 0, c->st>>>(
+      static_cast<uint16_t*>(dk), static_cast<uint16_t*>(dv),
+      c->d_pages + (size_t)row * g.n_layers * c->max_pages, g.n_layers, c->max_pages, c->bucket,
+      n_positions, g.n_kv_heads, g.head_dim);
+  CK(cudaGetLastError());
+  CK(cudaMemcpyAsync(k_host, dk, n * 2, cudaMemcpyDeviceToHost, c->st));
+  CK(cudaMemcpyAsync(v_host, dv, n * 2, cudaMemcpyDeviceToHost, c->st));
+  CK(cudaFreeAsync(dk, c->st));
+  CK(cudaFreeAsync(dv, c->st));
+  CK(cudaStreamSynchronize(c->st));
+  return leave(c);
+}
+
+// ------------------------------------------------------------ the frame ----
+static int attn_splits(const m3_ctx* c, int rows, int nb) {
+  const int pairs = rows * c->cfg.n_kv_heads;
+  int s = (2 * c->nsm + pairs - 1) / pairs;
+  const int tiles = nb * c->bucket / kAttnTile;
+  if (s > tiles) s = tiles;
+  if (s > c->max_splits) s = c->max_splits;
+  return s < 1 ? 1 : s;
+}
+
+// A GEMV over all `rows` batch rows, in launches of at most 4 rows.
+static int gemv_rows(m3_ctx* c, const DMat& M, int epi, int rows, const bf16* x, int ldx,
+                     const bf16* gamma, bf16* out, int ldo, const SampleArgs* smp, bool& pdl) {
+  for (int r0 = 0; r0 < rows; r0 += 4) {
+    GemvArgs a{};
+    a.w = M.w;
+    a.scales = M.s;
+    a.N = M.N;
+    a.K = M.K;
+    a.row0 = r0;
+    a.mr = rows - r0 < 4 ? rows - r0 : 4;
+    a.x = x + (size_t)r0 * ldx;
+    a.ldx = ldx;
+    a.gamma = gamma;
+    a.eps = c->cfg.rms_eps;
+    a.out = out ? out + (size_t)r0 * ldo : nullptr;
+    a.ldo = ldo;
+    a.fp = c->fp;
+    if (smp) a.smp = *smp;
+    a.err = c->err;
+    CK(launch_gemv(a, M.wf, epi, c->st, pdl, c->nsm));
+    pdl = true;
+  }
+  return M3_OK;
+}
+
+static int record_layer(m3_ctx* c, const DLayer& L, Acts& A, int rows, int H, int Hq, int Hkv,
+                        int d, int ffn, const unsigned long long* pages, int layer, int n_layers,
+                        int max_pages, int page_size, int kv_f16, int splits, int fixed_pos,
+                        const double* inv_freq, bool& pdl) {
+  const int ldqkv = (Hq + 2 * Hkv) * d;
+  CKR(gemv_rows(c, L.qkv, EPI_STORE, rows, A.x, H, L.attn_norm, A.qkv, ldqkv, nullptr, pdl));
+  AttnArgs at{};
+  at.qkv = A.qkv;
+  at.ldqkv = ldqkv;
+  at.q_norm = L.q_norm;
+  at.k_norm = L.k_norm;
+  at.eps = c->cfg.rms_eps;
+  at.inv_freq = inv_freq;
+  at.pages = pages;
+  at.layer = layer;
+  at.n_layers = n_layers;
+  at.max_pages = max_pages;
+  at.page_size = page_size;
+  at.Hq = Hq;
+  at.Hkv = Hkv;
+  at.part = A.apart;
+  at.counters = A.acnt;
+  at.out = A.o;
+  at.fp = c->fp;
+  at.fixed_pos = fixed_pos;
+  at.err = c->err;
+  CK(launch_attn(at, d, kv_f16, splits, rows, c->st, true));
+  CKR(gemv_rows(c, L.o, EPI_RESID, rows, A.o, Hq * d, nullptr, A.x, H, nullptr, pdl));
+  CKR(gemv_rows(c, L.gu, EPI_SWIGLU, rows, A.x, H, L.mlp_norm, A.act, ffn, nullptr, pdl));
+  CKR(gemv_rows(c, L.d, EPI_RESID, rows, A.act, ffn, nullptr, A.x, H, nullptr, pdl));
+  return M3_OK;
+}
+
+static int record_frame(m3_ctx* c, int rows, int nb) {
+  const m3_config& g = c->cfg;
+  const int splits = attn_splits(c, rows, nb);
+  bool pdl = false;  // the first kernel follows the parameter block in plain stream order
+  for (int l = 0; l < g.n_layers; ++l)
+    CKR(record_layer(c, c->L[l], c->A, rows, g.hidden, g.n_q_heads, g.n_kv_heads, g.head_dim,
+                     g.ffn, c->d_pages, l, g.n_layers, c->max_pages, c->bucket, c->kv_f16, splits,
+                     -1, c->inv_freq, pdl));
+  SampleArgs sa{};
+  sa.logits = c->logits;
+  sa.logits_ld = g.slice_len;
+  sa.codes = c->codes;
+  sa.code_stride = 1;
+  sa.index_base = (unsigned long long)g.slice_start;
+  sa.part_z = c->spz;
+  sa.part_i = c->spi;
+  sa.counter = c->scnt;
+  sa.h_out = c->h;
+  CKR(gemv_rows(c, c->lm, EPI_SAMPLE, rows, c->A.x, g.hidden, c->final_norm, nullptr, 0, &sa, pdl));
+  return M3_OK;
+}
+
+// Run `record` either directly or through a cached graph keyed by `key`.
+template <typename F>
+static int run_graph(m3_ctx* c, std::map<std::pair<int, int>, cudaGraphExec_t>& cache,
+                     std::pair<int, int> key, F record) {
+  if (!c->use_graphs) return record();
+  auto it = cache.find(key);
+  if (it == cache.end()) {
+    cudaGraph_t graph = nullptr;
+    CK(cudaStreamBeginCapture(c->st, cudaStreamCaptureModeThreadLocal));
+    int rc = record();
+    cudaError_t e = cudaStreamEndCapture(c->st, &graph);
+    if (rc != M3_OK) {
+      if (graph) cudaGraphDestroy(graph);
+      return rc;
+    }
+    if (e != cudaSuccess) return fail(M3_ECUDA, std::string("graph capture: ") + cudaGetErrorString(e));
+    cudaGraphExec_t exec = nullptr;
+    e = cudaGraphInstantiate(&exec, graph, 0);
+    cudaGraphDestroy(graph);
+    if (e != cudaSuccess) return fail(M3_ECUDA, std::string("graph instantiate: ") + cudaGetErrorString(e));
+    it = cache.emplace(key, exec).first;
+  }
+  CK(cudaGraphLaunch(it->second, c->st));
+  return M3_OK;
+}
+
+extern "C" int m3_decode_frame(m3_ctx* c, int rows, const int32_t* positions, uint64_t seed,
+                               uint64_t frame, const void* x_in, float cfg_scale,
+                               float temperature, int32_t* codes, void* h_out, float* logits) {
+  if (!c || !positions || !x_in || !codes) return fail(M3_EINVAL, "null argument");
+  const m3_config& g = c->cfg;
+  if (!c->d_pages) return fail(M3_ESTATE, "m3_kv_alloc first");
+  for (int l = 0; l < g.n_layers; ++l)
+    if (!c->loaded[l]) return fail(M3_ESTATE, "layer " + std::to_string(l) + " not loaded");
+  if (!c->head_loaded || !c->final_norm) return fail(M3_ESTATE, "lm_head / final norm not loaded");
+  if (rows < 1 || rows > c->kv_rows) return fail(M3_EINVAL, "rows out of 1..cache rows");
+  if (!(cfg_scale >= 0.0f) || !(temperature > 0.0f)) return fail(M3_EINVAL, "cfg_scale / temperature");
+  if (cfg_scale > 0.0f && rows % 2) return fail(M3_EINVAL, "cfg_scale > 0 needs (cond, uncond) row pairs");
+  FrameParams fp{};
+  fp.rows = rows;
+  fp.cfg_on = cfg_scale > 0.0f;
+  fp.cfg_scale = cfg_scale;
+  fp.temperature = temperature;
+  fp.seed = seed;
+  fp.frame = frame;
+  int maxpos = 0;
+  for (int r = 0; r < rows; ++r) {
+    if (positions[r] < 0 || positions[r] >= c->kv_max_pos)
+      return fail(M3_ECAPACITY, "position " + std::to_string(positions[r]) + " outside the KV capacity");
+    fp.pos[r] = positions[r];
+    maxpos = positions[r] > maxpos ? positions[r] : maxpos;
+  }
+  CKR(enter(c));
+  CKR(ensure_pages(c, maxpos + 1));
+  CK(cudaMemcpyAsync(c->A.x, x_in, sizeof(bf16) * rows * g.hidden, cudaMemcpyDeviceToDevice, c->st));
+  set_frame_params_kernel<<<1, 32, 0, c->st>>>(c->fp, fp);
+  CK(cudaGetLastError());
+  CKR(run_graph(c, c->graphs, {rows, c->n_buckets}, [&] { return record_frame(c, rows, c->n_buckets); }));
+  CK(cudaMemcpyAsync(codes, c->codes, sizeof(int) * rows, cudaMemcpyDeviceToDevice, c->st));
+  if (h_out)
+    CK(cudaMemcpyAsync(h_out, c->h, sizeof(bf16) * rows * g.hidden, cudaMemcpyDeviceToDevice, c->st));
+  if (logits)
+    CK(cudaMemcpyAsync(logits, c->logits, sizeof(float) * rows * g.slice_len,
+                       cudaMemcpyDeviceToDevice, c->st));
+  return leave(c);
+}
+
+// --------------------------------------------------------- depth decoder ---
+static int record_depth(m3_ctx* c, int rows, bool forced) {
+  const m3_config& g = c->cfg;
+  const int Dh = g.depth_hidden, NC = g.depth_codebooks, V = g.depth_vocab;
+  bool pdl = false;
+  CKR(gemv_rows(c, c->dproj, EPI_STORE, rows, c->dh, g.hidden, nullptr, c->DA.x, Dh, nullptr, pdl));
+  for (int j = 0; j <= NC; ++j) {
+    if (j >= 1) {
+      CK(launch_ex(embed_kernel, dim3(rows), dim3(128), 0, c->st, true, (const int*)c->dprev,
+                   (const bf16*)c->demb[j - 1], c->demb_rows[j - 1], 0, Dh, c->DA.x, c->err));
+    }
+    for (int l = 0; l < g.depth_layers; ++l)
+      CKR(record_layer(c, c->DL[l], c->DA, rows, Dh, g.depth_heads, g.depth_heads,
+                       g.depth_head_dim, g.depth_ffn, c->d_dpages, l, g.depth_layers, 1, 32, 0, 1,
+                       j, c->dinv_freq, pdl));
+    if (j >= 1) {
+      SampleArgs sa{};
+      sa.logits = c->dlogits + (size_t)(j - 1) * V;
+      sa.logits_ld = NC * V;
+      sa.codes = c->dcodes + (j - 1);
+      sa.code_stride = NC;
+      sa.prev = c->dprev;
+      sa.forced = forced ? c->dforced + (j - 1) : nullptr;
+      sa.forced_stride = NC;
+      sa.index_base = (unsigned long long)j << 32;
+      sa.part_z = c->spz;
+      sa.part_i = c->spi;
+      sa.counter = c->scnt + 1;
+      CKR(gemv_rows(c, c->dheads[j - 1], EPI_SAMPLE, rows, c->DA.x, Dh, c->dfinal, nullptr, 0, &sa, pdl));
+    }
+  }
+  return M3_OK;
+}
+
+extern "C" int m3_depth_decode(m3_ctx* c, int rows, const void* h_frame, const int32_t* code0,
+                               uint64_t seed, uint64_t frame, float cfg_scale, float temperature,
+                               const int32_t* forced, int32_t* codes, float* logits) {
+  if (!c || !h_frame || !code0 || !codes) return fail(M3_EINVAL, "null argument");
+  const m3_config& g = c->cfg;
+  if (!c->depth_loaded) return fail(M3_ESTATE, "depth decoder not loaded");
+  if (rows < 1 || rows > g.max_rows) return fail(M3_EINVAL, "rows out of 1..max_rows");
+  if (!(cfg_scale >= 0.0f) || !(temperature > 0.0f)) return fail(M3_EINVAL, "cfg_scale / temperature");
+  if (cfg_scale > 0.0f && rows % 2) return fail(M3_EINVAL, "cfg_scale > 0 needs (cond, uncond) row pairs");
+  const int NC = g.depth_codebooks;
+  FrameParams fp{};
+  fp.rows = rows;
+  fp.cfg_on = cfg_scale > 0.0f;
+  fp.cfg_scale = cfg_scale;
+  fp.temperature = temperature;
+  fp.seed = seed;
+  fp.frame = frame;
+  CKR(enter(c));
+  CK(cudaMemcpyAsync(c->dh, h_frame, sizeof(bf16) * rows * g.hidden, cudaMemcpyDeviceToDevice, c->st));
+  CK(cudaMemcpyAsync(c->dprev, code0, sizeof(int) * rows, cudaMemcpyDeviceToDevice, c->st));
+  if (forced)
+    CK(cudaMemcpyAsync(c->dforced, forced, sizeof(int) * rows * NC, cudaMemcpyDeviceToDevice, c->st));
+  set_frame_params_kernel<<<1, 32, 0, c->st>>>(c->fp, fp);
+  CK(cudaGetLastError());
+  const bool f = forced != nullptr;
+  CKR(run_graph(c, c->dgraphs, {rows, f ? 1 : 0}, [&] { return record_depth(c, rows, f); }));
+  CK(cudaMemcpyAsync(codes, c->dcodes, sizeof(int) * rows * NC, cudaMemcpyDeviceToDevice, c->st));
+  if (logits)
+    CK(cudaMemcpyAsync(logits, c->dlogits, sizeof(float) * rows * NC * g.depth_vocab,
+                       cudaMemcpyDeviceToDevice, c->st));
+  return leave(c);
+}
+
+// ------------------------------------------------------------- the rest ----
+extern "C" int m3_embed(m3_ctx* c, int rows, const int32_t* codes, const void* table, int offset,
+                        void* x_out) {
+  if (!c || !codes || !table || !x_out) return fail(M3_EINVAL, "null argument");
+  if (rows < 1 || rows > c->cfg.max_rows) return fail(M3_EINVAL, "rows");
+  CKR(enter(c));
+  CK(launch_ex(embed_kernel, dim3(rows), dim3(128), 0, c->st, false, codes,
+               static_cast<const bf16*>(table), 0x7fffffff, offset, c->cfg.hidden,
+               static_cast<bf16*>(x_out), c->err));
+  return leave(c);
+}
+
+extern "C" double m3_frame_bytes(const m3_ctx* c, int rows, int ctx_len) {
+  if (!c) return 0.0;
+  const m3_config& g = c->cfg;
+  const double esz = c->wdtype == M3_W_INT8 ? 1.0 : 2.0;
+  const double H = g.hidden, d = g.head_dim;
+  const double per_layer = H * (g.n_q_heads + 2.0 * g.n_kv_heads) * d + H * g.n_q_heads * d +
+                           3.0 * H * g.ffn;
+  double w = g.n_layers * per_layer * esz + (double)g.slice_len * H * esz;
+  if (c->wdtype == M3_W_INT8)
+    w += 4.0 * (g.n_layers * ((g.n_q_heads + 2.0 * g.n_kv_heads) * d + H + 2.0 * g.ffn + H) +
+                g.slice_len);
+  w += 2.0 * (g.n_layers * (2.0 * H + 2.0 * d) + H);  // norm gains
+  const double kv = (double)rows * (ctx_len + 1.0) * g.n_layers * 2.0 * g.n_kv_heads * d * 2.0;
+  return w + kv;
+}
+
+extern "C" int m3_sync_status(m3_ctx* c) {
+  if (!c) return fail(M3_EINVAL, "null ctx");
+  CK(cudaSetDevice(c->dev));
+  CK(cudaStreamSynchronize(c->st));
+  CK(cudaStreamSynchronize(c->user_st));
+  int e = 0;
+  CK(cudaMemcpy(&e, c->err, sizeof(int), cudaMemcpyDeviceToHost));
+  if (e != 0) {
+    CK(cudaMemset(c->err, 0, sizeof(int)));
+    if (e == kErrTimeout) return fail(M3_ETIMEOUT, "a device-side wait gave up");
+    return fail(M3_EDEVICE, "a kernel recorded an out-of-range index");
+  }
+  return M3_OK;
+}

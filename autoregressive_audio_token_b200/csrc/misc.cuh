@@ -1,0 +1,157 @@
+// misc.cuh -- the small kernels around the decode step: per-frame parameter
+// block, GPU int8 quantiser, embedding lookup, KV prefill / readback.
+#pragma once
+
+#include "common.cuh"
+#include "gemv.cuh"
+
+namespace m3 {
+
+// The frame's scalars go to a device block by a kernel launch (not a
+// host-to-device copy), so they are ordered on the stream like any kernel
+// and the captured graph reads them from a fixed address.
+__global__ void set_frame_params_kernel(FrameParams* dst, FrameParams v) {
+  if (threadIdx.x == 0) *dst = v;
+}
+
+// int8 weight-only quantisation ("MiniMax Music 3 on Metal", section
+// "Precision": one scale per row for the body and lm_head, per group of 128
+// for the depth decoder, quantised on the GPU at load):
+//   s = absmax / 127 (IEEE fp32 division), q = clamp(rint(w / s), -127, 127),
+//   s == 0 -> q = 0.
+// One CTA per (row, group) for groups >= 1024 elements; the output row r is
+// written at q + r * q_ld and its scales at s + r * s_ld.
+__global__ void quantize_rows_kernel(const __nv_bfloat16* __restrict__ w, int64_t cols,
+                                     int64_t group, int8_t* q, int64_t q_ld, float* s,
+                                     int64_t s_ld) {
+  const int64_t row = blockIdx.y;
+  const int64_t g = blockIdx.x;
+  const __nv_bfloat16* src = w + row * cols + g * group;
+  __shared__ float red[32];
+  float amax = 0.0f;
+  for (int64_t i = threadIdx.x; i < group; i += blockDim.x)
+    amax = fmaxf(amax, fabsf(__bfloat162float(src[i])));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float sc = __fdiv_rn(red[0], 127.0f);
+  if (threadIdx.x == 0) s[row * s_ld + g] = sc;
+  int8_t* dst = q + row * q_ld + g * group;
+  for (int64_t i = threadIdx.x; i < group; i += blockDim.x) {
+    int8_t v = 0;
+    if (sc != 0.0f) {
+      float r = rintf(__fdiv_rn(__bfloat162float(src[i]), sc));
+      r = fminf(127.0f, fmaxf(-127.0f, r));
+      v = (int8_t)r;
+    }
+    dst[i] = v;
+  }
+}
+
+// Groups of 128: one warp per (row, group), 4 elements per lane.
+__global__ void quantize_g128_kernel(const __nv_bfloat16* __restrict__ w, int64_t rows,
+                                     int64_t cols, int8_t* q, int64_t q_ld, float* s,
+                                     int64_t s_ld) {
+  const int64_t ng = cols / 128;
+  const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (gw >= rows * ng) return;
+  const int64_t row = gw / ng, g = gw % ng;
+  const __nv_bfloat16* src = w + row * cols + g * 128;
+  float v[4];
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[i] = __bfloat162float(src[lane + 32 * i]);
+    amax = fmaxf(amax, fabsf(v[i]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float sc = __fdiv_rn(amax, 127.0f);
+  if (lane == 0) s[row * s_ld + g] = sc;
+  int8_t* dst = q + row * q_ld + g * 128;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    int8_t qq = 0;
+    if (sc != 0.0f) {
+      float r = rintf(__fdiv_rn(v[i], sc));
+      r = fminf(127.0f, fmaxf(-127.0f, r));
+      qq = (int8_t)r;
+    }
+    dst[lane + 32 * i] = qq;
+  }
+}
+
+// x_out[r] = table[offset + codes[r]] for r < rows; an out-of-range code
+// records kErrBounds and yields a zero row.
+__global__ void embed_kernel(const int* __restrict__ codes, const __nv_bfloat16* __restrict__ table,
+                             int n_table, int offset, int H, __nv_bfloat16* x_out, int* err) {
+  const int r = blockIdx.x;
+  pdl_launch_dependents();
+  pdl_wait();
+  const int idx = offset + codes[r];
+  const bool ok = idx >= 0 && idx < n_table;
+  if (!ok && threadIdx.x == 0) record_error(err, kErrBounds);
+  for (int k = threadIdx.x * 8; k < H; k += blockDim.x * 8) {
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (ok) v = *reinterpret_cast<const uint4*>(table + (size_t)idx * H + k);
+    *reinterpret_cast<uint4*>(x_out + (size_t)r * H + k) = v;
+  }
+}
+
+// KV prefill: src bf16 [n_layers][n_pos][Hkv][D] -> pages, converted to the
+// cache type (bf16 copy or f16 round-to-nearest-even).
+__global__ void kv_set_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+                              const unsigned long long* __restrict__ pages, int n_layers,
+                              int max_pages, int page_size, int n_pos, int Hkv, int D, int f16) {
+  const int64_t total = (int64_t)n_layers * n_pos * Hkv * D;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int d = (int)(i % D);
+    const int hh = (int)((i / D) % Hkv);
+    const int p = (int)((i / ((int64_t)D * Hkv)) % n_pos);
+    const int l = (int)(i / ((int64_t)D * Hkv * n_pos));
+    uint16_t* base = reinterpret_cast<uint16_t*>(pages[(size_t)l * max_pages + p / page_size]);
+    const int off = p % page_size;
+    const float kf = __bfloat162float(k[i]), vf = __bfloat162float(v[i]);
+    uint16_t kb, vb;
+    if (f16) {
+      kb = __half_as_ushort(__float2half_rn(kf));
+      vb = __half_as_ushort(__float2half_rn(vf));
+    } else {
+      kb = __bfloat16_as_ushort(k[i]);
+      vb = __bfloat16_as_ushort(v[i]);
+    }
+    base[((size_t)hh * page_size + off) * D + d] = kb;
+    base[((size_t)(Hkv + hh) * page_size + off) * D + d] = vb;
+  }
+}
+
+// KV readback: pages -> raw cache-type bits [n_layers][n_pos][Hkv][D].
+__global__ void kv_get_kernel(uint16_t* k, uint16_t* v, const unsigned long long* __restrict__ pages,
+                              int n_layers, int max_pages, int page_size, int n_pos, int Hkv,
+                              int D) {
+  const int64_t total = (int64_t)n_layers * n_pos * Hkv * D;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int d = (int)(i % D);
+    const int hh = (int)((i / D) % Hkv);
+    const int p = (int)((i / ((int64_t)D * Hkv)) % n_pos);
+    const int l = (int)(i / ((int64_t)D * Hkv * n_pos));
+    const uint16_t* base =
+        reinterpret_cast<const uint16_t*>(pages[(size_t)l * max_pages + p / page_size]);
+    const int off = p % page_size;
+    k[i] = base[((size_t)hh * page_size + off) * D + d];
+    v[i] = base[((size_t)(Hkv + hh) * page_size + off) * D + d];
+  }
+}
+
+}  // namespace m3

@@ -1,0 +1,242 @@
+/*
+ * m3.h -- C ABI of the B200 (sm_100a) per-frame autoregressive decode of
+ * MiniMax Music 3's Qwen3-style 8B "Global LLM" and of its RVQ depth decoder.
+ *
+ * The operation and its sources (page title, section):
+ *  - One frame of the Global LLM: RMSNorm, fused QKV projection, per-head
+ *    q/k RMSNorm and RoPE (theta 1e6), GQA attention over the KV cache,
+ *    O projection + residual, RMSNorm, SwiGLU MLP + residual, over all
+ *    layers; then the final norm, the lm_head restricted to the sampleable
+ *    vocabulary rows, optional classifier-free guidance over (cond, uncond)
+ *    row pairs and a Gumbel-argmax draw.
+ *      "MiniMax-Music3 ... DiffSynth-Studio" (Chinese article), sections
+ *      "各子模型的结构要点" (Qwen3ForCausalLM, vocab 200000, hidden 4096,
+ *      36 layers, 32 heads / 8 KV heads, rope_theta 1e6) and "第二阶段"
+ *      (audio-code vocab mask, guided = uncond + c*(cond - uncond), depth
+ *      codes drawn one codebook at a time, 25 frames/s, 9000-frame cap).
+ *      "MiniMax Music 3 modular pipeline: 2.9x consumer-GPU speedup"
+ *      (diffusers issue), findings 2-4: static graph inputs, lm_head sliced
+ *      to the sampleable rows, Gumbel-argmax instead of softmax+multinomial,
+ *      K variations decoded in lockstep as 2K rows.
+ *  - Precision: bf16 activations rounded where torch rounds; fp32 norms,
+ *    softmax, rope and attention sums; int8 weight-only with one fp32 scale
+ *    per row (body, lm_head) or per group of 128 (depth decoder), quantised
+ *    on the GPU at load.
+ *      "MiniMax Music 3 on Metal" (TensorFold PR), section "Precision is
+ *      the reference's".
+ *  - Bucketed KV growth and an f16 KV cache option.
+ *      "MiniMax Music 3, local" (portfolio page), section "Where the time went".
+ *
+ * Conventions common to every call:
+ *  - Every call returns an m3_status; no exception crosses the ABI.  On a
+ *    non-zero status m3_last_error() returns a thread-local message.
+ *  - Calls are asynchronous on the context's CUDA stream (the stream given
+ *    to m3_create, as a cudaStream_t cast to void*).  Device output buffers
+ *    are written in stream order; the caller keeps them alive until the
+ *    stream has passed them.
+ *  - "dev" pointers are device memory; "host" pointers are host memory;
+ *    a `mem` argument (M3_MEM_HOST / M3_MEM_DEVICE) says which for a source.
+ *  - Weights and KV cache are owned by the library and freed by m3_destroy.
+ *  - Raw bf16 / f16 values are passed as 16-bit patterns (uint16_t).
+ */
+#ifndef M3_H_
+#define M3_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define M3_API __attribute__((visibility("default")))
+#else
+#define M3_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct m3_ctx m3_ctx;
+
+typedef enum {
+  M3_OK = 0,
+  M3_EINVAL = -1,     /* bad argument (null, size, shape, alignment)      */
+  M3_ENOMEM = -2,     /* device or host allocation failed                 */
+  M3_ECUDA = -3,      /* a CUDA runtime call failed                       */
+  M3_ESTATE = -4,     /* call out of order (no weights, no KV cache ...)  */
+  M3_ECAPACITY = -5,  /* a position is outside the KV cache capacity      */
+  M3_ETIMEOUT = -6,   /* a bounded device-side wait gave up               */
+  M3_EDEVICE = -7     /* a kernel recorded an error word on the device    */
+} m3_status;
+
+enum { M3_W_BF16 = 0, M3_W_INT8 = 1 };   /* weight storage of the body + lm_head */
+enum { M3_KV_BF16 = 0, M3_KV_F16 = 1 };  /* KV cache element type               */
+enum { M3_MEM_HOST = 0, M3_MEM_DEVICE = 1 };
+
+/* Model shape.  depth_layers == 0 means no depth decoder. */
+typedef struct {
+  int hidden;          /* H: 4096 for the 8B                                  */
+  int n_layers;        /* 36                                                  */
+  int n_q_heads;       /* 32                                                  */
+  int n_kv_heads;      /* 8 (GQA group n_q_heads / n_kv_heads)                */
+  int head_dim;        /* 128 (64 also supported)                             */
+  int ffn;             /* SwiGLU intermediate, 12288                          */
+  int vocab;           /* full vocabulary, 200000 (informational)             */
+  int slice_start;     /* first sampleable vocab row, e.g. 151675             */
+  int slice_len;       /* number of sampleable rows, e.g. 16384               */
+  double rope_theta;   /* 1e6                                                 */
+  float rms_eps;       /* 1e-6                                                */
+  int max_rows;        /* largest `rows` any call will use, 1..16             */
+  int depth_layers;    /* 4, or 0                                             */
+  int depth_hidden;    /* 1024                                                */
+  int depth_heads;     /* 16 (MHA)                                            */
+  int depth_head_dim;  /* 64                                                  */
+  int depth_ffn;       /* 2816                                                */
+  int depth_codebooks; /* 7 residual codebooks                                */
+  int depth_vocab;     /* 1024 entries per residual codebook                  */
+  double depth_rope_theta;
+} m3_config;
+
+/* One decoder layer's source tensors, bf16, row-major [out, in]. */
+typedef struct {
+  const void* attn_norm; /* [H]                 */
+  const void* wq;        /* [Hq*d, H]           */
+  const void* wk;        /* [Hkv*d, H]          */
+  const void* wv;        /* [Hkv*d, H]          */
+  const void* q_norm;    /* [d]                 */
+  const void* k_norm;    /* [d]                 */
+  const void* wo;        /* [H, Hq*d]           */
+  const void* mlp_norm;  /* [H]                 */
+  const void* wg;        /* [ffn, H]            */
+  const void* wu;        /* [ffn, H]            */
+  const void* wd;        /* [H, ffn]            */
+} m3_layer_src;
+
+/* Body weights.  layers[i] goes to layer first_layer + i, so a caller can
+ * load a model layer by layer.  final_norm [H] and lm_head [slice_len, H]
+ * (rows slice_start.. of the full lm_head) may be null to skip them. */
+typedef struct {
+  int first_layer;
+  int n_layers;
+  const m3_layer_src* layers;
+  const void* final_norm;
+  const void* lm_head;
+  int mem; /* M3_MEM_HOST or M3_MEM_DEVICE for every pointer above */
+} m3_weight_src;
+
+/* Depth-decoder weights, bf16 (quantised to int8, one scale per group of
+ * 128, on the GPU at load).  emb[0] is [slice_len, depth_hidden] (indexed by
+ * the slice-relative semantic code); emb[j], j>=1, and heads[j] are
+ * [depth_vocab, depth_hidden]; proj is [depth_hidden, hidden]. */
+typedef struct {
+  const m3_layer_src* layers; /* depth_layers entries, MHA shapes */
+  const void* proj;
+  const void* const* emb;     /* depth_codebooks tables */
+  const void* final_norm;     /* [depth_hidden] */
+  const void* const* heads;   /* depth_codebooks heads */
+  int mem;
+} m3_depth_src;
+
+/* Create a context bound to the current CUDA device and `cuda_stream`
+ * (cudaStream_t, may be 0 for the legacy default stream).  Allocates only
+ * the small per-frame activation buffers (sized by cfg->max_rows). */
+M3_API int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out);
+
+/* Copy (and, for M3_W_INT8, quantise on the GPU) body weights into
+ * library-owned device memory.  The first call fixes wdtype; the source
+ * may be freed once the call returns (host sources are copied
+ * synchronously; device sources in stream order before the call returns). */
+M3_API int m3_load_weights(m3_ctx* ctx, const m3_weight_src* src, int wdtype);
+
+/* Copy and quantise (int8, one fp32 scale per 128 inputs) the depth decoder. */
+M3_API int m3_load_depth_weights(m3_ctx* ctx, const m3_depth_src* src);
+
+/* Set up the paged KV cache: `rows` independent rows, each with
+ * capacity `max_positions` (<= 9000 for the 8B; any value fits memory).
+ * Pages of `bucket` positions (a multiple of 32; 256 recommended) are
+ * allocated lazily, one bucket for all rows and layers at a time, as frames
+ * reach them -- the cache grows without copying.  kvdtype M3_KV_BF16 or
+ * M3_KV_F16.  Replaces any previous cache. */
+M3_API int m3_kv_alloc(m3_ctx* ctx, int rows, int max_positions, int kvdtype, int bucket);
+
+/* Fill positions [0, n_positions) of `row` (prefill).  k, v: bf16
+ * [n_layers, n_positions, Hkv, d]; stored converted to the cache type
+ * (f16 by round-to-nearest-even).  Values are taken as already rotated. */
+M3_API int m3_kv_set(m3_ctx* ctx, int row, int n_positions, const void* k, const void* v, int mem);
+
+/* Read positions [0, n_positions) of `row` back in the m3_kv_set layout, as
+ * raw cache-type bits (bf16 or f16).  Synchronises the stream. */
+M3_API int m3_kv_get(m3_ctx* ctx, int row, int n_positions, void* k_host, void* v_host);
+
+/* Decode one frame for rows 0..rows-1 (rows <= cache rows and <= max_rows).
+ *  positions (HOST, [rows]): the position each row writes this frame; the
+ *    row attends to positions 0..positions[r] inclusive.  Every position must
+ *    be < max_positions or the call returns M3_ECAPACITY before any launch.
+ *  x_in (dev bf16 [rows, H]): the frame's input embedding per row; copied
+ *    into a library-owned graph-input buffer before the launch.
+ *  cfg_scale > 0: rows are (cond, uncond) pairs (rows must be even); the
+ *    guided logits uncond + cfg_scale*(cond - uncond) are drawn once per pair
+ *    with noise row key = pair index, and both rows receive the code.
+ *    cfg_scale == 0: each row draws from its own logits, row key = row.
+ *  temperature > 0: z_i = g_i / temperature + Gumbel(seed, frame, key, slice_start + i).
+ *  codes (dev int32 [rows]): slice-relative code (0..slice_len-1).
+ *  h_out (dev bf16 [rows, H], nullable): final-normed hidden state.
+ *  logits (dev fp32 [rows, slice_len], nullable): raw per-row logits.
+ * The whole frame runs as one CUDA graph per (rows, KV bucket count),
+ * captured on first use.  May allocate a new KV bucket (synchronising). */
+M3_API int m3_decode_frame(m3_ctx* ctx, int rows, const int32_t* positions, uint64_t seed,
+                    uint64_t frame, const void* x_in, float cfg_scale, float temperature,
+                    int32_t* codes, void* h_out, float* logits);
+
+/* The 7 residual codes of one frame from the depth decoder.
+ *  h_frame (dev bf16 [rows, H]): the frame's final-normed hidden state
+ *    (m3_decode_frame's h_out), projected to depth_hidden at position 0;
+ *  code0 (dev int32 [rows]): the frame's semantic code (slice-relative),
+ *    embedded with emb[0] at position 1;
+ *  position j (1..7) yields codebook j's logits from heads[j-1], drawn with
+ *    noise index (j << 32) | i, and E_j[code_j] is the input of position j+1;
+ *  forced (dev int32 [rows, codebooks], nullable): teacher forcing -- feed
+ *    these codes forward instead of the drawn ones;
+ *  codes (dev int32 [rows, codebooks]); logits (dev fp32
+ *    [rows, codebooks, depth_vocab], nullable).
+ * cfg_scale / temperature as in m3_decode_frame. */
+M3_API int m3_depth_decode(m3_ctx* ctx, int rows, const void* h_frame, const int32_t* code0,
+                    uint64_t seed, uint64_t frame, float cfg_scale, float temperature,
+                    const int32_t* forced, int32_t* codes, float* logits);
+
+/* Frame feedback by table lookup: x_out[r] = table[offset + codes[r]].
+ * table (dev bf16 [n, H]), codes (dev int32 [rows]), x_out (dev bf16 [rows, H]). */
+M3_API int m3_embed(m3_ctx* ctx, int rows, const int32_t* codes, const void* table, int offset,
+             void* x_out);
+
+/* Stateless int8 weight-only quantiser on the GPU.  w (dev bf16 [rows, cols]);
+ * group = cols (one scale per row) or 128 (cols % group == 0);
+ * s = absmax/127 in fp32, q = clamp(rint(w/s), -127, 127), s == 0 -> q = 0.
+ * q (dev int8 [rows, cols]); scales (dev fp32 [rows, cols/group]). */
+M3_API int m3_quantize_int8(const void* w, int64_t rows, int64_t cols, int64_t group, int8_t* q,
+                     float* scales, void* cuda_stream);
+
+/* Export a loaded, possibly quantised weight in its source layout, to host
+ * memory (synchronises).  which: 0 wq 1 wk 2 wv 3 wo 4 wg 5 wu 6 wd 7 lm_head,
+ * 8 + same for the depth decoder's layers, 16 depth proj, 17 + j depth head j.
+ * For int8, q_host gets int8 [rows, cols] and s_host fp32 scales; for bf16
+ * q_host gets the bf16 bits and s_host is ignored. */
+M3_API int m3_export_weight(m3_ctx* ctx, int which, int layer, void* q_host, float* s_host);
+
+/* Algorithmic HBM bytes of one frame: weights read once per frame plus the
+ * KV cache read for `rows` rows at context length ctx (positions 0..ctx). */
+M3_API double m3_frame_bytes(const m3_ctx* ctx, int rows, int ctx_len);
+
+/* Synchronise the stream and return the first error a kernel recorded on
+ * the device (M3_ETIMEOUT / M3_EDEVICE), clearing it, or M3_OK. */
+M3_API int m3_sync_status(m3_ctx* ctx);
+
+/* Thread-local message for the last failing call on this thread. */
+M3_API const char* m3_last_error(void);
+
+M3_API void m3_destroy(m3_ctx* ctx);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* M3_H_ */
