@@ -867,6 +867,72 @@ extern "C" double m3_frame_bytes(const m3_ctx* c, int rows, int ctx_len) {
   return w + kv;
 }
 
+extern "C" int m3_time_gemv(m3_ctx* c, int which, int rows, int iters, float* avg_ms,
+                            double* bytes_per_launch) {
+  if (!c || !avg_ms || !bytes_per_launch) return fail(M3_EINVAL, "null argument");
+  const m3_config& g = c->cfg;
+  if (which < 0 || which > 4 || iters < 1) return fail(M3_EINVAL, "which / iters");
+  if (rows < 1 || rows > g.max_rows) return fail(M3_EINVAL, "rows");
+  for (int l = 0; l < g.n_layers; ++l)
+    if (!c->loaded[l]) return fail(M3_ESTATE, "weights not loaded");
+  if (which == 4 && (!c->head_loaded || !c->final_norm)) return fail(M3_ESTATE, "lm_head not loaded");
+  CKR(enter(c));
+  // a neutral frame block (positions 0, no CFG) for the sampler's reads
+  FrameParams fp{};
+  fp.rows = rows;
+  fp.temperature = 1.0f;
+  set_frame_params_kernel<<<1, 32, 0, c->st>>>(c->fp, fp);
+  CK(cudaGetLastError());
+  cudaEvent_t e0, e1;
+  CK(cudaEventCreate(&e0));
+  CK(cudaEventCreate(&e1));
+  const int H = g.hidden, ld = (g.n_q_heads + 2 * g.n_kv_heads) * g.head_dim;
+  double bytes = 0.0;
+  bool pdl = false;
+  auto one = [&](int l) -> int {
+    const DLayer& L = c->L[l];
+    const DMat* M = nullptr;
+    switch (which) {
+      case 0: M = &L.qkv; CKR(gemv_rows(c, L.qkv, EPI_STORE, rows, c->A.x, H, L.attn_norm, c->A.qkv, ld, nullptr, pdl)); break;
+      case 1: M = &L.o; CKR(gemv_rows(c, L.o, EPI_RESID, rows, c->A.o, g.n_q_heads * g.head_dim, nullptr, c->A.x, H, nullptr, pdl)); break;
+      case 2: M = &L.gu; CKR(gemv_rows(c, L.gu, EPI_SWIGLU, rows, c->A.x, H, L.mlp_norm, c->A.act, g.ffn, nullptr, pdl)); break;
+      case 3: M = &L.d; CKR(gemv_rows(c, L.d, EPI_RESID, rows, c->A.act, g.ffn, nullptr, c->A.x, H, nullptr, pdl)); break;
+      default: {
+        M = &c->lm;
+        SampleArgs sa{};
+        sa.logits = c->logits;
+        sa.logits_ld = g.slice_len;
+        sa.codes = c->codes;
+        sa.code_stride = 1;
+        sa.index_base = (unsigned long long)g.slice_start;
+        sa.part_z = c->spz;
+        sa.part_i = c->spi;
+        sa.counter = c->scnt;
+        sa.h_out = c->h;
+        CKR(gemv_rows(c, c->lm, EPI_SAMPLE, rows, c->A.x, H, c->final_norm, nullptr, 0, &sa, pdl));
+      }
+    }
+    const double esz = M->wf == WF_BF16 ? 2.0 : 1.0;
+    const double nsc = M->wf == WF_I8ROW ? 1.0 : (M->wf == WF_I8G128 ? M->K / 128.0 : 0.0);
+    const double outs = which == 2 ? M->N / 2.0 : (which == 4 ? M->N * 2.0 : M->N);  // fp32 logits
+    bytes = (double)M->N * M->K * esz + 4.0 * M->N * nsc + 2.0 * rows * M->K + 2.0 * rows * outs +
+            (which == 1 || which == 3 ? 2.0 * rows * M->N : 0.0);
+    return M3_OK;
+  };
+  for (int i = 0; i < 3; ++i) CKR(one(i % g.n_layers));  // warm-up
+  CK(cudaEventRecord(e0, c->st));
+  for (int i = 0; i < iters; ++i) CKR(one(i % g.n_layers));
+  CK(cudaEventRecord(e1, c->st));
+  CK(cudaEventSynchronize(e1));
+  float ms = 0.0f;
+  CK(cudaEventElapsedTime(&ms, e0, e1));
+  cudaEventDestroy(e0);
+  cudaEventDestroy(e1);
+  *avg_ms = ms / iters;
+  *bytes_per_launch = bytes;
+  return leave(c);
+}
+
 extern "C" int m3_sync_status(m3_ctx* c) {
   if (!c) return fail(M3_EINVAL, "null ctx");
   CK(cudaSetDevice(c->dev));

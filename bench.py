@@ -1,0 +1,380 @@
+"""Throughput of the per-frame AR decode of the 36-layer 8B Global LLM on B200.
+
+Workload (default): the full 36-layer Qwen3-8B-shaped body (hidden 4096,
+32/8 heads of 128, SwiGLU 12288) + final RMSNorm + lm_head sliced to 16384
+of 200000 vocab rows + CFG 1.5 + Gumbel-argmax at T = 1, bf16 weights drawn
+N(0, 0.02^2) from a seed, bf16 KV cache of a 1500-frame (60 s) song grown
+in 256-frame buckets, 2 rows (one cond/uncond pair).
+
+A step is one frame.  The K timed frames sit at evenly spaced positions of
+the song, (i + 1/2) * 1500 / K, so their mean is the song's mean frame time
+whatever K is; the cache holds seeded N(0, 1) keys/values for earlier
+positions.  Weights (14 GB) are far larger than L2 (126 MB), so no flush is
+needed between frames.
+
+Prints one JSON line (rank 0).  Under torchrun each rank decodes its own
+independent 2-row replica on its GPU (no collective on the data path) and
+the timing is the max over ranks.  `--impl reference` times the CPU oracle
+on a bounded sample of the same frame.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+SONG_FRAMES = 1500
+ROWS = 2
+CFG_SCALE = 1.5
+METRIC = "AR frames/s per row (8B, bf16, 2 rows)"
+WORKLOAD = "qwen3-8b-36L-bf16-2rows-song1500-cfg1.5"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=60)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--wdtype", default="bf16", choices=["bf16", "int8"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--layers", type=int, default=36,
+                   help="body layers (36 = the workload; fewer only for profiling small cases)")
+    return p.parse_args()
+
+
+# ----------------------------------------------------------- distributed ----
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def replica_seed(rank: int) -> int:
+    """Each rank decodes an independent replica (its own seeds): weights are
+    shared in distribution, inputs and noise differ."""
+    return 1000 + rank
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def song_positions(k: int, song: int = SONG_FRAMES):
+    return [min(song - 1, int((i + 0.5) * song / k)) for i in range(k)]
+
+
+# ---------------------------------------------------------------- clocks ----
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int, path: str):
+        self.path = path
+        self.index = index
+        self.proc = None
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        # with one visible GPU nvidia-smi may still list several: keep ours
+        self.multi = vis is None or "," in vis
+        if vis is not None and "," not in vis and vis.strip().isdigit():
+            self.index = int(vis)
+            self.multi = True
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi",
+                                          f"--query-gpu={self.QUERY}", "--format=csv,noheader",
+                                          "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9 or (parts[0] != str(self.index) and len(parts[0]) > 0 and
+                                  self.multi):
+                continue
+            try:
+                sm.append(float(parts[1].split()[0]))
+                smax.append(float(parts[2].split()[0]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ our arm ------
+
+def build_model(torch, m3, synth, seed: int, wdtype: int, layers: int = 36):
+    import dataclasses
+    s = dataclasses.replace(synth.FULL8B, n_layers=layers)
+    cfg = m3.config_from_shapes(s, None, max_rows=ROWS)
+    ctx = m3.m3_create(cfg)
+    for l in range(s.n_layers):  # generate on the GPU, load layer by layer
+        Lw = synth.layer_weights(s, 0, l, device="cuda")
+        m3.m3_load_weights(ctx, [Lw], first_layer=l, wdtype=wdtype)
+        del Lw
+    m3.m3_load_weights(ctx, [], final_norm=synth.final_norm(s, 0, device="cuda"),
+                       lm_head=synth.lm_head_slice(s, 0, device="cuda"), wdtype=wdtype)
+    m3.m3_kv_alloc(ctx, ROWS, SONG_FRAMES, m3.M3_KV_BF16, 256)
+    K, V = synth.kv_prefill(s, ROWS, SONG_FRAMES, seed, device="cuda")
+    for r in range(ROWS):
+        m3.m3_kv_set(ctx, r, K[r], V[r])
+    del K, V
+    torch.cuda.synchronize()
+    return s, ctx
+
+
+def run_ours(args, rank, world, local):
+    import torch
+    from autoregressive_audio_token_b200 import m3
+    import synth
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    seed = replica_seed(rank)
+    wdtype = m3.M3_W_INT8 if args.wdtype == "int8" else m3.M3_W_BF16
+    s, ctx = build_model(torch, m3, synth, seed, wdtype, args.layers)
+    xs = synth.normal((64, ROWS, s.hidden), seed, "bench/x_in", std=0.02, device="cuda")
+    codes = torch.empty(ROWS, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def frame(i, pos):
+        m3.m3_decode_frame(ctx, [pos] * ROWS, seed, i, xs[i % 64], CFG_SCALE, 1.0, codes)
+
+    # capture every bucket's graph before timing, then warm up
+    for b in range(0, SONG_FRAMES, 256):
+        frame(0, b)
+    warm = song_positions(max(args.warmup, 3))
+    for i, p in enumerate(warm):
+        frame(i, p)
+    torch.cuda.synchronize()
+    m3.m3_sync_status(ctx)
+
+    # ---- device-timed region: inputs resident in HBM -----------------------
+    positions = song_positions(args.steps)
+    clocks = ClockSampler(local, f"/tmp/m3_clocks_rank{rank}.csv")
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i, p in enumerate(positions):
+        frame(i, p)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(world)
+    ms = e0.elapsed_time(e1)
+    m3.m3_sync_status(ctx)
+    ms_max = max_over_ranks(ms, world, torch.device("cuda", local))
+    ms_per_step = ms_max / args.steps
+
+    # ---- end to end through the C ABI with host buffers ---------------------
+    x_host = xs[:64].cpu().pin_memory()
+    codes_host = torch.empty((args.steps, ROWS), dtype=torch.int32).pin_memory()
+    x_dev = torch.empty((ROWS, s.hidden), dtype=torch.bfloat16, device="cuda")
+    barrier(world)
+    torch.cuda.synchronize()
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for i, p in enumerate(positions):
+        x_dev.copy_(x_host[i % 64], non_blocking=True)
+        m3.m3_decode_frame(ctx, [p] * ROWS, seed, i, x_dev, CFG_SCALE, 1.0, codes)
+        codes_host[i].copy_(codes, non_blocking=True)
+    e3.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e2.elapsed_time(e3), world, torch.device("cuda", local)) / args.steps
+
+    # ---- the dominant kernel in isolation (gate/up + SwiGLU GEMV) ----------
+    kernels = {}
+    for which, name in [(2, "gate_up_swiglu"), (3, "down"), (0, "qkv"), (1, "o_proj"),
+                        (4, "lm_head_sample")]:
+        kms, kbytes = m3.m3_time_gemv(ctx, which, ROWS, 72 if which != 4 else 20)
+        kernels[name] = {"ms": kms, "bytes": kbytes, "gbs": kbytes / kms / 1e6}
+
+    mean_ctx = sum(positions) / len(positions)
+    frame_bytes = m3.m3_frame_bytes(ctx, ROWS, int(round(mean_ctx)))
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except Exception:
+        pass
+    hbm_peak = peaks.get("hbm_gbs", 6650.0)
+    peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
+    dom = kernels["gate_up_swiglu"]
+    traffic = None
+    try:
+        prof = json.load(open(os.path.join(ROOT, "profiles", "gemv_traffic.json")))
+        src_hash = prof.get("source_sha256")
+        if src_hash == kernel_source_hash():
+            traffic = prof.get("gate_up_swiglu_bytes_per_launch")
+    except Exception:
+        pass
+
+    fps = 1000.0 / ms_per_step * world
+    out = {
+        "metric": METRIC if args.wdtype == "bf16" else METRIC.replace("bf16", "int8"),
+        "value": fps,
+        "unit": "frames/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": args.wdtype,
+        "data": "synthetic (seeded N(0,0.02^2) weights, N(0,1) KV prefill, random-init 8B shape)",
+        "config": {"workload": WORKLOAD if args.wdtype == "bf16" else WORKLOAD.replace("bf16", "int8"),
+                   "rows": ROWS, "song_frames": SONG_FRAMES, "mean_ctx": mean_ctx,
+                   "cfg_scale": CFG_SCALE, "temperature": 1.0, "kv": "bf16 pages of 256",
+                   "l2": "no flush: 14 GB of weights per frame >> 126 MB L2",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "gpu_launches": None,
+        "frame": {"algorithmic_bytes": frame_bytes, "achieved_gbs": frame_bytes / ms_per_step / 1e6,
+                  "frac_of_measured_hbm": frame_bytes / ms_per_step / 1e6 / hbm_peak,
+                  "frac_of_8tbs": frame_bytes / ms_per_step / 1e6 / 8000.0},
+        "roofline": {"bound": "hbm", "kernel": "gemv gate/up + SwiGLU (bf16, 2 rows)",
+                     "achieved": dom["gbs"], "peak": hbm_peak, "unit": "GB/s",
+                     "frac": dom["gbs"] / hbm_peak, "peak_source": peak_src,
+                     "traffic": traffic, "algorithmic_bytes_per_launch": dom["bytes"]},
+        "kernels": kernels,
+        "e2e": {"value": 1000.0 / e2e_ms * world, "unit": "frames/s",
+                "h2d_bytes_per_step": ROWS * s.hidden * 2 + 4 * ROWS,
+                "d2h_bytes_per_step": 4 * ROWS},
+        "clocks": clk,
+    }
+    # kernels per frame: 5 per layer (qkv, attention, o, gate/up, down) + lm_head + params
+    out["gpu_launches"] = (5 * s.n_layers + 1 + 1) * args.steps
+    m3.m3_destroy(ctx)
+    del xs
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(steps=1)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return out
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "autoregressive_audio_token_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        if f.startswith("gemv") or f in ("common.cuh",):
+            h.update(open(os.path.join(d, f), "rb").read())
+    return h.hexdigest()
+
+
+# -------------------------------------------------------- the oracle arm ----
+
+SAMPLE_LAYERS = 2
+
+
+def cpu_baseline(steps: int = 1) -> dict:
+    """The CPU oracle as it stands on this host's cores: a bounded sample of the
+    frame (SAMPLE_LAYERS of the 36 body layers at the song's mean context, plus
+    the final norm + sliced lm_head + CFG + Gumbel-argmax), scaled to a full
+    frame as 36/SAMPLE_LAYERS x body-sample time + head time."""
+    import numpy as np
+    import torch
+    import synth
+    from oracle import oracle as O
+
+    s = synth.FULL8B
+    import dataclasses
+    sub = dataclasses.replace(s, n_layers=SAMPLE_LAYERS)
+    layers = [synth.layer_weights(s, 0, l) for l in range(SAMPLE_LAYERS)]
+    body = O.Body(sub, layers, synth.final_norm(s, 0), synth.lm_head_slice(s, 0))
+    ctx = SONG_FRAMES // 2
+    kc, vc = body.new_cache(ROWS, ctx + 1)
+    K, V = synth.kv_prefill(sub, ROWS, ctx, 7)
+    kc[:, :, :ctx] = O.bits(K)
+    vc[:, :, :ctx] = O.bits(V)
+    x = O.bits(synth.frame_input(s, ROWS, 7, 0))
+    t_body, t_head = [], []
+    for i in range(steps):
+        t0 = time.perf_counter()
+        hx = body.body(kc, vc, [ctx] * ROWS, x)
+        t1 = time.perf_counter()
+        body.sample(hx, 7, i, cfg_scale=CFG_SCALE)
+        t2 = time.perf_counter()
+        t_body.append(t1 - t0)
+        t_head.append(t2 - t1)
+    frame_s = statistics.mean(t_body) * s.n_layers / SAMPLE_LAYERS + statistics.mean(t_head)
+    return {"value": 1.0 / frame_s, "unit": "frames/s", "cores": O.num_threads(),
+            "kind": "oracle", "ms_per_frame": frame_s * 1000.0,
+            "sample": f"{SAMPLE_LAYERS} of 36 layers at ctx {ctx} for 2 rows + lm_head/CFG/draw, "
+                      f"{steps} frame(s); full frame = 36/{SAMPLE_LAYERS} x body + head"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    cb = cpu_baseline(steps=max(1, args.steps if args.steps <= 3 else 3))
+    return {"metric": METRIC, "value": cb["value"], "unit": "frames/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": cb["ms_per_frame"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD, "rows": ROWS, "song_frames": SONG_FRAMES},
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": "frames/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+    else:
+        out = run_ours(args, rank, world, local)
+    if rank == 0 and out is not None:
+        print(json.dumps(out))
+
+
+if __name__ == "__main__":
+    main()

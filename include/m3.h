@@ -226,6 +226,17 @@ M3_API int m3_export_weight(m3_ctx* ctx, int which, int layer, void* q_host, flo
  * KV cache read for `rows` rows at context length ctx (positions 0..ctx). */
 M3_API double m3_frame_bytes(const m3_ctx* ctx, int rows, int ctx_len);
 
+/* Time one kind of the frame's GEMVs in isolation, for roofline accounting:
+ * which = 0 fused QKV, 1 O projection, 2 gate/up + SwiGLU, 3 down, 4 lm_head
+ * + sampler.  Launch i (i < iters) uses layer i % n_layers, so consecutive
+ * launches stream different weights (layers beyond L2); launches follow each
+ * other with programmatic dependent launch as inside a frame.  The region is
+ * bracketed by CUDA events on the context's stream (synchronises).  Writes
+ * the mean milliseconds per launch and the algorithmic bytes per launch
+ * (weights, scales and activations read plus outputs written). */
+M3_API int m3_time_gemv(m3_ctx* ctx, int which, int rows, int iters, float* avg_ms,
+                        double* bytes_per_launch);
+
 /* Synchronise the stream and return the first error a kernel recorded on
  * the device (M3_ETIMEOUT / M3_EDEVICE), clearing it, or M3_OK. */
 M3_API int m3_sync_status(m3_ctx* ctx);
