@@ -300,17 +300,28 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const Attn
   if (w < grp) {
     const int h = g * grp + w;
     const float* pp = a.part + ((size_t)r * a.Hq + h) * S * stride;
-    float M = -INFINITY;
-    for (int s2 = 0; s2 < S; ++s2) M = fmaxf(M, __ldcg(pp + s2 * stride));
-    float L = 0.0f, o[VPL];
+    // lanes hold the splits' (max, sum): S <= 64, two per lane at most
+    const float m0 = lane < S ? __ldcg(pp + lane * stride) : -INFINITY;
+    const float m1 = lane + 32 < S ? __ldcg(pp + (lane + 32) * stride) : -INFINITY;
+    const float l0 = lane < S ? __ldcg(pp + lane * stride + 1) : 0.0f;
+    const float l1 = lane + 32 < S ? __ldcg(pp + (lane + 32) * stride + 1) : 0.0f;
+    float M = fmaxf(m0, m1);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float f0 = m0 == -INFINITY ? 0.0f : expf(m0 - M);
+    const float f1 = m1 == -INFINITY ? 0.0f : expf(m1 - M);
+    float L = l0 * f0 + l1 * f1;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    float o[VPL];
 #pragma unroll
     for (int e = 0; e < VPL; ++e) o[e] = 0.0f;
+#pragma unroll 8
     for (int s2 = 0; s2 < S; ++s2) {
-      const float ms = __ldcg(pp + s2 * stride);
-      const float f = (ms == -INFINITY) ? 0.0f : expf(ms - M);
-      L = fmaf(__ldcg(pp + s2 * stride + 1), f, L);
+      const float f = __shfl_sync(0xffffffffu, s2 < 32 ? f0 : f1, s2 & 31);
+      const float* src = pp + s2 * stride + 2 + VPL * lane;
 #pragma unroll
-      for (int e = 0; e < VPL; ++e) o[e] = fmaf(__ldcg(pp + s2 * stride + 2 + VPL * lane + e), f, o[e]);
+      for (int e = 0; e < VPL; ++e) o[e] = fmaf(__ldcg(src + e), f, o[e]);
     }
     __nv_bfloat16* dst = a.out + (size_t)r * a.Hq * D + (size_t)h * D + VPL * lane;
 #pragma unroll

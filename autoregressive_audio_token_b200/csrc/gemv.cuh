@@ -30,11 +30,23 @@ namespace m3 {
 enum : int { EPI_STORE = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_SAMPLE = 3 };
 enum : int { WF_BF16 = 0, WF_I8ROW = 1, WF_I8G128 = 2 };
 
-constexpr int kConsumers = 256;
-constexpr int kGemvThreads = kConsumers + 32;
-constexpr int kStageBytes = 32768;
-constexpr int kStages = 3;
+constexpr int kConsumers = 256;                  // 8 compute warps
+constexpr int kEpiWarp = kConsumers / 32;        // warp 8: epilogue
+constexpr int kGemvThreads = kConsumers + 64;    // + epilogue warp + producer warp
+constexpr int kPartBufs = 4;                     // partial-sum buffers in flight
+#ifndef M3_STAGE_BYTES
+#define M3_STAGE_BYTES 32768
+#endif
+#ifndef M3_STAGES
+#define M3_STAGES 4
+#endif
+#ifndef M3_PREFETCH_AHEAD
+#define M3_PREFETCH_AHEAD 0
+#endif
+constexpr int kStageBytes = M3_STAGE_BYTES;
+constexpr int kStages = M3_STAGES;
 constexpr int kMaxRows = 16;
+constexpr int kPrefetchAhead = M3_PREFETCH_AHEAD;  // stages prefetched into L2 beyond the ring
 
 // Per-frame scalars, written once per frame by set_frame_params before the
 // frame's first kernel.
@@ -96,28 +108,63 @@ template <int MR, int TPR, int ESZ>
 __host__ __device__ constexpr size_t gemv_smem_bytes(int rows_cta_max) {
   using S = GemvShape<TPR, ESZ>;
   return (size_t)kStages * kStageBytes + 2 * kStages * sizeof(uint64_t) +
-         sizeof(float) * (2 * S::SLOTS * S::P * MR + 9 * MR + (size_t)rows_cta_max * MR) +
+         sizeof(float) * (kPartBufs * S::SLOTS * S::P * MR + 9 * MR + (size_t)rows_cta_max * MR) +
          (sizeof(float) + sizeof(int)) * S::R * MR + 64;
 }
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
 
+// Reduce V values (one per row-in-stage x batch row) over the 32 lanes of a
+// warp as a reduce-scatter: after the call lane l holds in v[0] the warp
+// total of value index l >> (5 - log2 V).  V - 1 + (5 - log2 V) shuffles
+// instead of 5 V.
+template <int V>
+__device__ __forceinline__ void warp_reduce_scatter(float* v, int lane) {
+  static_assert(V >= 1 && V <= 32 && (V & (V - 1)) == 0, "V must be a power of two <= 32");
+  int n = V;
+#pragma unroll
+  for (int half = 16; half >= 1; half >>= 1) {
+    if (n > 1) {
+      const bool up = (lane & half) != 0;
+      const int h = n / 2;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        if (i < h) {
+          const float send = up ? v[i] : v[i + h];
+          const float keep = up ? v[i + h] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, half);
+        }
+      }
+      n = h;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], half);
+    }
+  }
+}
+
 template <int MR, int WF, int EPI, int TPR>
-__global__ void __launch_bounds__(kGemvThreads, MR <= 2 ? 2 : 1) gemv_kernel(const GemvArgs a) {
+__global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvArgs a) {
   constexpr int ESZ = WF == WF_BF16 ? 2 : 1;
   using S = GemvShape<TPR, ESZ>;
   constexpr int KC = S::KC, G = S::G, R = S::R, P = S::P, W = S::W, SLOTS = S::SLOTS;
   constexpr int UNIT = EPI == EPI_SWIGLU ? 2 : 1;
+  constexpr int V = P * MR;  // partial sums per thread per stage
+  constexpr int LV = V == 1 ? 0 : V == 2 ? 1 : V == 4 ? 2 : V == 8 ? 3 : V == 16 ? 4 : 5;
+  constexpr bool kScatter = (W == 32) && (V <= 32);
+  // named barriers: 1 norm (compute warps); 2.. partial buffer full; 2+kPartBufs.. empty
+  constexpr int kBarNorm = 1, kBarFull = 2, kBarEmpty = 2 + kPartBufs;
+  constexpr int kPartThreads = kConsumers + 32;  // compute warps + epilogue warp
 
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* ring = smem;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
   uint64_t* empty = full + kStages;
-  float* part = reinterpret_cast<float*>(empty + kStages);  // [2][SLOTS][P][MR]
-  float* nrm = part + 2 * SLOTS * P * MR;                    // [8][MR] + [MR]
+  float* part = reinterpret_cast<float*>(empty + kStages);  // [kPartBufs][SLOTS][V]
+  float* nrm = part + kPartBufs * SLOTS * V;                 // [8][MR] + [MR]
   float* accr = nrm + 9 * MR;                                 // [rows_cta][MR]
 
   const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
   const int K = a.K;
   const int nkc = (K + KC - 1) / KC;
   const int U = a.N / UNIT;
@@ -127,6 +174,8 @@ __global__ void __launch_bounds__(kGemvThreads, MR <= 2 ? 2 : 1) gemv_kernel(con
   const int nrows = r_end - r_begin;
   const int spk = (nrows + R - 1) / R;
   const int nstages = spk * nkc;
+  float* sbz = accr + (size_t)spk * R * MR;            // sampler: best z per role
+  int* sbi = reinterpret_cast<int*>(sbz + R * MR);      // sampler: its index
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -135,34 +184,217 @@ __global__ void __launch_bounds__(kGemvThreads, MR <= 2 ? 2 : 1) gemv_kernel(con
     }
     fence_barrier_init();
   }
+  if constexpr (EPI == EPI_SAMPLE) {
+    for (int c = tid; c < R * MR; c += blockDim.x) {
+      sbz[c] = -INFINITY;
+      sbi[c] = 0x7fffffff;
+    }
+  }
   __syncthreads();
   pdl_launch_dependents();
 
   // ------------------------------------------------------------ producer --
-  if (tid >= kConsumers) {
-    if (tid == kConsumers) {
+  if (warp == kEpiWarp + 1) {
+    if (lane == 0) {
       const uint64_t pol = policy_evict_first();
       const uint8_t* wb = static_cast<const uint8_t*>(a.w);
+      auto seg = [&](int s, int& rs, int& re, int& kc, uint32_t& segb) {
+        kc = s / spk;
+        const int sr = s % spk;
+        rs = r_begin + sr * R;
+        re = min(rs + R, r_end);
+        segb = (uint32_t)(min(KC, K - kc * KC) * ESZ);
+      };
+      auto prefetch = [&](int s) {
+        int rs, re, kc;
+        uint32_t segb;
+        seg(s, rs, re, kc, segb);
+        for (int r = rs; r < re; ++r)
+          bulk_prefetch_l2(wb + ((size_t)r * K + (size_t)kc * KC) * ESZ, segb);
+      };
+      constexpr int PFD = kStages + kPrefetchAhead;
+      if (kPrefetchAhead > 0)
+        for (int s = kStages; s < min(PFD, nstages); ++s) prefetch(s);
       for (int s = 0; s < nstages; ++s) {
         const int slot = s % kStages;
         if (s >= kStages && !mbar_wait(&empty[slot], ((s / kStages) - 1) & 1, a.err)) break;
-        const int kc = s / spk, sr = s % spk;
-        const int rs = r_begin + sr * R, re = min(rs + R, r_end);
-        const int kel = min(KC, K - kc * KC);
-        const uint32_t segb = (uint32_t)(kel * ESZ);
+        int rs, re, kc;
+        uint32_t segb;
+        seg(s, rs, re, kc, segb);
         mbar_arrive_expect_tx(&full[slot], segb * (uint32_t)(re - rs));
         uint8_t* dst = ring + slot * kStageBytes;
         for (int r = rs; r < re; ++r)
           bulk_g2s(dst + (size_t)(r - rs) * KC * ESZ,
                    wb + ((size_t)r * K + (size_t)kc * KC) * ESZ, segb, &full[slot], pol);
+        if (kPrefetchAhead > 0 && s + PFD < nstages) prefetch(s + PFD);
       }
     }
     return;
   }
 
-  // ------------------------------------------------------------ consumers --
+  // ------------------------------------------------------------ epilogue --
+  // Sums the partials of each stage and applies the epilogue; the compute
+  // warps never wait on its global-memory round trips (kPartBufs stages of
+  // slack).
+  if (warp == kEpiWarp) {
+    pdl_wait();  // residual / outputs are shared with the previous kernel
+    const int mr = a.mr;
+    const int np = (EPI == EPI_SAMPLE) ? (a.fp->cfg_on ? mr / 2 : mr) : 0;
+    int s = 0;
+    for (int kc = 0; kc < nkc; ++kc) {
+      const bool last_kc = (kc == nkc - 1);
+      for (int sr = 0; sr < spk; ++sr, ++s) {
+        const int b = s % kPartBufs;
+        named_bar_sync(kBarFull + b, kPartThreads);
+        const float* pb = part + b * SLOTS * V;
+        const int rs = r_begin + sr * R;
+        const int nr = min(R, r_end - rs);
+        auto row_sum = [&](int rl, int m) -> float {
+          const int gg = rl % G, pp = rl / G;
+          constexpr int SPG = TPR / W;  // slots per row group
+          float y = 0.0f;
+#pragma unroll
+          for (int q = 0; q < SPG; ++q) y += pb[(gg * SPG + q) * V + pp * MR + m];
+          return y;
+        };
+        if constexpr (EPI == EPI_STORE || EPI == EPI_RESID) {
+          for (int c = lane; c < R * MR; c += 32) {
+            const int rl = c / MR, m = c % MR;
+            if (rl >= nr || m >= mr) continue;
+            float y = row_sum(rl, m);
+            if (nkc > 1) {
+              float* ar = accr + (size_t)(sr * R + rl) * MR + m;
+              if (kc > 0) y += *ar;
+              if (!last_kc) {
+                *ar = y;
+                continue;
+              }
+            }
+            const int n = rs + rl;
+            if constexpr (WF == WF_I8ROW) y *= __ldg(a.scales + n);
+            __nv_bfloat16* o = a.out + (size_t)m * a.ldo + n;
+            if constexpr (EPI == EPI_STORE) {
+              *o = __float2bfloat16_rn(y);
+            } else {
+              *o = __float2bfloat16_rn(__bfloat162float(*o) + round_bf16(y));
+            }
+          }
+        } else if constexpr (EPI == EPI_SWIGLU) {
+          for (int c = lane; c < (R / 2) * MR; c += 32) {
+            const int j = c / MR, m = c % MR;
+            if (2 * j >= nr || m >= mr) continue;
+            float yg = row_sum(2 * j, m), yu = row_sum(2 * j + 1, m);
+            if (nkc > 1) {
+              float* ag = accr + (size_t)(sr * R + 2 * j) * MR + m;
+              float* au = accr + (size_t)(sr * R + 2 * j + 1) * MR + m;
+              if (kc > 0) {
+                yg += *ag;
+                yu += *au;
+              }
+              if (!last_kc) {
+                *ag = yg;
+                *au = yu;
+                continue;
+              }
+            }
+            const int n = rs + 2 * j;
+            if constexpr (WF == WF_I8ROW) {
+              yg *= __ldg(a.scales + n);
+              yu *= __ldg(a.scales + n + 1);
+            }
+            const float gb = round_bf16(yg), ub = round_bf16(yu);
+            const float act = round_bf16(round_bf16(silu_f(gb)) * ub);
+            a.out[(size_t)m * a.ldo + n / 2] = __float2bfloat16_rn(act);
+          }
+        } else {  // EPI_SAMPLE (K fits one segment): roles (row-in-stage, key)
+          const bool cfg = a.fp->cfg_on != 0;
+          for (int c = lane; c < R * MR; c += 32) {
+            const int rl = c / MR, p = c % MR;
+            if (rl >= nr || p >= np) continue;
+            const int n = rs + rl;
+            const int m0 = cfg ? 2 * p : p;
+            float y0 = row_sum(rl, m0);
+            float y1 = cfg ? row_sum(rl, m0 + 1) : 0.0f;
+            if constexpr (WF == WF_I8ROW) {
+              const float sc = __ldg(a.scales + n);
+              y0 *= sc;
+              y1 *= sc;
+            }
+            if (a.smp.logits) {
+              a.smp.logits[(size_t)(a.row0 + m0) * a.smp.logits_ld + n] = y0;
+              if (cfg) a.smp.logits[(size_t)(a.row0 + m0 + 1) * a.smp.logits_ld + n] = y1;
+            }
+            float gl = y0;
+            if (cfg) gl = __fadd_rn(y1, __fmul_rn(a.fp->cfg_scale, __fsub_rn(y0, y1)));
+            const unsigned long long key = cfg ? (unsigned long long)(a.row0 / 2 + p)
+                                               : (unsigned long long)(a.row0 + p);
+            const float gn = gumbel_noise(a.fp->seed, a.fp->frame, key,
+                                          a.smp.index_base + (unsigned long long)n);
+            const float z = __fadd_rn(__fdiv_rn(gl, a.fp->temperature), gn);
+            if (z > sbz[c] || (z == sbz[c] && n < sbi[c])) {
+              sbz[c] = z;
+              sbi[c] = n;
+            }
+          }
+        }
+        if (s + kPartBufs < nstages) named_bar_arrive(kBarEmpty + b, kPartThreads);
+      }
+    }
+    if constexpr (EPI == EPI_SAMPLE) {
+      // CTA-level argmax per key, then the last CTA reduces over CTAs.
+      __syncwarp();
+      int last = 0;
+      if (lane < np) {
+        float bz = -INFINITY;
+        int bi = 0x7fffffff;
+        for (int rl = 0; rl < R; ++rl) {
+          const float z = sbz[rl * MR + lane];
+          const int i = sbi[rl * MR + lane];
+          if (z > bz || (z == bz && i < bi)) {
+            bz = z;
+            bi = i;
+          }
+        }
+        a.smp.part_z[blockIdx.x * kMaxRows + lane] = bz;
+        a.smp.part_i[blockIdx.x * kMaxRows + lane] = bi;
+        __threadfence();
+      }
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence();
+        const unsigned old = atomicAdd(a.smp.counter, 1u);
+        last = (old == gridDim.x - 1);
+      }
+      last = __shfl_sync(0xffffffffu, last, 0);
+      if (!last) return;
+      __threadfence();
+      if (lane < np) {
+        float bz = -INFINITY;
+        int bi = 0x7fffffff;
+        for (int bb = 0; bb < (int)gridDim.x; ++bb) {
+          const float z = __ldcg(a.smp.part_z + bb * kMaxRows + lane);
+          const int i = __ldcg(a.smp.part_i + bb * kMaxRows + lane);
+          if (z > bz || (z == bz && i < bi)) {
+            bz = z;
+            bi = i;
+          }
+        }
+        const bool cfg = a.fp->cfg_on != 0;
+        const int nm = cfg ? 2 : 1;
+        for (int q = 0; q < nm; ++q) {
+          const int r = a.row0 + (cfg ? 2 * lane + q : lane);
+          a.smp.codes[(size_t)r * a.smp.code_stride] = bi;
+          if (a.smp.prev)
+            a.smp.prev[r] = a.smp.forced ? a.smp.forced[(size_t)r * a.smp.forced_stride] : bi;
+        }
+      }
+      if (lane == 0) *a.smp.counter = 0u;
+    }
+    return;
+  }
+
+  // ------------------------------------------------------- compute warps --
   const int g = tid / TPR, t = tid % TPR;
-  const int lane = tid & 31, warp = tid >> 5;
   const int mr = a.mr;
   const __nv_bfloat16* __restrict__ x = a.x;
 
@@ -190,7 +422,7 @@ __global__ void __launch_bounds__(kGemvThreads, MR <= 2 ? 2 : 1) gemv_kernel(con
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
       if (lane == 0) nrm[warp * MR + m] = v;
     }
-    named_bar_sync(1, kConsumers);
+    named_bar_sync(kBarNorm, kConsumers);
 #pragma unroll
     for (int m = 0; m < MR; ++m) {
       float tot = 0.0f;
@@ -224,41 +456,33 @@ __global__ void __launch_bounds__(kGemvThreads, MR <= 2 ? 2 : 1) gemv_kernel(con
     }
   };
 
-  // sampler state: this thread's role (row-in-stage, key) is fixed
-  constexpr int NPMAX = MR;
-  float best_z = -INFINITY;
-  int best_i = 0x7fffffff;
-  const int np = (EPI == EPI_SAMPLE) ? (a.fp->cfg_on ? mr / 2 : mr) : 0;
-
-  int s = 0, buf = 0;
+  int s = 0;
   for (int kc = 0; kc < nkc; ++kc) {
     load_x(kc);
     const int kel = min(KC, K - kc * KC);
     for (int sr = 0; sr < spk; ++sr, ++s) {
       const int slot = s % kStages;
       // On a timeout the error word is set and the stage is consumed as is, so
-      // that every consumer still reaches the same named barriers.
+      // that every thread still reaches the same barriers.
       mbar_wait(&full[slot], (s / kStages) & 1, a.err);
       const int rs = r_begin + sr * R;
       const int nr = min(R, r_end - rs);
       const uint8_t* st = ring + slot * kStageBytes;
-      float acc[P][MR];
+      float acc[V];
 #pragma unroll
-      for (int p = 0; p < P; ++p)
-#pragma unroll
-        for (int m = 0; m < MR; ++m) acc[p][m] = 0.0f;
+      for (int i = 0; i < V; ++i) acc[i] = 0.0f;
 
 #pragma unroll
       for (int p = 0; p < P; ++p) {
         const int rl = p * G + g;
         if (rl < nr) {
-          const uint8_t* seg = st + (size_t)rl * KC * ESZ;
+          const uint8_t* sg = st + (size_t)rl * KC * ESZ;
           if constexpr (ESZ == 2) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               const int c = t + h * TPR;  // 16-byte chunk index in the segment
               if (8 * c < kel) {
-                const uint4 wv = *reinterpret_cast<const uint4*>(seg + 16 * c);
+                const uint4 wv = *reinterpret_cast<const uint4*>(sg + 16 * c);
                 const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
@@ -266,19 +490,19 @@ __global__ void __launch_bounds__(kGemvThreads, MR <= 2 ? 2 : 1) gemv_kernel(con
                   bf16x2_to_f32(ww[j], lo, hi);
 #pragma unroll
                   for (int m = 0; m < MR; ++m) {
-                    acc[p][m] = fmaf(lo, xr[m][8 * h + 2 * j], acc[p][m]);
-                    acc[p][m] = fmaf(hi, xr[m][8 * h + 2 * j + 1], acc[p][m]);
+                    acc[p * MR + m] = fmaf(lo, xr[m][8 * h + 2 * j], acc[p * MR + m]);
+                    acc[p * MR + m] = fmaf(hi, xr[m][8 * h + 2 * j + 1], acc[p * MR + m]);
                   }
                 }
               }
             }
           } else {
             if (16 * t < kel) {
-              const uint4 wv = *reinterpret_cast<const uint4*>(seg + 16 * t);
+              const uint4 wv = *reinterpret_cast<const uint4*>(sg + 16 * t);
               const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
-              float part_m[MR];
+              float pm[MR];
 #pragma unroll
-              for (int m = 0; m < MR; ++m) part_m[m] = 0.0f;
+              for (int m = 0; m < MR; ++m) pm[m] = 0.0f;
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
                 float f[4];
@@ -286,17 +510,17 @@ __global__ void __launch_bounds__(kGemvThreads, MR <= 2 ? 2 : 1) gemv_kernel(con
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
 #pragma unroll
-                  for (int m = 0; m < MR; ++m) part_m[m] = fmaf(f[q], xr[m][4 * j + q], part_m[m]);
+                  for (int m = 0; m < MR; ++m) pm[m] = fmaf(f[q], xr[m][4 * j + q], pm[m]);
               }
               if constexpr (WF == WF_I8G128) {
                 const int n = rs + rl;
                 const int kabs = kc * KC + 16 * t;
                 const float sc = __ldg(a.scales + (size_t)n * (K / 128) + kabs / 128);
 #pragma unroll
-                for (int m = 0; m < MR; ++m) acc[p][m] = fmaf(sc, part_m[m], acc[p][m]);
+                for (int m = 0; m < MR; ++m) acc[p * MR + m] = fmaf(sc, pm[m], acc[p * MR + m]);
               } else {
 #pragma unroll
-                for (int m = 0; m < MR; ++m) acc[p][m] += part_m[m];
+                for (int m = 0; m < MR; ++m) acc[p * MR + m] += pm[m];
               }
             }
           }
@@ -306,186 +530,29 @@ __global__ void __launch_bounds__(kGemvThreads, MR <= 2 ? 2 : 1) gemv_kernel(con
       if (lane == 0) mbar_arrive(&empty[slot]);
 
       // reduce over the TPR threads of each row: shuffles, then partial slots
+      const int b = s % kPartBufs;
+      float* pb = part + b * SLOTS * V;
+      if constexpr (kScatter) {
+        warp_reduce_scatter<V>(acc, lane);
+      } else {
 #pragma unroll
-      for (int p = 0; p < P; ++p)
-#pragma unroll
-        for (int m = 0; m < MR; ++m) {
-          float v = acc[p][m];
+        for (int i = 0; i < V; ++i) {
+          float v = acc[i];
 #pragma unroll
           for (int o = W / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o, W);
-          acc[p][m] = v;
+          acc[i] = v;
         }
-      float* pb = part + buf * SLOTS * P * MR;
-      if ((tid % W) == 0) {
-        const int sl = tid / W;
+      }
+      if (s >= kPartBufs) named_bar_sync(kBarEmpty + b, kPartThreads);
+      if constexpr (kScatter) {
+        if ((lane & ((32 >> LV) - 1)) == 0) pb[warp * V + (lane >> (5 - LV))] = acc[0];
+      } else {
+        if ((tid % W) == 0) {
 #pragma unroll
-        for (int p = 0; p < P; ++p)
-#pragma unroll
-          for (int m = 0; m < MR; ++m) pb[(sl * P + p) * MR + m] = acc[p][m];
-      }
-      named_bar_sync(1, kConsumers);
-
-      // full sum of (row-in-stage rl, batch row m) for this stage
-      auto row_sum = [&](int rl, int m) -> float {
-        const int gg = rl % G, pp = rl / G;
-        constexpr int SPG = TPR / W;  // slots per row group
-        float y = 0.0f;
-#pragma unroll
-        for (int q = 0; q < SPG; ++q) y += pb[((gg * SPG + q) * P + pp) * MR + m];
-        return y;
-      };
-      const bool last_kc = (kc == nkc - 1);
-
-      if constexpr (EPI == EPI_STORE || EPI == EPI_RESID) {
-        for (int c = tid; c < R * MR; c += kConsumers) {
-          const int rl = c / MR, m = c % MR;
-          if (rl >= nr || m >= mr) continue;
-          float y = row_sum(rl, m);
-          if (nkc > 1) {
-            float* ar = accr + (size_t)(sr * R + rl) * MR + m;
-            if (kc > 0) y += *ar;
-            if (!last_kc) {
-              *ar = y;
-              continue;
-            }
-          }
-          const int n = rs + rl;
-          if constexpr (WF == WF_I8ROW) y *= __ldg(a.scales + n);
-          __nv_bfloat16* o = a.out + (size_t)m * a.ldo + n;
-          if constexpr (EPI == EPI_STORE) {
-            *o = __float2bfloat16_rn(y);
-          } else {
-            *o = __float2bfloat16_rn(__bfloat162float(*o) + round_bf16(y));
-          }
-        }
-      } else if constexpr (EPI == EPI_SWIGLU) {
-        for (int c = tid; c < (R / 2) * MR; c += kConsumers) {
-          const int j = c / MR, m = c % MR;
-          if (2 * j >= nr || m >= mr) continue;
-          float yg = row_sum(2 * j, m), yu = row_sum(2 * j + 1, m);
-          if (nkc > 1) {
-            float* ag = accr + (size_t)(sr * R + 2 * j) * MR + m;
-            float* au = accr + (size_t)(sr * R + 2 * j + 1) * MR + m;
-            if (kc > 0) {
-              yg += *ag;
-              yu += *au;
-            }
-            if (!last_kc) {
-              *ag = yg;
-              *au = yu;
-              continue;
-            }
-          }
-          const int n = rs + 2 * j;
-          if constexpr (WF == WF_I8ROW) {
-            yg *= __ldg(a.scales + n);
-            yu *= __ldg(a.scales + n + 1);
-          }
-          const float gb = round_bf16(yg), ub = round_bf16(yu);
-          const float act = round_bf16(round_bf16(silu_f(gb)) * ub);
-          a.out[(size_t)m * a.ldo + n / 2] = __float2bfloat16_rn(act);
-        }
-      } else {  // EPI_SAMPLE: one role per thread
-        const int c = tid;
-        const int rl = c / NPMAX, p = c % NPMAX;
-        if (rl < nr && p < np && (nkc == 1 || last_kc)) {
-          const int n = rs + rl;
-          const bool cfg = a.fp->cfg_on != 0;
-          const int m0 = cfg ? 2 * p : p;
-          float y0 = row_sum(rl, m0);
-          float y1 = cfg ? row_sum(rl, m0 + 1) : 0.0f;
-          if (nkc > 1) {
-            y0 += accr[(size_t)(sr * R + rl) * MR + m0];
-            if (cfg) y1 += accr[(size_t)(sr * R + rl) * MR + m0 + 1];
-          }
-          if constexpr (WF == WF_I8ROW) {
-            const float sc = __ldg(a.scales + n);
-            y0 *= sc;
-            y1 *= sc;
-          }
-          if (a.smp.logits) {
-            a.smp.logits[(size_t)(a.row0 + m0) * a.smp.logits_ld + n] = y0;
-            if (cfg) a.smp.logits[(size_t)(a.row0 + m0 + 1) * a.smp.logits_ld + n] = y1;
-          }
-          float gl = y0;
-          if (cfg) gl = __fadd_rn(y1, __fmul_rn(a.fp->cfg_scale, __fsub_rn(y0, y1)));
-          const unsigned long long key = cfg ? (unsigned long long)(a.row0 / 2 + p)
-                                             : (unsigned long long)(a.row0 + p);
-          const float gn = gumbel_noise(a.fp->seed, a.fp->frame, key,
-                                        a.smp.index_base + (unsigned long long)n);
-          const float z = __fadd_rn(__fdiv_rn(gl, a.fp->temperature), gn);
-          if (z > best_z || (z == best_z && n < best_i)) {
-            best_z = z;
-            best_i = n;
-          }
-        } else if (nkc > 1 && !last_kc && rl < nr && p < np) {
-          // accumulate the K-chunk partials of the rows this role reads
-          const bool cfg = a.fp->cfg_on != 0;
-          const int m0 = cfg ? 2 * p : p;
-          float* a0 = accr + (size_t)(sr * R + rl) * MR + m0;
-          *a0 = (kc > 0 ? *a0 : 0.0f) + row_sum(rl, m0);
-          if (cfg) a0[1] = (kc > 0 ? a0[1] : 0.0f) + row_sum(rl, m0 + 1);
+          for (int i = 0; i < V; ++i) pb[(tid / W) * V + i] = acc[i];
         }
       }
-      buf ^= 1;
-    }
-  }
-
-  if constexpr (EPI == EPI_SAMPLE) {
-    // CTA-level argmax per key, then the last CTA reduces over CTAs.
-    float* sz = accr + (size_t)spk * R * MR;
-    int* si = reinterpret_cast<int*>(sz + R * MR);
-    __shared__ int s_last;
-    if (tid < R * NPMAX) {
-      sz[tid] = best_z;
-      si[tid] = best_i;
-    }
-    named_bar_sync(1, kConsumers);
-    if (tid < np) {
-      float bz = -INFINITY;
-      int bi = 0x7fffffff;
-      for (int rl = 0; rl < R; ++rl) {
-        const float z = sz[rl * NPMAX + tid];
-        const int i = si[rl * NPMAX + tid];
-        if (z > bz || (z == bz && i < bi)) {
-          bz = z;
-          bi = i;
-        }
-      }
-      a.smp.part_z[blockIdx.x * kMaxRows + tid] = bz;
-      a.smp.part_i[blockIdx.x * kMaxRows + tid] = bi;
-      __threadfence();
-    }
-    named_bar_sync(1, kConsumers);
-    if (tid == 0) {
-      __threadfence();
-      const unsigned old = atomicAdd(a.smp.counter, 1u);
-      s_last = (old == gridDim.x - 1);
-    }
-    named_bar_sync(1, kConsumers);
-    if (s_last) {
-      __threadfence();
-      if (tid < np) {
-        float bz = -INFINITY;
-        int bi = 0x7fffffff;
-        for (int b = 0; b < (int)gridDim.x; ++b) {
-          const float z = __ldcg(a.smp.part_z + b * kMaxRows + tid);
-          const int i = __ldcg(a.smp.part_i + b * kMaxRows + tid);
-          if (z > bz || (z == bz && i < bi)) {
-            bz = z;
-            bi = i;
-          }
-        }
-        const bool cfg = a.fp->cfg_on != 0;
-        const int nm = cfg ? 2 : 1;
-        for (int q = 0; q < nm; ++q) {
-          const int r = a.row0 + (cfg ? 2 * tid + q : tid);
-          a.smp.codes[(size_t)r * a.smp.code_stride] = bi;
-          if (a.smp.prev)
-            a.smp.prev[r] = a.smp.forced ? a.smp.forced[(size_t)r * a.smp.forced_stride] : bi;
-        }
-      }
-      if (tid == 0) *a.smp.counter = 0u;
+      named_bar_arrive(kBarFull + b, kPartThreads);
     }
   }
 }

@@ -12,7 +12,7 @@ cudaError_t launch_gemv_t(const GemvArgs& a, cudaStream_t st, bool pdl, int nsm)
   constexpr int ESZ = WF == WF_BF16 ? 2 : 1;
   using S = GemvShape<TPR, ESZ>;
   constexpr int UNIT = EPI == EPI_SWIGLU ? 2 : 1;
-  if (EPI == EPI_SAMPLE && S::R * MR > kConsumers) return cudaErrorInvalidValue;
+  if (EPI == EPI_SAMPLE && a.K > S::KC) return cudaErrorInvalidValue;  // one segment per row
   const int units = a.N / UNIT;
   const int grid = units < nsm ? units : nsm;
   const int per = (units + grid - 1) / grid * UNIT;
