@@ -8,6 +8,7 @@
 #include <cstdio>
 #include <cstring>
 #include <map>
+#include <mutex>
 #include <string>
 #include <tuple>
 #include <vector>
@@ -946,4 +947,95 @@ extern "C" int m3_sync_status(m3_ctx* c) {
     return fail(M3_EDEVICE, "a kernel recorded an out-of-range index");
   }
   return M3_OK;
+}
+
+// ------------------------------------------- allocation-free sampler -------
+// Scratch of m3_sample_noalloc: the frame-parameter block, the cross-CTA
+// argmax ticket and the per-CTA partial argmaxes live in this file-scope
+// device array instead of context-owned buffers.  Every GPU that loads the
+// library holds it (about 129 KB) until the process exits.
+namespace {
+constexpr int kNoAllocMaxCtas = 1024;
+constexpr size_t kNoAllocParamsOff = 0;
+constexpr size_t kNoAllocCounterOff = 256;
+constexpr size_t kNoAllocPartZOff = 512;
+constexpr size_t kNoAllocPartIOff = kNoAllocPartZOff + sizeof(float) * kNoAllocMaxCtas * kMaxRows;
+constexpr size_t kNoAllocBytes = kNoAllocPartIOff + sizeof(int) * kNoAllocMaxCtas * kMaxRows;
+static_assert(sizeof(FrameParams) <= 256, "frame params fit their slot");
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+// Device address of g_noalloc_scratch per device, looked up once per device
+// (the host-side name of the array is not a device address).
+static std::mutex g_noalloc_mu;
+static void* g_noalloc_ptr[64] = {};
+
+static int noalloc_scratch(int dev, unsigned char** out) {
+  if (dev < 0 || dev >= 64) return fail(M3_EINVAL, "device index beyond 63");
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess)
+      return fail(M3_ECUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = static_cast<unsigned char*>(g_noalloc_ptr[dev]);
+  return M3_OK;
+}
+
+extern "C" int m3_sample_noalloc(m3_ctx* c, int rows, const void* h, uint64_t seed,
+                                 uint64_t frame, float cfg_scale, float temperature,
+                                 int32_t* codes, float* logits) {
+  if (!c || !h || !codes) return fail(M3_EINVAL, "null argument");
+  const m3_config& g = c->cfg;
+  if (!c->head_loaded) return fail(M3_ESTATE, "lm_head not loaded");
+  if (rows < 1 || rows > kMaxRows || rows > g.max_rows)
+    return fail(M3_EINVAL, "rows must be in 1..min(16, max_rows)");
+  if (!(cfg_scale >= 0.0f) || !(temperature > 0.0f)) return fail(M3_EINVAL, "cfg_scale / temperature");
+  if (cfg_scale > 0.0f && rows % 2) return fail(M3_EINVAL, "cfg_scale > 0 needs (cond, uncond) row pairs");
+  const int grid = g.slice_len < c->nsm ? g.slice_len : c->nsm;
+  if (grid > kNoAllocMaxCtas) return fail(M3_EINVAL, "more CTAs than the static scratch holds");
+  CK(cudaSetDevice(c->dev));
+  unsigned char* scratch = nullptr;
+  CKR(noalloc_scratch(c->dev, &scratch));
+  CKR(enter(c));
+  FrameParams fp{};
+  fp.rows = rows;
+  fp.cfg_on = cfg_scale > 0.0f;
+  fp.cfg_scale = cfg_scale;
+  fp.temperature = temperature;
+  fp.seed = seed;
+  fp.frame = frame;
+  FrameParams* dfp = reinterpret_cast<FrameParams*>(scratch + kNoAllocParamsOff);
+  unsigned* counter = reinterpret_cast<unsigned*>(scratch + kNoAllocCounterOff);
+  set_frame_params_kernel<<<1, 32, 0, c->st>>>(dfp, fp);
+  CK(cudaGetLastError());
+  CK(cudaMemsetAsync(counter, 0, sizeof(unsigned), c->st));  // the ticket starts at zero
+  for (int r0 = 0; r0 < rows; r0 += 4) {
+    GemvArgs a{};
+    a.w = c->lm.w;
+    a.scales = c->lm.s;
+    a.N = c->lm.N;
+    a.K = c->lm.K;
+    a.row0 = r0;
+    a.mr = rows - r0 < 4 ? rows - r0 : 4;
+    a.x = static_cast<const bf16*>(h) + (size_t)r0 * g.hidden;
+    a.ldx = g.hidden;
+    a.gamma = nullptr;  // h is already the final-normed hidden state
+    a.eps = g.rms_eps;
+    a.fp = dfp;
+    a.smp.logits = logits;
+    a.smp.logits_ld = g.slice_len;
+    a.smp.codes = codes;
+    a.smp.code_stride = 1;
+    a.smp.index_base = (unsigned long long)g.slice_start;
+    a.smp.part_z = reinterpret_cast<float*>(scratch + kNoAllocPartZOff);
+    a.smp.part_i = reinterpret_cast<int*>(scratch + kNoAllocPartIOff);
+    a.smp.counter = counter;
+    a.err = c->err;
+    CK(launch_gemv(a, c->lm.wf, EPI_SAMPLE, c->st, false, c->nsm));
+  }
+  return leave(c);
 }

@@ -24,7 +24,8 @@ M3_MEM_HOST, M3_MEM_DEVICE = 0, 1
 
 EXPORTED = ("m3_create", "m3_load_weights", "m3_load_depth_weights", "m3_kv_alloc", "m3_kv_set",
             "m3_kv_get", "m3_decode_frame", "m3_depth_decode", "m3_embed", "m3_quantize_int8",
-            "m3_export_weight", "m3_frame_bytes", "m3_time_gemv", "m3_sync_status",
+            "m3_export_weight", "m3_frame_bytes", "m3_time_gemv", "m3_sample_noalloc",
+            "m3_sync_status",
             "m3_last_error", "m3_destroy")
 
 
@@ -85,6 +86,7 @@ def load_library() -> C.CDLL:
     L.m3_frame_bytes.argtypes = [vp, i32, i32]
     L.m3_frame_bytes.restype = C.c_double
     L.m3_time_gemv.argtypes = [vp, i32, i32, i32, C.POINTER(C.c_float), C.POINTER(C.c_double)]
+    L.m3_sample_noalloc.argtypes = [vp, i32, vp, u64, u64, f32, f32, vp, vp]
     L.m3_sync_status.argtypes = [vp]
     L.m3_last_error.restype = C.c_char_p
     L.m3_destroy.argtypes = [vp]
@@ -244,6 +246,14 @@ def m3_time_gemv(ctx: int, which: int, rows: int, iters: int):
     b = C.c_double()
     _check(lib.m3_time_gemv(ctx, which, rows, iters, C.byref(ms), C.byref(b)))
     return ms.value, b.value
+
+
+def m3_sample_noalloc(ctx: int, h: torch.Tensor, seed: int, frame: int, cfg_scale: float,
+                      temperature: float, codes: torch.Tensor,
+                      logits: torch.Tensor | None = None) -> None:
+    """The allocation-free draw on a final-normed hidden state (see m3.h)."""
+    _check(lib.m3_sample_noalloc(ctx, h.shape[0], _ptr(h), seed, frame, cfg_scale, temperature,
+                                 _ptr(codes), _ptr(logits)))
 
 
 def m3_sync_status(ctx: int) -> None:

@@ -237,6 +237,25 @@ M3_API double m3_frame_bytes(const m3_ctx* ctx, int rows, int ctx_len);
 M3_API int m3_time_gemv(m3_ctx* ctx, int which, int rows, int iters, float* avg_ms,
                         double* bytes_per_launch);
 
+/* The lm_head + CFG + Gumbel-argmax draw of m3_decode_frame on a given
+ * final-normed hidden state, for callers that must not allocate GPU memory
+ * on the decode thread (a real-time audio callback, a host thread that runs
+ * while a CUDA graph is being captured elsewhere, an embedder whose memory
+ * is budgeted up front): it calls no cudaMalloc / cudaFree and no
+ * allocating library routine.  The pages have no counterpart of this call.
+ *  h (dev bf16 [rows, H]): final-normed hidden state (m3_decode_frame's h_out);
+ *  rows <= 16 and <= max_rows, else M3_EINVAL; seed, frame, cfg_scale,
+ *  temperature, codes, logits as in m3_decode_frame (logits nullable).
+ * Its scratch (parameter block, argmax partials, ticket; about 129 KB) is a
+ * file-scope __device__ array that every GPU loading the library holds
+ * until exit.  The first call on a device looks up that array's device
+ * address, so make the first call before any stream capture.  All calls
+ * share the array and keep the last call's contents (the ticket is cleared
+ * by each call): calls that overlap on the GPU -- on different streams or
+ * contexts of one device -- race and must be ordered by the caller. */
+M3_API int m3_sample_noalloc(m3_ctx* ctx, int rows, const void* h, uint64_t seed, uint64_t frame,
+                             float cfg_scale, float temperature, int32_t* codes, float* logits);
+
 /* Synchronise the stream and return the first error a kernel recorded on
  * the device (M3_ETIMEOUT / M3_EDEVICE), clearing it, or M3_OK. */
 M3_API int m3_sync_status(m3_ctx* ctx);
