@@ -10,7 +10,22 @@ static cudaError_t launch_attn_t(const AttnArgs& a, int splits, int rows, cudaSt
   auto kern = attn_decode_kernel<D, KVF16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_ex(kern, dim3(splits, a.Hkv, rows), dim3(kAttnWarps * 32), smem, st, pdl, a);
+  if (splits < 1 || splits > kAttnMaxSplits) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(splits, a.Hkv, rows);
+  cfg.blockDim = dim3(kAttnWarps * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = splits;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 cudaError_t launch_attn(const AttnArgs& a, int D, int kv_f16, int splits, int rows,

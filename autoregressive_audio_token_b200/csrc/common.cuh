@@ -147,4 +147,14 @@ __device__ __forceinline__ void s8x4_to_f32(uint32_t w, float* f) {
   f[3] = __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7653)) - bias;
 }
 
+// Element offset of (head slot hs, page-local position off, dim d) in a KV
+// page laid out [2 * Hkv head slots][page_size][D]: the 16-byte chunk index
+// of d is XOR-ed with (off & 7), so that eight consecutive positions' chunk c
+// fall in eight different shared-memory bank groups once a tile is copied
+// linearly into shared memory (conflict-free ldmatrix).
+__host__ __device__ __forceinline__ size_t kv_elem_offset(int hs, int page_size, int off, int D,
+                                                         int d) {
+  return ((size_t)hs * page_size + off) * D + ((((d >> 3) ^ (off & 7))) << 3) + (d & 7);
+}
+
 }  // namespace m3

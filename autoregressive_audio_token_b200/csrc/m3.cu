@@ -56,8 +56,6 @@ struct DLayer {
 
 struct Acts {  // activation buffers of one stack (body or depth)
   bf16 *x = nullptr, *qkv = nullptr, *o = nullptr, *act = nullptr;
-  float* apart = nullptr;
-  unsigned* acnt = nullptr;
 };
 
 struct m3_ctx {
@@ -105,7 +103,7 @@ struct m3_ctx {
   unsigned* scnt = nullptr;
   FrameParams* fp = nullptr;
   int* err = nullptr;
-  int max_splits = 64;
+  int max_splits = kAttnMaxSplits;
   // depth buffers
   bf16* dh = nullptr;
   int* dcodes = nullptr;
@@ -166,16 +164,11 @@ static double* make_inv_freq(m3_ctx* c, int d, double theta, int* rc) {
   return p;
 }
 
-static int alloc_acts(m3_ctx* c, Acts& A, int rows, int H, int Hq, int Hkv, int d, int ffn,
-                      int splits) {
+static int alloc_acts(m3_ctx* c, Acts& A, int rows, int H, int Hq, int Hkv, int d, int ffn) {
   CKR(dalloc(c, &A.x, sizeof(bf16) * rows * H));
   CKR(dalloc(c, &A.qkv, sizeof(bf16) * rows * (Hq + 2 * Hkv) * d));
   CKR(dalloc(c, &A.o, sizeof(bf16) * rows * Hq * d));
   CKR(dalloc(c, &A.act, sizeof(bf16) * rows * ffn));
-  CKR(dalloc(c, &A.apart, sizeof(float) * rows * Hq * splits * (d + 2)));
-  void* cnt = nullptr;
-  CKR(dzalloc(c, &cnt, sizeof(unsigned) * rows * Hkv));
-  A.acnt = static_cast<unsigned*>(cnt);
   return M3_OK;
 }
 
@@ -226,8 +219,7 @@ extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) 
   int rc = M3_OK;
   c->inv_freq = make_inv_freq(c, g.head_dim, g.rope_theta, &rc);
   if (rc) return bail(rc);
-  if ((rc = alloc_acts(c, c->A, R, g.hidden, g.n_q_heads, g.n_kv_heads, g.head_dim, g.ffn,
-                       c->max_splits)))
+  if ((rc = alloc_acts(c, c->A, R, g.hidden, g.n_q_heads, g.n_kv_heads, g.head_dim, g.ffn)))
     return bail(rc);
   void* p = nullptr;
   if ((rc = dalloc(c, &c->h, sizeof(bf16) * R * g.hidden)) ||
@@ -248,7 +240,7 @@ extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) 
     c->dinv_freq = make_inv_freq(c, g.depth_head_dim, g.depth_rope_theta, &rc);
     if (rc) return bail(rc);
     if ((rc = alloc_acts(c, c->DA, R, Dh, g.depth_heads, g.depth_heads, g.depth_head_dim,
-                         g.depth_ffn, 1)) ||
+                         g.depth_ffn)) ||
         (rc = dalloc(c, &c->dh, sizeof(bf16) * R * g.hidden)) ||
         (rc = dalloc(c, &c->dcodes, sizeof(int) * R * NC)) ||
         (rc = dalloc(c, &c->dprev, sizeof(int) * R)) ||
@@ -671,8 +663,6 @@ static int record_layer(m3_ctx* c, const DLayer& L, Acts& A, int rows, int H, in
   at.page_size = page_size;
   at.Hq = Hq;
   at.Hkv = Hkv;
-  at.part = A.apart;
-  at.counters = A.acnt;
   at.out = A.o;
   at.fp = c->fp;
   at.fixed_pos = fixed_pos;

@@ -107,8 +107,9 @@ __global__ void embed_kernel(const int* __restrict__ codes, const __nv_bfloat16*
   }
 }
 
-// KV prefill: src bf16 [n_layers][n_pos][Hkv][D] -> pages, converted to the
-// cache type (bf16 copy or f16 round-to-nearest-even).
+// KV prefill: src bf16 [n_layers][n_pos][Hkv][D] -> pages (chunk-swizzled,
+// see kv_elem_offset), converted to the cache type (bf16 copy or f16
+// round-to-nearest-even).
 __global__ void kv_set_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                               const unsigned long long* __restrict__ pages, int n_layers,
                               int max_pages, int page_size, int n_pos, int Hkv, int D, int f16) {
@@ -130,8 +131,8 @@ __global__ void kv_set_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bf
       kb = __bfloat16_as_ushort(k[i]);
       vb = __bfloat16_as_ushort(v[i]);
     }
-    base[((size_t)hh * page_size + off) * D + d] = kb;
-    base[((size_t)(Hkv + hh) * page_size + off) * D + d] = vb;
+    base[kv_elem_offset(hh, page_size, off, D, d)] = kb;
+    base[kv_elem_offset(Hkv + hh, page_size, off, D, d)] = vb;
   }
 }
 
@@ -149,8 +150,8 @@ __global__ void kv_get_kernel(uint16_t* k, uint16_t* v, const unsigned long long
     const uint16_t* base =
         reinterpret_cast<const uint16_t*>(pages[(size_t)l * max_pages + p / page_size]);
     const int off = p % page_size;
-    k[i] = base[((size_t)hh * page_size + off) * D + d];
-    v[i] = base[((size_t)(Hkv + hh) * page_size + off) * D + d];
+    k[i] = base[kv_elem_offset(hh, page_size, off, D, d)];
+    v[i] = base[kv_elem_offset(Hkv + hh, page_size, off, D, d)];
   }
 }
 

@@ -82,6 +82,24 @@ def test_tiny_rows_and_cfg(ora, rows, cfg):
         m.close()
 
 
+@pytest.mark.parametrize("kv_f16", [False, True])
+def test_tiny_long_context_many_tiles(ora, kv_f16):
+    # positions up to 700 with bucket 256: several 32-position tiles per warp,
+    # splits crossing page boundaries, partial last tiles
+    s = synth.TINY
+    m = Model(s, seed=8, kv_f16=kv_f16, max_rows=2)
+    try:
+        kc, vc = m.kv_setup(rows=2, n_prefill=650, max_pos=768)
+        x = synth.frame_input(s, 2, 8, 0)
+        for f, pos in enumerate([[650, 651], [700, 37], [767, 255]]):
+            codes, h, lg = m.decode(pos, 3, f, x)
+            oc, oh, olg = m.ora.decode_frame(kc, vc, pos, 3, f, bits(x))
+            assert rel_err(lg, olg) <= TOL[0], (pos, rel_err(lg, olg))
+            check_codes_teacher_forced(m, h, codes, 3, f)
+    finally:
+        m.close()
+
+
 def test_kv_written_matches_oracle(ora):
     s = synth.TINY
     m = Model(s, seed=2, kv_f16=False)
@@ -162,10 +180,11 @@ def test_errors_are_status_codes(ora):
 
 # -------------------------------------------------- one 8B decoder layer ----
 
-@pytest.mark.parametrize("wdtype,rows", [(0, 1), (0, 2), (1, 1), (1, 2)])
-def test_layer8b_vs_oracle(ora, wdtype, rows):
+@pytest.mark.parametrize("wdtype,rows,kv_f16", [(0, 1, False), (0, 2, False), (1, 1, False),
+                                                (1, 2, True)])
+def test_layer8b_vs_oracle(ora, wdtype, rows, kv_f16):
     s = synth.LAYER8B
-    m = Model(s, seed=11, device="cuda", wdtype=wdtype, max_rows=2)
+    m = Model(s, seed=11, device="cuda", wdtype=wdtype, max_rows=2, kv_f16=kv_f16)
     try:
         kc, vc = m.kv_setup(rows=rows, n_prefill=1024, max_pos=1100)
         x = synth.frame_input(s, rows, 11, 0)
