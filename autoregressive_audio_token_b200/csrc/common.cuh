@@ -147,6 +147,45 @@ __device__ __forceinline__ void s8x4_to_f32(uint32_t w, float* f) {
   f[3] = __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7653)) - bias;
 }
 
+// ------------------------------------------- packed fp32 pairs (sm_100a) ---
+// Two fp32 values in one 64-bit register pair, for the packed f32x2 FMA/ADD
+// of sm_100 (one instruction for two lanes of arithmetic).
+__device__ __forceinline__ uint64_t pack_u32x2(uint32_t lo, uint32_t hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  return pack_u32x2(__float_as_uint(lo), __float_as_uint(hi));
+}
+
+__device__ __forceinline__ float2 unpack_f32x2(uint64_t v) {
+  uint32_t lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(v));
+  return make_float2(__uint_as_float(lo), __uint_as_float(hi));
+}
+
+// acc = a * b + acc, elementwise on (lo, hi), each with one rounding.
+__device__ __forceinline__ void ffma2(uint64_t& acc, uint64_t a, uint64_t b) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
+}
+
+__device__ __forceinline__ void fadd2(uint64_t& acc, uint64_t b) {
+  asm("add.rn.f32x2 %0, %0, %1;" : "+l"(acc) : "l"(b));
+}
+
+// Four int8 packed in w -> two exact fp32 pairs (q0, q1), (q2, q3), via the
+// 2^23 magic: float(0x4B000000 | (b ^ 0x80)) = 2^23 + 128 + q.
+__device__ __forceinline__ void s8x4_to_f32x2(uint32_t w, uint64_t& f01, uint64_t& f23) {
+  const uint32_t x = w ^ 0x80808080u;
+  const uint64_t nb = pack_f32x2(-8388736.0f, -8388736.0f);  // -(2^23 + 128)
+  f01 = pack_u32x2(__byte_perm(x, 0x4B000000u, 0x7650), __byte_perm(x, 0x4B000000u, 0x7651));
+  f23 = pack_u32x2(__byte_perm(x, 0x4B000000u, 0x7652), __byte_perm(x, 0x4B000000u, 0x7653));
+  fadd2(f01, nb);
+  fadd2(f23, nb);
+}
+
 // Element offset of (head slot hs, page-local position off, dim d) in a KV
 // page laid out [2 * Hkv head slots][page_size][D]: the 16-byte chunk index
 // of d is XOR-ed with (off & 7), so that eight consecutive positions' chunk c

@@ -35,10 +35,10 @@ constexpr int kEpiWarp = kConsumers / 32;        // warp 8: epilogue
 constexpr int kGemvThreads = kConsumers + 64;    // + epilogue warp + producer warp
 constexpr int kPartBufs = 4;                     // partial-sum buffers in flight
 #ifndef M3_STAGE_BYTES
-#define M3_STAGE_BYTES 32768
+#define M3_STAGE_BYTES 65536
 #endif
 #ifndef M3_STAGES
-#define M3_STAGES 4
+#define M3_STAGES 3
 #endif
 #ifndef M3_PREFETCH_AHEAD
 #define M3_PREFETCH_AHEAD 0
@@ -432,8 +432,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvArgs a)
     }
   }
 
-  // x in registers: this thread's 16 K positions of the current chunk.
-  float xr[MR][16];
+  // x in registers: this thread's 16 K positions of the current chunk, as 8
+  // packed fp32 pairs (even, odd) for the packed FMA.
+  uint64_t xr2[MR][8];
   auto elem_k = [&](int kc, int e) -> int {
     if (ESZ == 2) return kc * KC + (e < 8 ? 8 * t + e : 8 * (t + TPR) + (e - 8));
     return kc * KC + 16 * t + e;
@@ -441,18 +442,24 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvArgs a)
   auto load_x = [&](int kc) {
     const bool write_h = (EPI == EPI_SAMPLE) && a.smp.h_out && blockIdx.x == 0 && g == 0;
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const int k = elem_k(kc, e);
-      const bool ok = k < K;
-      const float gm = (a.gamma && ok) ? __bfloat162float(a.gamma[k]) : 1.0f;
+    for (int e2 = 0; e2 < 8; ++e2) {
+      float vv[MR][2];
 #pragma unroll
-      for (int m = 0; m < MR; ++m) {
-        float v = (ok && m < mr) ? __bfloat162float(x[(size_t)m * a.ldx + k]) : 0.0f;
-        if (a.gamma) v = round_bf16(gm * round_bf16(v * inv[m]));
-        xr[m][e] = v;
-        if (write_h && ok && m < mr)
-          a.smp.h_out[(size_t)(a.row0 + m) * K + k] = __float2bfloat16_rn(v);
+      for (int q = 0; q < 2; ++q) {
+        const int k = elem_k(kc, 2 * e2 + q);
+        const bool ok = k < K;
+        const float gm = (a.gamma && ok) ? __bfloat162float(a.gamma[k]) : 1.0f;
+#pragma unroll
+        for (int m = 0; m < MR; ++m) {
+          float v = (ok && m < mr) ? __bfloat162float(x[(size_t)m * a.ldx + k]) : 0.0f;
+          if (a.gamma) v = round_bf16(gm * round_bf16(v * inv[m]));
+          vv[m][q] = v;
+          if (write_h && ok && m < mr)
+            a.smp.h_out[(size_t)(a.row0 + m) * K + k] = __float2bfloat16_rn(v);
+        }
       }
+#pragma unroll
+      for (int m = 0; m < MR; ++m) xr2[m][e2] = pack_f32x2(vv[m][0], vv[m][1]);
     }
   };
 
@@ -468,9 +475,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvArgs a)
       const int rs = r_begin + sr * R;
       const int nr = min(R, r_end - rs);
       const uint8_t* st = ring + slot * kStageBytes;
-      float acc[V];
+      // packed (even, odd) partial sums per (row-in-pass, batch row)
+      uint64_t acc2[V];
 #pragma unroll
-      for (int i = 0; i < V; ++i) acc[i] = 0.0f;
+      for (int i = 0; i < V; ++i) acc2[i] = 0ull;
 
 #pragma unroll
       for (int p = 0; p < P; ++p) {
@@ -486,13 +494,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvArgs a)
                 const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                  float lo, hi;
-                  bf16x2_to_f32(ww[j], lo, hi);
+                  // (bf16 lo, bf16 hi) -> exact fp32 pair
+                  const uint64_t wp = pack_u32x2(ww[j] << 16, ww[j] & 0xFFFF0000u);
 #pragma unroll
-                  for (int m = 0; m < MR; ++m) {
-                    acc[p * MR + m] = fmaf(lo, xr[m][8 * h + 2 * j], acc[p * MR + m]);
-                    acc[p * MR + m] = fmaf(hi, xr[m][8 * h + 2 * j + 1], acc[p * MR + m]);
-                  }
+                  for (int m = 0; m < MR; ++m) ffma2(acc2[p * MR + m], wp, xr2[m][4 * h + j]);
                 }
               }
             }
@@ -500,31 +505,39 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvArgs a)
             if (16 * t < kel) {
               const uint4 wv = *reinterpret_cast<const uint4*>(sg + 16 * t);
               const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
-              float pm[MR];
+              uint64_t pm2[MR];
 #pragma unroll
-              for (int m = 0; m < MR; ++m) pm[m] = 0.0f;
+              for (int m = 0; m < MR; ++m) pm2[m] = 0ull;
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
-                float f[4];
-                s8x4_to_f32(ww[j], f);
+                uint64_t f01, f23;
+                s8x4_to_f32x2(ww[j], f01, f23);
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-#pragma unroll
-                  for (int m = 0; m < MR; ++m) pm[m] = fmaf(f[q], xr[m][4 * j + q], pm[m]);
+                for (int m = 0; m < MR; ++m) {
+                  ffma2(pm2[m], f01, xr2[m][2 * j]);
+                  ffma2(pm2[m], f23, xr2[m][2 * j + 1]);
+                }
               }
               if constexpr (WF == WF_I8G128) {
                 const int n = rs + rl;
                 const int kabs = kc * KC + 16 * t;
                 const float sc = __ldg(a.scales + (size_t)n * (K / 128) + kabs / 128);
+                const uint64_t sc2 = pack_f32x2(sc, sc);
 #pragma unroll
-                for (int m = 0; m < MR; ++m) acc[p * MR + m] = fmaf(sc, pm[m], acc[p * MR + m]);
+                for (int m = 0; m < MR; ++m) ffma2(acc2[p * MR + m], sc2, pm2[m]);
               } else {
 #pragma unroll
-                for (int m = 0; m < MR; ++m) acc[p * MR + m] += pm[m];
+                for (int m = 0; m < MR; ++m) fadd2(acc2[p * MR + m], pm2[m]);
               }
             }
           }
         }
+      }
+      float acc[V];
+#pragma unroll
+      for (int i = 0; i < V; ++i) {
+        const float2 f = unpack_f32x2(acc2[i]);
+        acc[i] = f.x + f.y;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
