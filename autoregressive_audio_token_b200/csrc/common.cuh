@@ -61,8 +61,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait for phase `parity` of `bar` to complete; false (and an error word)
 // if it does not within the spin limit.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
-  for (long long i = 0; i < kSpinLimit; ++i)
+  for (long long i = 0; i < kSpinLimit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
+    // once any wait of the launch has given up, give up at once too, so a
+    // failure ends the kernel in one spin limit rather than one per stage
+    if ((i & 1023) == 1023 && err && *reinterpret_cast<volatile int*>(err) != 0) return false;
+  }
   record_error(err, kErrTimeout);
   return false;
 }

@@ -53,3 +53,12 @@ cudaError_t launch_attn(const AttnArgs& a, int D, int kv_f16, int splits, int ro
                         cudaStream_t st, bool pdl);
 
 }  // namespace m3
+
+namespace m3 {
+struct FrameArgs;
+// Persistent whole-frame kernel (frame.cuh): cooperative launch of `grid`
+// CTAs (one per SM).
+cudaError_t launch_frame(const FrameArgs& a, int wf, int kv_f16, int rows_cta_max, int grid,
+                         cudaStream_t st);
+size_t frame_smem(int mr, int wf, int rows_cta_max);
+}  // namespace m3

@@ -16,6 +16,7 @@
 #include "m3.h"
 #include "launch.cuh"
 #include "misc.cuh"
+#include "frame.cuh"
 
 using namespace m3;
 typedef __nv_bfloat16 bf16;
@@ -115,6 +116,15 @@ struct m3_ctx {
 
   std::map<std::pair<int, int>, cudaGraphExec_t> graphs;
   std::map<std::pair<int, int>, cudaGraphExec_t> dgraphs;
+
+  // persistent whole-frame kernel (frame.cuh)
+  bool use_frame_kernel = false;  // opt in with M3_FRAME_KERNEL=1
+  bool phases_dirty = true;
+  FramePhase* d_phases = nullptr;
+  int nph = 0;
+  unsigned* d_bar = nullptr;
+  float* fapart = nullptr;
+  unsigned* facnt = nullptr;
 };
 
 template <typename T>
@@ -208,6 +218,7 @@ extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) 
   if (cudaDeviceGetAttribute(&c->nsm, cudaDevAttrMultiProcessorCount, c->dev) != cudaSuccess)
     return bail(fail(M3_ECUDA, "SM count"));
   if (const char* e = getenv("M3_NO_GRAPH")) c->use_graphs = (e[0] == '0');
+  if (const char* e = getenv("M3_FRAME_KERNEL")) c->use_frame_kernel = (e[0] == '1');
   if (cudaStreamCreateWithFlags(&c->st, cudaStreamNonBlocking) != cudaSuccess ||
       cudaEventCreateWithFlags(&c->ev_in, cudaEventDisableTiming) != cudaSuccess ||
       cudaEventCreateWithFlags(&c->ev_out, cudaEventDisableTiming) != cudaSuccess)
@@ -384,12 +395,14 @@ extern "C" int m3_load_weights(m3_ctx* c, const m3_weight_src* src, int wdtype) 
     CKR(load_layer(c, c->L[l], src->layers[i], src->mem, wf, g.hidden, g.n_q_heads, g.n_kv_heads,
                    g.head_dim, g.ffn));
     c->loaded[l] = 1;
+    c->phases_dirty = true;
   }
   if (src->final_norm) CKR(put_vec(c, &c->final_norm, src->final_norm, g.hidden, src->mem));
   if (src->lm_head) {
     if (!c->lm.w) CKR(alloc_mat(c, c->lm, g.slice_len, g.hidden, wf));
     CKR(put_rows(c, c->lm, src->lm_head, src->mem, g.slice_len, 0, 1));
     c->head_loaded = true;
+    c->phases_dirty = true;
   }
   CK(cudaStreamSynchronize(c->st));  // sources may be freed on return
   return leave(c);
@@ -722,6 +735,128 @@ static int run_graph(m3_ctx* c, std::map<std::pair<int, int>, cudaGraphExec_t>& 
   return M3_OK;
 }
 
+// ------------------------------------------ the persistent frame kernel -----
+// Used for up to 4 rows when every GEMV of the body streams 4096-wide
+// segments (K > 1024) and heads are 128 wide -- the 8B shapes; other shapes
+// take the per-kernel graph above; the frame kernel is opt-in (M3_FRAME_KERNEL=1)
+// until it beats that graph.
+static bool frame_kernel_ok(const m3_ctx* c, int rows) {
+  const m3_config& g = c->cfg;
+  return c->use_frame_kernel && rows <= 4 && g.head_dim == 128 && gemv_tpr(g.hidden) == 256 &&
+         gemv_tpr(g.n_q_heads * g.head_dim) == 256 && gemv_tpr(g.ffn) == 256 &&
+         c->nsm <= 1024;
+}
+
+static int frame_rows_cta_max(const m3_ctx* c) {
+  const m3_config& g = c->cfg;
+  const int esz = c->wdtype == M3_W_INT8 ? 1 : 2;
+  const int R = kStageBytes / (4096 * esz);
+  const int Ns[5] = {(g.n_q_heads + 2 * g.n_kv_heads) * g.head_dim, g.hidden, 2 * g.ffn, g.hidden,
+                     g.slice_len};
+  int best = 0;
+  for (int i = 0; i < 5; ++i) {
+    const int unit = i == 2 ? 2 : 1;
+    const int U = Ns[i] / unit;
+    const int per = (U + c->nsm - 1) / c->nsm * unit;
+    const int rm = (per + R - 1) / R * R;
+    best = rm > best ? rm : best;
+  }
+  return best;
+}
+
+static int build_frame_phases(m3_ctx* c) {
+  const m3_config& g = c->cfg;
+  const int H = g.hidden, d = g.head_dim;
+  const int ldqkv = (g.n_q_heads + 2 * g.n_kv_heads) * d;
+  std::vector<FramePhase> ph;
+  auto gemv_phase = [&](int kind, int layer, const DMat& M, const bf16* x, int ldx,
+                        const bf16* gamma, bf16* out, int ldo) {
+    FramePhase p{};
+    p.kind = kind;
+    p.layer = layer;
+    p.w = M.w;
+    p.scales = M.s;
+    p.N = M.N;
+    p.K = M.K;
+    p.x = x;
+    p.ldx = ldx;
+    p.gamma = gamma;
+    p.out = out;
+    p.ldo = ldo;
+    ph.push_back(p);
+  };
+  for (int l = 0; l < g.n_layers; ++l) {
+    const DLayer& L = c->L[l];
+    gemv_phase(PH_QKV, l, L.qkv, c->A.x, H, L.attn_norm, c->A.qkv, ldqkv);
+    FramePhase at{};
+    at.kind = PH_ATT;
+    at.layer = l;
+    at.q_norm = L.q_norm;
+    at.k_norm = L.k_norm;
+    ph.push_back(at);
+    gemv_phase(PH_O, l, L.o, c->A.o, g.n_q_heads * d, nullptr, c->A.x, H);
+    gemv_phase(PH_GU, l, L.gu, c->A.x, H, L.mlp_norm, c->A.act, g.ffn);
+    gemv_phase(PH_D, l, L.d, c->A.act, g.ffn, nullptr, c->A.x, H);
+  }
+  gemv_phase(PH_LM, g.n_layers, c->lm, c->A.x, H, c->final_norm, nullptr, 0);
+  if (!c->d_phases || c->nph != (int)ph.size()) {
+    CKR(dalloc(c, &c->d_phases, sizeof(FramePhase) * ph.size()));
+    CKR(dalloc(c, &c->d_bar, sizeof(unsigned) * ph.size()));
+  }
+  if (!c->fapart) {
+    CKR(dalloc(c, &c->fapart, sizeof(float) * g.max_rows * g.n_q_heads * 16 * (d + 2)));
+    void* p = nullptr;
+    CKR(dzalloc(c, &p, sizeof(unsigned) * g.max_rows * g.n_kv_heads));
+    c->facnt = static_cast<unsigned*>(p);
+  }
+  c->nph = (int)ph.size();
+  CK(cudaMemcpyAsync(c->d_phases, ph.data(), sizeof(FramePhase) * ph.size(),
+                     cudaMemcpyHostToDevice, c->st));
+  CK(cudaStreamSynchronize(c->st));
+  c->phases_dirty = false;
+  return M3_OK;
+}
+
+static int run_frame_kernel(m3_ctx* c, int rows) {
+  const m3_config& g = c->cfg;
+  if (c->phases_dirty) CKR(build_frame_phases(c));
+  FrameArgs a{};
+  a.ph = c->d_phases;
+  a.nph = c->nph;
+  a.mr = rows;
+  a.eps = g.rms_eps;
+  a.fp = c->fp;
+  a.qkv = c->A.qkv;
+  a.ldqkv = (g.n_q_heads + 2 * g.n_kv_heads) * g.head_dim;
+  a.inv_freq = c->inv_freq;
+  a.pages = c->d_pages;
+  a.n_layers = g.n_layers;
+  a.max_pages = c->max_pages;
+  a.page_size = c->bucket;
+  a.Hq = g.n_q_heads;
+  a.Hkv = g.n_kv_heads;
+  int splits = c->nsm / (rows * g.n_kv_heads);
+  a.splits = splits < 1 ? 1 : (splits > 16 ? 16 : splits);
+  a.apart = c->fapart;
+  a.acnt = c->facnt;
+  a.att_out = c->A.o;
+  a.smp.logits = c->logits;
+  a.smp.logits_ld = g.slice_len;
+  a.smp.codes = c->codes;
+  a.smp.code_stride = 1;
+  a.smp.index_base = (unsigned long long)g.slice_start;
+  a.smp.part_z = c->spz;
+  a.smp.part_i = c->spi;
+  a.smp.counter = c->scnt;
+  a.smp.h_out = c->h;
+  a.bar = c->d_bar;
+  a.err = c->err;
+  CK(cudaMemsetAsync(c->d_bar, 0, sizeof(unsigned) * c->nph, c->st));
+  const int wf = c->wdtype == M3_W_INT8 ? WF_I8ROW : WF_BF16;
+  CK(launch_frame(a, wf, c->kv_f16, frame_rows_cta_max(c), c->nsm, c->st));
+  return M3_OK;
+}
+
 extern "C" int m3_decode_frame(m3_ctx* c, int rows, const int32_t* positions, uint64_t seed,
                                uint64_t frame, const void* x_in, float cfg_scale,
                                float temperature, int32_t* codes, void* h_out, float* logits) {
@@ -753,7 +888,12 @@ extern "C" int m3_decode_frame(m3_ctx* c, int rows, const int32_t* positions, ui
   CK(cudaMemcpyAsync(c->A.x, x_in, sizeof(bf16) * rows * g.hidden, cudaMemcpyDeviceToDevice, c->st));
   set_frame_params_kernel<<<1, 32, 0, c->st>>>(c->fp, fp);
   CK(cudaGetLastError());
-  CKR(run_graph(c, c->graphs, {rows, c->n_buckets}, [&] { return record_frame(c, rows, c->n_buckets); }));
+  if (frame_kernel_ok(c, rows)) {
+    CKR(run_frame_kernel(c, rows));
+  } else {
+    CKR(run_graph(c, c->graphs, {rows, c->n_buckets},
+                  [&] { return record_frame(c, rows, c->n_buckets); }));
+  }
   CK(cudaMemcpyAsync(codes, c->codes, sizeof(int) * rows, cudaMemcpyDeviceToDevice, c->st));
   if (h_out)
     CK(cudaMemcpyAsync(h_out, c->h, sizeof(bf16) * rows * g.hidden, cudaMemcpyDeviceToDevice, c->st));

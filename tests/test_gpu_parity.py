@@ -180,9 +180,13 @@ def test_errors_are_status_codes(ora):
 
 # -------------------------------------------------- one 8B decoder layer ----
 
+@pytest.mark.parametrize("path", ["frame_kernel", "per_kernel"])
 @pytest.mark.parametrize("wdtype,rows,kv_f16", [(0, 1, False), (0, 2, False), (1, 1, False),
                                                 (1, 2, True)])
-def test_layer8b_vs_oracle(ora, wdtype, rows, kv_f16):
+def test_layer8b_vs_oracle(ora, wdtype, rows, kv_f16, path, monkeypatch):
+    # the 8B layer shape runs through the per-kernel CUDA graph by default;
+    # M3_FRAME_KERNEL=1 selects the persistent whole-frame kernel
+    monkeypatch.setenv("M3_FRAME_KERNEL", "1" if path == "frame_kernel" else "0")
     s = synth.LAYER8B
     m = Model(s, seed=11, device="cuda", wdtype=wdtype, max_rows=2, kv_f16=kv_f16)
     try:
