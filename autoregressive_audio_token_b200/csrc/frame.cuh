@@ -63,7 +63,20 @@ struct FrameArgs {
   int* err;
 };
 
-constexpr int kFrameThreads = kConsumers + 64;
+// The frame kernel keeps its own warp layout: 8 compute warps owning 16 K
+// positions each per 4096-wide segment (bf16: two 16-byte chunks), 1
+// epilogue warp, 1 producer warp.
+constexpr int kFC = 256;
+constexpr int kFEpi = kFC / 32;
+constexpr int kFrameThreads = kFC + 64;
+
+template <int ESZ>
+struct FrameShape {
+  static constexpr int KC = 4096;                      // K elements per segment
+  static constexpr int R = kStageBytes / (KC * ESZ);   // rows per stage
+  static constexpr int P = R;                          // one row group
+  static constexpr int SLOTS = kFC / 32;               // partial sums per row
+};
 
 // attention scratch of the frame kernel (head_dim 128): q, k, v of the new
 // token, per-warp (m, l, o), new-token scores
@@ -75,7 +88,7 @@ constexpr int kFrameAttFloats = kAttnWarps * 128 + 2 * 128 + kAttnWarps * kAttnW
 // sampler's per-role bests.
 template <int MR, int WF>
 __host__ __device__ constexpr size_t frame_smem_bytes(int rows_cta_max) {
-  using S = GemvShape<256, WF == WF_BF16 ? 2 : 1>;
+  using S = FrameShape<WF == WF_BF16 ? 2 : 1>;
   return (size_t)kStages * kStageBytes + 2 * kStages * sizeof(uint64_t) +
          sizeof(float) * ((size_t)kPartBufs * S::SLOTS * S::P * MR + 9 * MR + kFrameAttFloats +
                           (size_t)rows_cta_max * MR) +
@@ -92,13 +105,13 @@ template <int MR, int WF, int KVF16>
 __global__ void __launch_bounds__(kFrameThreads, 1) frame_kernel(const FrameArgs a) {
   constexpr int D = 128, TPR = 256;
   constexpr int ESZ = WF == WF_BF16 ? 2 : 1;
-  using S = GemvShape<TPR, ESZ>;
+  using S = FrameShape<ESZ>;
   constexpr int KC = S::KC, R = S::R, P = S::P, SLOTS = S::SLOTS;
   constexpr int V = P * MR;
   constexpr int LV = V == 1 ? 0 : V == 2 ? 1 : V == 4 ? 2 : V == 8 ? 3 : V == 16 ? 4 : 5;
   constexpr bool kScatter = V <= 32;
   constexpr int kBarCompute = 1, kBarFull = 2, kBarEmpty = 2 + kPartBufs;
-  constexpr int kPartThreads = kConsumers + 32;
+  constexpr int kPartThreads = kFC + 32;
   constexpr int VPL = D / 32, NT = D / 8, KS = D / 16;
   constexpr int TILE_BYTES = kAttnTile * D * 2;
   static_assert(2 * TILE_BYTES <= kStageBytes, "a K/V tile pair fits one ring stage");
@@ -147,14 +160,14 @@ __global__ void __launch_bounds__(kFrameThreads, 1) frame_kernel(const FrameArgs
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumers / 32);
+      mbar_init(&empty[s], kFC / 32);
     }
     fence_barrier_init();
   }
   __syncthreads();
 
   // =============================================================== producer
-  if (warp == kEpiWarp + 1) {
+  if (warp == kFEpi + 1) {
     if (lane != 0) return;
     const uint64_t pol = policy_evict_first();
     int s = 0;
@@ -211,7 +224,7 @@ __global__ void __launch_bounds__(kFrameThreads, 1) frame_kernel(const FrameArgs
   }
 
   // =============================================================== epilogue
-  if (warp == kEpiWarp) {
+  if (warp == kFEpi) {
     // total partial stages of this CTA (the compute warps wait on EMPTY only
     // for stages that have a successor kPartBufs later)
     int total_sp = 0;
@@ -403,7 +416,7 @@ __global__ void __launch_bounds__(kFrameThreads, 1) frame_kernel(const FrameArgs
         if ((it & 1023) == 0 && *reinterpret_cast<volatile int*>(a.err) != 0) break;
       }
     }
-    named_bar_sync(kBarCompute, kConsumers);
+    named_bar_sync(kBarCompute, kFC);
   };
 
   for (int p = 0; p < a.nph; ++p) {
@@ -472,7 +485,7 @@ __global__ void __launch_bounds__(kFrameThreads, 1) frame_kernel(const FrameArgs
             }
           }
         }
-        named_bar_sync(kBarCompute, kConsumers);
+        named_bar_sync(kBarCompute, kFC);
         if (is_q) {
           float pq = 0.0f;
 #pragma unroll
@@ -598,7 +611,7 @@ __global__ void __launch_bounds__(kFrameThreads, 1) frame_kernel(const FrameArgs
             wh[2 + 8 * j + 2 * tig + 1] = o_acc[j][1];
           }
         }
-        named_bar_sync(kBarCompute, kConsumers);
+        named_bar_sync(kBarCompute, kFC);
         const int stride = D + 2;
         if (is_q) {
           const int h = g * grp + warp;
@@ -632,13 +645,13 @@ __global__ void __launch_bounds__(kFrameThreads, 1) frame_kernel(const FrameArgs
           for (int e = 0; e < VPL; ++e) pp[2 + VPL * lane + e] = o[e];
           __threadfence();
         }
-        named_bar_sync(kBarCompute, kConsumers);
+        named_bar_sync(kBarCompute, kFC);
         if (tid == 0) {
           __threadfence();
           const unsigned old = atomicAdd(a.acnt + (size_t)r * a.Hkv + g, 1u);
           s_flag = (old == (unsigned)(a.splits - 1));
         }
-        named_bar_sync(kBarCompute, kConsumers);
+        named_bar_sync(kBarCompute, kFC);
         if (s_flag) {
           __threadfence();
           if (is_q) {
@@ -663,7 +676,7 @@ __global__ void __launch_bounds__(kFrameThreads, 1) frame_kernel(const FrameArgs
           }
           if (tid == 0) a.acnt[(size_t)r * a.Hkv + g] = 0u;
         }
-        named_bar_sync(kBarCompute, kConsumers);  // before the next item reuses q_s ...
+        named_bar_sync(kBarCompute, kFC);  // before the next item reuses q_s ...
       }
       if (tid == 0) {
         __threadfence();
@@ -688,7 +701,7 @@ __global__ void __launch_bounds__(kFrameThreads, 1) frame_kernel(const FrameArgs
       float ss[MR];
 #pragma unroll
       for (int m = 0; m < MR; ++m) ss[m] = 0.0f;
-      for (int k = tid; k < K; k += kConsumers) {
+      for (int k = tid; k < K; k += kFC) {
 #pragma unroll
         for (int m = 0; m < MR; ++m)
           if (m < mr) {
@@ -703,15 +716,15 @@ __global__ void __launch_bounds__(kFrameThreads, 1) frame_kernel(const FrameArgs
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
         if (lane == 0) nrm[warp * MR + m] = v;
       }
-      named_bar_sync(kBarCompute, kConsumers);
+      named_bar_sync(kBarCompute, kFC);
 #pragma unroll
       for (int m = 0; m < MR; ++m) {
         float tot = 0.0f;
 #pragma unroll
-        for (int w = 0; w < kConsumers / 32; ++w) tot += nrm[w * MR + m];
+        for (int w = 0; w < kFC / 32; ++w) tot += nrm[w * MR + m];
         inv[m] = 1.0f / sqrtf(tot / (float)K + a.eps);
       }
-      named_bar_sync(kBarCompute, kConsumers);  // nrm is reused by the next norm
+      named_bar_sync(kBarCompute, kFC);  // nrm is reused by the next norm
     }
     const bool write_h = ph.kind == PH_LM && a.smp.h_out && blockIdx.x == 0;
 

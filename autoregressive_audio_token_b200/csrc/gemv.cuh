@@ -30,7 +30,7 @@ namespace m3 {
 enum : int { EPI_STORE = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_SAMPLE = 3 };
 enum : int { WF_BF16 = 0, WF_I8ROW = 1, WF_I8G128 = 2 };
 
-constexpr int kConsumers = 256;                  // 8 compute warps
+constexpr int kConsumers = 512;                  // 16 compute warps
 constexpr int kEpiWarp = kConsumers / 32;        // warp 8: epilogue
 constexpr int kGemvThreads = kConsumers + 64;    // + epilogue warp + producer warp
 constexpr int kPartBufs = 4;                     // partial-sum buffers in flight
@@ -94,7 +94,8 @@ struct GemvArgs {
 
 template <int TPR, int ESZ>
 struct GemvShape {
-  static constexpr int KC = TPR * 16;                 // K elements per segment
+  static constexpr int EPT = 16 / ESZ;                // K elements per thread: one 16-B chunk
+  static constexpr int KC = TPR * EPT;                // K elements per segment
   static constexpr int G = kConsumers / TPR;          // rows in flight per pass
   static constexpr int R = kStageBytes / (KC * ESZ);  // rows (segments) per stage
   static constexpr int P = R / G;                     // passes per stage
@@ -108,7 +109,8 @@ template <int MR, int TPR, int ESZ>
 __host__ __device__ constexpr size_t gemv_smem_bytes(int rows_cta_max) {
   using S = GemvShape<TPR, ESZ>;
   return (size_t)kStages * kStageBytes + 2 * kStages * sizeof(uint64_t) +
-         sizeof(float) * (kPartBufs * S::SLOTS * S::P * MR + 9 * MR + (size_t)rows_cta_max * MR) +
+         sizeof(float) * (kPartBufs * S::SLOTS * S::P * MR + (kConsumers / 32 + 1) * MR +
+                          (size_t)rows_cta_max * MR) +
          (sizeof(float) + sizeof(int)) * S::R * MR + 64;
 }
 
@@ -147,6 +149,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvArgs a)
   constexpr int ESZ = WF == WF_BF16 ? 2 : 1;
   using S = GemvShape<TPR, ESZ>;
   constexpr int KC = S::KC, G = S::G, R = S::R, P = S::P, W = S::W, SLOTS = S::SLOTS;
+  constexpr int EPT = S::EPT;
   constexpr int UNIT = EPI == EPI_SWIGLU ? 2 : 1;
   constexpr int V = P * MR;  // partial sums per thread per stage
   constexpr int LV = V == 1 ? 0 : V == 2 ? 1 : V == 4 ? 2 : V == 8 ? 3 : V == 16 ? 4 : 5;
@@ -161,7 +164,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvArgs a)
   uint64_t* empty = full + kStages;
   float* part = reinterpret_cast<float*>(empty + kStages);  // [kPartBufs][SLOTS][V]
   float* nrm = part + kPartBufs * SLOTS * V;                 // [8][MR] + [MR]
-  float* accr = nrm + 9 * MR;                                 // [rows_cta][MR]
+  float* accr = nrm + (kConsumers / 32 + 1) * MR;              // [rows_cta][MR]
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -432,21 +435,17 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvArgs a)
     }
   }
 
-  // x in registers: this thread's 16 K positions of the current chunk, as 8
-  // packed fp32 pairs (even, odd) for the packed FMA.
-  uint64_t xr2[MR][8];
-  auto elem_k = [&](int kc, int e) -> int {
-    if (ESZ == 2) return kc * KC + (e < 8 ? 8 * t + e : 8 * (t + TPR) + (e - 8));
-    return kc * KC + 16 * t + e;
-  };
+  // x in registers: this thread's EPT K positions of the current segment
+  // (one 16-byte weight chunk per row), as packed fp32 pairs (even, odd).
+  uint64_t xr2[MR][EPT / 2];
   auto load_x = [&](int kc) {
     const bool write_h = (EPI == EPI_SAMPLE) && a.smp.h_out && blockIdx.x == 0 && g == 0;
 #pragma unroll
-    for (int e2 = 0; e2 < 8; ++e2) {
+    for (int e2 = 0; e2 < EPT / 2; ++e2) {
       float vv[MR][2];
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
-        const int k = elem_k(kc, 2 * e2 + q);
+        const int k = kc * KC + EPT * t + 2 * e2 + q;
         const bool ok = k < K;
         const float gm = (a.gamma && ok) ? __bfloat162float(a.gamma[k]) : 1.0f;
 #pragma unroll
@@ -475,69 +474,54 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvArgs a)
       const int rs = r_begin + sr * R;
       const int nr = min(R, r_end - rs);
       const uint8_t* st = ring + slot * kStageBytes;
-      // packed (even, odd) partial sums per (row-in-pass, batch row)
-      uint64_t acc2[V];
+      // per (row-in-pass, batch row) partial sums; each row's chunk is summed
+      // in packed (even, odd) pairs and folded into one float
+      float acc[V];
 #pragma unroll
-      for (int i = 0; i < V; ++i) acc2[i] = 0ull;
-
+      for (int i = 0; i < V; ++i) acc[i] = 0.0f;
+      const bool in_k = EPT * t < kel;
 #pragma unroll
       for (int p = 0; p < P; ++p) {
         const int rl = p * G + g;
-        if (rl < nr) {
-          const uint8_t* sg = st + (size_t)rl * KC * ESZ;
+        if (rl < nr && in_k) {
+          const uint4 wv = *reinterpret_cast<const uint4*>(st + (size_t)rl * KC * ESZ + 16 * t);
+          const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+          uint64_t pm2[MR];
+#pragma unroll
+          for (int m = 0; m < MR; ++m) pm2[m] = 0ull;
           if constexpr (ESZ == 2) {
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int c = t + h * TPR;  // 16-byte chunk index in the segment
-              if (8 * c < kel) {
-                const uint4 wv = *reinterpret_cast<const uint4*>(sg + 16 * c);
-                const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+            for (int j = 0; j < 4; ++j) {
+              // (bf16 lo, bf16 hi) -> exact fp32 pair
+              const uint64_t wp = pack_u32x2(ww[j] << 16, ww[j] & 0xFFFF0000u);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                  // (bf16 lo, bf16 hi) -> exact fp32 pair
-                  const uint64_t wp = pack_u32x2(ww[j] << 16, ww[j] & 0xFFFF0000u);
-#pragma unroll
-                  for (int m = 0; m < MR; ++m) ffma2(acc2[p * MR + m], wp, xr2[m][4 * h + j]);
-                }
-              }
+              for (int m = 0; m < MR; ++m) ffma2(pm2[m], wp, xr2[m][j]);
             }
           } else {
-            if (16 * t < kel) {
-              const uint4 wv = *reinterpret_cast<const uint4*>(sg + 16 * t);
-              const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
-              uint64_t pm2[MR];
 #pragma unroll
-              for (int m = 0; m < MR; ++m) pm2[m] = 0ull;
+            for (int j = 0; j < 4; ++j) {
+              uint64_t f01, f23;
+              s8x4_to_f32x2(ww[j], f01, f23);
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                uint64_t f01, f23;
-                s8x4_to_f32x2(ww[j], f01, f23);
-#pragma unroll
-                for (int m = 0; m < MR; ++m) {
-                  ffma2(pm2[m], f01, xr2[m][2 * j]);
-                  ffma2(pm2[m], f23, xr2[m][2 * j + 1]);
-                }
-              }
-              if constexpr (WF == WF_I8G128) {
-                const int n = rs + rl;
-                const int kabs = kc * KC + 16 * t;
-                const float sc = __ldg(a.scales + (size_t)n * (K / 128) + kabs / 128);
-                const uint64_t sc2 = pack_f32x2(sc, sc);
-#pragma unroll
-                for (int m = 0; m < MR; ++m) ffma2(acc2[p * MR + m], sc2, pm2[m]);
-              } else {
-#pragma unroll
-                for (int m = 0; m < MR; ++m) fadd2(acc2[p * MR + m], pm2[m]);
+              for (int m = 0; m < MR; ++m) {
+                ffma2(pm2[m], f01, xr2[m][2 * j]);
+                ffma2(pm2[m], f23, xr2[m][2 * j + 1]);
               }
             }
           }
-        }
-      }
-      float acc[V];
+          float sc = 1.0f;
+          if constexpr (WF == WF_I8G128) {
+            const int n = rs + rl;
+            const int kabs = kc * KC + 16 * t;
+            sc = __ldg(a.scales + (size_t)n * (K / 128) + kabs / 128);
+          }
 #pragma unroll
-      for (int i = 0; i < V; ++i) {
-        const float2 f = unpack_f32x2(acc2[i]);
-        acc[i] = f.x + f.y;
+          for (int m = 0; m < MR; ++m) {
+            const float2 f = unpack_f32x2(pm2[m]);
+            if constexpr (WF == WF_I8G128) acc[p * MR + m] = fmaf(sc, f.x + f.y, acc[p * MR + m]);
+            else acc[p * MR + m] += f.x + f.y;
+          }
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);

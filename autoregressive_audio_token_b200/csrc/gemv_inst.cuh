@@ -32,10 +32,15 @@ cudaError_t launch_gemv_mr(const GemvArgs& a, cudaStream_t st, bool pdl, int nsm
 
 template <int WF, int EPI>
 cudaError_t launch_gemv_k(const GemvArgs& a, cudaStream_t st, bool pdl, int nsm) {
-  switch (gemv_tpr(a.K)) {
-    case 16: return launch_gemv_mr<WF, EPI, 16>(a, st, pdl, nsm);
+  constexpr int ESZ = WF == WF_BF16 ? 2 : 1;
+  switch (gemv_tpr(a.K, ESZ)) {
+    case 32: return launch_gemv_mr<WF, EPI, 32>(a, st, pdl, nsm);
     case 64: return launch_gemv_mr<WF, EPI, 64>(a, st, pdl, nsm);
-    default: return launch_gemv_mr<WF, EPI, 256>(a, st, pdl, nsm);
+    case 128: return launch_gemv_mr<WF, EPI, 128>(a, st, pdl, nsm);
+    case 256: return launch_gemv_mr<WF, EPI, 256>(a, st, pdl, nsm);
+    default:
+      if constexpr (ESZ == 2) return launch_gemv_mr<WF, EPI, 512>(a, st, pdl, nsm);
+      return cudaErrorInvalidValue;
   }
 }
 

@@ -29,13 +29,15 @@ cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sm
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-// Threads per output row for a GEMV over K inputs (16 inputs per thread per
-// segment); K > 1024 streams in segments of 4096.
-inline int gemv_tpr(int K) { return K <= 256 ? 16 : (K <= 1024 ? 64 : 256); }
-
-inline int gemv_rows_per_stage(int K, int esz) {
-  const int kc = gemv_tpr(K) * 16;
-  return kStageBytes / (kc * esz);
+// Threads per output row for a GEMV over K inputs: one 16-byte chunk each
+// (8 bf16 or 16 int8 inputs), the fewest threads covering min(K, 4096);
+// K > 4096 streams in segments of 4096.
+inline int gemv_tpr(int K, int esz) {
+  const int ept = 16 / esz;
+  const int target = K < 4096 ? K : 4096;
+  int tpr = 32;
+  while (tpr * ept < target && tpr < 512) tpr *= 2;
+  return tpr;
 }
 
 cudaError_t launch_gemv_bf16(const GemvArgs& a, int epi, cudaStream_t st, bool pdl, int nsm);

@@ -742,9 +742,8 @@ static int run_graph(m3_ctx* c, std::map<std::pair<int, int>, cudaGraphExec_t>& 
 // until it beats that graph.
 static bool frame_kernel_ok(const m3_ctx* c, int rows) {
   const m3_config& g = c->cfg;
-  return c->use_frame_kernel && rows <= 4 && g.head_dim == 128 && gemv_tpr(g.hidden) == 256 &&
-         gemv_tpr(g.n_q_heads * g.head_dim) == 256 && gemv_tpr(g.ffn) == 256 &&
-         c->nsm <= 1024;
+  return c->use_frame_kernel && rows <= 4 && g.head_dim == 128 && g.hidden > 1024 &&
+         g.n_q_heads * g.head_dim > 1024 && g.ffn > 1024 && c->nsm <= 1024;
 }
 
 static int frame_rows_cta_max(const m3_ctx* c) {
