@@ -180,12 +180,6 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const Attn
                     bytes, &bars[b]);
   };
 
-  // Zero the tile buffers once: rows past the end of a partial tile are
-  // multiplied by p = 0 and must not hold NaN patterns.
-  for (int i = tid; i < kAttnBuf * 2 * TILE_ELEMS / 8; i += blockDim.x)
-    reinterpret_cast<uint4*>(kt)[i] = make_uint4(0, 0, 0, 0);
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  __syncthreads();
   if (tid == 0) {
     for (int b = 0; b < kAttnBuf; ++b) mbar_init(&bars[b], 1);
     fence_barrier_init();
@@ -291,6 +285,17 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const Attn
     const int b = t % kAttnBuf;
     mbar_wait(&bars[b], (t / kAttnBuf) & 1, a.err);
     const int nv = min(kAttnTile, jc1 - (j0 + t * kAttnTile));
+    if (nv < kAttnTile) {
+      // rows past the end of a partial tile hold stale (or never written)
+      // shared memory; zero them so that p = 0 never multiplies a NaN pattern
+      uint4* kz = reinterpret_cast<uint4*>(kt + b * TILE_ELEMS);
+      uint4* vz = reinterpret_cast<uint4*>(vt + b * TILE_ELEMS);
+      for (int c = nv * (D / 8) + lane; c < kAttnTile * (D / 8); c += 32) {
+        kz[c] = make_uint4(0, 0, 0, 0);
+        vz[c] = make_uint4(0, 0, 0, 0);
+      }
+      __syncwarp();
+    }
     const uint32_t kb = smem_u32(kt + b * TILE_ELEMS);
     const uint32_t vb = smem_u32(vt + b * TILE_ELEMS);
     // S = Q K^T: 4 n-tiles of 8 positions
@@ -422,33 +427,44 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const Attn
     for (int e = 0; e < VPL; ++e) cw[2 + VPL * lane + e] = o[e];
   }
 
-  // ---- the splits of (r, g) form one cluster: rank 0 merges them through
-  // distributed shared memory (log-sum-exp), then every CTA may exit ------
+  // ---- the splits of (r, g) form one cluster and merge through distributed
+  // shared memory (log-sum-exp): rank s finishes its slice of the group's
+  // (head, dim) outputs, reading every rank's partial in parallel ----------
   cg::cluster_group cluster = cg::this_cluster();
   cluster.sync();
-  if (sidx == 0 && w < grp) {
-    const int h = g * grp + w;
-    float M = -INFINITY;
-    for (int s2 = 0; s2 < S; ++s2) {
-      const float* rem = cluster.map_shared_rank(cp_s, s2) + w * stride;
-      M = fmaxf(M, rem[0]);
+  {
+    const int items = grp * D;
+    const int per = (items + S - 1) / S;
+    const int it_end = min(items, (sidx + 1) * per);
+    for (int it = sidx * per + tid; it < it_end; it += blockDim.x) {
+      const int hl = it / D, d = it % D;
+      float ms[kAttnMaxSplits], ls[kAttnMaxSplits], os[kAttnMaxSplits];
+#pragma unroll
+      for (int s2 = 0; s2 < kAttnMaxSplits; ++s2) {
+        if (s2 < S) {
+          const float* rem = cluster.map_shared_rank(cp_s, s2) + hl * stride;
+          ms[s2] = rem[0];
+          ls[s2] = rem[1];
+          os[s2] = rem[2 + d];
+        }
+      }
+      float M = -INFINITY;
+#pragma unroll
+      for (int s2 = 0; s2 < kAttnMaxSplits; ++s2)
+        if (s2 < S) M = fmaxf(M, ms[s2]);
+      float L = 0.0f, o = 0.0f;
+#pragma unroll
+      for (int s2 = 0; s2 < kAttnMaxSplits; ++s2) {
+        if (s2 < S) {
+          const float f = ms[s2] == -INFINITY ? 0.0f : expf(ms[s2] - M);
+          L = fmaf(ls[s2], f, L);
+          o = fmaf(os[s2], f, o);
+        }
+      }
+      a.out[(size_t)r * a.Hq * D + (size_t)(g * grp + hl) * D + d] = __float2bfloat16_rn(o / L);
     }
-    float L = 0.0f, o[VPL];
-#pragma unroll
-    for (int e = 0; e < VPL; ++e) o[e] = 0.0f;
-    for (int s2 = 0; s2 < S; ++s2) {
-      const float* rem = cluster.map_shared_rank(cp_s, s2) + w * stride;
-      const float ms = rem[0];
-      const float f = ms == -INFINITY ? 0.0f : expf(ms - M);
-      L = fmaf(rem[1], f, L);
-#pragma unroll
-      for (int e = 0; e < VPL; ++e) o[e] = fmaf(rem[2 + VPL * lane + e], f, o[e]);
-    }
-    __nv_bfloat16* dst = a.out + (size_t)r * a.Hq * D + (size_t)h * D + VPL * lane;
-#pragma unroll
-    for (int e = 0; e < VPL; ++e) dst[e] = __float2bfloat16_rn(o[e] / L);
   }
-  cluster.sync();
+  cluster.sync();  // no CTA leaves while another still reads its shared memory
 }
 
 }  // namespace m3
