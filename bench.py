@@ -47,6 +47,12 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--layers", type=int, default=36,
                    help="body layers (36 = the workload; fewer only for profiling small cases)")
+    p.add_argument("--kv", default="bf16", choices=["bf16", "f16"])
+    p.add_argument("--depth", action="store_true",
+                   help="run the RVQ depth decoder (7 codes) after every frame")
+    p.add_argument("--sweep", action="store_true",
+                   help="batched-variations sweep: rows 2..16 x context 1500/4500/9000, "
+                        "bf16 and int8; one JSON line per point")
     return p.parse_args()
 
 
@@ -141,10 +147,11 @@ class ClockSampler:
 
 # ------------------------------------------------------------ our arm ------
 
-def build_model(torch, m3, synth, seed: int, wdtype: int, layers: int = 36):
+def build_model(torch, m3, synth, seed: int, wdtype: int, layers: int = 36, depth: bool = False,
+                max_rows: int = ROWS):
     import dataclasses
     s = dataclasses.replace(synth.FULL8B, n_layers=layers)
-    cfg = m3.config_from_shapes(s, None, max_rows=ROWS)
+    cfg = m3.config_from_shapes(s, synth.DEPTH if depth else None, max_rows=max_rows)
     ctx = m3.m3_create(cfg)
     for l in range(s.n_layers):  # generate on the GPU, load layer by layer
         Lw = synth.layer_weights(s, 0, l, device="cuda")
@@ -152,13 +159,19 @@ def build_model(torch, m3, synth, seed: int, wdtype: int, layers: int = 36):
         del Lw
     m3.m3_load_weights(ctx, [], final_norm=synth.final_norm(s, 0, device="cuda"),
                        lm_head=synth.lm_head_slice(s, 0, device="cuda"), wdtype=wdtype)
-    m3.m3_kv_alloc(ctx, ROWS, SONG_FRAMES, m3.M3_KV_BF16, 256)
-    K, V = synth.kv_prefill(s, ROWS, SONG_FRAMES, seed, device="cuda")
-    for r in range(ROWS):
-        m3.m3_kv_set(ctx, r, K[r], V[r])
-    del K, V
+    if depth:
+        m3.m3_load_depth_weights(ctx, synth.depth_weights(synth.DEPTH, 0, device="cuda"))
     torch.cuda.synchronize()
     return s, ctx
+
+
+def prefill_kv(torch, m3, synth, s, ctx, rows: int, n_pos: int, seed: int, kv_f16: bool):
+    m3.m3_kv_alloc(ctx, rows, n_pos, m3.M3_KV_F16 if kv_f16 else m3.M3_KV_BF16, 256)
+    for r in range(rows):  # one row at a time bounds the staging memory
+        K, V = synth.kv_prefill(s, 1, n_pos, seed + 17 * r, device="cuda")
+        m3.m3_kv_set(ctx, r, K[0], V[0])
+        del K, V
+    torch.cuda.synchronize()
 
 
 def run_ours(args, rank, world, local):
@@ -174,13 +187,20 @@ def run_ours(args, rank, world, local):
                                 device_id=torch.device("cuda", local))
     seed = replica_seed(rank)
     wdtype = m3.M3_W_INT8 if args.wdtype == "int8" else m3.M3_W_BF16
-    s, ctx = build_model(torch, m3, synth, seed, wdtype, args.layers)
+    s, ctx = build_model(torch, m3, synth, seed, wdtype, args.layers, depth=args.depth)
+    prefill_kv(torch, m3, synth, s, ctx, ROWS, SONG_FRAMES, seed, args.kv == "f16")
     xs = synth.normal((64, ROWS, s.hidden), seed, "bench/x_in", std=0.02, device="cuda")
     codes = torch.empty(ROWS, dtype=torch.int32, device="cuda")
+    h_dev = torch.empty((ROWS, s.hidden), dtype=torch.bfloat16, device="cuda")
+    dcodes = torch.empty((ROWS, synth.DEPTH.codebooks), dtype=torch.int32, device="cuda")
     stream = torch.cuda.current_stream()
 
     def frame(i, pos):
-        m3.m3_decode_frame(ctx, [pos] * ROWS, seed, i, xs[i % 64], CFG_SCALE, 1.0, codes)
+        if args.depth:
+            m3.m3_decode_frame(ctx, [pos] * ROWS, seed, i, xs[i % 64], CFG_SCALE, 1.0, codes, h_dev)
+            m3.m3_depth_decode(ctx, h_dev, codes, seed, i, CFG_SCALE, 1.0, dcodes)
+        else:
+            m3.m3_decode_frame(ctx, [pos] * ROWS, seed, i, xs[i % 64], CFG_SCALE, 1.0, codes)
 
     # capture every bucket's graph before timing, then warm up
     for b in range(0, SONG_FRAMES, 256):
@@ -254,6 +274,7 @@ def run_ours(args, rank, world, local):
         pass
 
     fps = 1000.0 / ms_per_step * world
+    variant = workload_name(args)
     out = {
         "metric": METRIC if args.wdtype == "bf16" else METRIC.replace("bf16", "int8"),
         "value": fps,
@@ -267,9 +288,10 @@ def run_ours(args, rank, world, local):
         "vs_baseline": None,
         "dtype": args.wdtype,
         "data": "synthetic (seeded N(0,0.02^2) weights, N(0,1) KV prefill, random-init 8B shape)",
-        "config": {"workload": WORKLOAD if args.wdtype == "bf16" else WORKLOAD.replace("bf16", "int8"),
+        "config": {"workload": variant,
                    "rows": ROWS, "song_frames": SONG_FRAMES, "mean_ctx": mean_ctx,
-                   "cfg_scale": CFG_SCALE, "temperature": 1.0, "kv": "bf16 pages of 256",
+                   "cfg_scale": CFG_SCALE, "temperature": 1.0, "kv": f"{args.kv} pages of 256",
+                   "depth_decoder": bool(args.depth),
                    "l2": "no flush: 14 GB of weights per frame >> 126 MB L2",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "gpu_launches": None,
@@ -287,7 +309,11 @@ def run_ours(args, rank, world, local):
         "clocks": clk,
     }
     # kernels per frame: 5 per layer (qkv, attention, o, gate/up, down) + lm_head + params
-    out["gpu_launches"] = (5 * s.n_layers + 1 + 1) * args.steps
+    # per frame: parameter block + 5 kernels per layer + lm_head sampler; the
+    # depth decoder adds its parameter block, projection, 7 embeddings,
+    # 8 positions x layers x 5 kernels and 7 heads
+    depth_launches = (2 + 7 + 8 * synth.DEPTH.n_layers * 5 + 7) if args.depth else 0
+    out["gpu_launches"] = (5 * s.n_layers + 1 + 1 + depth_launches) * args.steps
     m3.m3_destroy(ctx)
     del xs
     torch.cuda.empty_cache()
@@ -365,9 +391,69 @@ def run_reference(args, rank, world):
                     "d2h_bytes_per_step": 0}}
 
 
+def workload_name(args) -> str:
+    name = WORKLOAD.replace("bf16", args.wdtype)
+    if args.kv != "bf16":
+        name += f"-{args.kv}kv"
+    if args.depth:
+        name += "-depth7"
+    return name
+
+
+def run_sweep(args):
+    """Batched-variations sweep: K = 1, 2, 4, 8 same-prompt variations decoded in
+    lockstep (rows = 2K), contexts 1500 / 4500 / 9000, bf16 and int8 weights,
+    bf16 KV; per point one JSON line with frames/s per row, ms/frame, the
+    frame's algorithmic bytes and GB/s, and the cost of each extra row pair
+    relative to the 2-row frame at the same context."""
+    import torch
+    from autoregressive_audio_token_b200 import m3
+    import synth
+    torch.cuda.set_device(0)
+    for wname in ("bf16", "int8"):
+        wd = m3.M3_W_INT8 if wname == "int8" else m3.M3_W_BF16
+        s, ctx = build_model(torch, m3, synth, 7, wd, max_rows=16)
+        for n_ctx in (1500, 4500, 9000):
+            base = None
+            for rows in (2, 4, 8, 16):
+                prefill_kv(torch, m3, synth, s, ctx, rows, n_ctx, 7, False)
+                xs = synth.normal((rows, s.hidden), 7, "sweep/x", std=0.02, device="cuda")
+                codes = torch.empty(rows, dtype=torch.int32, device="cuda")
+                pos = [n_ctx - 1] * rows
+                for i in range(3):
+                    m3.m3_decode_frame(ctx, pos, 7, i, xs, CFG_SCALE, 1.0, codes)
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                steps = 10
+                e0.record()
+                for i in range(steps):
+                    m3.m3_decode_frame(ctx, pos, 7, i, xs, CFG_SCALE, 1.0, codes)
+                e1.record()
+                torch.cuda.synchronize()
+                m3.m3_sync_status(ctx)
+                ms = e0.elapsed_time(e1) / steps
+                fb = m3.m3_frame_bytes(ctx, rows, n_ctx - 1)
+                if rows == 2:
+                    base = ms
+                print(json.dumps({"sweep": "batched variations", "weights": wname, "kv": "bf16",
+                                  "rows": rows, "variations": rows // 2, "ctx": n_ctx,
+                                  "ms_per_frame": ms, "frames_per_s_per_row": 1000.0 / ms,
+                                  "row_frames_per_s": rows * 1000.0 / ms,
+                                  "algorithmic_bytes": fb, "achieved_gbs": fb / ms / 1e6,
+                                  "extra_pair_cost_vs_2rows": (ms / base - 1.0) / max(1, rows // 2 - 1)
+                                  if rows > 2 else 0.0}), flush=True)
+                del xs
+        m3.m3_destroy(ctx)
+        torch.cuda.empty_cache()
+
+
 def main():
     args = parse()
     rank, world, local = dist_env()
+    if args.sweep:
+        if rank == 0:
+            run_sweep(args)
+        return
     if args.impl == "reference":
         out = run_reference(args, rank, world)
     else:
