@@ -92,33 +92,81 @@ def song_positions(k: int, song: int = SONG_FRAMES):
 # ---------------------------------------------------------------- clocks ----
 
 class ClockSampler:
+    """SM clock and clock-event reasons sampled DURING the timed region.
+
+    An NVML polling thread (every 5 ms, read-only queries) finds this
+    process's GPU by PCI bus id; where NVML is missing it falls back to an
+    `nvidia-smi -lms 200` child process."""
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index: int, path: str):
+    def __init__(self, local: int, path: str):
+        self.local = local
         self.path = path
-        self.index = index
+        self.samples = []
+        self.stop_flag = False
+        self.thread = None
         self.proc = None
-        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
-        # with one visible GPU nvidia-smi may still list several: keep ours
-        self.multi = vis is None or "," in vis
-        if vis is not None and "," not in vis and vis.strip().isdigit():
-            self.index = int(vis)
-            self.multi = True
+        self.nvml = None
+        self.handle = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            p = torch.cuda.get_device_properties(local)
+            want = (int(p.pci_domain_id), int(p.pci_bus_id), int(p.pci_device_id))
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                info = pynvml.nvmlDeviceGetPciInfo(h)
+                if (int(info.domain), int(info.bus), int(info.device)) == want:
+                    self.handle = h
+                    break
+            if self.handle is not None:
+                self.nvml = pynvml
+        except Exception:
+            self.nvml = None
+
+    def _poll(self):
+        nv = self.nvml
+        while not self.stop_flag:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                smax = nv.nvmlDeviceGetMaxClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                self.samples.append((float(sm), float(smax), int(rs)))
+            except Exception:
+                pass
+            time.sleep(0.005)
 
     def start(self):
+        if self.nvml is not None:
+            import threading
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return
         try:
             self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi",
+            self.proc = subprocess.Popen(["nvidia-smi", f"-i={self.local}",
                                           f"--query-gpu={self.QUERY}", "--format=csv,noheader",
                                           "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
     def stop(self) -> dict:
+        if self.thread is not None:
+            self.stop_flag = True
+            self.thread.join()
+            sm = [s for s, _, _ in self.samples]
+            smax = [m for _, m, _ in self.samples]
+            reasons = {n for _, _, r in self.samples for n, bit in self.REASONS if r & bit}
+            return {"sm_mhz": statistics.median(sm) if sm else None,
+                    "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                    "samples": len(sm), "source": "nvml, 5 ms"}
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -126,23 +174,21 @@ class ClockSampler:
             self.proc.kill()
         self.f.close()
         sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9 or (parts[0] != str(self.index) and len(parts[0]) > 0 and
-                                  self.multi):
+            if len(parts) < 9:
                 continue
             try:
                 sm.append(float(parts[1].split()[0]))
                 smax.append(float(parts[2].split()[0]))
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
+            for (n, _), v in zip(self.REASONS, parts[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvidia-smi, 200 ms"}
 
 
 # ------------------------------------------------------------ our arm ------
