@@ -23,7 +23,8 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]
 
-SOURCES = ["m3.cu", "attention.cu", "frame.cu", "gemv_bf16.cu", "gemv_i8row.cu", "gemv_i8g128.cu"]
+SOURCES = ["m3.cu", "attention.cu", "gemv_tile.cu", "gemv_bf16.cu", "gemv_i8row.cu",
+           "gemv_i8g128.cu"]
 
 
 def _deps_mtime() -> float:

@@ -90,6 +90,10 @@ struct GemvArgs {
   const FrameParams* fp;
   SampleArgs smp;
   int* err;
+  // tiled kernels (gemv_tile.cuh, gemv_dyn.cuh) only: CTAs per cluster,
+  // stage bytes, stages; the dynamic kernel's {claim, done} counter pair
+  int tc, tsb, tns;
+  unsigned* ctr;
 };
 
 template <int TPR, int ESZ>

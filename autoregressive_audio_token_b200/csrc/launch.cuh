@@ -51,16 +51,18 @@ inline cudaError_t launch_gemv(const GemvArgs& a, int wf, int epi, cudaStream_t 
   return launch_gemv_i8g128(a, epi, st, pdl, nsm);
 }
 
+// The tiled tensor-core GEMV (gemv_tile.cuh): its launch plan and launcher.
+struct TileLaunch {
+  int C = 1, grid = 0, sb = 0, ns = 0;
+  size_t smem = 0;
+  bool dyn = false;  // dynamic unit claiming (gemv_dyn.cuh): needs a counter pair
+};
+cudaError_t plan_gemv_tile(int N, int K, int mr, int wf, int epi, int nsm, int sb, int ns,
+                           bool dyn, TileLaunch* out);
+cudaError_t launch_gemv_tile(const GemvArgs& a, int wf, int epi, const TileLaunch& L,
+                             cudaStream_t st, bool pdl);
+
 cudaError_t launch_attn(const AttnArgs& a, int D, int kv_f16, int splits, int rows,
                         cudaStream_t st, bool pdl);
 
-}  // namespace m3
-
-namespace m3 {
-struct FrameArgs;
-// Persistent whole-frame kernel (frame.cuh): cooperative launch of `grid`
-// CTAs (one per SM).
-cudaError_t launch_frame(const FrameArgs& a, int wf, int kv_f16, int rows_cta_max, int grid,
-                         cudaStream_t st);
-size_t frame_smem(int mr, int wf, int rows_cta_max);
 }  // namespace m3

@@ -16,7 +16,7 @@
 #include "m3.h"
 #include "launch.cuh"
 #include "misc.cuh"
-#include "frame.cuh"
+#include "gemv_tile.cuh"
 
 using namespace m3;
 typedef __nv_bfloat16 bf16;
@@ -45,9 +45,10 @@ static int fail(int code, const std::string& msg) {
 
 // ------------------------------------------------------------------- state --
 struct DMat {
-  void* w = nullptr;   // [N][K] bf16 or int8
+  void* w = nullptr;   // [N][K] bf16 or int8: row-major, or tiled (gemv_tile.cuh)
   float* s = nullptr;  // int8 scales
   int N = 0, K = 0, wf = WF_BF16;
+  bool tiled = false;  // bf16 and int8-row matrices of the tensor-core GEMV
 };
 
 struct DLayer {
@@ -58,6 +59,10 @@ struct DLayer {
 struct Acts {  // activation buffers of one stack (body or depth)
   bf16 *x = nullptr, *qkv = nullptr, *o = nullptr, *act = nullptr;
 };
+
+// Counter pairs of the dynamically scheduled GEMV: far more than the
+// launches a stream can have in flight (a frame has ~5 per layer).
+constexpr int kTileCtrPairs = 4096;
 
 struct m3_ctx {
   m3_config cfg{};
@@ -117,14 +122,15 @@ struct m3_ctx {
   std::map<std::pair<int, int>, cudaGraphExec_t> graphs;
   std::map<std::pair<int, int>, cudaGraphExec_t> dgraphs;
 
-  // persistent whole-frame kernel (frame.cuh)
-  bool use_frame_kernel = false;  // opt in with M3_FRAME_KERNEL=1
-  bool phases_dirty = true;
-  FramePhase* d_phases = nullptr;
-  int nph = 0;
-  unsigned* d_bar = nullptr;
-  float* fapart = nullptr;
-  unsigned* facnt = nullptr;
+  // tiled GEMV: ring geometry and the launch plan per (N, K, rows, format, epilogue)
+  int tile_sb = 65536, tile_ns = 2;
+  bool tile_dyn = true;  // dynamic unit claiming where it applies
+  std::map<std::tuple<int, int, int, int, int>, TileLaunch> tile_plans;
+  // {claim, done} counter pairs of the dynamically scheduled GEMV, one per
+  // launch in flight: launches take pairs round-robin, the last CTA of a
+  // launch zeroes its pair
+  unsigned* tile_ctrs = nullptr;
+  unsigned tile_ctr_next = 0;
 };
 
 template <typename T>
@@ -218,7 +224,9 @@ extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) 
   if (cudaDeviceGetAttribute(&c->nsm, cudaDevAttrMultiProcessorCount, c->dev) != cudaSuccess)
     return bail(fail(M3_ECUDA, "SM count"));
   if (const char* e = getenv("M3_NO_GRAPH")) c->use_graphs = (e[0] == '0');
-  if (const char* e = getenv("M3_FRAME_KERNEL")) c->use_frame_kernel = (e[0] == '1');
+  if (const char* e = getenv("M3_GEMV_STAGE_KB")) c->tile_sb = atoi(e) * 1024;
+  if (const char* e = getenv("M3_GEMV_STAGES")) c->tile_ns = atoi(e);
+  if (const char* e = getenv("M3_GEMV_DYN")) c->tile_dyn = (e[0] == '1');
   if (cudaStreamCreateWithFlags(&c->st, cudaStreamNonBlocking) != cudaSuccess ||
       cudaEventCreateWithFlags(&c->ev_in, cudaEventDisableTiming) != cudaSuccess ||
       cudaEventCreateWithFlags(&c->ev_out, cudaEventDisableTiming) != cudaSuccess)
@@ -241,6 +249,8 @@ extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) 
       (rc = dzalloc(c, &p, sizeof(unsigned) * 64)) )
     return bail(rc);
   c->scnt = static_cast<unsigned*>(p);
+  if ((rc = dzalloc(c, &p, sizeof(unsigned) * 2 * kTileCtrPairs))) return bail(rc);
+  c->tile_ctrs = static_cast<unsigned*>(p);
   if ((rc = dzalloc(c, &p, sizeof(FrameParams)))) return bail(rc);
   c->fp = static_cast<FrameParams*>(p);
   if ((rc = dzalloc(c, &p, sizeof(int)))) return bail(rc);
@@ -313,16 +323,33 @@ static int put_rows(m3_ctx* c, DMat& M, const void* src, int mem, int rows, int 
   const void* dsrc = nullptr;
   void* owned = nullptr;
   CKR(stage_src(c, src, bytes, mem, &dsrc, &owned));
-  if (M.wf == WF_BF16) {
+  const unsigned tgrid = (unsigned)(c->nsm * 8);
+  if (M.wf == WF_BF16 && M.tiled) {
+    tile_rows_kernel<uint16_t><<<tgrid, 256, 0, c->st>>>(
+        static_cast<const uint16_t*>(dsrc), rows, cols, static_cast<uint8_t*>(M.w), dst_row0,
+        row_step);
+    CK(cudaGetLastError());
+  } else if (M.wf == WF_BF16) {
     CK(cudaMemcpy2DAsync(static_cast<bf16*>(M.w) + (size_t)dst_row0 * cols,
                          sizeof(bf16) * cols * row_step, dsrc, sizeof(bf16) * cols,
                          sizeof(bf16) * cols, rows, cudaMemcpyDeviceToDevice, c->st));
   } else if (M.wf == WF_I8ROW) {
-    quantize_rows_kernel<<<dim3(1, rows), 256, 0, c->st>>>(
-        static_cast<const bf16*>(dsrc), cols, cols,
-        static_cast<int8_t*>(M.w) + (size_t)dst_row0 * cols, (int64_t)cols * row_step,
-        M.s + dst_row0, row_step);
+    // quantise row-major (into a staging buffer when the matrix is tiled)
+    void* q = nullptr;
+    if (M.tiled) CK(cudaMallocAsync(&q, (size_t)rows * cols, c->st));
+    int8_t* qdst = M.tiled ? static_cast<int8_t*>(q) : static_cast<int8_t*>(M.w) + (size_t)dst_row0 * cols;
+    const int64_t q_ld = M.tiled ? cols : (int64_t)cols * row_step;
+    quantize_rows_kernel<<<dim3(1, rows), 256, 0, c->st>>>(static_cast<const bf16*>(dsrc), cols,
+                                                           cols, qdst, q_ld, M.s + dst_row0,
+                                                           row_step);
     CK(cudaGetLastError());
+    if (M.tiled) {
+      tile_rows_kernel<int8_t><<<tgrid, 256, 0, c->st>>>(static_cast<const int8_t*>(q), rows, cols,
+                                                         static_cast<uint8_t*>(M.w), dst_row0,
+                                                         row_step);
+      CK(cudaGetLastError());
+      CK(cudaFreeAsync(q, c->st));
+    }
   } else {
     const int ng = cols / 128;
     const int64_t warps = (int64_t)rows * ng;
@@ -340,8 +367,12 @@ static int alloc_mat(m3_ctx* c, DMat& M, int N, int K, int wf) {
   M.N = N;
   M.K = K;
   M.wf = wf;
+  M.tiled = wf != WF_I8G128;
   const size_t esz = wf == WF_BF16 ? 2 : 1;
-  CKR(dalloc(c, &M.w, esz * (size_t)N * K));
+  // tiled: rows padded to whole 16-row units with zeros
+  const size_t rows = M.tiled ? (size_t)(N + kUnitRows - 1) / kUnitRows * kUnitRows : (size_t)N;
+  CKR(dalloc(c, &M.w, esz * rows * K));
+  if (M.tiled && rows != (size_t)N) CK(cudaMemset(M.w, 0, esz * rows * K));
   if (wf == WF_I8ROW) CKR(dalloc(c, &M.s, sizeof(float) * N));
   if (wf == WF_I8G128) CKR(dalloc(c, &M.s, sizeof(float) * (size_t)N * (K / 128)));
   return M3_OK;
@@ -395,14 +426,12 @@ extern "C" int m3_load_weights(m3_ctx* c, const m3_weight_src* src, int wdtype) 
     CKR(load_layer(c, c->L[l], src->layers[i], src->mem, wf, g.hidden, g.n_q_heads, g.n_kv_heads,
                    g.head_dim, g.ffn));
     c->loaded[l] = 1;
-    c->phases_dirty = true;
   }
   if (src->final_norm) CKR(put_vec(c, &c->final_norm, src->final_norm, g.hidden, src->mem));
   if (src->lm_head) {
     if (!c->lm.w) CKR(alloc_mat(c, c->lm, g.slice_len, g.hidden, wf));
     CKR(put_rows(c, c->lm, src->lm_head, src->mem, g.slice_len, 0, 1));
     c->head_loaded = true;
-    c->phases_dirty = true;
   }
   CK(cudaStreamSynchronize(c->st));  // sources may be freed on return
   return leave(c);
@@ -501,8 +530,19 @@ extern "C" int m3_export_weight(m3_ctx* c, int which, int layer, void* q_host, f
   CK(cudaStreamSynchronize(c->st));
   const size_t esz = M->wf == WF_BF16 ? 2 : 1;
   const size_t rb = esz * M->K;
-  CK(cudaMemcpy2D(q_host, rb, static_cast<const char*>(M->w) + (size_t)row0 * rb, rb * step, rb,
-                  rows, cudaMemcpyDeviceToHost));
+  if (M->tiled) {
+    // whole tiled matrix to the host, then the requested rows back to row-major
+    std::vector<uint8_t> t(esz * (size_t)(M->N + kUnitRows - 1) / kUnitRows * kUnitRows * M->K);
+    CK(cudaMemcpy(t.data(), M->w, t.size(), cudaMemcpyDeviceToHost));
+    uint8_t* q = static_cast<uint8_t*>(q_host);
+    for (int r = 0; r < rows; ++r)
+      for (int k = 0; k < M->K; ++k)
+        memcpy(q + (size_t)r * rb + k * esz,
+               t.data() + tile_byte_offset(row0 + r * step, k, M->K, (int)esz), esz);
+  } else {
+    CK(cudaMemcpy2D(q_host, rb, static_cast<const char*>(M->w) + (size_t)row0 * rb, rb * step, rb,
+                    rows, cudaMemcpyDeviceToHost));
+  }
   if (M->wf != WF_BF16 && s_host) {
     const int ns = M->wf == WF_I8ROW ? 1 : M->K / 128;
     CK(cudaMemcpy2D(s_host, sizeof(float) * ns, M->s + (size_t)row0 * ns,
@@ -630,27 +670,49 @@ static int attn_splits(const m3_ctx* c, int rows, int nb) {
   return s < 1 ? 1 : s;
 }
 
-// A GEMV over all `rows` batch rows, in launches of at most 4 rows.
+// A GEMV over all `rows` batch rows: one launch of the tiled tensor-core
+// kernel, or launches of at most 4 rows of the CUDA-core kernel (int8 with
+// group-128 scales).
 static int gemv_rows(m3_ctx* c, const DMat& M, int epi, int rows, const bf16* x, int ldx,
-                     const bf16* gamma, bf16* out, int ldo, const SampleArgs* smp, bool& pdl) {
-  for (int r0 = 0; r0 < rows; r0 += 4) {
+                     const bf16* gamma, bf16* out, int ldo, const SampleArgs* smp, bool& pdl,
+                     const FrameParams* fp = nullptr, bool cache_plan = true) {
+  const int step = M.tiled ? rows : 4;
+  for (int r0 = 0; r0 < rows; r0 += step) {
     GemvArgs a{};
     a.w = M.w;
     a.scales = M.s;
     a.N = M.N;
     a.K = M.K;
     a.row0 = r0;
-    a.mr = rows - r0 < 4 ? rows - r0 : 4;
+    a.mr = rows - r0 < step ? rows - r0 : step;
     a.x = x + (size_t)r0 * ldx;
     a.ldx = ldx;
     a.gamma = gamma;
     a.eps = c->cfg.rms_eps;
     a.out = out ? out + (size_t)r0 * ldo : nullptr;
     a.ldo = ldo;
-    a.fp = c->fp;
+    a.fp = fp ? fp : c->fp;
     if (smp) a.smp = *smp;
     a.err = c->err;
-    CK(launch_gemv(a, M.wf, epi, c->st, pdl, c->nsm));
+    if (M.tiled) {
+      const auto key = std::make_tuple(M.N, M.K, a.mr, M.wf, epi);
+      auto it = c->tile_plans.find(key);
+      TileLaunch L;
+      if (it != c->tile_plans.end()) {
+        L = it->second;
+      } else {
+        CK(plan_gemv_tile(M.N, M.K, a.mr, M.wf, epi, c->nsm, c->tile_sb, c->tile_ns,
+                          c->tile_dyn && a.ldx % 8 == 0, &L));
+        if (cache_plan) c->tile_plans.emplace(key, L);
+      }
+      if (L.dyn) {
+        a.ctr = c->tile_ctrs + 2 * (c->tile_ctr_next % kTileCtrPairs);
+        ++c->tile_ctr_next;
+      }
+      CK(launch_gemv_tile(a, M.wf, epi, L, c->st, pdl));
+    } else {
+      CK(launch_gemv(a, M.wf, epi, c->st, pdl, c->nsm));
+    }
     pdl = true;
   }
   return M3_OK;
@@ -735,127 +797,6 @@ static int run_graph(m3_ctx* c, std::map<std::pair<int, int>, cudaGraphExec_t>& 
   return M3_OK;
 }
 
-// ------------------------------------------ the persistent frame kernel -----
-// Used for up to 4 rows when every GEMV of the body streams 4096-wide
-// segments (K > 1024) and heads are 128 wide -- the 8B shapes; other shapes
-// take the per-kernel graph above; the frame kernel is opt-in (M3_FRAME_KERNEL=1)
-// until it beats that graph.
-static bool frame_kernel_ok(const m3_ctx* c, int rows) {
-  const m3_config& g = c->cfg;
-  return c->use_frame_kernel && rows <= 4 && g.head_dim == 128 && g.hidden > 1024 &&
-         g.n_q_heads * g.head_dim > 1024 && g.ffn > 1024 && c->nsm <= 1024;
-}
-
-static int frame_rows_cta_max(const m3_ctx* c) {
-  const m3_config& g = c->cfg;
-  const int esz = c->wdtype == M3_W_INT8 ? 1 : 2;
-  const int R = kStageBytes / (4096 * esz);
-  const int Ns[5] = {(g.n_q_heads + 2 * g.n_kv_heads) * g.head_dim, g.hidden, 2 * g.ffn, g.hidden,
-                     g.slice_len};
-  int best = 0;
-  for (int i = 0; i < 5; ++i) {
-    const int unit = i == 2 ? 2 : 1;
-    const int U = Ns[i] / unit;
-    const int per = (U + c->nsm - 1) / c->nsm * unit;
-    const int rm = (per + R - 1) / R * R;
-    best = rm > best ? rm : best;
-  }
-  return best;
-}
-
-static int build_frame_phases(m3_ctx* c) {
-  const m3_config& g = c->cfg;
-  const int H = g.hidden, d = g.head_dim;
-  const int ldqkv = (g.n_q_heads + 2 * g.n_kv_heads) * d;
-  std::vector<FramePhase> ph;
-  auto gemv_phase = [&](int kind, int layer, const DMat& M, const bf16* x, int ldx,
-                        const bf16* gamma, bf16* out, int ldo) {
-    FramePhase p{};
-    p.kind = kind;
-    p.layer = layer;
-    p.w = M.w;
-    p.scales = M.s;
-    p.N = M.N;
-    p.K = M.K;
-    p.x = x;
-    p.ldx = ldx;
-    p.gamma = gamma;
-    p.out = out;
-    p.ldo = ldo;
-    ph.push_back(p);
-  };
-  for (int l = 0; l < g.n_layers; ++l) {
-    const DLayer& L = c->L[l];
-    gemv_phase(PH_QKV, l, L.qkv, c->A.x, H, L.attn_norm, c->A.qkv, ldqkv);
-    FramePhase at{};
-    at.kind = PH_ATT;
-    at.layer = l;
-    at.q_norm = L.q_norm;
-    at.k_norm = L.k_norm;
-    ph.push_back(at);
-    gemv_phase(PH_O, l, L.o, c->A.o, g.n_q_heads * d, nullptr, c->A.x, H);
-    gemv_phase(PH_GU, l, L.gu, c->A.x, H, L.mlp_norm, c->A.act, g.ffn);
-    gemv_phase(PH_D, l, L.d, c->A.act, g.ffn, nullptr, c->A.x, H);
-  }
-  gemv_phase(PH_LM, g.n_layers, c->lm, c->A.x, H, c->final_norm, nullptr, 0);
-  if (!c->d_phases || c->nph != (int)ph.size()) {
-    CKR(dalloc(c, &c->d_phases, sizeof(FramePhase) * ph.size()));
-    CKR(dalloc(c, &c->d_bar, sizeof(unsigned) * ph.size()));
-  }
-  if (!c->fapart) {
-    CKR(dalloc(c, &c->fapart, sizeof(float) * g.max_rows * g.n_q_heads * 16 * (d + 2)));
-    void* p = nullptr;
-    CKR(dzalloc(c, &p, sizeof(unsigned) * g.max_rows * g.n_kv_heads));
-    c->facnt = static_cast<unsigned*>(p);
-  }
-  c->nph = (int)ph.size();
-  CK(cudaMemcpyAsync(c->d_phases, ph.data(), sizeof(FramePhase) * ph.size(),
-                     cudaMemcpyHostToDevice, c->st));
-  CK(cudaStreamSynchronize(c->st));
-  c->phases_dirty = false;
-  return M3_OK;
-}
-
-static int run_frame_kernel(m3_ctx* c, int rows) {
-  const m3_config& g = c->cfg;
-  if (c->phases_dirty) CKR(build_frame_phases(c));
-  FrameArgs a{};
-  a.ph = c->d_phases;
-  a.nph = c->nph;
-  a.mr = rows;
-  a.eps = g.rms_eps;
-  a.fp = c->fp;
-  a.qkv = c->A.qkv;
-  a.ldqkv = (g.n_q_heads + 2 * g.n_kv_heads) * g.head_dim;
-  a.inv_freq = c->inv_freq;
-  a.pages = c->d_pages;
-  a.n_layers = g.n_layers;
-  a.max_pages = c->max_pages;
-  a.page_size = c->bucket;
-  a.Hq = g.n_q_heads;
-  a.Hkv = g.n_kv_heads;
-  int splits = c->nsm / (rows * g.n_kv_heads);
-  a.splits = splits < 1 ? 1 : (splits > 16 ? 16 : splits);
-  a.apart = c->fapart;
-  a.acnt = c->facnt;
-  a.att_out = c->A.o;
-  a.smp.logits = c->logits;
-  a.smp.logits_ld = g.slice_len;
-  a.smp.codes = c->codes;
-  a.smp.code_stride = 1;
-  a.smp.index_base = (unsigned long long)g.slice_start;
-  a.smp.part_z = c->spz;
-  a.smp.part_i = c->spi;
-  a.smp.counter = c->scnt;
-  a.smp.h_out = c->h;
-  a.bar = c->d_bar;
-  a.err = c->err;
-  CK(cudaMemsetAsync(c->d_bar, 0, sizeof(unsigned) * c->nph, c->st));
-  const int wf = c->wdtype == M3_W_INT8 ? WF_I8ROW : WF_BF16;
-  CK(launch_frame(a, wf, c->kv_f16, frame_rows_cta_max(c), c->nsm, c->st));
-  return M3_OK;
-}
-
 extern "C" int m3_decode_frame(m3_ctx* c, int rows, const int32_t* positions, uint64_t seed,
                                uint64_t frame, const void* x_in, float cfg_scale,
                                float temperature, int32_t* codes, void* h_out, float* logits) {
@@ -887,12 +828,8 @@ extern "C" int m3_decode_frame(m3_ctx* c, int rows, const int32_t* positions, ui
   CK(cudaMemcpyAsync(c->A.x, x_in, sizeof(bf16) * rows * g.hidden, cudaMemcpyDeviceToDevice, c->st));
   set_frame_params_kernel<<<1, 32, 0, c->st>>>(c->fp, fp);
   CK(cudaGetLastError());
-  if (frame_kernel_ok(c, rows)) {
-    CKR(run_frame_kernel(c, rows));
-  } else {
-    CKR(run_graph(c, c->graphs, {rows, c->n_buckets},
-                  [&] { return record_frame(c, rows, c->n_buckets); }));
-  }
+  CKR(run_graph(c, c->graphs, {rows, c->n_buckets},
+                [&] { return record_frame(c, rows, c->n_buckets); }));
   CK(cudaMemcpyAsync(codes, c->codes, sizeof(int) * rows, cudaMemcpyDeviceToDevice, c->st));
   if (h_out)
     CK(cudaMemcpyAsync(h_out, c->h, sizeof(bf16) * rows * g.hidden, cudaMemcpyDeviceToDevice, c->st));
@@ -1072,6 +1009,8 @@ extern "C" int m3_sync_status(m3_ctx* c) {
   CK(cudaMemcpy(&e, c->err, sizeof(int), cudaMemcpyDeviceToHost));
   if (e != 0) {
     CK(cudaMemset(c->err, 0, sizeof(int)));
+    // a launch that gave up may have left its claim counters set
+    CK(cudaMemset(c->tile_ctrs, 0, sizeof(unsigned) * 2 * kTileCtrPairs));
     if (e == kErrTimeout) return fail(M3_ETIMEOUT, "a device-side wait gave up");
     return fail(M3_EDEVICE, "a kernel recorded an out-of-range index");
   }
@@ -1142,29 +1081,19 @@ extern "C" int m3_sample_noalloc(m3_ctx* c, int rows, const void* h, uint64_t se
   set_frame_params_kernel<<<1, 32, 0, c->st>>>(dfp, fp);
   CK(cudaGetLastError());
   CK(cudaMemsetAsync(counter, 0, sizeof(unsigned), c->st));  // the ticket starts at zero
-  for (int r0 = 0; r0 < rows; r0 += 4) {
-    GemvArgs a{};
-    a.w = c->lm.w;
-    a.scales = c->lm.s;
-    a.N = c->lm.N;
-    a.K = c->lm.K;
-    a.row0 = r0;
-    a.mr = rows - r0 < 4 ? rows - r0 : 4;
-    a.x = static_cast<const bf16*>(h) + (size_t)r0 * g.hidden;
-    a.ldx = g.hidden;
-    a.gamma = nullptr;  // h is already the final-normed hidden state
-    a.eps = g.rms_eps;
-    a.fp = dfp;
-    a.smp.logits = logits;
-    a.smp.logits_ld = g.slice_len;
-    a.smp.codes = codes;
-    a.smp.code_stride = 1;
-    a.smp.index_base = (unsigned long long)g.slice_start;
-    a.smp.part_z = reinterpret_cast<float*>(scratch + kNoAllocPartZOff);
-    a.smp.part_i = reinterpret_cast<int*>(scratch + kNoAllocPartIOff);
-    a.smp.counter = counter;
-    a.err = c->err;
-    CK(launch_gemv(a, c->lm.wf, EPI_SAMPLE, c->st, false, c->nsm));
-  }
+  SampleArgs sa{};
+  sa.logits = logits;
+  sa.logits_ld = g.slice_len;
+  sa.codes = codes;
+  sa.code_stride = 1;
+  sa.index_base = (unsigned long long)g.slice_start;
+  sa.part_z = reinterpret_cast<float*>(scratch + kNoAllocPartZOff);
+  sa.part_i = reinterpret_cast<int*>(scratch + kNoAllocPartIOff);
+  sa.counter = counter;
+  bool pdl = false;
+  // h is already the final-normed hidden state: no gain; launch plans are
+  // looked up, not cached, so this call allocates nothing on the host either
+  CKR(gemv_rows(c, c->lm, EPI_SAMPLE, rows, static_cast<const bf16*>(h), g.hidden, nullptr,
+                nullptr, 0, &sa, pdl, dfp, false));
   return leave(c);
 }

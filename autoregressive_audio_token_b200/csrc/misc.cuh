@@ -4,6 +4,7 @@
 
 #include "common.cuh"
 #include "gemv.cuh"
+#include "gemv_tile.cuh"
 
 namespace m3 {
 
@@ -87,6 +88,20 @@ __global__ void quantize_g128_kernel(const __nv_bfloat16* __restrict__ w, int64_
       qq = (int8_t)r;
     }
     dst[lane + 32 * i] = qq;
+  }
+}
+
+// Row-major [rows][K] weights (bf16 or int8) -> the tiled layout of
+// gemv_tile.cuh, source row r going to matrix row dst_row0 + r * row_step.
+template <typename T>
+__global__ void tile_rows_kernel(const T* __restrict__ src, int rows, int K, uint8_t* dst,
+                                 int dst_row0, int row_step) {
+  const int64_t total = (int64_t)rows * K;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int r = (int)(i / K), k = (int)(i % K);
+    const int n = dst_row0 + r * row_step;
+    *reinterpret_cast<T*>(dst + tile_byte_offset(n, k, K, (int)sizeof(T))) = src[i];
   }
 }
 

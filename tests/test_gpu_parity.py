@@ -82,6 +82,41 @@ def test_tiny_rows_and_cfg(ora, rows, cfg):
         m.close()
 
 
+@pytest.mark.parametrize("rows,cfg,wdtype", [(9, 0.0, 0), (16, 1.5, 0), (16, 0.0, 1),
+                                              (12, 1.5, 1)])
+def test_tiny_many_rows(ora, rows, cfg, wdtype):
+    # 9..16 activation rows: the MMA's second row half (rows 8..15) in use
+    s = synth.TINY
+    m = Model(s, seed=12, max_rows=16, wdtype=wdtype)
+    try:
+        kc, vc = m.kv_setup(rows=rows, n_prefill=33, max_pos=100)
+        pos = [33 + (r % 5) for r in range(rows)]
+        x = synth.frame_input(s, rows, 12, 0)
+        codes, h, lg = m.decode(pos, seed=8, frame=2, x_in=x, cfg_scale=cfg)
+        oc, oh, olg = m.ora.decode_frame(kc, vc, pos, 8, 2, bits(x), cfg_scale=cfg)
+        assert rel_err(lg, olg) <= TOL[wdtype], rel_err(lg, olg)
+        check_codes_teacher_forced(m, h, codes, 8, 2, cfg_scale=cfg)
+    finally:
+        m.close()
+
+
+def test_tiny_ragged_vocab_slice(ora):
+    # a sampled slice of 500 rows: the last 8-row weight unit is partly padding
+    import dataclasses
+    s = dataclasses.replace(synth.TINY, slice_len=500)
+    m = Model(s, seed=13, max_rows=2)
+    try:
+        kc, vc = m.kv_setup(rows=2, n_prefill=20, max_pos=64)
+        x = synth.frame_input(s, 2, 13, 0)
+        codes, h, lg = m.decode([20, 20], seed=4, frame=1, x_in=x, cfg_scale=1.5)
+        oc, oh, olg = m.ora.decode_frame(kc, vc, [20, 20], 4, 1, bits(x), cfg_scale=1.5)
+        assert lg.shape[-1] == 500
+        assert rel_err(lg, olg) <= TOL[0], rel_err(lg, olg)
+        check_codes_teacher_forced(m, h, codes, 4, 1, cfg_scale=1.5)
+    finally:
+        m.close()
+
+
 @pytest.mark.parametrize("kv_f16", [False, True])
 def test_tiny_long_context_many_tiles(ora, kv_f16):
     # positions up to 700 with bucket 256: several 32-position tiles per warp,
@@ -180,13 +215,16 @@ def test_errors_are_status_codes(ora):
 
 # -------------------------------------------------- one 8B decoder layer ----
 
-@pytest.mark.parametrize("path", ["frame_kernel", "per_kernel"])
+@pytest.mark.parametrize("ring", ["64x2", "8x4"])
 @pytest.mark.parametrize("wdtype,rows,kv_f16", [(0, 1, False), (0, 2, False), (1, 1, False),
                                                 (1, 2, True)])
-def test_layer8b_vs_oracle(ora, wdtype, rows, kv_f16, path, monkeypatch):
-    # the 8B layer shape runs through the per-kernel CUDA graph by default;
-    # M3_FRAME_KERNEL=1 selects the persistent whole-frame kernel
-    monkeypatch.setenv("M3_FRAME_KERNEL", "1" if path == "frame_kernel" else "0")
+def test_layer8b_vs_oracle(ora, wdtype, rows, kv_f16, ring, monkeypatch):
+    # with 64 KB stages a 16-row unit of K = 4096 is one stage and the down
+    # projection (K = 12288) streams each unit in six parts; with 8 KB stages
+    # every GEMV splits its units into many parts
+    kb, ns = ring.split("x")
+    monkeypatch.setenv("M3_GEMV_STAGE_KB", kb)
+    monkeypatch.setenv("M3_GEMV_STAGES", ns)
     s = synth.LAYER8B
     m = Model(s, seed=11, device="cuda", wdtype=wdtype, max_rows=2, kv_f16=kv_f16)
     try:
