@@ -10,6 +10,11 @@ static cudaError_t launch_attn_t(const AttnArgs& a, int splits, int rows, cudaSt
   auto kern = attn_decode_kernel<D, KVF16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  // the whole unified L1 as shared memory, so that the next kernel's CTA
+  // fits beside this one
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
   if (splits < 1 || splits > kAttnMaxSplits) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(splits, a.Hkv, rows);

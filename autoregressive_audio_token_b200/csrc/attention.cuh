@@ -209,14 +209,22 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const Attn
   pdl_wait();  // q, k, v of the new token come from the QKV projection
 
   // ---- new token: q/k RMSNorm + RoPE (lane l holds dims l + 32i) --------
-  auto norm_rope = [&](const __nv_bfloat16* src, const float* gamma, float* dst) {
-    float v[VPL];
+  // every load of the new token is issued before any of them is used
+  const __nv_bfloat16* row_qkv = a.qkv + (size_t)r * a.ldqkv;
+  const __nv_bfloat16* qraw = row_qkv + (size_t)(g * grp + w) * D;
+  const __nv_bfloat16* kraw = row_qkv + (size_t)a.Hq * D + (size_t)g * D;
+  const __nv_bfloat16* vraw = row_qkv + (size_t)(a.Hq + a.Hkv) * D + (size_t)g * D;
+  float qin[VPL], kin[VPL], vin[VPL];  // a warp may hold a query head and the key
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    qin[i] = is_q ? __bfloat162float(qraw[lane + 32 * i]) : 0.0f;
+    kin[i] = is_k ? __bfloat162float(kraw[lane + 32 * i]) : 0.0f;
+    vin[i] = is_k ? __bfloat162float(vraw[lane + 32 * i]) : 0.0f;
+  }
+  auto norm_rope = [&](float* v, const float* gamma, float* dst) {
     float ss = 0.0f;
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      v[i] = __bfloat162float(src[lane + 32 * i]);
-      ss = fmaf(v[i], v[i], ss);
-    }
+    for (int i = 0; i < VPL; ++i) ss = fmaf(v[i], v[i], ss);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const float inv = 1.0f / sqrtf(ss / (float)D + a.eps);
@@ -233,18 +241,15 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const Attn
     for (int i = 0; i < VPL; ++i) dst[lane + 32 * i] = round_bf16(v[i]);
   };
 
-  const __nv_bfloat16* row_qkv = a.qkv + (size_t)r * a.ldqkv;
-  if (is_q) norm_rope(row_qkv + (size_t)(g * grp + w) * D, gq, q_s + w * D);
+  if (is_q) norm_rope(qin, gq, q_s + w * D);
   if (is_k) {
     // the key (and value) of the new token, as they will be stored
-    const __nv_bfloat16* kraw = row_qkv + (size_t)a.Hq * D + (size_t)g * D;
-    const __nv_bfloat16* vraw = row_qkv + (size_t)(a.Hq + a.Hkv) * D + (size_t)g * D;
-    norm_rope(kraw, gk, k_s);
+    norm_rope(kin, gk, k_s);
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       const int dim = lane + 32 * i;
       const uint16_t kb = f32_to_kv<KVF16>(k_s[dim]);
-      const uint16_t vb = f32_to_kv<KVF16>(__bfloat162float(vraw[dim]));
+      const uint16_t vb = f32_to_kv<KVF16>(vin[i]);
       k_s[dim] = kv_to_f32<KVF16>(kb);
       v_s[dim] = kv_to_f32<KVF16>(vb);
       if (sidx == 0) {

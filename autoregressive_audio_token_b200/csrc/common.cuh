@@ -175,6 +175,24 @@ __device__ __forceinline__ void ffma2(uint64_t& acc, uint64_t a, uint64_t b) {
   asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
 }
 
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// (bf16 lo, bf16 hi) packed -> the exact fp32 pair
+__device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t w) {
+  return pack_u32x2(w << 16, w & 0xFFFF0000u);
+}
+
+// fp32 pair -> (bf16 lo, bf16 hi) packed, each rounded to nearest even
+__device__ __forceinline__ uint32_t f32x2_to_bf16x2(uint64_t v) {
+  const float2 f = unpack_f32x2(v);
+  const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
+  return *reinterpret_cast<const uint32_t*>(&b);
+}
+
 __device__ __forceinline__ void fadd2(uint64_t& acc, uint64_t b) {
   asm("add.rn.f32x2 %0, %0, %1;" : "+l"(acc) : "l"(b));
 }

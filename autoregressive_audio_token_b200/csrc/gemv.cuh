@@ -94,6 +94,12 @@ struct GemvArgs {
   // stage bytes, stages; the dynamic kernel's {claim, done} counter pair
   int tc, tsb, tns;
   unsigned* ctr;
+  // RMSNorm partials: a residual-add launch writes sum(x_new^2) per (row m,
+  // 16-row unit u) at ssq_out[m * units + u]; a normalising launch reads
+  // ssq_n such partials per row from ssq_in (either may be null)
+  float* ssq_out;
+  const float* ssq_in;
+  int ssq_n;
 };
 
 template <int TPR, int ESZ>

@@ -56,7 +56,7 @@ __host__ __device__ __forceinline__ size_t dyn_smem_bytes(const DynPlan& d, int 
 }
 
 template <int WF, int EPI>
-__global__ void __launch_bounds__(kDThreads, 1) gemv_dyn_kernel(const GemvArgs a) {
+__global__ void __maxnreg__(128) gemv_dyn_kernel(const GemvArgs a) {
   static_assert(WF == WF_BF16 || WF == WF_I8ROW, "tiled formats: bf16, int8 row scale");
   static_assert(EPI == EPI_STORE || EPI == EPI_RESID || EPI == EPI_SWIGLU, "no sampler here");
   constexpr int ESZ = WF == WF_BF16 ? 2 : 1;
@@ -173,16 +173,31 @@ __global__ void __launch_bounds__(kDThreads, 1) gemv_dyn_kernel(const GemvArgs a
           a.out[(size_t)m * a.ldo + n / 2] = __float2bfloat16_rn(act);
         }
       } else {
-        for (int e = lane; e < WU; e += 32) {
+        // WU = 16 mr is a multiple of 16: each pass covers two rows, one per
+        // half-warp, so the RMSNorm partial of (row, unit) is a 16-lane sum
+        for (int e0 = 0; e0 < WU; e0 += 32) {
+          const int e = e0 + lane;
           const int m = e / kUnitRows, n = u * kUnitRows + e % kUnitRows;
-          float y = 0.0f;
+          float y = 0.0f, o2 = 0.0f;
+          if (e < WU) {
 #pragma unroll
-          for (int w = 0; w < kDW; ++w) y += pb[(size_t)w * WU + e];
-          if (n >= a.N) continue;
-          if constexpr (WF == WF_I8ROW) y = y * rpow[m] * __ldg(a.scales + n);
-          __nv_bfloat16* o = a.out + (size_t)m * a.ldo + n;
-          if constexpr (EPI == EPI_STORE) *o = __float2bfloat16_rn(y);
-          else *o = __float2bfloat16_rn(__bfloat162float(*o) + round_bf16(y));
+            for (int w = 0; w < kDW; ++w) y += pb[(size_t)w * WU + e];
+          }
+          if (e < WU && n < a.N) {
+            if constexpr (WF == WF_I8ROW) y = y * rpow[m] * __ldg(a.scales + n);
+            __nv_bfloat16* o = a.out + (size_t)m * a.ldo + n;
+            __nv_bfloat16 ob;
+            if constexpr (EPI == EPI_STORE) ob = __float2bfloat16_rn(y);
+            else ob = __float2bfloat16_rn(__bfloat162float(*o) + round_bf16(y));
+            *o = ob;
+            const float of = __bfloat162float(ob);
+            o2 = of * of;
+          }
+          if (EPI == EPI_RESID && a.ssq_out) {
+#pragma unroll
+            for (int off = 8; off > 0; off >>= 1) o2 += __shfl_xor_sync(0xffffffffu, o2, off);
+            if ((lane & 15) == 0 && e < WU) a.ssq_out[(size_t)m * U + u] = o2;
+          }
         }
       }
       __syncwarp();
@@ -191,8 +206,12 @@ __global__ void __launch_bounds__(kDThreads, 1) gemv_dyn_kernel(const GemvArgs a
   } else {
     // --------------------------------------------------------- consumers --
     pdl_wait();  // the activations come from the previous kernel
-    stage_activations<WF>(a, mr, 0, T, rinv, rpow, reinterpret_cast<float*>(xs), xs, nullptr, tid,
-                          NT);
+    if (a.gamma)
+      stage_activations<WF, 4, true>(a, mr, 0, T, rinv, rpow, reinterpret_cast<float*>(xs), xs,
+                                     nullptr, tid, NT);
+    else
+      stage_activations<WF, 8, false>(a, mr, 0, T, rinv, rpow, reinterpret_cast<float*>(xs), xs,
+                                      nullptr, tid, NT);
     const int g = lane >> 2, t = lane & 3;
     const uint2* xl = g < mr ? xs + g * 4 + t : zpad;  // B fragment stream of batch row g
     const int xsl = g < mr ? mr * 4 : 0;

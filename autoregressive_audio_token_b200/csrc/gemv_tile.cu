@@ -20,6 +20,11 @@ cudaError_t launch_tile_t(const GemvArgs& a0, const TileLaunch& L, cudaStream_t 
   auto kern = a.mr > 8 ? gemv_tile_kernel<WF, EPI, true> : gemv_tile_kernel<WF, EPI, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.smem);
   if (e != cudaSuccess) return e;
+  // the whole unified L1 as shared memory, so that the next kernel's CTA
+  // fits beside this one
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(L.grid);
   cfg.blockDim = dim3(kTThreads);
@@ -41,6 +46,11 @@ template <int WF, int EPI>
 cudaError_t max_clusters_t(int C, size_t smem, int* n) {
   auto kern = gemv_tile_kernel<WF, EPI, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  // the whole unified L1 as shared memory, so that the next kernel's CTA
+  // fits beside this one
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(C);
@@ -64,6 +74,11 @@ cudaError_t launch_dyn_t(const GemvArgs& a0, const TileLaunch& L, cudaStream_t s
   a.tns = L.ns;
   auto kern = gemv_dyn_kernel<WF, EPI>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.smem);
+  if (e != cudaSuccess) return e;
+  // the whole unified L1 as shared memory, so that the next kernel's CTA
+  // fits beside this one
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   return launch_ex(kern, dim3(L.grid), dim3(kDThreads), L.smem, st, pdl, a);
 }

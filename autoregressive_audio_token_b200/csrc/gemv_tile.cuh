@@ -199,45 +199,45 @@ __device__ __forceinline__ void unpack16(const uint4& lo, const uint4& hi, float
   for (int i = 0; i < 8; ++i) bf16x2_to_f32(w[i], v[2 * i], v[2 * i + 1]);
 }
 
+// Per-row reduction of vals[m * n + j] over j < n (sum or max) by warps in a
+// fixed order (lane-strided, then a shuffle tree); lane 0 of warp m stores
+// f(result).  Deterministic for a given n.
+template <bool MAX, typename F>
+__device__ __forceinline__ void rows_reduce(const float* vals, int n, int mr, int warp, int nwarps,
+                                            int lane, F store) {
+  for (int m = warp; m < mr; m += nwarps) {
+    float s = 0.0f;
+#pragma unroll 8
+    for (int j = lane; j < n; j += 32) s = MAX ? fmaxf(s, vals[m * n + j]) : s + vals[m * n + j];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float y = __shfl_xor_sync(0xffffffffu, s, o);
+      s = MAX ? fmaxf(s, y) : s + y;
+    }
+    if (lane == 0) store(m, s);
+  }
+}
+
 // The consumer threads' setup of one launch (nt threads, named barrier 1):
 // RMSNorm statistics over the whole K (when a.gamma), the int8 scale
 // exponent, and the activations of tiles [kt0, kt0 + Tr) in B-fragment
 // order, xs[j][m][t] = {(k, k+1), (k+8, k+9)} with k = 16 (kt0 + j) + 2t,
-// normalised as out = bf16(gamma * bf16(x / rms)).  Loads go out four items
-// (16 inputs of one row) per thread at a time.  `sq` is scratch of T * mr
-// floats that may alias xs.
-template <int WF>
+// normalised as out = bf16(gamma * bf16(x / rms)).
+// The sum of squares comes from a.ssq_in when the previous kernel left
+// per-unit partials there ([mr][a.ssq_n], summed here in a fixed order),
+// else from a pass over x.  Each thread holds up to NB items (16 inputs of
+// one row) in registers, so with the partials the setup is one round trip
+// to L2.  `sq` is scratch of T * mr floats that may alias xs.
+template <int WF, int NB, bool GAMMA>
 __device__ __forceinline__ void stage_activations(const GemvArgs& a, int mr, int kt0, int Tr,
                                                   float* rinv, float* rpow, float* sq, uint2* xs,
                                                   __nv_bfloat16* h_out, int tid, int nt) {
   const int K = a.K, T = K >> 4;
   const int warp = tid >> 5, lane = tid & 31, nwarps = nt >> 5;
   const __nv_bfloat16* __restrict__ x = a.x;
-  const __nv_bfloat16* __restrict__ gm = a.gamma;
-  // per-row reduction of sq[m * T + j] over j (sum or max), in a fixed order
-  auto row_reduce = [&](bool is_max, float* dst, bool to_pow) {
-    named_bar_sync(1, nt);
-    for (int m = warp; m < mr; m += nwarps) {
-      float s = 0.0f;
-      for (int j = lane; j < T; j += 32) s = is_max ? fmaxf(s, sq[m * T + j]) : s + sq[m * T + j];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float y = __shfl_xor_sync(0xffffffffu, s, o);
-        s = is_max ? fmaxf(s, y) : s + y;
-      }
-      if (lane == 0) {
-        if (!to_pow) {
-          dst[m] = 1.0f / sqrtf(s / (float)K + a.eps);
-        } else {
-          int e = 0;  // largest magnitude below 2^15 after scaling by 2^-e
-          if (s >= 32768.0f) e = ilogbf(s) - 14;
-          dst[m] = ldexpf(1.0f, e);
-        }
-      }
-    }
-    named_bar_sync(1, nt);
-  };
-  // normalised inputs 16 j .. 16 j + 15 of row m from raw loads
+  const __nv_bfloat16* __restrict__ gm = GAMMA ? a.gamma : nullptr;
+  const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+  auto set_rinv = [&](int m, float s) { rinv[m] = 1.0f / sqrtf(s / (float)K + a.eps); };
   auto normalise = [&](int m, const uint4& xl, const uint4& xh, const uint4& gl, const uint4& gh,
                        float* v) {
     unpack16(xl, xh, v);
@@ -249,18 +249,18 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, int mr, int
       for (int i = 0; i < 16; ++i) v[i] = round_bf16(g[i] * round_bf16(v[i] * r));
     }
   };
-  const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-  if (gm) {  // sum of squares per (row, 16 inputs)
-    for (int i0 = tid; i0 < T * mr; i0 += 4 * nt) {
-      uint4 xl[4], xh[4];
+  const bool have_ss = gm && a.ssq_in;
+  if (gm && !have_ss) {  // sum of squares per (row, 16 inputs), then per row
+    for (int i0 = tid; i0 < T * mr; i0 += NB * nt) {
+      uint4 xl[NB], xh[NB];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < NB; ++q) {
         const int i = i0 + q * nt;
         xl[q] = xh[q] = z4;
         if (i < T * mr) load16(x + (size_t)(i / T) * a.ldx + 16 * (i % T), xl[q], xh[q]);
       }
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < NB; ++q) {
         const int i = i0 + q * nt;
         if (i >= T * mr) continue;
         float v[16];
@@ -271,13 +271,19 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, int mr, int
         sq[i] = s;
       }
     }
-    row_reduce(false, rinv, false);
+    named_bar_sync(1, nt);
+    rows_reduce<false>(sq, T, mr, warp, nwarps, lane, set_rinv);
+    named_bar_sync(1, nt);
   }
   if constexpr (WF == WF_I8ROW) {  // largest normalised magnitude per row
-    for (int i0 = tid; i0 < T * mr; i0 += 4 * nt) {
-      uint4 xl[4], xh[4], gl[4], gh[4];
+    if (have_ss) {
+      rows_reduce<false>(a.ssq_in, a.ssq_n, mr, warp, nwarps, lane, set_rinv);
+      named_bar_sync(1, nt);
+    }
+    for (int i0 = tid; i0 < T * mr; i0 += NB * nt) {
+      uint4 xl[NB], xh[NB], gl[NB], gh[NB];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < NB; ++q) {
         const int i = i0 + q * nt;
         xl[q] = xh[q] = gl[q] = gh[q] = z4;
         if (i < T * mr) {
@@ -286,7 +292,7 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, int mr, int
         }
       }
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < NB; ++q) {
         const int i = i0 + q * nt;
         if (i >= T * mr) continue;
         float v[16];
@@ -297,48 +303,89 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, int mr, int
         sq[i] = mx;
       }
     }
-    row_reduce(true, rpow, true);
+    named_bar_sync(1, nt);
+    rows_reduce<true>(sq, T, mr, warp, nwarps, lane, [&](int m, float s) {
+      int e = 0;  // largest magnitude below 2^15 after scaling by 2^-e
+      if (s >= 32768.0f) e = ilogbf(s) - 14;
+      rpow[m] = ldexpf(1.0f, e);
+    });
+    named_bar_sync(1, nt);
   }
-  // the slice in B-fragment order
-  for (int i0 = tid; i0 < Tr * mr; i0 += 4 * nt) {
-    uint4 xl[4], xh[4], gl[4], gh[4];
+  // the slice in B-fragment order, NB items per thread per batch; item i is
+  // (tile jj = i / mr, row m = i % mr), so a warp's stores are 32-byte
+  // steps and its loads 32-byte sectors
+  uint4 xl[NB], xh[NB], gl[NB], gh[NB];
+  auto load_batch = [&](int i0) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < NB; ++q) {
       const int i = i0 + q * nt;
       xl[q] = xh[q] = gl[q] = gh[q] = z4;
       if (i < Tr * mr) {
-        const int m = i / Tr, j = kt0 + i % Tr;
+        const int m = i % mr, j = kt0 + i / mr;
         load16(x + (size_t)m * a.ldx + 16 * j, xl[q], xh[q]);
         if (gm) load16(gm + 16 * j, gl[q], gh[q]);
       }
     }
+  };
+  auto store_batch = [&](int i0) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < NB; ++q) {
       const int i = i0 + q * nt;
       if (i >= Tr * mr) continue;
-      const int m = i / Tr, jj = i % Tr;
-      float v[16];
-      normalise(m, xl[q], xh[q], gl[q], gh[q], v);
-      if (h_out) {
-        __nv_bfloat16* h = h_out + (size_t)m * K + 16 * (kt0 + jj);
+      const int m = i % mr, jj = i / mr;
+      // w[p] = inputs (2p, 2p+1) of the item, p < 8
+      uint32_t w[8] = {xl[q].x, xl[q].y, xl[q].z, xl[q].w, xh[q].x, xh[q].y, xh[q].z, xh[q].w};
+      if constexpr (WF == WF_BF16) {
+        if (gm) {
+          const uint32_t gw[8] = {gl[q].x, gl[q].y, gl[q].z, gl[q].w,
+                                  gh[q].x, gh[q].y, gh[q].z, gh[q].w};
+          const uint64_t r2 = pack_f32x2(rinv[m], rinv[m]);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) h[e] = __float2bfloat16_rn(v[e]);
-      }
-      float sc = 1.0f;
-      if constexpr (WF == WF_I8ROW) sc = 1.0f / rpow[m];  // a power of two: exact
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        uint2 f;
-        if constexpr (WF == WF_I8ROW) {
-          f.x = pack_f16x2(v[2 * t] * sc, v[2 * t + 1] * sc);
-          f.y = pack_f16x2(v[2 * t + 8] * sc, v[2 * t + 9] * sc);
-        } else {
-          f.x = pack_bf16x2(v[2 * t], v[2 * t + 1]);
-          f.y = pack_bf16x2(v[2 * t + 8], v[2 * t + 9]);
+          for (int p = 0; p < 8; ++p) {
+            const uint32_t t1 = f32x2_to_bf16x2(fmul2(bf16x2_to_f32x2(w[p]), r2));
+            w[p] = f32x2_to_bf16x2(fmul2(bf16x2_to_f32x2(gw[p]), bf16x2_to_f32x2(t1)));
+          }
         }
-        xs[((size_t)jj * mr + m) * 4 + t] = f;
+        if (h_out) {
+          uint4* h = reinterpret_cast<uint4*>(h_out + (size_t)m * K + 16 * (kt0 + jj));
+          h[0] = make_uint4(w[0], w[1], w[2], w[3]);
+          h[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(xs + ((size_t)jj * mr + m) * 4);
+        dst[0] = make_uint4(w[0], w[4], w[1], w[5]);
+        dst[1] = make_uint4(w[2], w[6], w[3], w[7]);
+      } else {
+        float v[16];
+        normalise(m, xl[q], xh[q], gl[q], gh[q], v);
+        if (h_out) {
+          __nv_bfloat16* h = h_out + (size_t)m * K + 16 * (kt0 + jj);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) h[e] = __float2bfloat16_rn(v[e]);
+        }
+        const float sc = 1.0f / rpow[m];  // a power of two: exact
+        uint32_t f[8];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          f[2 * t] = pack_f16x2(v[2 * t] * sc, v[2 * t + 1] * sc);
+          f[2 * t + 1] = pack_f16x2(v[2 * t + 8] * sc, v[2 * t + 9] * sc);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(xs + ((size_t)jj * mr + m) * 4);
+        dst[0] = make_uint4(f[0], f[1], f[2], f[3]);
+        dst[1] = make_uint4(f[4], f[5], f[6], f[7]);
       }
     }
+  };
+  load_batch(tid);
+  if (WF != WF_I8ROW && have_ss) {
+    // the row statistics from the previous kernel's partials, while this
+    // thread's first loads are in flight
+    rows_reduce<false>(a.ssq_in, a.ssq_n, mr, warp, nwarps, lane, set_rinv);
+    named_bar_sync(1, nt);
+  }
+  store_batch(tid);
+  for (int i0 = tid + NB * nt; i0 < Tr * mr; i0 += NB * nt) {
+    load_batch(i0);
+    store_batch(i0);
   }
   named_bar_sync(1, nt);
 }
@@ -414,8 +461,12 @@ __global__ void __launch_bounds__(kTThreads, 1) gemv_tile_kernel(const GemvArgs 
     pdl_wait();  // the activations come from the previous kernel
     __nv_bfloat16* h_out =
         (EPI == EPI_SAMPLE && a.smp.h_out && cl == 0) ? a.smp.h_out + (size_t)a.row0 * a.K : nullptr;
-    stage_activations<WF>(a, mr, kt0, P.Tr, rinv, rpow, reinterpret_cast<float*>(xs), xs, h_out,
-                          tid, NT);
+    if (a.gamma)
+      stage_activations<WF, 4, true>(a, mr, kt0, P.Tr, rinv, rpow, reinterpret_cast<float*>(xs),
+                                     xs, h_out, tid, NT);
+    else
+      stage_activations<WF, 8, false>(a, mr, kt0, P.Tr, rinv, rpow, reinterpret_cast<float*>(xs),
+                                      xs, h_out, tid, NT);
 
     const int g = lane >> 2, t = lane & 3;
     // this lane's B-fragment streams: batch rows g and g + 8, or the zero pad

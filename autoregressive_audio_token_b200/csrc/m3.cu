@@ -131,6 +131,14 @@ struct m3_ctx {
   // launch zeroes its pair
   unsigned* tile_ctrs = nullptr;
   unsigned tile_ctr_next = 0;
+  // RMSNorm partials of the residual stream between a residual-add launch
+  // and the normalising launch after it (recording a frame only): two
+  // [max_rows][units] buffers used alternately; ssq_cur is the one that
+  // holds the current stream's partials, or null
+  float* ssq_buf[2] = {nullptr, nullptr};
+  float* ssq_cur = nullptr;
+  int ssq_n = 0;
+  bool ssq_track = false;
 };
 
 template <typename T>
@@ -251,6 +259,9 @@ extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) 
   c->scnt = static_cast<unsigned*>(p);
   if ((rc = dzalloc(c, &p, sizeof(unsigned) * 2 * kTileCtrPairs))) return bail(rc);
   c->tile_ctrs = static_cast<unsigned*>(p);
+  for (int i = 0; i < 2; ++i)
+    if ((rc = dalloc(c, &c->ssq_buf[i], sizeof(float) * R * ((g.hidden + kUnitRows - 1) / kUnitRows))))
+      return bail(rc);
   if ((rc = dzalloc(c, &p, sizeof(FrameParams)))) return bail(rc);
   c->fp = static_cast<FrameParams*>(p);
   if ((rc = dzalloc(c, &p, sizeof(int)))) return bail(rc);
@@ -709,7 +720,22 @@ static int gemv_rows(m3_ctx* c, const DMat& M, int epi, int rows, const bf16* x,
         a.ctr = c->tile_ctrs + 2 * (c->tile_ctr_next % kTileCtrPairs);
         ++c->tile_ctr_next;
       }
+      float* ssq_written = nullptr;
+      if (c->ssq_track) {
+        if (gamma && c->ssq_cur) {
+          a.ssq_in = c->ssq_cur;
+          a.ssq_n = c->ssq_n;
+        }
+        if (epi == EPI_RESID && L.dyn && M.N == c->cfg.hidden) {
+          ssq_written = c->ssq_cur == c->ssq_buf[0] ? c->ssq_buf[1] : c->ssq_buf[0];
+          a.ssq_out = ssq_written;
+        }
+      }
       CK(launch_gemv_tile(a, M.wf, epi, L, c->st, pdl));
+      if (epi == EPI_RESID) {
+        c->ssq_cur = ssq_written;  // a residual add without partials invalidates them
+        c->ssq_n = (M.N + kUnitRows - 1) / kUnitRows;
+      }
     } else {
       CK(launch_gemv(a, M.wf, epi, c->st, pdl, c->nsm));
     }
@@ -753,6 +779,16 @@ static int record_frame(m3_ctx* c, int rows, int nb) {
   const m3_config& g = c->cfg;
   const int splits = attn_splits(c, rows, nb);
   bool pdl = false;  // the first kernel follows the parameter block in plain stream order
+  // the frame's input was copied in: no partials for the first norm
+  c->ssq_cur = nullptr;
+  c->ssq_track = true;
+  struct Untrack {
+    m3_ctx* c;
+    ~Untrack() {
+      c->ssq_track = false;
+      c->ssq_cur = nullptr;
+    }
+  } untrack{c};
   for (int l = 0; l < g.n_layers; ++l)
     CKR(record_layer(c, c->L[l], c->A, rows, g.hidden, g.n_q_heads, g.n_kv_heads, g.head_dim,
                      g.ffn, c->d_pages, l, g.n_layers, c->max_pages, c->bucket, c->kv_f16, splits,
