@@ -49,6 +49,7 @@ struct AttnArgs {
   const __nv_bfloat16* k_norm;  // [D]
   float eps;
   const double* inv_freq;     // [D/2] theta^(-2i/D)
+  const float2* rope;         // nullable: this frame's (cos, sin) [rows][D/2]
   const unsigned long long* pages;  // [rows][n_layers][max_pages] page base addresses
   int layer, n_layers, max_pages, page_size;
   int Hq, Hkv;
@@ -201,9 +202,15 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const Attn
   if (is_q || is_k) {
 #pragma unroll
     for (int i = 0; i < VPL / 2; ++i) {
-      const double ang = (double)pos * a.inv_freq[lane + 32 * i];
-      rc[i] = (float)cos(ang);
-      rs[i] = (float)sin(ang);
+      if (a.rope) {
+        const float2 cs = a.rope[(size_t)r * (D / 2) + lane + 32 * i];
+        rc[i] = cs.x;
+        rs[i] = cs.y;
+      } else {
+        const double ang = (double)pos * a.inv_freq[lane + 32 * i];
+        rc[i] = (float)cos(ang);
+        rs[i] = (float)sin(ang);
+      }
     }
   }
   pdl_wait();  // q, k, v of the new token come from the QKV projection

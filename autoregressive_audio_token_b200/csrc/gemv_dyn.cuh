@@ -205,7 +205,6 @@ __global__ void __maxnreg__(128) gemv_dyn_kernel(const GemvArgs a) {
     }
   } else {
     // --------------------------------------------------------- consumers --
-    pdl_wait();  // the activations come from the previous kernel
     if (a.gamma)
       stage_activations<WF, 4, true>(a, mr, 0, T, rinv, rpow, reinterpret_cast<float*>(xs), xs,
                                      nullptr, tid, NT);

@@ -218,7 +218,8 @@ __device__ __forceinline__ void rows_reduce(const float* vals, int n, int mr, in
   }
 }
 
-// The consumer threads' setup of one launch (nt threads, named barrier 1):
+// The consumer threads' setup of one launch (nt threads, named barrier 1),
+// which also waits for the previous kernel (after fetching static gains):
 // RMSNorm statistics over the whole K (when a.gamma), the int8 scale
 // exponent, and the activations of tiles [kt0, kt0 + Tr) in B-fragment
 // order, xs[j][m][t] = {(k, k+1), (k+8, k+9)} with k = 16 (kt0 + j) + 2t,
@@ -249,6 +250,19 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, int mr, int
       for (int i = 0; i < 16; ++i) v[i] = round_bf16(g[i] * round_bf16(v[i] * r));
     }
   };
+  // the gains are static: their first batch is fetched (from HBM, the
+  // slowest load here) before waiting for the previous kernel
+  uint4 xl[NB], xh[NB], gl[NB], gh[NB];
+  auto load_gamma = [&](int i0) {
+#pragma unroll
+    for (int q = 0; q < NB; ++q) {
+      const int i = i0 + q * nt;
+      gl[q] = gh[q] = z4;
+      if (gm && i < Tr * mr) load16(gm + 16 * (kt0 + i / mr), gl[q], gh[q]);
+    }
+  };
+  load_gamma(tid);
+  pdl_wait();  // the activations come from the previous kernel
   const bool have_ss = gm && a.ssq_in;
   if (gm && !have_ss) {  // sum of squares per (row, 16 inputs), then per row
     for (int i0 = tid; i0 < T * mr; i0 += NB * nt) {
@@ -314,17 +328,12 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, int mr, int
   // the slice in B-fragment order, NB items per thread per batch; item i is
   // (tile jj = i / mr, row m = i % mr), so a warp's stores are 32-byte
   // steps and its loads 32-byte sectors
-  uint4 xl[NB], xh[NB], gl[NB], gh[NB];
-  auto load_batch = [&](int i0) {
+  auto load_x = [&](int i0) {
 #pragma unroll
     for (int q = 0; q < NB; ++q) {
       const int i = i0 + q * nt;
-      xl[q] = xh[q] = gl[q] = gh[q] = z4;
-      if (i < Tr * mr) {
-        const int m = i % mr, j = kt0 + i / mr;
-        load16(x + (size_t)m * a.ldx + 16 * j, xl[q], xh[q]);
-        if (gm) load16(gm + 16 * j, gl[q], gh[q]);
-      }
+      xl[q] = xh[q] = z4;
+      if (i < Tr * mr) load16(x + (size_t)(i % mr) * a.ldx + 16 * (kt0 + i / mr), xl[q], xh[q]);
     }
   };
   auto store_batch = [&](int i0) {
@@ -375,16 +384,39 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, int mr, int
       }
     }
   };
-  load_batch(tid);
+  load_x(tid);
   if (WF != WF_I8ROW && have_ss) {
-    // the row statistics from the previous kernel's partials, while this
-    // thread's first loads are in flight
-    rows_reduce<false>(a.ssq_in, a.ssq_n, mr, warp, nwarps, lane, set_rinv);
+    // the row statistics from the previous kernel's partials, loaded while
+    // this thread's first activations are in flight: one partial per thread
+    // and row, a shuffle tree per warp, the warps in order
+    const int n = a.ssq_n;
+    if (mr <= 4 && n <= nt) {
+      float v[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) v[m] = (m < mr && tid < n) ? a.ssq_in[m * n + tid] : 0.0f;
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v[m] += __shfl_xor_sync(0xffffffffu, v[m], o);
+      if (lane == 0)
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+          if (m < mr) sq[warp * 16 + m] = v[m];
+      named_bar_sync(1, nt);
+      if (tid < mr) {
+        float t = 0.0f;
+        for (int w = 0; w < nwarps; ++w) t += sq[w * 16 + tid];
+        set_rinv(tid, t);
+      }
+    } else {
+      rows_reduce<false>(a.ssq_in, n, mr, warp, nwarps, lane, set_rinv);
+    }
     named_bar_sync(1, nt);
   }
   store_batch(tid);
   for (int i0 = tid + NB * nt; i0 < Tr * mr; i0 += NB * nt) {
-    load_batch(i0);
+    load_gamma(i0);
+    load_x(i0);
     store_batch(i0);
   }
   named_bar_sync(1, nt);
@@ -458,7 +490,6 @@ __global__ void __launch_bounds__(kTThreads, 1) gemv_tile_kernel(const GemvArgs 
     }
   } else {
     // --------------------------------------------------------- consumers --
-    pdl_wait();  // the activations come from the previous kernel
     __nv_bfloat16* h_out =
         (EPI == EPI_SAMPLE && a.smp.h_out && cl == 0) ? a.smp.h_out + (size_t)a.row0 * a.K : nullptr;
     if (a.gamma)

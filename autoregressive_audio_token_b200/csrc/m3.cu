@@ -139,6 +139,7 @@ struct m3_ctx {
   float* ssq_cur = nullptr;
   int ssq_n = 0;
   bool ssq_track = false;
+  float2* rope = nullptr;  // this frame's RoPE (cos, sin) [max_rows][head_dim / 2]
 };
 
 template <typename T>
@@ -262,6 +263,7 @@ extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) 
   for (int i = 0; i < 2; ++i)
     if ((rc = dalloc(c, &c->ssq_buf[i], sizeof(float) * R * ((g.hidden + kUnitRows - 1) / kUnitRows))))
       return bail(rc);
+  if ((rc = dalloc(c, &c->rope, sizeof(float2) * R * (g.head_dim / 2)))) return bail(rc);
   if ((rc = dzalloc(c, &p, sizeof(FrameParams)))) return bail(rc);
   c->fp = static_cast<FrameParams*>(p);
   if ((rc = dzalloc(c, &p, sizeof(int)))) return bail(rc);
@@ -747,7 +749,7 @@ static int gemv_rows(m3_ctx* c, const DMat& M, int epi, int rows, const bf16* x,
 static int record_layer(m3_ctx* c, const DLayer& L, Acts& A, int rows, int H, int Hq, int Hkv,
                         int d, int ffn, const unsigned long long* pages, int layer, int n_layers,
                         int max_pages, int page_size, int kv_f16, int splits, int fixed_pos,
-                        const double* inv_freq, bool& pdl) {
+                        const double* inv_freq, const float2* rope, bool& pdl) {
   const int ldqkv = (Hq + 2 * Hkv) * d;
   CKR(gemv_rows(c, L.qkv, EPI_STORE, rows, A.x, H, L.attn_norm, A.qkv, ldqkv, nullptr, pdl));
   AttnArgs at{};
@@ -757,6 +759,7 @@ static int record_layer(m3_ctx* c, const DLayer& L, Acts& A, int rows, int H, in
   at.k_norm = L.k_norm;
   at.eps = c->cfg.rms_eps;
   at.inv_freq = inv_freq;
+  at.rope = rope;
   at.pages = pages;
   at.layer = layer;
   at.n_layers = n_layers;
@@ -792,7 +795,7 @@ static int record_frame(m3_ctx* c, int rows, int nb) {
   for (int l = 0; l < g.n_layers; ++l)
     CKR(record_layer(c, c->L[l], c->A, rows, g.hidden, g.n_q_heads, g.n_kv_heads, g.head_dim,
                      g.ffn, c->d_pages, l, g.n_layers, c->max_pages, c->bucket, c->kv_f16, splits,
-                     -1, c->inv_freq, pdl));
+                     -1, c->inv_freq, c->rope, pdl));
   SampleArgs sa{};
   sa.logits = c->logits;
   sa.logits_ld = g.slice_len;
@@ -864,6 +867,8 @@ extern "C" int m3_decode_frame(m3_ctx* c, int rows, const int32_t* positions, ui
   CK(cudaMemcpyAsync(c->A.x, x_in, sizeof(bf16) * rows * g.hidden, cudaMemcpyDeviceToDevice, c->st));
   set_frame_params_kernel<<<1, 32, 0, c->st>>>(c->fp, fp);
   CK(cudaGetLastError());
+  rope_table_kernel<<<rows, 64, 0, c->st>>>(fp, c->inv_freq, g.head_dim / 2, c->rope);
+  CK(cudaGetLastError());
   CKR(run_graph(c, c->graphs, {rows, c->n_buckets},
                 [&] { return record_frame(c, rows, c->n_buckets); }));
   CK(cudaMemcpyAsync(codes, c->codes, sizeof(int) * rows, cudaMemcpyDeviceToDevice, c->st));
@@ -889,7 +894,7 @@ static int record_depth(m3_ctx* c, int rows, bool forced) {
     for (int l = 0; l < g.depth_layers; ++l)
       CKR(record_layer(c, c->DL[l], c->DA, rows, Dh, g.depth_heads, g.depth_heads,
                        g.depth_head_dim, g.depth_ffn, c->d_dpages, l, g.depth_layers, 1, 32, 0, 1,
-                       j, c->dinv_freq, pdl));
+                       j, c->dinv_freq, nullptr, pdl));
     if (j >= 1) {
       SampleArgs sa{};
       sa.logits = c->dlogits + (size_t)(j - 1) * V;

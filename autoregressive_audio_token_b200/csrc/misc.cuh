@@ -15,6 +15,18 @@ __global__ void set_frame_params_kernel(FrameParams* dst, FrameParams v) {
   if (threadIdx.x == 0) *dst = v;
 }
 
+// The frame's RoPE rotations, (cos, sin) of pos[r] * inv_freq[i] (fp64,
+// then fp32), for rows r < v.rows and i < half: one table per frame instead
+// of the trigonometry in every attention CTA of every layer.
+__global__ void rope_table_kernel(FrameParams v, const double* __restrict__ inv_freq, int half,
+                                  float2* table) {
+  const int r = blockIdx.x;
+  for (int i = threadIdx.x; i < half; i += blockDim.x) {
+    const double ang = (double)v.pos[r] * inv_freq[i];
+    table[(size_t)r * half + i] = make_float2((float)cos(ang), (float)sin(ang));
+  }
+}
+
 // int8 weight-only quantisation ("MiniMax Music 3 on Metal", section
 // "Precision": one scale per row for the body and lm_head, per group of 128
 // for the depth decoder, quantised on the GPU at load):
