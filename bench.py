@@ -314,7 +314,7 @@ def run_ours(args, rank, world, local):
     try:
         prof = json.load(open(os.path.join(ROOT, "profiles", "gemv_traffic.json")))
         src_hash = prof.get("source_sha256")
-        if src_hash == kernel_source_hash():
+        if src_hash == kernel_source_hash() and args.wdtype == "bf16":
             traffic = prof.get("gate_up_swiglu_bytes_per_launch")
     except Exception:
         pass
@@ -344,7 +344,8 @@ def run_ours(args, rank, world, local):
         "frame": {"algorithmic_bytes": frame_bytes, "achieved_gbs": frame_bytes / ms_per_step / 1e6,
                   "frac_of_measured_hbm": frame_bytes / ms_per_step / 1e6 / hbm_peak,
                   "frac_of_8tbs": frame_bytes / ms_per_step / 1e6 / 8000.0},
-        "roofline": {"bound": "hbm", "kernel": "gemv gate/up + SwiGLU (bf16, 2 rows)",
+        "roofline": {"bound": "hbm",
+                     "kernel": f"gemv_dyn_kernel gate/up + SwiGLU ({args.wdtype}, {ROWS} rows)",
                      "achieved": dom["gbs"], "peak": hbm_peak, "unit": "GB/s",
                      "frac": dom["gbs"] / hbm_peak, "peak_source": peak_src,
                      "traffic": traffic, "algorithmic_bytes_per_launch": dom["bytes"]},
