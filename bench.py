@@ -355,12 +355,12 @@ def run_ours(args, rank, world, local):
                 "d2h_bytes_per_step": 4 * ROWS},
         "clocks": clk,
     }
-    # kernels per frame: 5 per layer (qkv, attention, o, gate/up, down) + lm_head + params
-    # per frame: parameter block + 5 kernels per layer + lm_head sampler; the
-    # depth decoder adds its parameter block, projection, 7 embeddings,
-    # 8 positions x layers x 5 kernels and 7 heads
+    # per frame: parameter block + RoPE table + 5 kernels per layer (qkv,
+    # attention, o, gate/up, down) + lm_head sampler; the depth decoder adds
+    # its parameter block, projection, 7 embeddings, 8 positions x layers x 5
+    # kernels and 7 heads
     depth_launches = (2 + 7 + 8 * synth.DEPTH.n_layers * 5 + 7) if args.depth else 0
-    out["gpu_launches"] = (5 * s.n_layers + 1 + 1 + depth_launches) * args.steps
+    out["gpu_launches"] = (5 * s.n_layers + 1 + 2 + depth_launches) * args.steps
     m3.m3_destroy(ctx)
     del xs
     torch.cuda.empty_cache()
