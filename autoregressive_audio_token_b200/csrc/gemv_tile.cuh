@@ -264,6 +264,10 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, int mr, int
   load_gamma(tid);
   pdl_wait();  // the activations come from the previous kernel
   const bool have_ss = gm && a.ssq_in;
+  // int8 with the whole K in one batch per thread: the row maxima come from
+  // the normalised values held in registers (no extra pass over x)
+  const bool fast8 = (WF == WF_I8ROW) && Tr == T && Tr * mr <= NB * nt;
+  if (fast8 && tid < 16) rpow[tid] = 0.0f;  // row maxima (as bits) until the scale
   if (gm && !have_ss) {  // sum of squares per (row, 16 inputs), then per row
     for (int i0 = tid; i0 < T * mr; i0 += NB * nt) {
       uint4 xl[NB], xh[NB];
@@ -289,7 +293,7 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, int mr, int
     rows_reduce<false>(sq, T, mr, warp, nwarps, lane, set_rinv);
     named_bar_sync(1, nt);
   }
-  if constexpr (WF == WF_I8ROW) {  // largest normalised magnitude per row
+  if (WF == WF_I8ROW && !fast8) {  // largest normalised magnitude per row
     if (have_ss) {
       rows_reduce<false>(a.ssq_in, a.ssq_n, mr, warp, nwarps, lane, set_rinv);
       named_bar_sync(1, nt);
@@ -385,7 +389,7 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, int mr, int
     }
   };
   load_x(tid);
-  if (WF != WF_I8ROW && have_ss) {
+  if ((WF != WF_I8ROW || fast8) && have_ss) {
     // the row statistics from the previous kernel's partials, loaded while
     // this thread's first activations are in flight: one partial per thread
     // and row, a shuffle tree per warp, the warps in order
@@ -413,7 +417,65 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, int mr, int
     }
     named_bar_sync(1, nt);
   }
-  store_batch(tid);
+  if (fast8) {
+    named_bar_sync(1, nt);  // the maxima are zero
+    // normalised bf16 words of the thread's items, their row maxima
+    uint32_t ww[NB][8];
+#pragma unroll
+    for (int q = 0; q < NB; ++q) {
+      const int i = tid + q * nt;
+      const uint32_t wx[8] = {xl[q].x, xl[q].y, xl[q].z, xl[q].w, xh[q].x, xh[q].y, xh[q].z, xh[q].w};
+      const uint32_t gw[8] = {gl[q].x, gl[q].y, gl[q].z, gl[q].w, gh[q].x, gh[q].y, gh[q].z, gh[q].w};
+      const int m = i % mr;
+      const uint64_t r2 = gm ? pack_f32x2(rinv[m], rinv[m]) : 0ull;
+      uint32_t mx = 0u;
+#pragma unroll
+      for (int p = 0; p < 8; ++p) {
+        uint32_t w = wx[p];
+        if (gm) {
+          const uint32_t t1 = f32x2_to_bf16x2(fmul2(bf16x2_to_f32x2(w), r2));
+          w = f32x2_to_bf16x2(fmul2(bf16x2_to_f32x2(gw[p]), bf16x2_to_f32x2(t1)));
+        }
+        ww[q][p] = w;
+        // |bf16| bits as fp32 bits order like the magnitudes
+        mx = max(mx, max((w << 16) & 0x7FFFFFFFu, w & 0x7FFF0000u));
+      }
+      if (i < Tr * mr) atomicMax(reinterpret_cast<unsigned*>(rpow) + m, mx);
+    }
+    named_bar_sync(1, nt);
+    if (tid < mr) {
+      const float mxf = __uint_as_float(reinterpret_cast<unsigned*>(rpow)[tid]);
+      int e = 0;  // largest magnitude below 2^15 after scaling by 2^-e
+      if (mxf >= 32768.0f) e = ilogbf(mxf) - 14;
+      rpow[tid] = ldexpf(1.0f, e);
+    }
+    named_bar_sync(1, nt);
+#pragma unroll
+    for (int q = 0; q < NB; ++q) {
+      const int i = tid + q * nt;
+      if (i >= Tr * mr) continue;
+      const int m = i % mr, jj = i / mr;
+      if (h_out) {
+        uint4* h = reinterpret_cast<uint4*>(h_out + (size_t)m * K + 16 * (kt0 + jj));
+        h[0] = make_uint4(ww[q][0], ww[q][1], ww[q][2], ww[q][3]);
+        h[1] = make_uint4(ww[q][4], ww[q][5], ww[q][6], ww[q][7]);
+      }
+      const float sc = 1.0f / rpow[m];  // a power of two: exact
+      const uint64_t s2 = pack_f32x2(sc, sc);
+      uint32_t f[8];
+#pragma unroll
+      for (int p = 0; p < 8; ++p) {
+        const float2 v = unpack_f32x2(fmul2(bf16x2_to_f32x2(ww[q][p]), s2));
+        f[p] = pack_f16x2(v.x, v.y);
+      }
+      // f[p] = inputs (2p, 2p+1): entry t = {pair t, pair t + 4}
+      uint4* dst = reinterpret_cast<uint4*>(xs + ((size_t)jj * mr + m) * 4);
+      dst[0] = make_uint4(f[0], f[4], f[1], f[5]);
+      dst[1] = make_uint4(f[2], f[6], f[3], f[7]);
+    }
+  } else {
+    store_batch(tid);
+  }
   for (int i0 = tid + NB * nt; i0 < Tr * mr; i0 += NB * nt) {
     load_gamma(i0);
     load_x(i0);
