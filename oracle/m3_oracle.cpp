@@ -370,6 +370,57 @@ static int64_t gumbel_argmax(const float* g, int64_t n, float temperature, uint6
   return best;
 }
 
+// Top-k filtering before the draw (the AR sampler's "CFG 1.5, top-k 50,
+// multinomial" in the DiffSynth-Studio article, "第二阶段"): keep the k
+// largest guided logits -- ties at the k-th value broken towards the lower
+// index -- and draw among them by Gumbel-argmax; k <= 0 or k >= n keeps all.
+// The kept indices, ascending.
+static std::vector<int64_t> topk_set(const float* g, int64_t n, int64_t k) {
+  std::vector<int64_t> idx(n);
+  for (int64_t i = 0; i < n; ++i) idx[i] = i;
+  std::stable_sort(idx.begin(), idx.end(), [&](int64_t a, int64_t b) { return g[a] > g[b]; });
+  idx.resize(k);
+  std::sort(idx.begin(), idx.end());
+  return idx;
+}
+
+// The draw over the kept set; margin_out (nullable): best minus second-best z
+// over the kept set.
+static int64_t topk_gumbel_argmax(const float* g, int64_t n, int64_t k, float temperature,
+                                  uint64_t seed, uint64_t frame, uint64_t key_row,
+                                  uint64_t index_base, float* margin_out) {
+  std::vector<int64_t> keep;
+  if (k > 0 && k < n) {
+    keep = topk_set(g, n, k);
+  } else {
+    keep.resize(n);
+    for (int64_t i = 0; i < n; ++i) keep[i] = i;
+  }
+  int64_t best = -1;
+  float b1 = -INFINITY, b2 = -INFINITY;
+  for (int64_t i : keep) {
+    float z = g[i] / temperature + ora_gumbel(seed, frame, key_row, index_base + (uint64_t)i);
+    if (best < 0 || z > b1) {
+      b2 = b1;
+      b1 = z;
+      best = i;
+    } else if (z > b2) {
+      b2 = z;
+    }
+  }
+  if (margin_out) *margin_out = b1 - b2;
+  return best;
+}
+
+// Repeated top-k draws from fixed logits (frame = frame0 + t, key_row 0).
+void ora_topk_draws(const float* logits, int64_t n, int64_t k, float temperature, uint64_t seed,
+                    uint64_t frame0, int64_t ndraws, int32_t* out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < ndraws; ++t)
+    out[t] = (int32_t)topk_gumbel_argmax(logits, n, k, temperature, seed, frame0 + (uint64_t)t, 0,
+                                         0, nullptr);
+}
+
 // Repeated draws from fixed logits: draw t uses frame = frame0 + t and
 // key_row 0.  Used to check the draw against the categorical distribution.
 void ora_gumbel_argmax_draws(const float* logits, int64_t n, float temperature, uint64_t seed,
@@ -388,7 +439,7 @@ void ora_gumbel_argmax_draws(const float* logits, int64_t n, float temperature, 
 // logits (nullable) receives the raw per-row logits [rows, slice_len];
 // margin (nullable) receives per row the gap between the best and second-best z.
 int ora_sample(const OraCfg* cfg, OraMat lm, int rows, const bf16_t* hf, uint64_t seed,
-               uint64_t frame, float cfg_scale, float temperature, int32_t* codes,
+               uint64_t frame, float cfg_scale, float temperature, int top_k, int32_t* codes,
                float* logits, float* margin) {
   const int H = cfg->hidden, S = cfg->slice_len;
   if (cfg_scale > 0.0f && (rows % 2)) return -1;
@@ -408,16 +459,12 @@ int ora_sample(const OraCfg* cfg, OraMat lm, int rows, const bf16_t* hf, uint64_
     } else {
       std::memcpy(g.data(), &L[(size_t)p * S], sizeof(float) * S);
     }
-    int64_t best = gumbel_argmax(g.data(), S, temperature, seed, frame, (uint64_t)p,
-                                 (uint64_t)cfg->slice_start, nullptr);
+    float mg = 0.0f;
+    int64_t best = topk_gumbel_argmax(g.data(), S, top_k, temperature, seed, frame, (uint64_t)p,
+                                      (uint64_t)cfg->slice_start, &mg);
     if (margin) {
-      float b1 = -INFINITY, b2 = -INFINITY;
-      for (int i = 0; i < S; ++i) {
-        float zz = g[i] / temperature + ora_gumbel(seed, frame, p, cfg->slice_start + i);
-        if (zz > b1) { b2 = b1; b1 = zz; } else if (zz > b2) { b2 = zz; }
-      }
-      if (cfg_scale > 0.0f) { margin[2 * p] = b1 - b2; margin[2 * p + 1] = b1 - b2; }
-      else margin[p] = b1 - b2;
+      if (cfg_scale > 0.0f) { margin[2 * p] = mg; margin[2 * p + 1] = mg; }
+      else margin[p] = mg;
     }
     if (cfg_scale > 0.0f) {
       codes[2 * p] = (int32_t)best;
@@ -474,8 +521,8 @@ int ora_sample_full_masked(const OraCfg* cfg, const bf16_t* lm_full, int vocab, 
 int ora_decode_frame(const OraCfg* cfg, const OraLayer* layers, const bf16_t* final_norm,
                      OraMat lm, int rows, int64_t max_pos, uint16_t* kcache, uint16_t* vcache,
                      const int32_t* positions, uint64_t seed, uint64_t frame, const bf16_t* x_in,
-                     float cfg_scale, float temperature, int32_t* codes, bf16_t* h_out,
-                     float* logits) {
+                     float cfg_scale, float temperature, int top_k, int32_t* codes,
+                     bf16_t* h_out, float* logits) {
   const int H = cfg->hidden, d = cfg->head_dim, Hkv = cfg->n_kv_heads;
   for (int r = 0; r < rows; ++r)
     if (positions[r] < 0 || positions[r] >= max_pos) return -5;
@@ -492,8 +539,8 @@ int ora_decode_frame(const OraCfg* cfg, const OraLayer* layers, const bf16_t* fi
     for (int i = 0; i < H; ++i) hf[(size_t)r * H + i] = f2bf(t[i]);
   }
   if (h_out) std::memcpy(h_out, hf.data(), sizeof(bf16_t) * hf.size());
-  return ora_sample(cfg, lm, rows, hf.data(), seed, frame, cfg_scale, temperature, codes, logits,
-                    nullptr);
+  return ora_sample(cfg, lm, rows, hf.data(), seed, frame, cfg_scale, temperature, top_k, codes,
+                    logits, nullptr);
 }
 
 // Only the layers (no sampler): used by tests that pin the residual wiring.

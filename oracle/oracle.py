@@ -75,15 +75,15 @@ def lib():
         L.ora_attention.restype = None
         L.ora_attention.argtypes = [vp, vp, vp, i64, C.c_int, vp]
         L.ora_sample.restype = C.c_int
-        L.ora_sample.argtypes = [C.POINTER(OraCfg), OraMat, C.c_int, vp, u64, u64, f32, f32, vp,
-                                 vp, vp]
+        L.ora_sample.argtypes = [C.POINTER(OraCfg), OraMat, C.c_int, vp, u64, u64, f32, f32,
+                                 C.c_int, vp, vp, vp]
         L.ora_sample_full_masked.restype = C.c_int
         L.ora_sample_full_masked.argtypes = [C.POINTER(OraCfg), vp, C.c_int, C.c_int, vp, u64,
                                              u64, f32, f32, vp]
         L.ora_decode_frame.restype = C.c_int
         L.ora_decode_frame.argtypes = [C.POINTER(OraCfg), C.POINTER(OraLayer), vp, OraMat,
-                                       C.c_int, i64, vp, vp, vp, u64, u64, vp, f32, f32, vp, vp,
-                                       vp]
+                                       C.c_int, i64, vp, vp, vp, u64, u64, vp, f32, f32, C.c_int,
+                                       vp, vp, vp]
         L.ora_body.restype = C.c_int
         L.ora_body.argtypes = [C.POINTER(OraCfg), C.POINTER(OraLayer), C.c_int, i64, vp, vp, vp,
                                vp, vp]
@@ -92,6 +92,8 @@ def lib():
                                        vp, vp, vp]
         L.ora_gumbel_argmax_draws.restype = None
         L.ora_gumbel_argmax_draws.argtypes = [vp, i64, f32, u64, u64, i64, vp]
+        L.ora_topk_draws.restype = None
+        L.ora_topk_draws.argtypes = [vp, i64, i64, f32, u64, u64, i64, vp]
         L.ora_num_threads.restype = C.c_int
         L.ora_set_num_threads.argtypes = [C.c_int]
         _lib = L
@@ -179,6 +181,13 @@ def gumbel_argmax_draws(logits, temperature, seed, frame0, ndraws) -> np.ndarray
     return out
 
 
+def topk_draws(logits, k, temperature, seed, frame0, ndraws) -> np.ndarray:
+    lg = np.ascontiguousarray(logits, np.float32)
+    out = np.empty(ndraws, np.int32)
+    lib().ora_topk_draws(_p(lg), lg.size, k, temperature, seed, frame0, ndraws, _p(out))
+    return out
+
+
 def set_threads(n: int) -> None:
     lib().ora_set_num_threads(int(n))
 
@@ -235,7 +244,7 @@ class Body:
         return np.zeros(shp, np.uint16), np.zeros(shp, np.uint16)
 
     def decode_frame(self, kc, vc, positions, seed, frame, x_in_bits, cfg_scale=0.0,
-                     temperature=1.0):
+                     temperature=1.0, top_k=0):
         rows = x_in_bits.shape[0]
         pos = np.ascontiguousarray(positions, np.int32)
         x = np.ascontiguousarray(x_in_bits, np.uint16)
@@ -244,7 +253,8 @@ class Body:
         lg = np.empty((rows, self.shape.slice_len), np.float32)
         rc = lib().ora_decode_frame(C.byref(self.cfg), self.layers, _p(self.final_norm), self.lm,
                                     rows, kc.shape[2], _p(kc), _p(vc), _p(pos), seed, frame,
-                                    _p(x), cfg_scale, temperature, _p(codes), _p(h), _p(lg))
+                                    _p(x), cfg_scale, temperature, top_k, _p(codes), _p(h),
+                                    _p(lg))
         if rc != 0:
             raise RuntimeError(f"ora_decode_frame: {rc}")
         return codes, h, lg
@@ -258,14 +268,16 @@ class Body:
                        _p(pos), _p(x), _p(out))
         return out
 
-    def sample(self, h_bits, seed, frame, cfg_scale=0.0, temperature=1.0, with_margin=False):
+    def sample(self, h_bits, seed, frame, cfg_scale=0.0, temperature=1.0, with_margin=False,
+               top_k=0):
         h = np.ascontiguousarray(h_bits, np.uint16)
         rows = h.shape[0]
         codes = np.empty(rows, np.int32)
         lg = np.empty((rows, self.shape.slice_len), np.float32)
         mg = np.empty(rows, np.float32)
         rc = lib().ora_sample(C.byref(self.cfg), self.lm, rows, _p(h), seed, frame, cfg_scale,
-                              temperature, _p(codes), _p(lg), _p(mg) if with_margin else None)
+                              temperature, top_k, _p(codes), _p(lg),
+                              _p(mg) if with_margin else None)
         if rc != 0:
             raise RuntimeError(f"ora_sample: {rc}")
         return (codes, lg, mg) if with_margin else (codes, lg)

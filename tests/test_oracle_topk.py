@@ -1,0 +1,88 @@
+"""Pins for the oracle's top-k filtered draw: the DiffSynth-Studio article's
+AR sampler ("第二阶段": CFG 1.5, top-k 50, multinomial), with the multinomial
+as Gumbel-argmax (the diffusers issue, finding 3).  Top-k keeps the k largest
+guided logits, ties at the k-th value going to the lower index.
+"""
+import numpy as np
+import pytest
+
+import synth
+from test_oracle_frame import _bits, _tiny_body
+
+
+def _softmax(x, T):
+    z = np.exp((x - x.max()) / T)
+    return z / z.sum()
+
+
+def test_top1_is_greedy(ora):
+    rng = np.random.default_rng(3)
+    for trial in range(20):
+        lg = rng.standard_normal(64).astype(np.float32)
+        d = ora.topk_draws(lg, 1, 1.0, trial, 0, 50)
+        assert np.all(d == int(np.argmax(lg)))
+
+
+def test_k_at_least_n_is_plain_draw(ora):
+    rng = np.random.default_rng(4)
+    lg = rng.standard_normal(32).astype(np.float32)
+    for k in (0, 32, 100):
+        assert np.array_equal(ora.topk_draws(lg, k, 0.8, 7, 3, 500),
+                              ora.gumbel_argmax_draws(lg, 0.8, 7, 3, 500))
+
+
+@pytest.mark.parametrize("k,T", [(5, 1.0), (3, 0.7)])
+def test_topk_distribution(ora, k, T):
+    rng = np.random.default_rng(5)
+    lg = (rng.standard_normal(16) * 1.5).astype(np.float32)
+    n = 100_000
+    d = ora.topk_draws(lg, k, T, 11, 0, n)
+    keep = np.sort(np.argsort(-lg, kind="stable")[:k])
+    assert set(np.unique(d)) <= set(keep.tolist())
+    p = np.zeros(16)
+    p[keep] = _softmax(lg[keep].astype(np.float64), T)
+    emp = np.bincount(d, minlength=16) / n
+    assert np.abs(emp - p).sum() < 0.02
+
+
+def test_ties_at_the_threshold_keep_lower_indices(ora):
+    lg = np.array([3.0, 1.0, 2.0, 2.0, 2.0, 0.0], np.float32)
+    d = ora.topk_draws(lg, 3, 1.0, 2, 0, 20_000)
+    assert set(np.unique(d)) == {0, 2, 3}
+
+
+@pytest.mark.parametrize("cfg_scale", [0.0, 1.5])
+def test_sampler_top1_is_guided_argmax(ora, cfg_scale):
+    s = synth.TINY
+    body, *_ = _tiny_body(ora)
+    rng = np.random.default_rng(6)
+    for trial in range(8):
+        h = ((rng.standard_normal((2, s.hidden)).astype(np.float32).view(np.uint32)) >> 16).astype(np.uint16)
+        codes, lg = body.sample(h, seed=trial, frame=trial, cfg_scale=cfg_scale, top_k=1)
+        if cfg_scale > 0:
+            g = lg[1] + np.float32(cfg_scale) * (lg[0] - lg[1])
+            assert codes[0] == codes[1] == int(np.argmax(g))
+        else:
+            assert codes[0] == int(np.argmax(lg[0])) and codes[1] == int(np.argmax(lg[1]))
+
+
+def test_sampler_topk_draws_within_the_kept_set(ora):
+    s = synth.TINY
+    body, *_ = _tiny_body(ora)
+    rng = np.random.default_rng(7)
+    h = ((rng.standard_normal((2, s.hidden)).astype(np.float32).view(np.uint32)) >> 16).astype(np.uint16)
+    _, lg = body.sample(h, seed=0, frame=0, cfg_scale=1.5)
+    g = lg[1] + np.float32(1.5) * (lg[0] - lg[1])
+    keep = set(np.argsort(-g, kind="stable")[:50].tolist())
+    seen = set()
+    for f in range(300):
+        codes, _ = body.sample(h, seed=1, frame=f, cfg_scale=1.5, top_k=50)
+        assert int(codes[0]) in keep
+        seen.add(int(codes[0]))
+    assert len(seen) > 10  # it does draw, not only take the top
+    # with no top-k the draws leave the set at times
+    outside = 0
+    for f in range(300):
+        codes, _ = body.sample(h, seed=1, frame=f, cfg_scale=1.5)
+        outside += int(codes[0]) not in keep
+    assert outside > 0
