@@ -58,6 +58,7 @@ struct FrameParams {
   unsigned long long seed;
   unsigned long long frame;
   int pos[kMaxRows];
+  int top_k;  // the lm_head draw keeps the top_k guided logits; 0 keeps all
 };
 
 struct SampleArgs {
@@ -73,6 +74,7 @@ struct SampleArgs {
   int* part_i;                // [grid][kMaxRows] scratch
   unsigned int* counter;      // zero at rest; the last CTA resets it
   __nv_bfloat16* h_out;       // nullable: normalised input [rows][K] (CTA 0 writes)
+  float* gbuf;                // nullable: [keys][N] guided logits for the top-k draw
 };
 
 struct GemvArgs {

@@ -484,6 +484,96 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, int mr, int
   named_bar_sync(1, nt);
 }
 
+// ------------------------------------------------------------ top-k draw --
+// Order-preserving bits of a float (larger float, larger unsigned).
+__device__ __forceinline__ uint32_t f32_order(float f) {
+  const uint32_t b = __float_as_uint(f == 0.0f ? 0.0f : f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// One key's top-k draw over the guided logits g = smp.gbuf[p][0, N), by one
+// CTA (nt threads): radix select (8 bits per pass, most significant first)
+// of the k-th largest value T; the kept set is every index with g > T plus
+// the lowest-indexed ties at T that fill k; then Gumbel-argmax over the kept
+// set (the lowest index on equal z) and the code written for the key's rows.
+static __device__ __noinline__ void topk_draw(const GemvArgs& a, int p, int k, bool cfg, int tid, int nt,
+                          unsigned long long* best) {
+  __shared__ unsigned hist[256];
+  __shared__ unsigned sel[2];        // prefix of T, ties still to take
+  __shared__ unsigned eq_before[kTThreads + 1];
+  const int N = a.N;
+  const float* g = a.smp.gbuf + (size_t)p * N;
+  if (tid == 0) {
+    sel[0] = 0u;
+    sel[1] = (unsigned)k;
+    best[0] = 0ull;
+  }
+  uint32_t mask = 0u;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = tid; b < 256; b += nt) hist[b] = 0u;
+    __syncthreads();
+    const uint32_t prefix = sel[0];
+    for (int i = tid; i < N; i += nt) {
+      const uint32_t v = f32_order(__ldcg(g + i));
+      if ((v & mask) == prefix) atomicAdd(&hist[(v >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      unsigned need = sel[1], cum = 0u;
+      for (int b = 255; b >= 0; --b) {
+        if (cum + hist[b] >= need) {
+          sel[0] = prefix | ((uint32_t)b << shift);
+          sel[1] = need - cum;  // taken from inside bin b
+          break;
+        }
+        cum += hist[b];
+      }
+    }
+    mask |= 255u << shift;
+    __syncthreads();
+  }
+  const uint32_t T = sel[0];
+  const unsigned ties = sel[1];  // the lowest-indexed `ties` values equal to T are kept
+  // ties before each thread's contiguous chunk of indices
+  const int chunk = (N + nt - 1) / nt;
+  const int c0 = min(N, tid * chunk), c1 = min(N, c0 + chunk);
+  unsigned eq = 0u;
+  for (int i = c0; i < c1; ++i) eq += f32_order(__ldcg(g + i)) == T;
+  eq_before[tid + 1] = eq;
+  __syncthreads();
+  if (tid == 0) {
+    eq_before[0] = 0u;
+    for (int t = 1; t <= nt; ++t) eq_before[t] += eq_before[t - 1];
+  }
+  __syncthreads();
+  const unsigned long long key = cfg ? (unsigned long long)(a.row0 / 2 + p)
+                                     : (unsigned long long)(a.row0 + p);
+  unsigned rank = eq_before[tid];
+  for (int i = c0; i < c1; ++i) {
+    const float gi = __ldcg(g + i);
+    const uint32_t v = f32_order(gi);
+    bool keep = v > T;
+    if (v == T) keep = rank++ < ties;
+    if (!keep) continue;
+    const float gn = gumbel_noise(a.fp->seed, a.fp->frame, key,
+                                  a.smp.index_base + (unsigned long long)i);
+    const float z = __fadd_rn(__fdiv_rn(gi, a.fp->temperature), gn);
+    atomicMax(&best[0], argmax_key(z, i));
+  }
+  __syncthreads();
+  if (tid == 0) {
+    const int bi = key_idx(best[0]);
+    const int nm = cfg ? 2 : 1;
+    for (int q = 0; q < nm; ++q) {
+      const int r = a.row0 + (cfg ? 2 * p + q : p);
+      a.smp.codes[(size_t)r * a.smp.code_stride] = bi;
+      if (a.smp.prev)
+        a.smp.prev[r] = a.smp.forced ? a.smp.forced[(size_t)r * a.smp.forced_stride] : bi;
+    }
+  }
+  __syncthreads();
+}
+
 // ------------------------------------------------------- static kernel ----
 // HI: more than 8 batch rows (a second MMA per tile for rows 8..15).
 template <int WF, int EPI, bool HI>
@@ -674,6 +764,9 @@ __global__ void __launch_bounds__(kTThreads, 1) gemv_tile_kernel(const GemvArgs 
   } else {  // EPI_SAMPLE: all of the CTA's outputs in parallel, then argmax
     const bool cfg = a.fp->cfg_on != 0;
     const int np = cfg ? mr / 2 : mr;
+    // top-k: the guided logits go to smp.gbuf and the last CTA selects and
+    // draws (k < N; the host passes 0 for "keep all")
+    const int topk = a.smp.gbuf ? a.fp->top_k : 0;
     for (int e = tid; e < nown * kUnitRows * np; e += kTThreads) {
       const int ul = rank + (e / (kUnitRows * np)) * C, r = e % (kUnitRows * np);
       const int p = r / kUnitRows, nn = r % kUnitRows;
@@ -693,6 +786,10 @@ __global__ void __launch_bounds__(kTThreads, 1) gemv_tile_kernel(const GemvArgs 
       }
       float gl = y0;
       if (cfg) gl = __fadd_rn(y1, __fmul_rn(a.fp->cfg_scale, __fsub_rn(y0, y1)));
+      if (topk > 0) {
+        a.smp.gbuf[(size_t)p * a.N + n] = gl;
+        continue;
+      }
       const unsigned long long key = cfg ? (unsigned long long)(a.row0 / 2 + p)
                                          : (unsigned long long)(a.row0 + p);
       const float gn = gumbel_noise(a.fp->seed, a.fp->frame, key,
@@ -705,8 +802,8 @@ __global__ void __launch_bounds__(kTThreads, 1) gemv_tile_kernel(const GemvArgs 
       const unsigned long long b = best[tid];
       a.smp.part_z[blockIdx.x * kMaxRows + tid] = b ? key_z(b) : -INFINITY;
       a.smp.part_i[blockIdx.x * kMaxRows + tid] = b ? key_idx(b) : 0x7fffffff;
-      __threadfence();
     }
+    __threadfence();
     __syncthreads();
     if (tid == 0) {
       __threadfence();
@@ -714,7 +811,12 @@ __global__ void __launch_bounds__(kTThreads, 1) gemv_tile_kernel(const GemvArgs 
       *flag = old == gridDim.x - 1;
     }
     __syncthreads();
-    if (*flag) {  // the last CTA: argmax over the CTAs' winners
+    if (*flag && topk > 0) {  // the last CTA: top-k selection and draw per key
+      __threadfence();
+      for (int p = 0; p < np; ++p)
+        topk_draw(a, p, topk, cfg, tid, kTThreads, best);
+      if (tid == 0) *a.smp.counter = 0u;
+    } else if (*flag) {  // the last CTA: argmax over the CTAs' winners
       __threadfence();
       if (tid < np) {
         float bz = -INFINITY;

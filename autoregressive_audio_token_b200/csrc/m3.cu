@@ -140,6 +140,8 @@ struct m3_ctx {
   int ssq_n = 0;
   bool ssq_track = false;
   float2* rope = nullptr;  // this frame's RoPE (cos, sin) [max_rows][head_dim / 2]
+  int top_k = 0;           // the frame draw keeps the top_k guided logits (0: all)
+  float* gbuf = nullptr;   // the guided logits of the top-k draw [max_rows][slice_len]
 };
 
 template <typename T>
@@ -264,6 +266,7 @@ extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) 
     if ((rc = dalloc(c, &c->ssq_buf[i], sizeof(float) * R * ((g.hidden + kUnitRows - 1) / kUnitRows))))
       return bail(rc);
   if ((rc = dalloc(c, &c->rope, sizeof(float2) * R * (g.head_dim / 2)))) return bail(rc);
+  if ((rc = dalloc(c, &c->gbuf, sizeof(float) * R * g.slice_len))) return bail(rc);
   if ((rc = dzalloc(c, &p, sizeof(FrameParams)))) return bail(rc);
   c->fp = static_cast<FrameParams*>(p);
   if ((rc = dzalloc(c, &p, sizeof(int)))) return bail(rc);
@@ -310,6 +313,13 @@ extern "C" void m3_destroy(m3_ctx* c) {
 }
 
 extern "C" const char* m3_last_error(void) { return g_err.c_str(); }
+
+extern "C" int m3_set_top_k(m3_ctx* c, int top_k) {
+  if (!c) return fail(M3_EINVAL, "null ctx");
+  if (top_k < 0) return fail(M3_EINVAL, "top_k < 0");
+  c->top_k = top_k >= c->cfg.slice_len ? 0 : top_k;  // keeping every logit is no filter
+  return M3_OK;
+}
 
 // ----------------------------------------------------------------- weights --
 // Copy a bf16 [rows, cols] source into device staging memory (or use it as is).
@@ -806,6 +816,7 @@ static int record_frame(m3_ctx* c, int rows, int nb) {
   sa.part_i = c->spi;
   sa.counter = c->scnt;
   sa.h_out = c->h;
+  sa.gbuf = c->gbuf;
   CKR(gemv_rows(c, c->lm, EPI_SAMPLE, rows, c->A.x, g.hidden, c->final_norm, nullptr, 0, &sa, pdl));
   return M3_OK;
 }
@@ -855,6 +866,7 @@ extern "C" int m3_decode_frame(m3_ctx* c, int rows, const int32_t* positions, ui
   fp.temperature = temperature;
   fp.seed = seed;
   fp.frame = frame;
+  fp.top_k = c->top_k;
   int maxpos = 0;
   for (int r = 0; r < rows; ++r) {
     if (positions[r] < 0 || positions[r] >= c->kv_max_pos)

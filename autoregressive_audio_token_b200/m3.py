@@ -24,7 +24,7 @@ M3_MEM_HOST, M3_MEM_DEVICE = 0, 1
 
 EXPORTED = ("m3_create", "m3_load_weights", "m3_load_depth_weights", "m3_kv_alloc", "m3_kv_set",
             "m3_kv_get", "m3_decode_frame", "m3_depth_decode", "m3_embed", "m3_quantize_int8",
-            "m3_export_weight", "m3_frame_bytes", "m3_time_gemv", "m3_sample_noalloc",
+            "m3_export_weight", "m3_frame_bytes", "m3_time_gemv", "m3_sample_noalloc", "m3_set_top_k",
             "m3_sync_status",
             "m3_last_error", "m3_destroy")
 
@@ -76,6 +76,7 @@ def load_library() -> C.CDLL:
     L.m3_load_weights.argtypes = [vp, C.POINTER(m3_weight_src), i32]
     L.m3_load_depth_weights.argtypes = [vp, C.POINTER(m3_depth_src)]
     L.m3_kv_alloc.argtypes = [vp, i32, i32, i32, i32]
+    L.m3_set_top_k.argtypes = [vp, i32]
     L.m3_kv_set.argtypes = [vp, i32, i32, vp, vp, i32]
     L.m3_kv_get.argtypes = [vp, i32, i32, vp, vp]
     L.m3_decode_frame.argtypes = [vp, i32, vp, u64, u64, vp, f32, f32, vp, vp, vp]
@@ -254,6 +255,11 @@ def m3_sample_noalloc(ctx: int, h: torch.Tensor, seed: int, frame: int, cfg_scal
     """The allocation-free draw on a final-normed hidden state (see m3.h)."""
     _check(lib.m3_sample_noalloc(ctx, h.shape[0], _ptr(h), seed, frame, cfg_scale, temperature,
                                  _ptr(codes), _ptr(logits)))
+
+
+def m3_set_top_k(ctx: int, top_k: int) -> None:
+    """Top-k filter of the frame draw (0 keeps every logit); see m3.h."""
+    _check(lib.m3_set_top_k(ctx, top_k))
 
 
 def m3_sync_status(ctx: int) -> None:

@@ -48,6 +48,9 @@ def parse():
     p.add_argument("--layers", type=int, default=36,
                    help="body layers (36 = the workload; fewer only for profiling small cases)")
     p.add_argument("--kv", default="bf16", choices=["bf16", "f16"])
+    p.add_argument("--top-k", type=int, default=0,
+                   help="top-k filter of the frame draw (0 keeps every logit, as the timed "
+                        "configs do)")
     p.add_argument("--depth", action="store_true",
                    help="run the RVQ depth decoder (7 codes) after every frame")
     p.add_argument("--sweep", action="store_true",
@@ -234,6 +237,7 @@ def run_ours(args, rank, world, local):
     seed = replica_seed(rank)
     wdtype = m3.M3_W_INT8 if args.wdtype == "int8" else m3.M3_W_BF16
     s, ctx = build_model(torch, m3, synth, seed, wdtype, args.layers, depth=args.depth)
+    m3.m3_set_top_k(ctx, args.top_k)
     prefill_kv(torch, m3, synth, s, ctx, ROWS, SONG_FRAMES, seed, args.kv == "f16")
     xs = synth.normal((64, ROWS, s.hidden), seed, "bench/x_in", std=0.02, device="cuda")
     codes = torch.empty(ROWS, dtype=torch.int32, device="cuda")
@@ -337,7 +341,7 @@ def run_ours(args, rank, world, local):
         "config": {"workload": variant,
                    "rows": ROWS, "song_frames": SONG_FRAMES, "mean_ctx": mean_ctx,
                    "cfg_scale": CFG_SCALE, "temperature": 1.0, "kv": f"{args.kv} pages of 256",
-                   "depth_decoder": bool(args.depth),
+                   "depth_decoder": bool(args.depth), "top_k": args.top_k,
                    "l2": "no flush: 14 GB of weights per frame >> 126 MB L2",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "gpu_launches": None,
@@ -444,6 +448,8 @@ def workload_name(args) -> str:
         name += f"-{args.kv}kv"
     if args.depth:
         name += "-depth7"
+    if args.top_k:
+        name += f"-top{args.top_k}"
     return name
 
 

@@ -167,6 +167,15 @@ M3_API int m3_kv_set(m3_ctx* ctx, int row, int n_positions, const void* k, const
  * raw cache-type bits (bf16 or f16).  Synchronises the stream. */
 M3_API int m3_kv_get(m3_ctx* ctx, int row, int n_positions, void* k_host, void* v_host);
 
+/* Top-k filter of the frame draw (the AR sampler's "CFG 1.5, top-k 50,
+ * multinomial", DiffSynth-Studio article, "第二阶段"): m3_decode_frame keeps
+ * the top_k largest guided logits per key -- ties at the k-th value going to
+ * the lower index -- and draws among them by Gumbel-argmax.  0 (the default)
+ * or top_k >= slice_len keeps every logit.  Applies to the calls that follow;
+ * the depth decoder and m3_sample_noalloc always keep every logit.
+ * Returns M3_EINVAL for top_k < 0. */
+M3_API int m3_set_top_k(m3_ctx* ctx, int top_k);
+
 /* Decode one frame for rows 0..rows-1 (rows <= cache rows and <= max_rows).
  *  positions (HOST, [rows]): the position each row writes this frame; the
  *    row attends to positions 0..positions[r] inclusive.  Every position must

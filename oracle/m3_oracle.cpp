@@ -412,6 +412,14 @@ static int64_t topk_gumbel_argmax(const float* g, int64_t n, int64_t k, float te
   return best;
 }
 
+// One top-k draw from given guided logits g [n] (the sampler's decision on
+// another implementation's logits).
+int32_t ora_topk_draw(const float* g, int64_t n, int64_t k, float temperature, uint64_t seed,
+                      uint64_t frame, uint64_t key_row, uint64_t index_base) {
+  return (int32_t)topk_gumbel_argmax(g, n, k, temperature, seed, frame, key_row, index_base,
+                                     nullptr);
+}
+
 // Repeated top-k draws from fixed logits (frame = frame0 + t, key_row 0).
 void ora_topk_draws(const float* logits, int64_t n, int64_t k, float temperature, uint64_t seed,
                     uint64_t frame0, int64_t ndraws, int32_t* out) {

@@ -92,6 +92,8 @@ def lib():
                                        vp, vp, vp]
         L.ora_gumbel_argmax_draws.restype = None
         L.ora_gumbel_argmax_draws.argtypes = [vp, i64, f32, u64, u64, i64, vp]
+        L.ora_topk_draw.restype = C.c_int32
+        L.ora_topk_draw.argtypes = [vp, i64, i64, f32, u64, u64, u64, u64]
         L.ora_topk_draws.restype = None
         L.ora_topk_draws.argtypes = [vp, i64, i64, f32, u64, u64, i64, vp]
         L.ora_num_threads.restype = C.c_int
@@ -179,6 +181,12 @@ def gumbel_argmax_draws(logits, temperature, seed, frame0, ndraws) -> np.ndarray
     out = np.empty(ndraws, np.int32)
     lib().ora_gumbel_argmax_draws(_p(lg), lg.size, temperature, seed, frame0, ndraws, _p(out))
     return out
+
+
+def topk_draw(g, k, temperature, seed, frame, key_row, index_base) -> int:
+    gg = np.ascontiguousarray(g, np.float32)
+    return int(lib().ora_topk_draw(_p(gg), gg.size, k, temperature, seed, frame, key_row,
+                                   index_base))
 
 
 def topk_draws(logits, k, temperature, seed, frame0, ndraws) -> np.ndarray:

@@ -100,6 +100,55 @@ def test_tiny_many_rows(ora, rows, cfg, wdtype):
         m.close()
 
 
+def _guided(lg, p, cfg):
+    # the kernel's guided logits, in the same fp32 operations
+    if cfg > 0:
+        return lg[2 * p + 1] + np.float32(cfg) * (lg[2 * p] - lg[2 * p + 1])
+    return lg[p]
+
+
+def _check_topk_codes(ora, codes, lg, k, seed, frame, cfg, slice_start):
+    # decision-level parity: the oracle's top-k draw on the GPU's own logits
+    npick = lg.shape[0] // 2 if cfg > 0 else lg.shape[0]
+    for p in range(npick):
+        want = ora.topk_draw(_guided(lg, p, cfg), k, 1.0, seed, frame, p, slice_start)
+        rows = (2 * p, 2 * p + 1) if cfg > 0 else (p,)
+        for r in rows:
+            assert codes[r] == want, (p, k, codes, want)
+
+
+@pytest.mark.parametrize("rows,cfg,k", [(2, 1.5, 50), (1, 0.0, 7), (2, 1.5, 1), (4, 1.5, 50),
+                                        (3, 0.0, 511)])
+def test_tiny_topk_draw(ora, rows, cfg, k):
+    s = synth.TINY
+    m = Model(s, seed=14, max_rows=4, oracle=False)
+    try:
+        m.m3.m3_set_top_k(m.ctx, k)
+        m.kv_setup(rows=rows, n_prefill=30, max_pos=100)
+        x = synth.frame_input(s, rows, 14, 0)
+        for f in range(6):
+            pos = [30 + f] * rows
+            codes, h, lg = m.decode(pos, seed=3, frame=f, x_in=x, cfg_scale=cfg)
+            _check_topk_codes(ora, codes, lg, k, 3, f, cfg, s.slice_start)
+        # back to the plain draw: some code outside the top-k shows up over frames
+        m.m3.m3_set_top_k(m.ctx, 0)
+        codes, h, lg = m.decode([40] * rows, seed=3, frame=9, x_in=x, cfg_scale=cfg)
+        _check_topk_codes(ora, codes, lg, 0, 3, 9, cfg, s.slice_start)
+    finally:
+        m.close()
+
+
+def test_topk_rejects_negative(ora):
+    from autoregressive_audio_token_b200 import m3
+    m = Model(synth.TINY, seed=15, oracle=False)
+    try:
+        with pytest.raises(m3.M3Error) as e:
+            m3.m3_set_top_k(m.ctx, -1)
+        assert e.value.code == m3.M3_EINVAL
+    finally:
+        m.close()
+
+
 def test_tiny_ragged_vocab_slice(ora):
     # a sampled slice of 500 rows: the last 8-row weight unit is partly padding
     import dataclasses
@@ -235,6 +284,12 @@ def test_layer8b_vs_oracle(ora, wdtype, rows, kv_f16, ring, monkeypatch):
         oc, oh, olg = m.ora.decode_frame(kc, vc, pos, 77, 0, bits(x))
         assert rel_err(lg, olg) <= TOL[wdtype], rel_err(lg, olg)
         check_codes_teacher_forced(m, h, codes, 77, 0)
+        if ring == "64x2":
+            # the top-k 50 draw over the 16384-row slice, on the GPU's own logits
+            m.m3.m3_set_top_k(m.ctx, 50)
+            codes, h, lg = m.decode([p + 1 for p in pos], 77, 1, x)
+            _check_topk_codes(ora, codes, lg, 50, 77, 1, 0.0, s.slice_start)
+            m.m3.m3_set_top_k(m.ctx, 0)
         if wdtype == 1:
             # the GPU's quantised weights are the oracle's, bit for bit
             L0 = m.layers[0]
