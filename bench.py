@@ -54,7 +54,7 @@ def parse():
     p.add_argument("--depth", action="store_true",
                    help="run the RVQ depth decoder (7 codes) after every frame")
     p.add_argument("--sweep", action="store_true",
-                   help="batched-variations sweep: rows 2..16 x context 1500/4500/9000, "
+                   help="batched-variations sweep: rows 1..16 x context 1500/4500/9000, "
                         "bf16 and int8; one JSON line per point")
     return p.parse_args()
 
@@ -454,11 +454,12 @@ def workload_name(args) -> str:
 
 
 def run_sweep(args):
-    """Batched-variations sweep: K = 1, 2, 4, 8 same-prompt variations decoded in
-    lockstep (rows = 2K), contexts 1500 / 4500 / 9000, bf16 and int8 weights,
-    bf16 KV; per point one JSON line with frames/s per row, ms/frame, the
-    frame's algorithmic bytes and GB/s, and the cost of each extra row pair
-    relative to the 2-row frame at the same context."""
+    """Batched-variations sweep: one unguided row (CFG off), then K = 1, 2, 4, 8
+    same-prompt variations decoded in lockstep (rows = 2K, CFG on), contexts
+    1500 / 4500 / 9000, bf16 and int8 weights, bf16 KV; per point one JSON line
+    with frames/s per row, ms/frame, the frame's algorithmic bytes and GB/s,
+    T_rows / T_1, and the cost of each extra row (pair) relative to the 1-row
+    (2-row) frame at the same context."""
     import torch
     from autoregressive_audio_token_b200 import m3
     import synth
@@ -468,24 +469,28 @@ def run_sweep(args):
         s, ctx = build_model(torch, m3, synth, 7, wd, max_rows=16)
         for n_ctx in (1500, 4500, 9000):
             base = None
-            for rows in (2, 4, 8, 16):
+            t1 = None
+            for rows in (1, 2, 4, 8, 16):
                 prefill_kv(torch, m3, synth, s, ctx, rows, n_ctx, 7, False)
                 xs = synth.normal((rows, s.hidden), 7, "sweep/x", std=0.02, device="cuda")
                 codes = torch.empty(rows, dtype=torch.int32, device="cuda")
                 pos = [n_ctx - 1] * rows
+                cfg = CFG_SCALE if rows % 2 == 0 else 0.0
                 for i in range(3):
-                    m3.m3_decode_frame(ctx, pos, 7, i, xs, CFG_SCALE, 1.0, codes)
+                    m3.m3_decode_frame(ctx, pos, 7, i, xs, cfg, 1.0, codes)
                 torch.cuda.synchronize()
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 steps = 10
                 e0.record()
                 for i in range(steps):
-                    m3.m3_decode_frame(ctx, pos, 7, i, xs, CFG_SCALE, 1.0, codes)
+                    m3.m3_decode_frame(ctx, pos, 7, i, xs, cfg, 1.0, codes)
                 e1.record()
                 torch.cuda.synchronize()
                 m3.m3_sync_status(ctx)
                 ms = e0.elapsed_time(e1) / steps
                 fb = m3.m3_frame_bytes(ctx, rows, n_ctx - 1)
+                if rows == 1:
+                    t1 = ms
                 if rows == 2:
                     base = ms
                 print(json.dumps({"sweep": "batched variations", "weights": wname, "kv": "bf16",
@@ -493,6 +498,9 @@ def run_sweep(args):
                                   "ms_per_frame": ms, "frames_per_s_per_row": 1000.0 / ms,
                                   "row_frames_per_s": rows * 1000.0 / ms,
                                   "algorithmic_bytes": fb, "achieved_gbs": fb / ms / 1e6,
+                                  "cfg_scale": cfg,
+                                  "t_rows_over_t1": ms / t1,
+                                  "extra_row_cost_vs_1row": (ms / t1 - 1.0) / max(1, rows - 1),
                                   "extra_pair_cost_vs_2rows": (ms / base - 1.0) / max(1, rows // 2 - 1)
                                   if rows > 2 else 0.0}), flush=True)
                 del xs
