@@ -282,6 +282,12 @@ struct OraCfg {
   float rms_eps;
   int wfmt;    // 0 bf16, 1 int8 per row
   int kv_f16;  // 0 bf16 cache, 1 f16 cache
+  // The end token (DiffSynth-Studio article, "第二阶段": the vocab mask
+  // leaves the audio codes and the end token sampleable): with has_end the
+  // lm_head holds slice_len + 1 rows, the last being vocab row end_token,
+  // drawn as slice-relative code slice_len.
+  int has_end;
+  int end_token;
 };
 
 struct OraLayer {
@@ -384,11 +390,20 @@ static std::vector<int64_t> topk_set(const float* g, int64_t n, int64_t k) {
   return idx;
 }
 
+// Noise index of candidate i of a draw: index_base + i, except candidate
+// end_i (the end token, when the draw has one), whose index is end_index.
+struct NoiseIndex {
+  uint64_t base;
+  int64_t end_i;  // -1: none
+  uint64_t end_index;
+  uint64_t at(int64_t i) const { return i == end_i ? end_index : base + (uint64_t)i; }
+};
+
 // The draw over the kept set; margin_out (nullable): best minus second-best z
 // over the kept set.
 static int64_t topk_gumbel_argmax(const float* g, int64_t n, int64_t k, float temperature,
                                   uint64_t seed, uint64_t frame, uint64_t key_row,
-                                  uint64_t index_base, float* margin_out) {
+                                  NoiseIndex index, float* margin_out) {
   std::vector<int64_t> keep;
   if (k > 0 && k < n) {
     keep = topk_set(g, n, k);
@@ -399,7 +414,7 @@ static int64_t topk_gumbel_argmax(const float* g, int64_t n, int64_t k, float te
   int64_t best = -1;
   float b1 = -INFINITY, b2 = -INFINITY;
   for (int64_t i : keep) {
-    float z = g[i] / temperature + ora_gumbel(seed, frame, key_row, index_base + (uint64_t)i);
+    float z = g[i] / temperature + ora_gumbel(seed, frame, key_row, index.at(i));
     if (best < 0 || z > b1) {
       b2 = b1;
       b1 = z;
@@ -416,8 +431,8 @@ static int64_t topk_gumbel_argmax(const float* g, int64_t n, int64_t k, float te
 // another implementation's logits).
 int32_t ora_topk_draw(const float* g, int64_t n, int64_t k, float temperature, uint64_t seed,
                       uint64_t frame, uint64_t key_row, uint64_t index_base) {
-  return (int32_t)topk_gumbel_argmax(g, n, k, temperature, seed, frame, key_row, index_base,
-                                     nullptr);
+  return (int32_t)topk_gumbel_argmax(g, n, k, temperature, seed, frame, key_row,
+                                     NoiseIndex{index_base, -1, 0}, nullptr);
 }
 
 // Repeated top-k draws from fixed logits (frame = frame0 + t, key_row 0).
@@ -426,7 +441,7 @@ void ora_topk_draws(const float* logits, int64_t n, int64_t k, float temperature
 #pragma omp parallel for schedule(static)
   for (int64_t t = 0; t < ndraws; ++t)
     out[t] = (int32_t)topk_gumbel_argmax(logits, n, k, temperature, seed, frame0 + (uint64_t)t, 0,
-                                         0, nullptr);
+                                         NoiseIndex{0, -1, 0}, nullptr);
 }
 
 // Repeated draws from fixed logits: draw t uses frame = frame0 + t and
@@ -444,12 +459,17 @@ void ora_gumbel_argmax_draws(const float* logits, int64_t n, float temperature, 
 // are (cond, uncond) pairs and g = l_u + c (l_c - l_u) is drawn once per pair
 // with key_row = pair index, both rows receiving the code; else g = l with
 // key_row = row.  Codes are slice-relative.  Noise index = slice_start + i.
-// logits (nullable) receives the raw per-row logits [rows, slice_len];
+// With the end token (cfg->has_end) there are S + 1 candidates, the last one
+// being the end token (code S, noise index end_token); ties between it and a
+// code go to the code.
+// logits (nullable) receives the raw per-row logits [rows, S (+1)];
 // margin (nullable) receives per row the gap between the best and second-best z.
 int ora_sample(const OraCfg* cfg, OraMat lm, int rows, const bf16_t* hf, uint64_t seed,
                uint64_t frame, float cfg_scale, float temperature, int top_k, int32_t* codes,
                float* logits, float* margin) {
-  const int H = cfg->hidden, S = cfg->slice_len;
+  const int H = cfg->hidden, S = cfg->slice_len + (cfg->has_end ? 1 : 0);
+  const NoiseIndex ni{(uint64_t)cfg->slice_start, cfg->has_end ? (int64_t)cfg->slice_len : -1,
+                      (uint64_t)cfg->end_token};
   if (cfg_scale > 0.0f && (rows % 2)) return -1;
   std::vector<float> L((size_t)rows * S), h(H);
   for (int r = 0; r < rows; ++r) {
@@ -469,7 +489,7 @@ int ora_sample(const OraCfg* cfg, OraMat lm, int rows, const bf16_t* hf, uint64_
     }
     float mg = 0.0f;
     int64_t best = topk_gumbel_argmax(g.data(), S, top_k, temperature, seed, frame, (uint64_t)p,
-                                      (uint64_t)cfg->slice_start, &mg);
+                                      ni, &mg);
     if (margin) {
       if (cfg_scale > 0.0f) { margin[2 * p] = mg; margin[2 * p + 1] = mg; }
       else margin[p] = mg;
@@ -485,11 +505,13 @@ int ora_sample(const OraCfg* cfg, OraMat lm, int rows, const bf16_t* hf, uint64_
 }
 
 // The same draw over the FULL vocabulary [vocab, H] with every row outside the
-// slice masked to -inf (the unsliced reference form).  Returns codes relative
-// to slice_start so they are directly comparable with ora_sample.
+// slice -- other than the end token, when there is one -- masked to -inf (the
+// unsliced reference form), top-k over the whole guided vector.  Returns codes
+// relative to slice_start (the end token as slice_len) so they are directly
+// comparable with ora_sample.
 int ora_sample_full_masked(const OraCfg* cfg, const bf16_t* lm_full, int vocab, int rows,
                            const bf16_t* hf, uint64_t seed, uint64_t frame, float cfg_scale,
-                           float temperature, int32_t* codes) {
+                           float temperature, int top_k, int32_t* codes) {
   const int H = cfg->hidden;
   if (cfg_scale > 0.0f && (rows % 2)) return -1;
   OraMat lm{lm_full, nullptr, nullptr, 0};
@@ -497,9 +519,11 @@ int ora_sample_full_masked(const OraCfg* cfg, const bf16_t* lm_full, int vocab, 
   for (int r = 0; r < rows; ++r) {
     for (int i = 0; i < H; ++i) h[i] = bf2f(hf[(size_t)r * H + i]);
     gemv(lm, vocab, H, h.data(), &L[(size_t)r * vocab]);
-    for (int i = 0; i < vocab; ++i)
-      if (i < cfg->slice_start || i >= cfg->slice_start + cfg->slice_len)
-        L[(size_t)r * vocab + i] = -INFINITY;
+    for (int i = 0; i < vocab; ++i) {
+      const bool in_slice = i >= cfg->slice_start && i < cfg->slice_start + cfg->slice_len;
+      const bool is_end = cfg->has_end && i == cfg->end_token;
+      if (!in_slice && !is_end) L[(size_t)r * vocab + i] = -INFINITY;
+    }
   }
   int npick = cfg_scale > 0.0f ? rows / 2 : rows;
   std::vector<float> g(vocab);
@@ -512,8 +536,10 @@ int ora_sample_full_masked(const OraCfg* cfg, const bf16_t* lm_full, int vocab, 
         g[i] = L[(size_t)p * vocab + i];
       }
     }
-    int64_t best = gumbel_argmax(g.data(), vocab, temperature, seed, frame, (uint64_t)p, 0, nullptr);
-    int32_t rel = (int32_t)(best - cfg->slice_start);
+    int64_t best = topk_gumbel_argmax(g.data(), vocab, top_k, temperature, seed, frame,
+                                      (uint64_t)p, NoiseIndex{0, -1, 0}, nullptr);
+    int32_t rel = (cfg->has_end && best == cfg->end_token) ? (int32_t)cfg->slice_len
+                                                            : (int32_t)(best - cfg->slice_start);
     if (cfg_scale > 0.0f) { codes[2 * p] = rel; codes[2 * p + 1] = rel; }
     else codes[p] = rel;
   }
@@ -525,7 +551,7 @@ int ora_sample_full_masked(const OraCfg* cfg, const bf16_t* lm_full, int vocab, 
 //   positions[r]: the position this frame writes (attends 0..positions[r]);
 //   x_in: [rows, H] bf16; codes: [rows] slice-relative;
 //   h_out (nullable): [rows, H] bf16 final-normed hidden state;
-//   logits (nullable): [rows, slice_len] fp32.
+//   logits (nullable): [rows, slice_len (+1 with the end token)] fp32.
 int ora_decode_frame(const OraCfg* cfg, const OraLayer* layers, const bf16_t* final_norm,
                      OraMat lm, int rows, int64_t max_pos, uint16_t* kcache, uint16_t* vcache,
                      const int32_t* positions, uint64_t seed, uint64_t frame, const bf16_t* x_in,
@@ -587,6 +613,8 @@ struct OraDepth {
   const bf16_t* const* emb; // codebooks tables: emb[0] [sem_vocab, hidden], emb[j] [vocab, hidden]
   const bf16_t* final_norm; // [hidden]
   const OraMat* heads;      // codebooks heads [vocab, hidden]
+  int sem_vocab;            // rows of emb[0]; code0 == sem_vocab (the end token's
+                            // code) feeds a zero vector at position 1
 };
 
 // codes_out: [rows, codebooks]; forced (nullable): [rows, codebooks] codes to
@@ -615,8 +643,12 @@ int ora_depth_decode(const OraDepth* D, int rows, const bf16_t* h_frame, const i
     for (int r = 0; r < rows; ++r) {
       float* xr = &x[(size_t)r * H];
       if (j > 0) {
-        const bf16_t* e = D->emb[j - 1] + (size_t)prev[r] * H;
-        for (int i = 0; i < H; ++i) xr[i] = bf2f(e[i]);
+        if (j == 1 && prev[r] == D->sem_vocab) {
+          for (int i = 0; i < H; ++i) xr[i] = 0.0f;
+        } else {
+          const bf16_t* e = D->emb[j - 1] + (size_t)prev[r] * H;
+          for (int i = 0; i < H; ++i) xr[i] = bf2f(e[i]);
+        }
       }
       for (int l = 0; l < D->n_layers; ++l) {
         size_t off = ((size_t)r * D->n_layers + l) * lstride;
@@ -651,6 +683,122 @@ int ora_depth_decode(const OraDepth* D, int rows, const bf16_t* h_frame, const i
       }
     }
   }
+  return 0;
+}
+
+// ------------------------------------------------- the multi-frame loop ----
+// The autoregressive loop of the Global LLM (DiffSynth-Studio article,
+// "第二阶段": each frame's codes are embedded back as the next input and the
+// loop stops early at the end token, an error if no frame came out;
+// "MiniMax Music 3 on Metal": position, step and count advance frame by
+// frame).  Frame f = 0, 1, ... runs every row at position positions[r] + f
+// with noise frame frame0 + f:
+//   1. the Global LLM frame gives code0 per row and its final hidden state hf;
+//   2. with a depth decoder (D non-null), its NC residual codes from (hf, code0);
+//   3. the next input (the article's embed_audio_frame): the token embedding
+//      of code0 plus the residual codebooks' audio embeddings, scaled by
+//      (1 + NC)^-0.5 -- the article's 8^-0.5 for its 8 codebooks:
+//        x = bf16(s * (tok_emb[code0] + audio_emb[0][code_1] + ... + audio_emb[NC-1][code_NC]))
+//      with the sum in fp32 in that order and s = fp32(1 / sqrt(1 + NC)).
+// A key (a CFG pair, or a row without CFG) stops at the first frame whose
+// code0 is the end token (code slice_len); its count is the number of frames
+// before that one.  The loop ends once every key has stopped, or after
+// max_frames frames.  A stopped key's rows keep being computed, on a zero
+// input, as rows of a lockstep batch are.
+//   tok_emb [slice_len, H] bf16: embed_tokens rows slice_start..;
+//   audio_emb: NC tables [D->vocab, H] bf16 (unused without D);
+//   forced (nullable) [max_frames, rows, 1 + NC]: teacher forcing -- these
+//     codes are fed forward (and stopped on) instead of the drawn ones;
+//   codes_out [max_frames, rows, 1 + NC]: the drawn code0 and residual codes
+//     of every frame a row's key runs; on its end frame the residual entries
+//     are -1; -1 everywhere after that;
+//   h_hist (nullable) [max_frames, rows, H] bf16: hf of every frame a row's
+//     key runs (end frame included), zeros after;
+//   n_frames [keys].
+// Returns 0; -1 on bad arguments or a fed code out of range; -5 if a
+// position would reach max_pos; -8 if some key stopped at frame 0.
+int ora_generate(const OraCfg* cfg, const OraLayer* layers, const bf16_t* final_norm, OraMat lm,
+                 const OraDepth* D, const bf16_t* tok_emb, const bf16_t* const* audio_emb,
+                 int rows, int64_t max_pos, uint16_t* kcache, uint16_t* vcache,
+                 const int32_t* positions, uint64_t seed, uint64_t frame0, const bf16_t* x_in,
+                 float cfg_scale, float temperature, int top_k, int max_frames,
+                 const int32_t* forced, int32_t* codes_out, bf16_t* h_hist, int32_t* n_frames) {
+  const int H = cfg->hidden, S = cfg->slice_len;
+  const int NC = D ? D->codebooks : 0, W = 1 + NC;
+  const bool cfg_on = cfg_scale > 0.0f;
+  if (rows < 1 || max_frames < 0 || (cfg_on && (rows % 2))) return -1;
+  const int keys = cfg_on ? rows / 2 : rows;
+  for (int r = 0; r < rows; ++r)
+    if (positions[r] < 0 || (int64_t)positions[r] + max_frames > max_pos) return -5;
+  const float sc = (float)(1.0 / std::sqrt((double)(1 + NC)));
+  std::vector<bf16_t> x(x_in, x_in + (size_t)rows * H), hf((size_t)rows * H);
+  std::vector<int32_t> pos(rows), code0(rows), c0(rows), fed((size_t)rows * W);
+  std::vector<int32_t> dcodes((size_t)rows * (NC ? NC : 1)), fz((size_t)rows * (NC ? NC : 1));
+  std::vector<int> active(keys, 1);
+  for (int k = 0; k < keys; ++k) n_frames[k] = 0;
+  for (size_t i = 0; i < (size_t)max_frames * rows * W; ++i) codes_out[i] = -1;
+  if (h_hist) std::memset(h_hist, 0, sizeof(bf16_t) * (size_t)max_frames * rows * H);
+  for (int f = 0; f < max_frames; ++f) {
+    bool any = false;
+    for (int k = 0; k < keys; ++k) any = any || active[k];
+    if (!any) break;
+    const uint64_t frame = frame0 + (uint64_t)f;
+    for (int r = 0; r < rows; ++r) pos[r] = positions[r] + f;
+    int rc = ora_decode_frame(cfg, layers, final_norm, lm, rows, max_pos, kcache, vcache,
+                              pos.data(), seed, frame, x.data(), cfg_scale, temperature, top_k,
+                              code0.data(), hf.data(), nullptr);
+    if (rc) return rc;
+    const int32_t* fr = forced ? forced + (size_t)f * rows * W : nullptr;
+    for (int r = 0; r < rows; ++r) c0[r] = fr ? fr[(size_t)r * W] : code0[r];
+    if (NC) {
+      for (int r = 0; r < rows; ++r)
+        for (int j = 0; j < NC; ++j) fz[(size_t)r * NC + j] = fr ? fr[(size_t)r * W + 1 + j] : 0;
+      rc = ora_depth_decode(D, rows, hf.data(), c0.data(), seed, frame, cfg_scale, temperature,
+                            fr ? fz.data() : nullptr, dcodes.data(), nullptr);
+      if (rc) return rc;
+    }
+    for (int r = 0; r < rows; ++r) {
+      fed[(size_t)r * W] = c0[r];
+      for (int j = 0; j < NC; ++j)
+        fed[(size_t)r * W + 1 + j] = fr ? fz[(size_t)r * NC + j] : dcodes[(size_t)r * NC + j];
+    }
+    // this frame's record, for the rows whose key still runs
+    for (int r = 0; r < rows; ++r) {
+      if (!active[cfg_on ? r / 2 : r]) continue;
+      const bool ends = cfg->has_end && fed[(size_t)r * W] == S;
+      int32_t* out = codes_out + ((size_t)f * rows + r) * W;
+      out[0] = code0[r];
+      for (int j = 0; j < NC; ++j) out[1 + j] = ends ? -1 : dcodes[(size_t)r * NC + j];
+      if (h_hist)
+        std::memcpy(h_hist + ((size_t)f * rows + r) * H, &hf[(size_t)r * H], sizeof(bf16_t) * H);
+    }
+    // the stop rule and the counts
+    for (int k = 0; k < keys; ++k) {
+      if (!active[k]) continue;
+      const int r = cfg_on ? 2 * k : k;
+      if (cfg->has_end && fed[(size_t)r * W] == S) active[k] = 0;
+      else n_frames[k] += 1;
+    }
+    // the next frame's input
+    for (int r = 0; r < rows; ++r) {
+      bf16_t* xr = &x[(size_t)r * H];
+      if (!active[cfg_on ? r / 2 : r]) {
+        for (int i = 0; i < H; ++i) xr[i] = 0;
+        continue;
+      }
+      const int32_t* cr = &fed[(size_t)r * W];
+      if (cr[0] < 0 || cr[0] >= S) return -1;
+      for (int j = 0; j < NC; ++j)
+        if (cr[1 + j] < 0 || cr[1 + j] >= D->vocab) return -1;
+      for (int i = 0; i < H; ++i) {
+        float t = bf2f(tok_emb[(size_t)cr[0] * H + i]);
+        for (int j = 0; j < NC; ++j) t += bf2f(audio_emb[j][(size_t)cr[1 + j] * H + i]);
+        xr[i] = f2bf(t * sc);
+      }
+    }
+  }
+  for (int k = 0; k < keys; ++k)
+    if (n_frames[k] == 0) return -8;
   return 0;
 }
 

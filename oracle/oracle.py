@@ -24,7 +24,8 @@ class OraCfg(C.Structure):
     _fields_ = [("hidden", C.c_int), ("n_layers", C.c_int), ("n_q_heads", C.c_int),
                 ("n_kv_heads", C.c_int), ("head_dim", C.c_int), ("ffn", C.c_int),
                 ("slice_start", C.c_int), ("slice_len", C.c_int), ("rope_theta", C.c_double),
-                ("rms_eps", C.c_float), ("wfmt", C.c_int), ("kv_f16", C.c_int)]
+                ("rms_eps", C.c_float), ("wfmt", C.c_int), ("kv_f16", C.c_int),
+                ("has_end", C.c_int), ("end_token", C.c_int)]
 
 
 class OraLayer(C.Structure):
@@ -39,7 +40,7 @@ class OraDepth(C.Structure):
                 ("vocab", C.c_int), ("in_hidden", C.c_int), ("rope_theta", C.c_double),
                 ("rms_eps", C.c_float), ("layers", C.POINTER(OraLayer)), ("proj", OraMat),
                 ("emb", C.POINTER(C.c_void_p)), ("final_norm", C.c_void_p),
-                ("heads", C.POINTER(OraMat))]
+                ("heads", C.POINTER(OraMat)), ("sem_vocab", C.c_int)]
 
 
 def lib():
@@ -79,7 +80,12 @@ def lib():
                                  C.c_int, vp, vp, vp]
         L.ora_sample_full_masked.restype = C.c_int
         L.ora_sample_full_masked.argtypes = [C.POINTER(OraCfg), vp, C.c_int, C.c_int, vp, u64,
-                                             u64, f32, f32, vp]
+                                             u64, f32, f32, C.c_int, vp]
+        L.ora_generate.restype = C.c_int
+        L.ora_generate.argtypes = [C.POINTER(OraCfg), C.POINTER(OraLayer), vp, OraMat,
+                                   C.POINTER(OraDepth), vp, C.POINTER(C.c_void_p), C.c_int, i64,
+                                   vp, vp, vp, u64, u64, vp, f32, f32, C.c_int, C.c_int, vp, vp,
+                                   vp, vp]
         L.ora_decode_frame.restype = C.c_int
         L.ora_decode_frame.argtypes = [C.POINTER(OraCfg), C.POINTER(OraLayer), vp, OraMat,
                                        C.c_int, i64, vp, vp, vp, u64, u64, vp, f32, f32, C.c_int,
@@ -228,13 +234,22 @@ class Body:
     """The oracle's copy of a body: weights as raw bits, optionally int8-quantised
     by the oracle's own quantiser (wfmt 1 = one scale per row)."""
 
-    def __init__(self, shape, layers: list, final_norm, lm_slice, wfmt=0, kv_f16=False):
+    def __init__(self, shape, layers: list, final_norm, lm_slice, wfmt=0, kv_f16=False,
+                 lm_end_row=None):
+        """lm_end_row: the end token's lm_head row [H] when shape.end_token >= 0
+        (drawn as code slice_len)."""
         self.shape = shape
         self.keep = _Keep()
         k = self.keep
+        self.has_end = getattr(shape, "end_token", -1) >= 0
+        self.n_cand = shape.slice_len + (1 if self.has_end else 0)
         self.cfg = OraCfg(shape.hidden, shape.n_layers, shape.n_q_heads, shape.n_kv_heads,
                           shape.head_dim, shape.ffn, shape.slice_start, shape.slice_len,
-                          shape.rope_theta, shape.rms_eps, wfmt, int(kv_f16))
+                          shape.rope_theta, shape.rms_eps, wfmt, int(kv_f16),
+                          int(self.has_end), int(getattr(shape, "end_token", -1)))
+        if self.has_end and lm_slice is not None:
+            assert lm_end_row is not None, "the end token needs its lm_head row"
+            lm_slice = np.concatenate([bits(lm_slice), bits(lm_end_row).reshape(1, -1)], 0)
         arr = (OraLayer * len(layers))()
         for i, Lw in enumerate(layers):
             b = {n: bits(t) for n, t in Lw.items()}
@@ -258,7 +273,7 @@ class Body:
         x = np.ascontiguousarray(x_in_bits, np.uint16)
         codes = np.empty(rows, np.int32)
         h = np.empty((rows, self.shape.hidden), np.uint16)
-        lg = np.empty((rows, self.shape.slice_len), np.float32)
+        lg = np.empty((rows, self.n_cand), np.float32)
         rc = lib().ora_decode_frame(C.byref(self.cfg), self.layers, _p(self.final_norm), self.lm,
                                     rows, kc.shape[2], _p(kc), _p(vc), _p(pos), seed, frame,
                                     _p(x), cfg_scale, temperature, top_k, _p(codes), _p(h),
@@ -281,7 +296,7 @@ class Body:
         h = np.ascontiguousarray(h_bits, np.uint16)
         rows = h.shape[0]
         codes = np.empty(rows, np.int32)
-        lg = np.empty((rows, self.shape.slice_len), np.float32)
+        lg = np.empty((rows, self.n_cand), np.float32)
         mg = np.empty(rows, np.float32)
         rc = lib().ora_sample(C.byref(self.cfg), self.lm, rows, _p(h), seed, frame, cfg_scale,
                               temperature, top_k, _p(codes), _p(lg),
@@ -291,16 +306,47 @@ class Body:
         return (codes, lg, mg) if with_margin else (codes, lg)
 
     def sample_full_masked(self, lm_full_bits, h_bits, seed, frame, cfg_scale=0.0,
-                           temperature=1.0):
+                           temperature=1.0, top_k=0):
         h = np.ascontiguousarray(h_bits, np.uint16)
         W = np.ascontiguousarray(lm_full_bits, np.uint16)
         rows = h.shape[0]
         codes = np.empty(rows, np.int32)
         rc = lib().ora_sample_full_masked(C.byref(self.cfg), _p(W), W.shape[0], rows, _p(h), seed,
-                                          frame, cfg_scale, temperature, _p(codes))
+                                          frame, cfg_scale, temperature, top_k, _p(codes))
         if rc != 0:
             raise RuntimeError(f"ora_sample_full_masked: {rc}")
         return codes
+
+    def generate(self, kc, vc, positions, seed, frame0, x_in_bits, max_frames, tok_emb,
+                 depth=None, audio_emb=None, cfg_scale=0.0, temperature=1.0, top_k=0,
+                 forced=None, with_h=False):
+        """The multi-frame loop (ora_generate).  Returns (rc, codes [F, rows, 1+NC],
+        n_frames [keys], h_hist [F, rows, H] bf16 bits or None); rc is 0 or -8
+        (a key stopped at frame 0)."""
+        s = self.shape
+        rows = x_in_bits.shape[0]
+        nc = depth.shape.codebooks if depth is not None else 0
+        keys = rows // 2 if cfg_scale > 0 else rows
+        pos = np.ascontiguousarray(positions, np.int32)
+        x = np.ascontiguousarray(x_in_bits, np.uint16)
+        te = np.ascontiguousarray(bits(tok_emb), np.uint16)
+        ae = [np.ascontiguousarray(bits(a), np.uint16) for a in (audio_emb or [])]
+        ap = (C.c_void_p * max(1, len(ae)))()
+        for j, a in enumerate(ae):
+            ap[j] = _p(a).value
+        codes = np.empty((max_frames, rows, 1 + nc), np.int32)
+        nf = np.empty(keys, np.int32)
+        hh = np.empty((max_frames, rows, s.hidden), np.uint16) if with_h else None
+        fc = None if forced is None else np.ascontiguousarray(forced, np.int32)
+        rc = lib().ora_generate(C.byref(self.cfg), self.layers, _p(self.final_norm), self.lm,
+                                C.byref(depth.D) if depth is not None else None, _p(te), ap,
+                                rows, kc.shape[2], _p(kc), _p(vc), _p(pos), seed, frame0, _p(x),
+                                cfg_scale, temperature, top_k, max_frames,
+                                _p(fc) if fc is not None else None, _p(codes),
+                                _p(hh) if hh is not None else None, _p(nf))
+        if rc not in (0, -8):
+            raise RuntimeError(f"ora_generate: {rc}")
+        return rc, codes, nf, hh
 
 
 class Depth:
@@ -330,7 +376,7 @@ class Depth:
         self.D = OraDepth(shape.hidden, shape.n_layers, shape.n_heads, shape.head_dim, shape.ffn,
                           shape.codebooks, shape.vocab, shape.in_hidden, shape.rope_theta,
                           shape.rms_eps, arr, _mat(k, bits(w["proj"]), 2), emb,
-                          k(bits(w["final_norm"])), heads)
+                          k(bits(w["final_norm"])), heads, shape.sem_vocab)
 
     def decode(self, h_frame_bits, code0, seed, frame, cfg_scale=0.0, temperature=1.0,
                forced=None):

@@ -31,6 +31,7 @@ class BodyShape:
     slice_len: int
     rope_theta: float = 1.0e6
     rms_eps: float = 1.0e-6
+    end_token: int = -1  # vocab row of the end token, sampleable with the slice; -1: none
 
 
 @dataclasses.dataclass(frozen=True)
@@ -58,6 +59,10 @@ LAYER8B = BodyShape(hidden=4096, n_layers=1, n_q_heads=32, n_kv_heads=8, head_di
 # The full 36-layer 8B body with its sliced lm_head.
 FULL8B = BodyShape(hidden=4096, n_layers=36, n_q_heads=32, n_kv_heads=8, head_dim=128,
                    ffn=12288, vocab=200000, slice_start=151675, slice_len=16384)
+# The same with the end token sampleable (the generation loop's stop code).
+FULL8B_END = dataclasses.replace(FULL8B, end_token=151670)
+# TINY with an end token four rows below the code block, as in the 8B vocab.
+TINY_END = dataclasses.replace(TINY, end_token=1019)
 DEPTH = DepthShape()
 
 LAYER_TENSORS = ("attn_norm", "wq", "wk", "wv", "q_norm", "k_norm", "wo", "mlp_norm",
@@ -138,9 +143,34 @@ def lm_head_full(s: BodyShape, seed: int, device="cpu") -> torch.Tensor:
     return lm_head_rows(s, seed, 0, s.vocab, device)
 
 
+def lm_head_end_row(s: BodyShape, seed: int, device="cpu") -> torch.Tensor:
+    """The end token's row [hidden] of the full lm_head."""
+    return lm_head_rows(s, seed, s.end_token, 1, device)[0].contiguous()
+
+
 def embedding(s: BodyShape, seed: int, device="cpu") -> torch.Tensor:
     """Token-embedding table [vocab, hidden] used to feed a drawn code back."""
     return normal((s.vocab, s.hidden), seed, "embed_tokens", std=0.02, device=device)
+
+
+def embedding_slice(s: BodyShape, seed: int, device="cpu") -> torch.Tensor:
+    """The code block's rows [slice_len, hidden] of a token-embedding table,
+    drawn in blocks of 1024 vocab rows (the generation loop's feedback table;
+    not the same values as embedding())."""
+    blocks = []
+    b0, b1 = s.slice_start // 1024, (s.slice_start + s.slice_len - 1) // 1024
+    for b in range(b0, b1 + 1):
+        n = min(1024, s.vocab - b * 1024)
+        blocks.append(normal((n, s.hidden), seed, f"embed_tokens/block{b}", std=0.02,
+                             device=device))
+    off = s.slice_start - b0 * 1024
+    return torch.cat(blocks, 0)[off:off + s.slice_len].contiguous()
+
+
+def audio_embeddings(d: DepthShape, hidden: int, seed: int, device="cpu") -> list:
+    """The residual codebooks' audio-embedding tables, d.codebooks x [d.vocab, hidden]."""
+    return [normal((d.vocab, hidden), seed, f"audio_emb{j}", std=0.02, device=device)
+            for j in range(d.codebooks)]
 
 
 def kv_prefill(s, rows: int, n_pos: int, seed: int, device="cpu"):
