@@ -75,7 +75,15 @@ struct SampleArgs {
   unsigned int* counter;      // zero at rest; the last CTA resets it
   __nv_bfloat16* h_out;       // nullable: normalised input [rows][K] (CTA 0 writes)
   float* gbuf;                // nullable: [keys][N] guided logits for the top-k draw
+  int end_row1;               // 1 + the output row that is the end token (0: none)
+  unsigned long long end_index;  // that row's noise index (its vocab row)
 };
+
+// Noise index of output row n of a draw: the code block's vocab rows
+// index_base + n, and the end token's own vocab row for the end candidate.
+__device__ __forceinline__ unsigned long long smp_index(const SampleArgs& s, int n) {
+  return n == s.end_row1 - 1 ? s.end_index : s.index_base + (unsigned long long)n;
+}
 
 struct GemvArgs {
   const void* w;              // [N][K] row-major, bf16 or int8
@@ -343,8 +351,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvArgs a)
             if (cfg) gl = __fadd_rn(y1, __fmul_rn(a.fp->cfg_scale, __fsub_rn(y0, y1)));
             const unsigned long long key = cfg ? (unsigned long long)(a.row0 / 2 + p)
                                                : (unsigned long long)(a.row0 + p);
-            const float gn = gumbel_noise(a.fp->seed, a.fp->frame, key,
-                                          a.smp.index_base + (unsigned long long)n);
+            const float gn = gumbel_noise(a.fp->seed, a.fp->frame, key, smp_index(a.smp, n));
             const float z = __fadd_rn(__fdiv_rn(gl, a.fp->temperature), gn);
             if (z > sbz[c] || (z == sbz[c] && n < sbi[c])) {
               sbz[c] = z;

@@ -555,8 +555,7 @@ static __device__ __noinline__ void topk_draw(const GemvArgs& a, int p, int k, b
     bool keep = v > T;
     if (v == T) keep = rank++ < ties;
     if (!keep) continue;
-    const float gn = gumbel_noise(a.fp->seed, a.fp->frame, key,
-                                  a.smp.index_base + (unsigned long long)i);
+    const float gn = gumbel_noise(a.fp->seed, a.fp->frame, key, smp_index(a.smp, i));
     const float z = __fadd_rn(__fdiv_rn(gi, a.fp->temperature), gn);
     atomicMax(&best[0], argmax_key(z, i));
   }
@@ -792,8 +791,7 @@ __global__ void __launch_bounds__(kTThreads, 1) gemv_tile_kernel(const GemvArgs 
       }
       const unsigned long long key = cfg ? (unsigned long long)(a.row0 / 2 + p)
                                          : (unsigned long long)(a.row0 + p);
-      const float gn = gumbel_noise(a.fp->seed, a.fp->frame, key,
-                                    a.smp.index_base + (unsigned long long)n);
+      const float gn = gumbel_noise(a.fp->seed, a.fp->frame, key, smp_index(a.smp, n));
       const float z = __fadd_rn(__fdiv_rn(gl, a.fp->temperature), gn);
       atomicMax(&best[p], argmax_key(z, n));
     }

@@ -4,6 +4,7 @@
 // and per (rows, teacher forcing) for the depth decoder, error plumbing.
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -141,7 +142,15 @@ struct m3_ctx {
   bool ssq_track = false;
   float2* rope = nullptr;  // this frame's RoPE (cos, sin) [max_rows][head_dim / 2]
   int top_k = 0;           // the frame draw keeps the top_k guided logits (0: all)
-  float* gbuf = nullptr;   // the guided logits of the top-k draw [max_rows][slice_len]
+  // generation loop: feedback tables, device state, its host copy, graphs
+  bf16* fb_tok = nullptr;          // [slice_len][H]
+  std::vector<bf16*> fb_aud;       // depth_codebooks tables [depth_vocab][H]
+  bf16** d_fb_aud = nullptr;       // device array of the fb_aud pointers
+  LoopState* loop = nullptr;
+  LoopState* h_loop = nullptr;     // pinned
+  int* h_err = nullptr;            // pinned
+  std::map<std::pair<int, int>, cudaGraphExec_t> lgraphs;
+  float* gbuf = nullptr;   // the guided logits of the top-k draw [max_rows][candidates]
 };
 
 template <typename T>
@@ -178,6 +187,8 @@ static void drop_graphs(m3_ctx* c) {
   c->graphs.clear();
   for (auto& kv : c->dgraphs) cudaGraphExecDestroy(kv.second);
   c->dgraphs.clear();
+  for (auto& kv : c->lgraphs) cudaGraphExecDestroy(kv.second);
+  c->lgraphs.clear();
 }
 
 static double* make_inv_freq(m3_ctx* c, int d, double theta, int* rc) {
@@ -199,6 +210,10 @@ static int alloc_acts(m3_ctx* c, Acts& A, int rows, int H, int Hq, int Hkv, int 
   return M3_OK;
 }
 
+// Rows of the lm_head the draw chooses among: the code block, and the end
+// token after it when the config has one.
+static inline int n_cand(const m3_config& g) { return g.slice_len + (g.has_end_token ? 1 : 0); }
+
 // ------------------------------------------------------------- validation --
 static bool valid_cfg(const m3_config* g, std::string& why) {
   if (g->hidden <= 0 || g->n_layers <= 0 || g->n_q_heads <= 0 || g->n_kv_heads <= 0 ||
@@ -210,6 +225,9 @@ static bool valid_cfg(const m3_config* g, std::string& why) {
     why = "hidden, ffn and n_q_heads*head_dim must be multiples of 16"; return false; }
   if (g->max_rows < 1 || g->max_rows > kMaxRows) { why = "max_rows must be in 1..16"; return false; }
   if (g->slice_len <= 0 || g->slice_start < 0) { why = "bad vocab slice"; return false; }
+  if (g->has_end_token && (g->end_token < 0 || (g->end_token >= g->slice_start &&
+                                                g->end_token < g->slice_start + g->slice_len))) {
+    why = "end_token must be a vocab row outside the slice"; return false; }
   if (g->depth_layers > 0) {
     if (g->depth_head_dim != 64 && g->depth_head_dim != 128) { why = "depth_head_dim"; return false; }
     if (g->depth_hidden % 128 || g->depth_ffn % 128 || g->hidden % 128 ||
@@ -253,7 +271,7 @@ extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) 
     return bail(rc);
   void* p = nullptr;
   if ((rc = dalloc(c, &c->h, sizeof(bf16) * R * g.hidden)) ||
-      (rc = dalloc(c, &c->logits, sizeof(float) * R * g.slice_len)) ||
+      (rc = dalloc(c, &c->logits, sizeof(float) * R * n_cand(g))) ||
       (rc = dalloc(c, &c->codes, sizeof(int) * R)) ||
       (rc = dalloc(c, &c->spz, sizeof(float) * 1024 * kMaxRows)) ||
       (rc = dalloc(c, &c->spi, sizeof(int) * 1024 * kMaxRows)) ||
@@ -266,7 +284,7 @@ extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) 
     if ((rc = dalloc(c, &c->ssq_buf[i], sizeof(float) * R * ((g.hidden + kUnitRows - 1) / kUnitRows))))
       return bail(rc);
   if ((rc = dalloc(c, &c->rope, sizeof(float2) * R * (g.head_dim / 2)))) return bail(rc);
-  if ((rc = dalloc(c, &c->gbuf, sizeof(float) * R * g.slice_len))) return bail(rc);
+  if ((rc = dalloc(c, &c->gbuf, sizeof(float) * R * n_cand(g)))) return bail(rc);
   if ((rc = dzalloc(c, &p, sizeof(FrameParams)))) return bail(rc);
   c->fp = static_cast<FrameParams*>(p);
   if ((rc = dzalloc(c, &p, sizeof(int)))) return bail(rc);
@@ -306,6 +324,8 @@ extern "C" void m3_destroy(m3_ctx* c) {
   drop_graphs(c);
   for (void* p : c->buckets) cudaFree(p);
   for (void* p : c->allocs) cudaFree(p);
+  if (c->h_loop) cudaFreeHost(c->h_loop);
+  if (c->h_err) cudaFreeHost(c->h_err);
   if (c->ev_in) cudaEventDestroy(c->ev_in);
   if (c->ev_out) cudaEventDestroy(c->ev_out);
   if (c->st) cudaStreamDestroy(c->st);
@@ -317,7 +337,7 @@ extern "C" const char* m3_last_error(void) { return g_err.c_str(); }
 extern "C" int m3_set_top_k(m3_ctx* c, int top_k) {
   if (!c) return fail(M3_EINVAL, "null ctx");
   if (top_k < 0) return fail(M3_EINVAL, "top_k < 0");
-  c->top_k = top_k >= c->cfg.slice_len ? 0 : top_k;  // keeping every logit is no filter
+  c->top_k = top_k >= n_cand(c->cfg) ? 0 : top_k;  // keeping every logit is no filter
   return M3_OK;
 }
 
@@ -452,8 +472,11 @@ extern "C" int m3_load_weights(m3_ctx* c, const m3_weight_src* src, int wdtype) 
   }
   if (src->final_norm) CKR(put_vec(c, &c->final_norm, src->final_norm, g.hidden, src->mem));
   if (src->lm_head) {
-    if (!c->lm.w) CKR(alloc_mat(c, c->lm, g.slice_len, g.hidden, wf));
+    if (g.has_end_token && !src->lm_end_row)
+      return fail(M3_EINVAL, "the config has an end token: lm_end_row is needed with lm_head");
+    if (!c->lm.w) CKR(alloc_mat(c, c->lm, n_cand(g), g.hidden, wf));
     CKR(put_rows(c, c->lm, src->lm_head, src->mem, g.slice_len, 0, 1));
+    if (g.has_end_token) CKR(put_rows(c, c->lm, src->lm_end_row, src->mem, 1, g.slice_len, 1));
     c->head_loaded = true;
   }
   CK(cudaStreamSynchronize(c->st));  // sources may be freed on return
@@ -808,10 +831,12 @@ static int record_frame(m3_ctx* c, int rows, int nb) {
                      -1, c->inv_freq, c->rope, pdl));
   SampleArgs sa{};
   sa.logits = c->logits;
-  sa.logits_ld = g.slice_len;
+  sa.logits_ld = n_cand(g);
   sa.codes = c->codes;
   sa.code_stride = 1;
   sa.index_base = (unsigned long long)g.slice_start;
+  sa.end_row1 = g.has_end_token ? g.slice_len + 1 : 0;
+  sa.end_index = (unsigned long long)g.end_token;
   sa.part_z = c->spz;
   sa.part_i = c->spi;
   sa.counter = c->scnt;
@@ -879,7 +904,7 @@ extern "C" int m3_decode_frame(m3_ctx* c, int rows, const int32_t* positions, ui
   CK(cudaMemcpyAsync(c->A.x, x_in, sizeof(bf16) * rows * g.hidden, cudaMemcpyDeviceToDevice, c->st));
   set_frame_params_kernel<<<1, 32, 0, c->st>>>(c->fp, fp);
   CK(cudaGetLastError());
-  rope_table_kernel<<<rows, 64, 0, c->st>>>(fp, c->inv_freq, g.head_dim / 2, c->rope);
+  rope_table_kernel<<<rows, 64, 0, c->st>>>(c->fp, c->inv_freq, g.head_dim / 2, c->rope);
   CK(cudaGetLastError());
   CKR(run_graph(c, c->graphs, {rows, c->n_buckets},
                 [&] { return record_frame(c, rows, c->n_buckets); }));
@@ -887,21 +912,26 @@ extern "C" int m3_decode_frame(m3_ctx* c, int rows, const int32_t* positions, ui
   if (h_out)
     CK(cudaMemcpyAsync(h_out, c->h, sizeof(bf16) * rows * g.hidden, cudaMemcpyDeviceToDevice, c->st));
   if (logits)
-    CK(cudaMemcpyAsync(logits, c->logits, sizeof(float) * rows * g.slice_len,
+    CK(cudaMemcpyAsync(logits, c->logits, sizeof(float) * rows * n_cand(g),
                        cudaMemcpyDeviceToDevice, c->st));
   return leave(c);
 }
 
 // --------------------------------------------------------- depth decoder ---
-static int record_depth(m3_ctx* c, int rows, bool forced) {
+// hin: the frame's final-normed hidden state [rows][hidden]; the semantic
+// code is in dprev.
+static int record_depth(m3_ctx* c, int rows, bool forced, const bf16* hin) {
   const m3_config& g = c->cfg;
   const int Dh = g.depth_hidden, NC = g.depth_codebooks, V = g.depth_vocab;
   bool pdl = false;
-  CKR(gemv_rows(c, c->dproj, EPI_STORE, rows, c->dh, g.hidden, nullptr, c->DA.x, Dh, nullptr, pdl));
+  CKR(gemv_rows(c, c->dproj, EPI_STORE, rows, hin, g.hidden, nullptr, c->DA.x, Dh, nullptr, pdl));
   for (int j = 0; j <= NC; ++j) {
     if (j >= 1) {
+      // the end token's code (slice_len) has no semantic embedding: a zero input
+      const int zero_code = j == 1 && g.has_end_token ? g.slice_len : INT_MIN;
       CK(launch_ex(embed_kernel, dim3(rows), dim3(128), 0, c->st, true, (const int*)c->dprev,
-                   (const bf16*)c->demb[j - 1], c->demb_rows[j - 1], 0, Dh, c->DA.x, c->err));
+                   (const bf16*)c->demb[j - 1], c->demb_rows[j - 1], 0, Dh, c->DA.x, c->err,
+                   zero_code));
     }
     for (int l = 0; l < g.depth_layers; ++l)
       CKR(record_layer(c, c->DL[l], c->DA, rows, Dh, g.depth_heads, g.depth_heads,
@@ -951,12 +981,153 @@ extern "C" int m3_depth_decode(m3_ctx* c, int rows, const void* h_frame, const i
   set_frame_params_kernel<<<1, 32, 0, c->st>>>(c->fp, fp);
   CK(cudaGetLastError());
   const bool f = forced != nullptr;
-  CKR(run_graph(c, c->dgraphs, {rows, f ? 1 : 0}, [&] { return record_depth(c, rows, f); }));
+  CKR(run_graph(c, c->dgraphs, {rows, f ? 1 : 0}, [&] { return record_depth(c, rows, f, c->dh); }));
   CK(cudaMemcpyAsync(codes, c->dcodes, sizeof(int) * rows * NC, cudaMemcpyDeviceToDevice, c->st));
   if (logits)
     CK(cudaMemcpyAsync(logits, c->dlogits, sizeof(float) * rows * NC * g.depth_vocab,
                        cudaMemcpyDeviceToDevice, c->st));
   return leave(c);
+}
+
+// ------------------------------------------------------ generation loop ----
+constexpr int kLoopChunk = 16;  // frames between reads of the loop state
+
+extern "C" int m3_load_feedback(m3_ctx* c, const void* tok_emb, const void* const* audio_emb,
+                                int mem) {
+  if (!c || !tok_emb) return fail(M3_EINVAL, "null argument");
+  const m3_config& g = c->cfg;
+  const int nc = g.depth_layers > 0 ? g.depth_codebooks : 0;
+  if (nc && !audio_emb) return fail(M3_EINVAL, "the depth decoder's codebooks need audio_emb");
+  for (int j = 0; j < nc; ++j)
+    if (!audio_emb[j]) return fail(M3_EINVAL, "null audio_emb table");
+  const cudaMemcpyKind kind = mem == M3_MEM_DEVICE ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
+  CKR(enter(c));
+  const size_t tb = sizeof(bf16) * (size_t)g.slice_len * g.hidden;
+  if (!c->fb_tok) CKR(dalloc(c, &c->fb_tok, tb));
+  CK(cudaMemcpyAsync(c->fb_tok, tok_emb, tb, kind, c->st));
+  if (nc) {
+    const size_t ab = sizeof(bf16) * (size_t)g.depth_vocab * g.hidden;
+    c->fb_aud.resize(nc, nullptr);
+    for (int j = 0; j < nc; ++j) {
+      if (!c->fb_aud[j]) CKR(dalloc(c, &c->fb_aud[j], ab));
+      CK(cudaMemcpyAsync(c->fb_aud[j], audio_emb[j], ab, kind, c->st));
+    }
+    if (!c->d_fb_aud) CKR(dalloc(c, &c->d_fb_aud, sizeof(bf16*) * nc));
+    CK(cudaMemcpyAsync(c->d_fb_aud, c->fb_aud.data(), sizeof(bf16*) * nc, cudaMemcpyHostToDevice,
+                       c->st));
+  }
+  CK(cudaStreamSynchronize(c->st));  // sources may be freed on return
+  return leave(c);
+}
+
+// One frame of the loop: RoPE table from the device positions, the frame,
+// the depth decoder, the feedback input and the loop state's advance.
+static int record_loop_frame(m3_ctx* c, int rows, int nb, bool depth) {
+  const m3_config& g = c->cfg;
+  rope_table_kernel<<<rows, 64, 0, c->st>>>(c->fp, c->inv_freq, g.head_dim / 2, c->rope);
+  CK(cudaGetLastError());
+  CKR(record_frame(c, rows, nb));
+  const int nc = depth ? g.depth_codebooks : 0;
+  if (depth) {
+    CK(cudaMemcpyAsync(c->dprev, c->codes, sizeof(int) * rows, cudaMemcpyDeviceToDevice, c->st));
+    CKR(record_depth(c, rows, false, c->h));
+  }
+  LoopArgs la{};
+  la.fp = c->fp;
+  la.ls = c->loop;
+  la.codes = c->codes;
+  la.dcodes = c->dcodes;
+  la.h = c->h;
+  la.tok = c->fb_tok;
+  la.aud = c->d_fb_aud;
+  la.x = c->A.x;
+  la.err = c->err;
+  la.nc = nc;
+  la.V = g.depth_vocab;
+  la.H = g.hidden;
+  la.S = g.slice_len;
+  la.has_end = g.has_end_token ? 1 : 0;
+  la.scale = (float)(1.0 / std::sqrt((double)(1 + nc)));
+  loop_feedback_kernel<<<rows, 128, 0, c->st>>>(la);
+  CK(cudaGetLastError());
+  loop_advance_kernel<<<1, 32, 0, c->st>>>(la);
+  CK(cudaGetLastError());
+  return M3_OK;
+}
+
+extern "C" int m3_generate(m3_ctx* c, int rows, const int32_t* positions, uint64_t seed,
+                           uint64_t frame0, const void* x_in, float cfg_scale, float temperature,
+                           int max_frames, int32_t* codes, void* h_hist, int32_t* n_frames) {
+  if (!c || !positions || !x_in || !codes || !n_frames) return fail(M3_EINVAL, "null argument");
+  const m3_config& g = c->cfg;
+  if (!c->d_pages) return fail(M3_ESTATE, "m3_kv_alloc first");
+  for (int l = 0; l < g.n_layers; ++l)
+    if (!c->loaded[l]) return fail(M3_ESTATE, "layer " + std::to_string(l) + " not loaded");
+  if (!c->head_loaded || !c->final_norm) return fail(M3_ESTATE, "lm_head / final norm not loaded");
+  if (!c->fb_tok) return fail(M3_ESTATE, "m3_load_feedback first");
+  const bool depth = c->depth_loaded;
+  if (depth && !c->d_fb_aud) return fail(M3_ESTATE, "m3_load_feedback without audio tables");
+  if (rows < 1 || rows > c->kv_rows) return fail(M3_EINVAL, "rows out of 1..cache rows");
+  if (max_frames < 1) return fail(M3_EINVAL, "max_frames < 1");
+  if (!(cfg_scale >= 0.0f) || !(temperature > 0.0f)) return fail(M3_EINVAL, "cfg_scale / temperature");
+  if (cfg_scale > 0.0f && rows % 2) return fail(M3_EINVAL, "cfg_scale > 0 needs (cond, uncond) row pairs");
+  FrameParams fp{};
+  fp.rows = rows;
+  fp.cfg_on = cfg_scale > 0.0f;
+  fp.cfg_scale = cfg_scale;
+  fp.temperature = temperature;
+  fp.seed = seed;
+  fp.frame = frame0;
+  fp.top_k = c->top_k;
+  int maxpos = 0;
+  for (int r = 0; r < rows; ++r) {
+    if (positions[r] < 0 || (long long)positions[r] + max_frames > c->kv_max_pos)
+      return fail(M3_ECAPACITY, "positions[" + std::to_string(r) + "] + max_frames outside the KV capacity");
+    fp.pos[r] = positions[r];
+    maxpos = positions[r] > maxpos ? positions[r] : maxpos;
+  }
+  const int nc = depth ? g.depth_codebooks : 0;
+  const int keys = fp.cfg_on ? rows / 2 : rows;
+  LoopState ls{};
+  ls.keys = keys;
+  for (int k = 0; k < keys; ++k) ls.active[k] = 1;
+  ls.codes_out = codes;
+  ls.h_hist = static_cast<bf16*>(h_hist);
+  if (!c->loop) {
+    void* p = nullptr;
+    CKR(dzalloc(c, &p, sizeof(LoopState)));
+    c->loop = static_cast<LoopState*>(p);
+  }
+  if (!c->h_loop) CK(cudaMallocHost(&c->h_loop, sizeof(LoopState)));
+  if (!c->h_err) CK(cudaMallocHost(&c->h_err, sizeof(int)));
+  CKR(enter(c));
+  CK(cudaMemcpyAsync(c->A.x, x_in, sizeof(bf16) * rows * g.hidden, cudaMemcpyDeviceToDevice, c->st));
+  CK(cudaMemsetAsync(codes, 0xFF, sizeof(int32_t) * (size_t)max_frames * rows * (1 + nc), c->st));
+  if (h_hist) CK(cudaMemsetAsync(h_hist, 0, sizeof(bf16) * (size_t)max_frames * rows * g.hidden, c->st));
+  set_frame_params_kernel<<<1, 32, 0, c->st>>>(c->fp, fp);
+  CK(cudaGetLastError());
+  loop_init_kernel<<<1, 32, 0, c->st>>>(c->loop, ls);
+  CK(cudaGetLastError());
+  for (int s0 = 0; s0 < max_frames; s0 += kLoopChunk) {
+    const int n = max_frames - s0 < kLoopChunk ? max_frames - s0 : kLoopChunk;
+    CKR(ensure_pages(c, maxpos + s0 + n));
+    for (int i = 0; i < n; ++i)
+      CKR(run_graph(c, c->lgraphs, {rows, 2 * c->n_buckets + (depth ? 1 : 0)},
+                    [&] { return record_loop_frame(c, rows, c->n_buckets, depth); }));
+    CK(cudaMemcpyAsync(c->h_loop, c->loop, sizeof(LoopState), cudaMemcpyDeviceToHost, c->st));
+    CK(cudaMemcpyAsync(c->h_err, c->err, sizeof(int), cudaMemcpyDeviceToHost, c->st));
+    CK(cudaStreamSynchronize(c->st));
+    if (*c->h_err) break;
+    bool any = false;
+    for (int k = 0; k < keys; ++k) any = any || c->h_loop->active[k];
+    if (!any) break;
+  }
+  for (int k = 0; k < keys; ++k) n_frames[k] = c->h_loop->count[k];
+  CKR(leave(c));
+  if (*c->h_err) return m3_sync_status(c);
+  for (int k = 0; k < keys; ++k)
+    if (n_frames[k] == 0) return fail(M3_EEMPTY, "key " + std::to_string(k) + " drew the end token at its first frame");
+  return M3_OK;
 }
 
 // ------------------------------------------------------------- the rest ----
@@ -967,7 +1138,7 @@ extern "C" int m3_embed(m3_ctx* c, int rows, const int32_t* codes, const void* t
   CKR(enter(c));
   CK(launch_ex(embed_kernel, dim3(rows), dim3(128), 0, c->st, false, codes,
                static_cast<const bf16*>(table), 0x7fffffff, offset, c->cfg.hidden,
-               static_cast<bf16*>(x_out), c->err));
+               static_cast<bf16*>(x_out), c->err, INT_MIN));
   return leave(c);
 }
 
@@ -978,10 +1149,10 @@ extern "C" double m3_frame_bytes(const m3_ctx* c, int rows, int ctx_len) {
   const double H = g.hidden, d = g.head_dim;
   const double per_layer = H * (g.n_q_heads + 2.0 * g.n_kv_heads) * d + H * g.n_q_heads * d +
                            3.0 * H * g.ffn;
-  double w = g.n_layers * per_layer * esz + (double)g.slice_len * H * esz;
+  double w = g.n_layers * per_layer * esz + (double)n_cand(g) * H * esz;
   if (c->wdtype == M3_W_INT8)
     w += 4.0 * (g.n_layers * ((g.n_q_heads + 2.0 * g.n_kv_heads) * d + H + 2.0 * g.ffn + H) +
-                g.slice_len);
+                n_cand(g));
   w += 2.0 * (g.n_layers * (2.0 * H + 2.0 * d) + H);  // norm gains
   const double kv = (double)rows * (ctx_len + 1.0) * g.n_layers * 2.0 * g.n_kv_heads * d * 2.0;
   return w + kv;
@@ -1021,10 +1192,12 @@ extern "C" int m3_time_gemv(m3_ctx* c, int which, int rows, int iters, float* av
         M = &c->lm;
         SampleArgs sa{};
         sa.logits = c->logits;
-        sa.logits_ld = g.slice_len;
+        sa.logits_ld = n_cand(g);
         sa.codes = c->codes;
         sa.code_stride = 1;
         sa.index_base = (unsigned long long)g.slice_start;
+        sa.end_row1 = g.has_end_token ? g.slice_len + 1 : 0;
+        sa.end_index = (unsigned long long)g.end_token;
         sa.part_z = c->spz;
         sa.part_i = c->spi;
         sa.counter = c->scnt;
@@ -1116,7 +1289,7 @@ extern "C" int m3_sample_noalloc(m3_ctx* c, int rows, const void* h, uint64_t se
     return fail(M3_EINVAL, "rows must be in 1..min(16, max_rows)");
   if (!(cfg_scale >= 0.0f) || !(temperature > 0.0f)) return fail(M3_EINVAL, "cfg_scale / temperature");
   if (cfg_scale > 0.0f && rows % 2) return fail(M3_EINVAL, "cfg_scale > 0 needs (cond, uncond) row pairs");
-  const int grid = g.slice_len < c->nsm ? g.slice_len : c->nsm;
+  const int grid = n_cand(g) < c->nsm ? n_cand(g) : c->nsm;
   if (grid > kNoAllocMaxCtas) return fail(M3_EINVAL, "more CTAs than the static scratch holds");
   CK(cudaSetDevice(c->dev));
   unsigned char* scratch = nullptr;
@@ -1136,10 +1309,12 @@ extern "C" int m3_sample_noalloc(m3_ctx* c, int rows, const void* h, uint64_t se
   CK(cudaMemsetAsync(counter, 0, sizeof(unsigned), c->st));  // the ticket starts at zero
   SampleArgs sa{};
   sa.logits = logits;
-  sa.logits_ld = g.slice_len;
+  sa.logits_ld = n_cand(g);
   sa.codes = codes;
   sa.code_stride = 1;
   sa.index_base = (unsigned long long)g.slice_start;
+  sa.end_row1 = g.has_end_token ? g.slice_len + 1 : 0;
+  sa.end_index = (unsigned long long)g.end_token;
   sa.part_z = reinterpret_cast<float*>(scratch + kNoAllocPartZOff);
   sa.part_i = reinterpret_cast<int*>(scratch + kNoAllocPartIOff);
   sa.counter = counter;

@@ -16,13 +16,16 @@ __global__ void set_frame_params_kernel(FrameParams* dst, FrameParams v) {
 }
 
 // The frame's RoPE rotations, (cos, sin) of pos[r] * inv_freq[i] (fp64,
-// then fp32), for rows r < v.rows and i < half: one table per frame instead
-// of the trigonometry in every attention CTA of every layer.
-__global__ void rope_table_kernel(FrameParams v, const double* __restrict__ inv_freq, int half,
-                                  float2* table) {
+// then fp32), for rows r < rows and i < half: one table per frame instead
+// of the trigonometry in every attention CTA of every layer.  The positions
+// are read from the frame's parameter block on the device, so a captured
+// loop of frames sees the positions the loop advanced.
+__global__ void rope_table_kernel(const FrameParams* __restrict__ fp,
+                                  const double* __restrict__ inv_freq, int half, float2* table) {
   const int r = blockIdx.x;
+  const int pos = fp->pos[r];
   for (int i = threadIdx.x; i < half; i += blockDim.x) {
-    const double ang = (double)v.pos[r] * inv_freq[i];
+    const double ang = (double)pos * inv_freq[i];
     table[(size_t)r * half + i] = make_float2((float)cos(ang), (float)sin(ang));
   }
 }
@@ -119,14 +122,19 @@ __global__ void tile_rows_kernel(const T* __restrict__ src, int rows, int K, uin
 
 // x_out[r] = table[offset + codes[r]] for r < rows; an out-of-range code
 // records kErrBounds and yields a zero row.
+// A code equal to zero_code (the end token's code, at the depth decoder's
+// first lookup) gives a zero row without an error.
 __global__ void embed_kernel(const int* __restrict__ codes, const __nv_bfloat16* __restrict__ table,
-                             int n_table, int offset, int H, __nv_bfloat16* x_out, int* err) {
+                             int n_table, int offset, int H, __nv_bfloat16* x_out, int* err,
+                             int zero_code) {
   const int r = blockIdx.x;
   pdl_launch_dependents();
   pdl_wait();
-  const int idx = offset + codes[r];
-  const bool ok = idx >= 0 && idx < n_table;
-  if (!ok && threadIdx.x == 0) record_error(err, kErrBounds);
+  const int code = codes[r];
+  const int idx = offset + code;
+  const bool zero = code == zero_code;
+  const bool ok = !zero && idx >= 0 && idx < n_table;
+  if (!ok && !zero && threadIdx.x == 0) record_error(err, kErrBounds);
   for (int k = threadIdx.x * 8; k < H; k += blockDim.x * 8) {
     uint4 v = make_uint4(0, 0, 0, 0);
     if (ok) v = *reinterpret_cast<const uint4*>(table + (size_t)idx * H + k);
@@ -179,6 +187,131 @@ __global__ void kv_get_kernel(uint16_t* k, uint16_t* v, const unsigned long long
     const int off = p % page_size;
     k[i] = base[kv_elem_offset(hh, page_size, off, D, d)];
     v[i] = base[kv_elem_offset(Hkv + hh, page_size, off, D, d)];
+  }
+}
+
+// ------------------------------------------------------ generation loop --
+// Device state of a generation loop ("第二阶段" of the DiffSynth-Studio
+// article: each frame's codes are embedded back as the next input until the
+// end token; "MiniMax Music 3 on Metal": position, step and count advance
+// on the GPU, the host reading the state every 16 frames).
+struct LoopState {
+  int step;               // frames run so far
+  int keys;               // CFG pairs, or rows without CFG
+  int active[kMaxRows];   // per key: still generating
+  int count[kMaxRows];    // per key: frames generated before the end token
+  int* codes_out;         // [max_frames][rows][1 + nc], filled with -1 beforehand
+  __nv_bfloat16* h_hist;  // nullable: [max_frames][rows][H]
+};
+
+struct LoopArgs {
+  FrameParams* fp;
+  LoopState* ls;
+  const int* codes;                 // [rows] this frame's semantic code
+  const int* dcodes;                // [rows][nc] its residual codes
+  const __nv_bfloat16* h;           // [rows][H] its final-normed hidden state
+  const __nv_bfloat16* tok;         // [S][H] token embeddings of the code block
+  const __nv_bfloat16* const* aud;  // nc audio-embedding tables [V][H]
+  __nv_bfloat16* x;                 // [rows][H] the next frame's input
+  int* err;
+  int nc, V, H, S, has_end;
+  float scale;                      // (1 + nc)^-0.5
+};
+
+__global__ void loop_init_kernel(LoopState* dst, LoopState v) {
+  if (threadIdx.x == 0) *dst = v;
+}
+
+// One CTA per row.  For a row whose key still runs: record the frame (its
+// codes, the residual ones -1 on the end frame, and its hidden state) at
+// index step.  Then the next input: bf16(scale * (tok[c0] + aud[0][c1] + ...
+// + aud[nc-1][c_nc])) with the sum in fp32 in that order, or zeros for a key
+// that has stopped (now or before).
+__global__ void loop_feedback_kernel(LoopArgs a) {
+  __shared__ int cs[32];
+  __shared__ int feed_s;
+  const int r = blockIdx.x;
+  const int rows = a.fp->rows;
+  const int key = a.fp->cfg_on ? r / 2 : r;
+  const LoopState* ls = a.ls;
+  const int step = ls->step;
+  const bool act = ls->active[key] != 0;
+  const int c0 = a.codes[r];
+  const bool ends = a.has_end && c0 == a.S;
+  const int W = 1 + a.nc;
+  if (threadIdx.x == 0) {
+    cs[0] = c0;
+    for (int j = 0; j < a.nc; ++j) cs[1 + j] = a.dcodes[r * a.nc + j];
+    if (act) {
+      int* out = ls->codes_out + ((size_t)step * rows + r) * W;
+      out[0] = c0;
+      for (int j = 0; j < a.nc; ++j) out[1 + j] = ends ? -1 : cs[1 + j];
+    }
+    bool feed = act && !ends;
+    if (feed) {  // the codes fed forward must index the tables
+      bool ok = c0 >= 0 && c0 < a.S;
+      for (int j = 0; j < a.nc; ++j) ok = ok && cs[1 + j] >= 0 && cs[1 + j] < a.V;
+      if (!ok) record_error(a.err, kErrBounds);
+      feed = ok;
+    }
+    feed_s = feed;
+  }
+  if (act && ls->h_hist) {
+    const uint4* src = reinterpret_cast<const uint4*>(a.h + (size_t)r * a.H);
+    uint4* dst = reinterpret_cast<uint4*>(ls->h_hist + ((size_t)step * rows + r) * a.H);
+    for (int k = threadIdx.x; k < a.H / 8; k += blockDim.x) dst[k] = src[k];
+  }
+  __syncthreads();
+  const bool feed = feed_s != 0;
+  for (int k = threadIdx.x * 8; k < a.H; k += blockDim.x * 8) {
+    uint4 o = make_uint4(0u, 0u, 0u, 0u);
+    if (feed) {
+      float t[8];
+      const uint4 e = *reinterpret_cast<const uint4*>(a.tok + (size_t)cs[0] * a.H + k);
+      const uint32_t ew[4] = {e.x, e.y, e.z, e.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        t[2 * q] = __uint_as_float(ew[q] << 16);
+        t[2 * q + 1] = __uint_as_float(ew[q] & 0xFFFF0000u);
+      }
+      for (int j = 0; j < a.nc; ++j) {
+        const uint4 v = *reinterpret_cast<const uint4*>(a.aud[j] + (size_t)cs[1 + j] * a.H + k);
+        const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          t[2 * q] = __fadd_rn(t[2 * q], __uint_as_float(vw[q] << 16));
+          t[2 * q + 1] = __fadd_rn(t[2 * q + 1], __uint_as_float(vw[q] & 0xFFFF0000u));
+        }
+      }
+      uint32_t ow[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(t[2 * q], a.scale)));
+        const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(t[2 * q + 1], a.scale)));
+        ow[q] = lo | (hi << 16);
+      }
+      o = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+    }
+    *reinterpret_cast<uint4*>(a.x + (size_t)r * a.H + k) = o;
+  }
+}
+
+// One warp: the stop rule and the counts per key, then the next frame's
+// positions, noise frame and step.
+__global__ void loop_advance_kernel(LoopArgs a) {
+  FrameParams* fp = a.fp;
+  LoopState* ls = a.ls;
+  const int t = threadIdx.x;
+  if (t < ls->keys && ls->active[t]) {
+    const int r = fp->cfg_on ? 2 * t : t;
+    if (a.has_end && a.codes[r] == a.S) ls->active[t] = 0;
+    else ls->count[t] += 1;
+  }
+  if (t < fp->rows) fp->pos[t] += 1;
+  __syncwarp();
+  if (t == 0) {
+    ls->step += 1;
+    fp->frame += 1ull;
   }
 }
 

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libm3.so")
 
 M3_OK, M3_EINVAL, M3_ENOMEM, M3_ECUDA, M3_ESTATE, M3_ECAPACITY, M3_ETIMEOUT, M3_EDEVICE = \
     0, -1, -2, -3, -4, -5, -6, -7
+M3_EEMPTY = -8
 M3_W_BF16, M3_W_INT8 = 0, 1
 M3_KV_BF16, M3_KV_F16 = 0, 1
 M3_MEM_HOST, M3_MEM_DEVICE = 0, 1
@@ -25,7 +26,7 @@ M3_MEM_HOST, M3_MEM_DEVICE = 0, 1
 EXPORTED = ("m3_create", "m3_load_weights", "m3_load_depth_weights", "m3_kv_alloc", "m3_kv_set",
             "m3_kv_get", "m3_decode_frame", "m3_depth_decode", "m3_embed", "m3_quantize_int8",
             "m3_export_weight", "m3_frame_bytes", "m3_time_gemv", "m3_sample_noalloc", "m3_set_top_k",
-            "m3_sync_status",
+            "m3_load_feedback", "m3_generate", "m3_sync_status",
             "m3_last_error", "m3_destroy")
 
 
@@ -43,7 +44,8 @@ class m3_config(C.Structure):
                 ("depth_layers", C.c_int), ("depth_hidden", C.c_int), ("depth_heads", C.c_int),
                 ("depth_head_dim", C.c_int), ("depth_ffn", C.c_int),
                 ("depth_codebooks", C.c_int), ("depth_vocab", C.c_int),
-                ("depth_rope_theta", C.c_double)]
+                ("depth_rope_theta", C.c_double), ("has_end_token", C.c_int),
+                ("end_token", C.c_int)]
 
 
 LAYER_FIELDS = ("attn_norm", "wq", "wk", "wv", "q_norm", "k_norm", "wo", "mlp_norm", "wg",
@@ -57,7 +59,7 @@ class m3_layer_src(C.Structure):
 class m3_weight_src(C.Structure):
     _fields_ = [("first_layer", C.c_int), ("n_layers", C.c_int),
                 ("layers", C.POINTER(m3_layer_src)), ("final_norm", C.c_void_p),
-                ("lm_head", C.c_void_p), ("mem", C.c_int)]
+                ("lm_head", C.c_void_p), ("mem", C.c_int), ("lm_end_row", C.c_void_p)]
 
 
 class m3_depth_src(C.Structure):
@@ -88,6 +90,8 @@ def load_library() -> C.CDLL:
     L.m3_frame_bytes.restype = C.c_double
     L.m3_time_gemv.argtypes = [vp, i32, i32, i32, C.POINTER(C.c_float), C.POINTER(C.c_double)]
     L.m3_sample_noalloc.argtypes = [vp, i32, vp, u64, u64, f32, f32, vp, vp]
+    L.m3_load_feedback.argtypes = [vp, vp, C.POINTER(vp), i32]
+    L.m3_generate.argtypes = [vp, i32, vp, u64, u64, vp, f32, f32, i32, vp, vp, vp]
     L.m3_sync_status.argtypes = [vp]
     L.m3_last_error.restype = C.c_char_p
     L.m3_destroy.argtypes = [vp]
@@ -139,22 +143,24 @@ def _layer_src(t: dict, keep: list) -> m3_layer_src:
 
 
 def m3_load_weights(ctx: int, layers: list, first_layer: int = 0, final_norm=None, lm_head=None,
-                    wdtype: int = M3_W_BF16) -> None:
-    """layers: list of dicts of bf16 tensors (all on the host or all on the GPU)."""
+                    wdtype: int = M3_W_BF16, lm_end_row=None) -> None:
+    """layers: list of dicts of bf16 tensors (all on the host or all on the GPU);
+    lm_end_row: the end token's lm_head row [H] when the config has one."""
     keep = []
     arr = (m3_layer_src * max(1, len(layers)))()
     dev = None
     for i, t in enumerate(layers):
         arr[i] = _layer_src(t, keep)
         dev = t["wq"].is_cuda
-    for t in (final_norm, lm_head):
+    for t in (final_norm, lm_head, lm_end_row):
         if t is not None:
             keep.append(t.contiguous())
             dev = t.is_cuda if dev is None else dev
     src = m3_weight_src(first_layer, len(layers), arr,
                         _ptr(final_norm.contiguous()) if final_norm is not None else None,
                         _ptr(lm_head.contiguous()) if lm_head is not None else None,
-                        M3_MEM_DEVICE if dev else M3_MEM_HOST)
+                        M3_MEM_DEVICE if dev else M3_MEM_HOST,
+                        _ptr(lm_end_row.contiguous()) if lm_end_row is not None else None)
     if final_norm is not None:
         keep.append(final_norm)
     _check(lib.m3_load_weights(ctx, C.byref(src), wdtype))
@@ -262,6 +268,33 @@ def m3_set_top_k(ctx: int, top_k: int) -> None:
     _check(lib.m3_set_top_k(ctx, top_k))
 
 
+def m3_load_feedback(ctx: int, tok_emb: torch.Tensor, audio_emb=None) -> None:
+    """The generation loop's feedback tables (see m3.h): tok_emb [slice_len, H]
+    and the residual codebooks' audio_emb tables [depth_vocab, H], bf16."""
+    keep = [tok_emb.contiguous()] + [a.contiguous() for a in (audio_emb or [])]
+    arr = (C.c_void_p * max(1, len(keep) - 1))(*[t.data_ptr() for t in keep[1:]])
+    _check(lib.m3_load_feedback(ctx, keep[0].data_ptr(), arr if audio_emb else None,
+                                M3_MEM_DEVICE if tok_emb.is_cuda else M3_MEM_HOST))
+
+
+def m3_generate(ctx: int, positions, seed: int, frame0: int, x_in: torch.Tensor,
+                cfg_scale: float, temperature: float, max_frames: int, codes: torch.Tensor,
+                h_hist: torch.Tensor | None = None):
+    """The GPU generation loop (see m3.h).  codes: int32 [max_frames, rows, 1 + NC]
+    on the GPU.  Returns (status, n_frames per key): status is M3_OK or M3_EEMPTY;
+    any other status raises."""
+    rows = x_in.shape[0]
+    keys = rows // 2 if cfg_scale > 0 else rows
+    pos = (C.c_int32 * rows)(*[int(p) for p in positions])
+    nf = (C.c_int32 * keys)()
+    rc = lib.m3_generate(ctx, rows, C.cast(pos, C.c_void_p), seed, frame0, _ptr(x_in), cfg_scale,
+                         temperature, max_frames, _ptr(codes), _ptr(h_hist),
+                         C.cast(nf, C.c_void_p))
+    if rc not in (M3_OK, M3_EEMPTY):
+        _check(rc)
+    return rc, [int(v) for v in nf]
+
+
 def m3_sync_status(ctx: int) -> None:
     _check(lib.m3_sync_status(ctx))
 
@@ -277,6 +310,8 @@ def config_from_shapes(body, depth=None, max_rows: int = 2) -> m3_config:
                                                     body.head_dim, body.ffn)
     c.vocab, c.slice_start, c.slice_len = body.vocab, body.slice_start, body.slice_len
     c.rope_theta, c.rms_eps, c.max_rows = body.rope_theta, body.rms_eps, max_rows
+    end = getattr(body, "end_token", -1)
+    c.has_end_token, c.end_token = (1, end) if end >= 0 else (0, 0)
     if depth is not None:
         c.depth_layers, c.depth_hidden, c.depth_heads = depth.n_layers, depth.hidden, depth.n_heads
         c.depth_head_dim, c.depth_ffn = depth.head_dim, depth.ffn

@@ -65,7 +65,9 @@ typedef enum {
   M3_ESTATE = -4,     /* call out of order (no weights, no KV cache ...)  */
   M3_ECAPACITY = -5,  /* a position is outside the KV cache capacity      */
   M3_ETIMEOUT = -6,   /* a bounded device-side wait gave up               */
-  M3_EDEVICE = -7     /* a kernel recorded an error word on the device    */
+  M3_EDEVICE = -7,    /* a kernel recorded an error word on the device    */
+  M3_EEMPTY = -8      /* m3_generate: a key drew the end token at its first
+                         frame, so nothing was generated for it           */
 } m3_status;
 
 enum { M3_W_BF16 = 0, M3_W_INT8 = 1 };   /* weight storage of the body + lm_head */
@@ -94,6 +96,8 @@ typedef struct {
   int depth_codebooks; /* 7 residual codebooks                                */
   int depth_vocab;     /* 1024 entries per residual codebook                  */
   double depth_rope_theta;
+  int has_end_token;   /* 1: the end token is sampleable besides the code block */
+  int end_token;       /* its vocab row, e.g. 151670 (outside the slice)        */
 } m3_config;
 
 /* One decoder layer's source tensors, bf16, row-major [out, in]. */
@@ -113,14 +117,17 @@ typedef struct {
 
 /* Body weights.  layers[i] goes to layer first_layer + i, so a caller can
  * load a model layer by layer.  final_norm [H] and lm_head [slice_len, H]
- * (rows slice_start.. of the full lm_head) may be null to skip them. */
+ * (rows slice_start.. of the full lm_head) may be null to skip them; with
+ * cfg.has_end_token, lm_end_row [H] (row end_token of the full lm_head) must
+ * come with lm_head. */
 typedef struct {
   int first_layer;
   int n_layers;
   const m3_layer_src* layers;
   const void* final_norm;
   const void* lm_head;
-  int mem; /* M3_MEM_HOST or M3_MEM_DEVICE for every pointer above */
+  int mem; /* M3_MEM_HOST or M3_MEM_DEVICE for every pointer here */
+  const void* lm_end_row;
 } m3_weight_src;
 
 /* Depth-decoder weights, bf16 (quantised to int8, one scale per group of
@@ -167,12 +174,20 @@ M3_API int m3_kv_set(m3_ctx* ctx, int row, int n_positions, const void* k, const
  * raw cache-type bits (bf16 or f16).  Synchronises the stream. */
 M3_API int m3_kv_get(m3_ctx* ctx, int row, int n_positions, void* k_host, void* v_host);
 
+/* The end token.  With cfg.has_end_token the draw of m3_decode_frame chooses
+ * among slice_len + 1 candidates: the code block and, as slice-relative code
+ * slice_len, the end token (noise index end_token); the vocabulary mask of
+ * "第二阶段" in the DiffSynth-Studio article, which leaves the audio codes and
+ * the end token sampleable.  Ties between the end token and a code go to the
+ * code.  Logit buffers are then slice_len + 1 wide. */
+
 /* Top-k filter of the frame draw (the AR sampler's "CFG 1.5, top-k 50,
  * multinomial", DiffSynth-Studio article, "第二阶段"): m3_decode_frame keeps
  * the top_k largest guided logits per key -- ties at the k-th value going to
  * the lower index -- and draws among them by Gumbel-argmax.  0 (the default)
  * or top_k >= slice_len keeps every logit.  Applies to the calls that follow;
- * the depth decoder and m3_sample_noalloc always keep every logit.
+ * the depth decoder and m3_sample_noalloc always keep every logit; the
+ * generation loop (m3_generate) keeps the setting.
  * Returns M3_EINVAL for top_k < 0. */
 M3_API int m3_set_top_k(m3_ctx* ctx, int top_k);
 
@@ -187,9 +202,11 @@ M3_API int m3_set_top_k(m3_ctx* ctx, int top_k);
  *    with noise row key = pair index, and both rows receive the code.
  *    cfg_scale == 0: each row draws from its own logits, row key = row.
  *  temperature > 0: z_i = g_i / temperature + Gumbel(seed, frame, key, slice_start + i).
- *  codes (dev int32 [rows]): slice-relative code (0..slice_len-1).
+ *  codes (dev int32 [rows]): slice-relative code (0..slice_len-1; slice_len
+ *    is the end token when the config has one).
  *  h_out (dev bf16 [rows, H], nullable): final-normed hidden state.
- *  logits (dev fp32 [rows, slice_len], nullable): raw per-row logits.
+ *  logits (dev fp32 [rows, slice_len (+1 with the end token)], nullable):
+ *    raw per-row logits.
  * The whole frame runs as one CUDA graph per (rows, KV bucket count),
  * captured on first use.  May allocate a new KV bucket (synchronising). */
 M3_API int m3_decode_frame(m3_ctx* ctx, int rows, const int32_t* positions, uint64_t seed,
@@ -200,7 +217,8 @@ M3_API int m3_decode_frame(m3_ctx* ctx, int rows, const int32_t* positions, uint
  *  h_frame (dev bf16 [rows, H]): the frame's final-normed hidden state
  *    (m3_decode_frame's h_out), projected to depth_hidden at position 0;
  *  code0 (dev int32 [rows]): the frame's semantic code (slice-relative),
- *    embedded with emb[0] at position 1;
+ *    embedded with emb[0] at position 1 (the end token's code, slice_len,
+ *    gives a zero vector there);
  *  position j (1..7) yields codebook j's logits from heads[j-1], drawn with
  *    noise index (j << 32) | i, and E_j[code_j] is the input of position j+1;
  *  forced (dev int32 [rows, codebooks], nullable): teacher forcing -- feed
@@ -211,6 +229,46 @@ M3_API int m3_decode_frame(m3_ctx* ctx, int rows, const int32_t* positions, uint
 M3_API int m3_depth_decode(m3_ctx* ctx, int rows, const void* h_frame, const int32_t* code0,
                     uint64_t seed, uint64_t frame, float cfg_scale, float temperature,
                     const int32_t* forced, int32_t* codes, float* logits);
+
+/* Tables of the generation loop's feedback embedding (the DiffSynth-Studio
+ * article's embed_audio_frame, "第二阶段"), copied into library memory:
+ *  tok_emb [slice_len, H] bf16: embed_tokens rows slice_start.. (the code
+ *    block's token embeddings);
+ *  audio_emb: depth_codebooks tables [depth_vocab, H] bf16, the residual
+ *    codebooks' audio embeddings; null when the config has no depth decoder.
+ * Returns M3_EINVAL for a null table the config needs. */
+M3_API int m3_load_feedback(m3_ctx* ctx, const void* tok_emb, const void* const* audio_emb,
+                            int mem);
+
+/* The autoregressive generation loop on the GPU: frame f = 0, 1, ... runs
+ * every row at position positions[r] + f with noise frame frame0 + f, as
+ * m3_decode_frame; with the depth decoder loaded, m3_depth_decode follows on
+ * the frame's hidden state and code.  The next frame's input is, per row,
+ *   x = bf16((tok_emb[c0] + audio_emb[0][c1] + ... + audio_emb[NC-1][cNC]) * (1 + NC)^-0.5)
+ * (fp32 sum in that order; NC = depth_codebooks, or 0 without the depth
+ * decoder: x = tok_emb[c0]; the article's 8^-0.5 for its 8 codebooks).
+ * A key (a CFG pair, or a row without CFG) stops at the first frame whose
+ * code is the end token (slice_len; needs cfg.has_end_token); its count is
+ * the frames before that one.  Positions, the noise frame, the step and the
+ * counts advance on the GPU; the host reads the loop state every 16 frames
+ * and stops once every key has stopped, or after max_frames.  Rows of a
+ * stopped key keep being computed, on a zero input.
+ *  positions (HOST, [rows]): each row's first position; positions[r] +
+ *    max_frames must be <= max_positions, else M3_ECAPACITY before any launch.
+ *  x_in (dev bf16 [rows, H]): the first frame's input.
+ *  cfg_scale, temperature: as in m3_decode_frame; the top-k setting applies.
+ *  codes (dev int32 [max_frames, rows, 1 + NC]): per frame and row the semantic
+ *    code and the residual codes while the row's key runs; on its end frame
+ *    the semantic code is slice_len and the residual entries -1; -1 after.
+ *  h_hist (dev bf16 [max_frames, rows, H], nullable): each frame's
+ *    final-normed hidden state while the row's key runs; zeros after.
+ *  n_frames (HOST int32 [keys]): frames generated per key.
+ * Synchronises the stream (every 16 frames and at the end).  Returns
+ * M3_EEMPTY, with every output written, when some key drew the end token at
+ * its first frame; a device-side error as m3_sync_status reports it. */
+M3_API int m3_generate(m3_ctx* ctx, int rows, const int32_t* positions, uint64_t seed,
+                       uint64_t frame0, const void* x_in, float cfg_scale, float temperature,
+                       int max_frames, int32_t* codes, void* h_hist, int32_t* n_frames);
 
 /* Frame feedback by table lookup: x_out[r] = table[offset + codes[r]].
  * table (dev bf16 [n, H]), codes (dev int32 [rows]), x_out (dev bf16 [rows, H]). */

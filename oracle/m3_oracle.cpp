@@ -708,7 +708,10 @@ int ora_depth_decode(const OraDepth* D, int rows, const bf16_t* h_frame, const i
 //   tok_emb [slice_len, H] bf16: embed_tokens rows slice_start..;
 //   audio_emb: NC tables [D->vocab, H] bf16 (unused without D);
 //   forced (nullable) [max_frames, rows, 1 + NC]: teacher forcing -- these
-//     codes are fed forward (and stopped on) instead of the drawn ones;
+//     codes are fed forward (and stopped on) instead of the drawn ones; a
+//     negative entry (as in this loop's own -1 fill) stands for the drawn
+//     semantic code, or for residual code 0 (only ever read for rows whose
+//     output is not recorded);
 //   codes_out [max_frames, rows, 1 + NC]: the drawn code0 and residual codes
 //     of every frame a row's key runs; on its end frame the residual entries
 //     are -1; -1 everywhere after that;
@@ -749,10 +752,12 @@ int ora_generate(const OraCfg* cfg, const OraLayer* layers, const bf16_t* final_
                               code0.data(), hf.data(), nullptr);
     if (rc) return rc;
     const int32_t* fr = forced ? forced + (size_t)f * rows * W : nullptr;
-    for (int r = 0; r < rows; ++r) c0[r] = fr ? fr[(size_t)r * W] : code0[r];
+    for (int r = 0; r < rows; ++r)
+      c0[r] = fr && fr[(size_t)r * W] >= 0 ? fr[(size_t)r * W] : code0[r];
     if (NC) {
       for (int r = 0; r < rows; ++r)
-        for (int j = 0; j < NC; ++j) fz[(size_t)r * NC + j] = fr ? fr[(size_t)r * W + 1 + j] : 0;
+        for (int j = 0; j < NC; ++j)
+          fz[(size_t)r * NC + j] = fr && fr[(size_t)r * W + 1 + j] > 0 ? fr[(size_t)r * W + 1 + j] : 0;
       rc = ora_depth_decode(D, rows, hf.data(), c0.data(), seed, frame, cfg_scale, temperature,
                             fr ? fz.data() : nullptr, dcodes.data(), nullptr);
       if (rc) return rc;

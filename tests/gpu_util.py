@@ -26,7 +26,7 @@ class Model:
     """Body weights drawn once; handed to the library and to the oracle."""
 
     def __init__(self, shape, seed=0, device="cpu", wdtype=0, kv_f16=False, max_rows=2,
-                 depth=None, depth_seed=None, layers=None, oracle=True):
+                 depth=None, depth_seed=None, layers=None, oracle=True, end_row=None):
         from autoregressive_audio_token_b200 import m3
         self.m3 = m3
         self.shape = shape
@@ -34,6 +34,10 @@ class Model:
             [synth.layer_weights(shape, seed, l, device=device) for l in range(shape.n_layers)]
         self.final_norm = synth.final_norm(shape, seed, device=device)
         self.lm = synth.lm_head_slice(shape, seed, device=device)
+        self.has_end = getattr(shape, "end_token", -1) >= 0
+        self.n_cand = shape.slice_len + (1 if self.has_end else 0)
+        self.lm_end = (end_row if end_row is not None else
+                       synth.lm_head_end_row(shape, seed, device=device)) if self.has_end else None
         self.wdtype = wdtype
         self.kv_f16 = kv_f16
         self.depth_shape = depth
@@ -43,7 +47,8 @@ class Model:
         self.ctx = m3.m3_create(cfg)
         m3.m3_load_weights(self.ctx, [{k: v.cuda() for k, v in L.items()} for L in self.layers]
                            if device == "cpu" else self.layers, 0, self.final_norm.cuda(),
-                           self.lm.cuda(), wdtype=wdtype)
+                           self.lm.cuda(), wdtype=wdtype,
+                           lm_end_row=self.lm_end.cuda() if self.has_end else None)
         if self.dw is not None:
             dwc = {"layers": [{k: v.cuda() for k, v in L.items()} for L in self.dw["layers"]],
                    "proj": self.dw["proj"].cuda(), "emb": [e.cuda() for e in self.dw["emb"]],
@@ -55,7 +60,8 @@ class Model:
             from oracle import oracle as O
             self.ora = O.Body(shape, [{k: v.cpu() for k, v in L.items()} for L in self.layers],
                               self.final_norm.cpu(), self.lm.cpu(), wfmt=1 if wdtype else 0,
-                              kv_f16=kv_f16)
+                              kv_f16=kv_f16,
+                              lm_end_row=self.lm_end.cpu() if self.has_end else None)
             self.ora_depth = O.Depth(depth, {"layers": [{k: v.cpu() for k, v in L.items()}
                                                         for L in self.dw["layers"]],
                                              "proj": self.dw["proj"].cpu(),
@@ -93,7 +99,7 @@ class Model:
         s = self.shape
         codes = torch.empty(rows, dtype=torch.int32, device="cuda")
         h = torch.empty((rows, s.hidden), dtype=torch.bfloat16, device="cuda")
-        lg = torch.empty((rows, s.slice_len), dtype=torch.float32, device="cuda")
+        lg = torch.empty((rows, self.n_cand), dtype=torch.float32, device="cuda")
         self.m3.m3_decode_frame(self.ctx, positions, seed, frame, x_in.cuda().contiguous(),
                                 cfg_scale, temperature, codes, h, lg)
         torch.cuda.synchronize()
