@@ -53,6 +53,9 @@ def parse():
                         "configs do)")
     p.add_argument("--depth", action="store_true",
                    help="run the RVQ depth decoder (7 codes) after every frame")
+    p.add_argument("--generate", type=int, default=0, metavar="F",
+                   help="time the GPU generation loop (m3_generate) over F frames of a song "
+                        "after a 300-position prompt, against host-driven m3_decode_frame")
     p.add_argument("--sweep", action="store_true",
                    help="batched-variations sweep: rows 1..16 x context 1500/4500/9000, "
                         "bf16 and int8; one JSON line per point")
@@ -197,9 +200,9 @@ class ClockSampler:
 # ------------------------------------------------------------ our arm ------
 
 def build_model(torch, m3, synth, seed: int, wdtype: int, layers: int = 36, depth: bool = False,
-                max_rows: int = ROWS):
+                max_rows: int = ROWS, end_token: bool = False):
     import dataclasses
-    s = dataclasses.replace(synth.FULL8B, n_layers=layers)
+    s = dataclasses.replace(synth.FULL8B_END if end_token else synth.FULL8B, n_layers=layers)
     cfg = m3.config_from_shapes(s, synth.DEPTH if depth else None, max_rows=max_rows)
     ctx = m3.m3_create(cfg)
     for l in range(s.n_layers):  # generate on the GPU, load layer by layer
@@ -207,7 +210,9 @@ def build_model(torch, m3, synth, seed: int, wdtype: int, layers: int = 36, dept
         m3.m3_load_weights(ctx, [Lw], first_layer=l, wdtype=wdtype)
         del Lw
     m3.m3_load_weights(ctx, [], final_norm=synth.final_norm(s, 0, device="cuda"),
-                       lm_head=synth.lm_head_slice(s, 0, device="cuda"), wdtype=wdtype)
+                       lm_head=synth.lm_head_slice(s, 0, device="cuda"), wdtype=wdtype,
+                       lm_end_row=synth.lm_head_end_row(s, 0, device="cuda") if end_token
+                       else None)
     if depth:
         m3.m3_load_depth_weights(ctx, synth.depth_weights(synth.DEPTH, 0, device="cuda"))
     torch.cuda.synchronize()
@@ -508,9 +513,90 @@ def run_sweep(args):
         torch.cuda.empty_cache()
 
 
+def run_generate(args):
+    """The GPU generation loop over a whole song on the full 8B: F frames from
+    position 300 (a prompt's worth of N(0,1) KV), 2 rows (one CFG pair), the
+    end token sampleable, feedback through the token and audio embeddings.
+    Timed with CUDA events around one m3_generate call (graphs captured by
+    an untimed run first), and against the same frames driven from the host
+    one m3_decode_frame (+ m3_depth_decode) call at a time."""
+    import torch
+    from autoregressive_audio_token_b200 import m3
+    import synth
+    torch.cuda.set_device(0)
+    F, P = args.generate, 300
+    wdtype = m3.M3_W_INT8 if args.wdtype == "int8" else m3.M3_W_BF16
+    s, ctx = build_model(torch, m3, synth, 0, wdtype, args.layers, depth=args.depth,
+                         end_token=True)
+    m3.m3_set_top_k(ctx, args.top_k)
+    nc = synth.DEPTH.codebooks if args.depth else 0
+    m3.m3_load_feedback(ctx, synth.embedding_slice(s, 0, device="cuda"),
+                        synth.audio_embeddings(synth.DEPTH, s.hidden, 0, device="cuda")
+                        if args.depth else None)
+    prefill_kv(torch, m3, synth, s, ctx, ROWS, P + F + 1, 0, args.kv == "f16")
+    x0 = synth.normal((ROWS, s.hidden), 0, "bench/x0", std=0.02, device="cuda")
+    codes = torch.empty((F, ROWS, 1 + nc), dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+    m3.m3_generate(ctx, [P] * ROWS, 1, 0, x0, CFG_SCALE, 1.0, F, codes)  # capture, warm
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0, "/tmp/m3_clocks_gen.csv")
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    rc, nf = m3.m3_generate(ctx, [P] * ROWS, 1, 0, x0, CFG_SCALE, 1.0, F, codes)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    m3.m3_sync_status(ctx)
+    ms = e0.elapsed_time(e1)
+    # frames the loop ran: all F, or up to the 16-frame read after the end
+    ran = F if nf[0] >= F else min(F, 16 * ((nf[0] + 1 + 15) // 16))
+    # the same frames driven from the host, one call per frame
+    xs = torch.empty((ROWS, s.hidden), dtype=torch.bfloat16, device="cuda")
+    c1 = torch.empty(ROWS, dtype=torch.int32, device="cuda")
+    h1 = torch.empty((ROWS, s.hidden), dtype=torch.bfloat16, device="cuda")
+    d1 = torch.empty((ROWS, max(nc, 1)), dtype=torch.int32, device="cuda")
+    xs.copy_(x0)
+
+    def host_frame(i):
+        m3.m3_decode_frame(ctx, [P + i] * ROWS, 1, i, xs, CFG_SCALE, 1.0, c1, h1)
+        if nc:
+            m3.m3_depth_decode(ctx, h1, c1, 1, i, CFG_SCALE, 1.0, d1)
+
+    for i in range(3):
+        host_frame(i)
+    torch.cuda.synchronize()
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for i in range(ran):
+        host_frame(i)
+    e3.record(stream)
+    torch.cuda.synchronize()
+    m3.m3_sync_status(ctx)
+    ms_host = e2.elapsed_time(e3)
+    mean_ctx = P + (ran - 1) / 2.0
+    fb = m3.m3_frame_bytes(ctx, ROWS, int(round(mean_ctx)))
+    name = workload_name(args).replace("song1500", f"generate{F}-prompt{P}") + "-end"
+    print(json.dumps({
+        "metric": "AR frames/s per row, GPU generation loop (8B, 2 rows)",
+        "value": 1000.0 * ran / ms, "unit": "frames/s", "n_gpus": 1, "higher_is_better": True,
+        "ms_per_frame": ms / ran, "dtype": args.wdtype, "data": "synthetic",
+        "config": {"workload": name, "frames": F, "prompt_positions": P, "rows": ROWS,
+                   "cfg_scale": CFG_SCALE, "top_k": args.top_k, "depth_decoder": bool(nc),
+                   "status": rc, "n_frames": nf, "frames_run": ran},
+        "frame_bytes_mean_ctx": fb, "achieved_gbs": fb / (ms / ran) / 1e6,
+        "host_driven": {"ms_per_frame": ms_host / ran, "frames_per_s": 1000.0 * ran / ms_host},
+        "clocks": clk}))
+    m3.m3_destroy(ctx)
+
+
 def main():
     args = parse()
     rank, world, local = dist_env()
+    if args.generate:
+        if rank == 0:
+            run_generate(args)
+        return
     if args.sweep:
         if rank == 0:
             run_sweep(args)
