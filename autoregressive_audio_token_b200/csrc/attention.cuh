@@ -57,6 +57,10 @@ struct AttnArgs {
   const FrameParams* fp;
   int fixed_pos;              // >= 0: every row is at this position (depth decoder)
   int* err;
+  // L2 prefetch of the weights the next kernels stream (HBM is nearly idle
+  // while attention runs): up to two byte ranges, split evenly over the CTAs
+  const uint8_t* pf[2];
+  size_t pf_bytes[2];
 };
 
 template <int D>
@@ -185,6 +189,17 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const Attn
     for (int b = 0; b < kAttnBuf; ++b) mbar_init(&bars[b], 1);
     fence_barrier_init();
     for (int t = 0; t < min(kAttnBuf, ntiles); ++t) issue_tile(t);
+  } else if (tid == 32) {
+    const size_t nb = (size_t)gridDim.x * gridDim.y * gridDim.z;
+    const size_t b = ((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      if (!a.pf_bytes[q]) continue;
+      const size_t per = (a.pf_bytes[q] / nb + 255) & ~(size_t)255;
+      const size_t lo = b * per, hi = min(lo + per, a.pf_bytes[q]);
+      for (size_t o = lo; o < hi; o += 65536)
+        bulk_prefetch_l2(a.pf[q] + o, (uint32_t)min((size_t)65536, hi - o));
+    }
   }
   __syncthreads();
   pdl_launch_dependents();

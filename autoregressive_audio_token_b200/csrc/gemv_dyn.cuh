@@ -110,32 +110,54 @@ __global__ void __maxnreg__(128) gemv_dyn_kernel(const GemvArgs a) {
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
       const uint8_t* wb = static_cast<const uint8_t*>(a.w);
-      int s = 0;
-      bool ok = true;
-      int u = (int)atomicAdd(claim, 1u);
-      while (ok) {
-        const int un = u < U ? (int)atomicAdd(claim, 1u) : U;  // one unit ahead
-        const int nparts = u < U ? ppr : 1;                     // the end tag takes a stage
-        for (int p = 0; p < nparts; ++p, ++s) {
-          const int slot = s % ns;
-          if (s >= ns && !mbar_wait(&empty[slot], ((s / ns) - 1) & 1, a.err)) {
-            ok = false;
-            break;
-          }
-          if (u >= U) {
-            tag[slot] = -1;
-            mbar_arrive(&full[slot]);
-            ok = false;
-            break;
-          }
-          const int t0 = p * pt, t1 = min(T, t0 + pt);
-          const uint32_t bytes = (uint32_t)((t1 - t0) * TB);
-          tag[slot] = u * ppr + p;
-          mbar_arrive_expect_tx(&full[slot], bytes);
-          bulk_g2s(ring + (size_t)slot * D.stage, wb + ((size_t)u * T + t0) * TB, bytes,
-                   &full[slot], pol);
+      const int pfa = a.pfa < ppr ? a.pfa : ppr;  // at most into the next unit
+      // Before the consumers run, a CTA claims only its first unit: claiming
+      // ahead that early would let the CTAs that launch first take two units
+      // each before the others start, which unbalances launches of about two
+      // units per CTA.  Once a slot has come back (the consumers run), the
+      // next unit is claimed as soon as the current one starts.
+      int u = (int)atomicAdd(claim, 1u);  // the unit being loaded; -1: take the next
+      int un = -1;                         // the next unit, once claimed
+      int p = 0;                           // next part of u
+      bool started = false;                // a slot has come back
+      for (int s = 0;; ++s) {
+        const int slot = s % ns;
+        if (s >= ns) {
+          if (!mbar_wait(&empty[slot], ((s / ns) - 1) & 1, a.err)) break;
+          started = true;
         }
-        u = un;
+        if (u < 0) {
+          u = un >= 0 ? un : (int)atomicAdd(claim, 1u);
+          un = -1;
+          p = 0;
+        }
+        if ((started || !a.lazy_claim) && un < 0 && u < U) un = (int)atomicAdd(claim, 1u);
+        if (u >= U) {  // the end tag takes a stage
+          tag[slot] = -1;
+          mbar_arrive(&full[slot]);
+          break;
+        }
+        const int t0 = p * pt, t1 = min(T, t0 + pt);
+        const uint32_t bytes = (uint32_t)((t1 - t0) * TB);
+        tag[slot] = u * ppr + p;
+        mbar_arrive_expect_tx(&full[slot], bytes);
+        bulk_g2s(ring + (size_t)slot * D.stage, wb + ((size_t)u * T + t0) * TB, bytes,
+                 &full[slot], pol);
+        // keep HBM busy past the ring: the part pfa stages later in this
+        // CTA's sequence (in this unit or the one claimed next) goes to L2,
+        // so that the ring's refill of it hits L2
+        if (pfa > 0) {
+          int q = p + pfa, uq = u;
+          if (q >= ppr) {
+            q -= ppr;
+            uq = un;
+          }
+          if (uq >= 0 && uq < U && q < ppr) {
+            const int q0 = q * pt, q1 = min(T, q0 + pt);
+            bulk_prefetch_l2(wb + ((size_t)uq * T + q0) * TB, (uint32_t)((q1 - q0) * TB));
+          }
+        }
+        if (++p == ppr) u = -1;
       }
       // this CTA claims no more; the last CTA to stop resets the pair
       if (atomicAdd(done, 1u) == gridDim.x - 1) {

@@ -735,15 +735,31 @@ __global__ void __launch_bounds__(kTThreads, 1) gemv_tile_kernel(const GemvArgs 
   // this CTA finalises local units ul = rank, rank + C, ...
   const int nown = nu > rank ? (nu - rank + C - 1) / C : 0;
   if constexpr (EPI == EPI_STORE || EPI == EPI_RESID) {
+    // a unit's 16 rows of one batch row are 16 consecutive items, held by a
+    // half-warp (kTThreads is a multiple of 16): it sums their squares for
+    // the next norm's partials
+    static_assert(kTThreads % 16 == 0, "half-warp per (unit, row)");
     for (int e = tid; e < nown * WU; e += kTThreads) {
       const int ul = rank + (e / WU) * C, r = e % WU, m = r / kUnitRows;
       const int n = (u0 + ul) * kUnitRows + r % kUnitRows;
-      if (n >= a.N) continue;
-      float y = usum(ul, r);
-      if constexpr (WF == WF_I8ROW) y = y * rpow[m] * __ldg(a.scales + n);
-      __nv_bfloat16* o = a.out + (size_t)m * a.ldo + n;
-      if constexpr (EPI == EPI_STORE) *o = __float2bfloat16_rn(y);
-      else *o = __float2bfloat16_rn(__bfloat162float(*o) + round_bf16(y));
+      float o2 = 0.0f;
+      if (n < a.N) {
+        float y = usum(ul, r);
+        if constexpr (WF == WF_I8ROW) y = y * rpow[m] * __ldg(a.scales + n);
+        __nv_bfloat16* o = a.out + (size_t)m * a.ldo + n;
+        __nv_bfloat16 ob;
+        if constexpr (EPI == EPI_STORE) ob = __float2bfloat16_rn(y);
+        else ob = __float2bfloat16_rn(__bfloat162float(*o) + round_bf16(y));
+        *o = ob;
+        const float of = __bfloat162float(ob);
+        o2 = of * of;
+      }
+      if (EPI == EPI_RESID && a.ssq_out) {
+        const unsigned hm = 0xFFFFu << (tid & 16);
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) o2 += __shfl_xor_sync(hm, o2, off);
+        if ((tid & 15) == 0) a.ssq_out[(size_t)m * P.U + u0 + ul] = o2;
+      }
     }
   } else if constexpr (EPI == EPI_SWIGLU) {
     constexpr int HP = kUnitRows / 2;  // (gate, up) row pairs per unit

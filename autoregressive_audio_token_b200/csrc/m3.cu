@@ -124,8 +124,11 @@ struct m3_ctx {
   std::map<std::pair<int, int>, cudaGraphExec_t> dgraphs;
 
   // tiled GEMV: ring geometry and the launch plan per (N, K, rows, format, epilogue)
-  int tile_sb = 65536, tile_ns = 2;
+  int tile_sb = 65536, tile_ns = 3;
+  int tile_ns_o = 3;  // ring stages of the O projection (2 would let it sit beside attention)
   bool tile_dyn = true;  // dynamic unit claiming where it applies
+  int tile_pfa = 0;       // dynamic GEMV: L2 prefetch this many ring stages ahead
+  int tile_lazy = 1;      // dynamic GEMV: claim ahead only once the consumers run
   std::map<std::tuple<int, int, int, int, int>, TileLaunch> tile_plans;
   // {claim, done} counter pairs of the dynamically scheduled GEMV, one per
   // launch in flight: launches take pairs round-robin, the last CTA of a
@@ -142,6 +145,10 @@ struct m3_ctx {
   bool ssq_track = false;
   float2* rope = nullptr;  // this frame's RoPE (cos, sin) [max_rows][head_dim / 2]
   int top_k = 0;           // the frame draw keeps the top_k guided logits (0: all)
+  // L2 prefetch from the attention kernel: the O projection's tail and the
+  // first attn_pf_bytes of gate/up
+  bool attn_pf = false;
+  size_t attn_pf_bytes = (size_t)16 << 20;
   // generation loop: feedback tables, device state, its host copy, graphs
   bf16* fb_tok = nullptr;          // [slice_len][H]
   std::vector<bf16*> fb_aud;       // depth_codebooks tables [depth_vocab][H]
@@ -255,7 +262,12 @@ extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) 
   if (const char* e = getenv("M3_NO_GRAPH")) c->use_graphs = (e[0] == '0');
   if (const char* e = getenv("M3_GEMV_STAGE_KB")) c->tile_sb = atoi(e) * 1024;
   if (const char* e = getenv("M3_GEMV_STAGES")) c->tile_ns = atoi(e);
+  if (const char* e = getenv("M3_GEMV_STAGES_O")) c->tile_ns_o = atoi(e);
   if (const char* e = getenv("M3_GEMV_DYN")) c->tile_dyn = (e[0] == '1');
+  if (const char* e = getenv("M3_ATTN_PF")) c->attn_pf = (e[0] == '1');
+  if (const char* e = getenv("M3_GEMV_PF")) c->tile_pfa = atoi(e);
+  if (const char* e = getenv("M3_GEMV_LAZY")) c->tile_lazy = atoi(e);
+  if (const char* e = getenv("M3_ATTN_PF_MB")) c->attn_pf_bytes = (size_t)atoi(e) << 20;
   if (cudaStreamCreateWithFlags(&c->st, cudaStreamNonBlocking) != cudaSuccess ||
       cudaEventCreateWithFlags(&c->ev_in, cudaEventDisableTiming) != cudaSuccess ||
       cudaEventCreateWithFlags(&c->ev_out, cudaEventDisableTiming) != cudaSuccess)
@@ -721,7 +733,8 @@ static int attn_splits(const m3_ctx* c, int rows, int nb) {
 // group-128 scales).
 static int gemv_rows(m3_ctx* c, const DMat& M, int epi, int rows, const bf16* x, int ldx,
                      const bf16* gamma, bf16* out, int ldo, const SampleArgs* smp, bool& pdl,
-                     const FrameParams* fp = nullptr, bool cache_plan = true) {
+                     const FrameParams* fp = nullptr, bool cache_plan = true, int ring_ns = 0) {
+  const int ns = ring_ns > 0 ? ring_ns : c->tile_ns;
   const int step = M.tiled ? rows : 4;
   for (int r0 = 0; r0 < rows; r0 += step) {
     GemvArgs a{};
@@ -741,18 +754,20 @@ static int gemv_rows(m3_ctx* c, const DMat& M, int epi, int rows, const bf16* x,
     if (smp) a.smp = *smp;
     a.err = c->err;
     if (M.tiled) {
-      const auto key = std::make_tuple(M.N, M.K, a.mr, M.wf, epi);
+      const auto key = std::make_tuple(M.N, M.K, a.mr, M.wf, epi * 16 + ns);
       auto it = c->tile_plans.find(key);
       TileLaunch L;
       if (it != c->tile_plans.end()) {
         L = it->second;
       } else {
-        CK(plan_gemv_tile(M.N, M.K, a.mr, M.wf, epi, c->nsm, c->tile_sb, c->tile_ns,
+        CK(plan_gemv_tile(M.N, M.K, a.mr, M.wf, epi, c->nsm, c->tile_sb, ns,
                           c->tile_dyn && a.ldx % 8 == 0, &L));
         if (cache_plan) c->tile_plans.emplace(key, L);
       }
       if (L.dyn) {
         a.ctr = c->tile_ctrs + 2 * (c->tile_ctr_next % kTileCtrPairs);
+        a.pfa = c->tile_pfa;
+        a.lazy_claim = c->tile_lazy;
         ++c->tile_ctr_next;
       }
       float* ssq_written = nullptr;
@@ -761,7 +776,7 @@ static int gemv_rows(m3_ctx* c, const DMat& M, int epi, int rows, const bf16* x,
           a.ssq_in = c->ssq_cur;
           a.ssq_n = c->ssq_n;
         }
-        if (epi == EPI_RESID && L.dyn && M.N == c->cfg.hidden) {
+        if (epi == EPI_RESID && M.N == c->cfg.hidden) {
           ssq_written = c->ssq_cur == c->ssq_buf[0] ? c->ssq_buf[1] : c->ssq_buf[0];
           a.ssq_out = ssq_written;
         }
@@ -804,8 +819,26 @@ static int record_layer(m3_ctx* c, const DLayer& L, Acts& A, int rows, int H, in
   at.fp = c->fp;
   at.fixed_pos = fixed_pos;
   at.err = c->err;
+  if (fixed_pos < 0 && c->attn_pf) {
+    // the O projection past what its CTAs load before their wait, and the
+    // first attn_pf_bytes of gate/up
+    const size_t esz = L.o.wf == WF_BF16 ? 2 : 1;
+    const size_t ob = esz * (size_t)(L.o.N + kUnitRows - 1) / kUnitRows * kUnitRows * L.o.K;
+    // (a 3-stage ring does not fit beside attention: nothing is loaded before)
+    const size_t pre = c->tile_ns_o <= 2 ? (size_t)c->nsm * c->tile_sb * c->tile_ns_o : 0;
+    if (ob > pre) {
+      at.pf[0] = static_cast<const uint8_t*>(L.o.w) + pre;
+      at.pf_bytes[0] = ob - pre;
+    }
+    const size_t gb = esz * (size_t)(L.gu.N + kUnitRows - 1) / kUnitRows * kUnitRows * L.gu.K;
+    at.pf[1] = static_cast<const uint8_t*>(L.gu.w);
+    at.pf_bytes[1] = (c->attn_pf_bytes < gb ? c->attn_pf_bytes : gb) & ~(size_t)255;
+  }
   CK(launch_attn(at, d, kv_f16, splits, rows, c->st, true));
-  CKR(gemv_rows(c, L.o, EPI_RESID, rows, A.o, Hq * d, nullptr, A.x, H, nullptr, pdl));
+  // the projection after attention: a ring small enough for its CTAs to
+  // sit beside the attention CTAs and stream while attention runs
+  CKR(gemv_rows(c, L.o, EPI_RESID, rows, A.o, Hq * d, nullptr, A.x, H, nullptr, pdl, nullptr,
+                true, fixed_pos < 0 ? c->tile_ns_o : 0));
   CKR(gemv_rows(c, L.gu, EPI_SWIGLU, rows, A.x, H, L.mlp_norm, A.act, ffn, nullptr, pdl));
   CKR(gemv_rows(c, L.d, EPI_RESID, rows, A.act, ffn, nullptr, A.x, H, nullptr, pdl));
   return M3_OK;
@@ -1185,7 +1218,7 @@ extern "C" int m3_time_gemv(m3_ctx* c, int which, int rows, int iters, float* av
     const DMat* M = nullptr;
     switch (which) {
       case 0: M = &L.qkv; CKR(gemv_rows(c, L.qkv, EPI_STORE, rows, c->A.x, H, L.attn_norm, c->A.qkv, ld, nullptr, pdl)); break;
-      case 1: M = &L.o; CKR(gemv_rows(c, L.o, EPI_RESID, rows, c->A.o, g.n_q_heads * g.head_dim, nullptr, c->A.x, H, nullptr, pdl)); break;
+      case 1: M = &L.o; CKR(gemv_rows(c, L.o, EPI_RESID, rows, c->A.o, g.n_q_heads * g.head_dim, nullptr, c->A.x, H, nullptr, pdl, nullptr, true, c->tile_ns_o)); break;
       case 2: M = &L.gu; CKR(gemv_rows(c, L.gu, EPI_SWIGLU, rows, c->A.x, H, L.mlp_norm, c->A.act, g.ffn, nullptr, pdl)); break;
       case 3: M = &L.d; CKR(gemv_rows(c, L.d, EPI_RESID, rows, c->A.act, g.ffn, nullptr, c->A.x, H, nullptr, pdl)); break;
       default: {

@@ -264,13 +264,15 @@ def test_errors_are_status_codes(ora):
 
 # -------------------------------------------------- one 8B decoder layer ----
 
-@pytest.mark.parametrize("ring", ["64x2", "8x4"])
+@pytest.mark.parametrize("ring", ["64x3", "64x2", "8x4"])
 @pytest.mark.parametrize("wdtype,rows,kv_f16", [(0, 1, False), (0, 2, False), (1, 1, False),
                                                 (1, 2, True)])
 def test_layer8b_vs_oracle(ora, wdtype, rows, kv_f16, ring, monkeypatch):
-    # with 64 KB stages a 16-row unit of K = 4096 is one stage and the down
-    # projection (K = 12288) streams each unit in six parts; with 8 KB stages
-    # every GEMV splits its units into many parts
+    # 64 KB x 3 is the default ring (the down projection, whose activations
+    # leave no room for it, takes the cluster-split kernel); with 64 KB x 2 a
+    # 16-row unit of K = 4096 is two bf16 stages or one int8 stage and the
+    # down projection streams each unit in six or three parts; with 8 KB
+    # stages every GEMV splits its units into many parts
     kb, ns = ring.split("x")
     monkeypatch.setenv("M3_GEMV_STAGE_KB", kb)
     monkeypatch.setenv("M3_GEMV_STAGES", ns)
@@ -284,7 +286,7 @@ def test_layer8b_vs_oracle(ora, wdtype, rows, kv_f16, ring, monkeypatch):
         oc, oh, olg = m.ora.decode_frame(kc, vc, pos, 77, 0, bits(x))
         assert rel_err(lg, olg) <= TOL[wdtype], rel_err(lg, olg)
         check_codes_teacher_forced(m, h, codes, 77, 0)
-        if ring == "64x2":
+        if ring == "64x3":
             # the top-k 50 draw over the 16384-row slice, on the GPU's own logits
             m.m3.m3_set_top_k(m.ctx, 50)
             codes, h, lg = m.decode([p + 1 for p in pos], 77, 1, x)
