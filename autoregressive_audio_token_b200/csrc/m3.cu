@@ -127,6 +127,10 @@ struct m3_ctx {
   int tile_sb = 65536, tile_ns = 3;
   int tile_ns_o = 3;  // ring stages of the O projection (2 would let it sit beside attention)
   bool tile_dyn = true;  // dynamic unit claiming where it applies
+  // ... for the epilogues whose bit is set: the store (QKV) and SwiGLU
+  // (gate/up) launches; the residual projections (O, down) balance better
+  // split over clusters (measured)
+  int tile_dyn_mask = (1 << EPI_STORE) | (1 << EPI_SWIGLU);
   int tile_pfa = 0;       // dynamic GEMV: L2 prefetch this many ring stages ahead
   int tile_lazy = 1;      // dynamic GEMV: claim ahead only once the consumers run
   std::map<std::tuple<int, int, int, int, int>, TileLaunch> tile_plans;
@@ -264,6 +268,7 @@ extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) 
   if (const char* e = getenv("M3_GEMV_STAGES")) c->tile_ns = atoi(e);
   if (const char* e = getenv("M3_GEMV_STAGES_O")) c->tile_ns_o = atoi(e);
   if (const char* e = getenv("M3_GEMV_DYN")) c->tile_dyn = (e[0] == '1');
+  if (const char* e = getenv("M3_GEMV_DYN_MASK")) c->tile_dyn_mask = atoi(e);
   if (const char* e = getenv("M3_ATTN_PF")) c->attn_pf = (e[0] == '1');
   if (const char* e = getenv("M3_GEMV_PF")) c->tile_pfa = atoi(e);
   if (const char* e = getenv("M3_GEMV_LAZY")) c->tile_lazy = atoi(e);
@@ -761,7 +766,8 @@ static int gemv_rows(m3_ctx* c, const DMat& M, int epi, int rows, const bf16* x,
         L = it->second;
       } else {
         CK(plan_gemv_tile(M.N, M.K, a.mr, M.wf, epi, c->nsm, c->tile_sb, ns,
-                          c->tile_dyn && a.ldx % 8 == 0, &L));
+                          c->tile_dyn && ((c->tile_dyn_mask >> epi) & 1) && a.ldx % 8 == 0,
+                          &L));
         if (cache_plan) c->tile_plans.emplace(key, L);
       }
       if (L.dyn) {
