@@ -111,20 +111,20 @@ __device__ __forceinline__ void mma_f16(float* c, uint4 a, uint32_t b0, uint32_t
       : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
 }
 
-// Four int8 (q0, q1, q2, q3) -> f16 pairs (q0, q1), (q2, q3), exact:
-// f16 bits 0x6400 | (q ^ 0x80) = 1024 + 128 + q, minus 1152.
-__device__ __forceinline__ void s8x4_to_f16x2(uint32_t w, uint32_t& b0, uint32_t& b1) {
-  const uint32_t x = w ^ 0x80808080u;
-  const uint32_t lo = __byte_perm(x, 0x64646464u, 0x5140);  // bytes q0, q1 under 0x64
-  const uint32_t hi = __byte_perm(x, 0x64646464u, 0x7362);  // bytes q2, q3 under 0x64
-  const __half2 bias = __half2half2(__ushort_as_half((unsigned short)0x6480));  // 1152
-  const __half2 l = __hsub2(*reinterpret_cast<const __half2*>(&lo), bias);
-  const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&hi), bias);
-  b0 = *reinterpret_cast<const uint32_t*>(&l);
-  b1 = *reinterpret_cast<const uint32_t*>(&h);
+// int8 weights of the tiled GEMVs are stored biased, byte = q + 128 (q ^ 0x80).
+// Under the f16 exponent pattern 0x64 a byte b reads as 1024 + b = 1152 + q,
+// exact, so four weights become two f16 pairs in two byte permutes; the
+// 1152 is taken out again by a second MMA with every A entry -1152, so the
+// accumulator holds sum (1152 + q) x - 1152 x = sum q x.
+__device__ __forceinline__ void u8x4_to_f16x2_biased(uint32_t w, uint32_t& b0, uint32_t& b1) {
+  b0 = __byte_perm(w, 0x64646464u, 0x5140);  // bytes b0, b1 under 0x64
+  b1 = __byte_perm(w, 0x64646464u, 0x7362);  // bytes b2, b3 under 0x64
 }
 
-// One lane's A fragment of a weight tile in shared memory.
+// One lane's A fragment of a weight tile in shared memory (int8: 1152 + q).
+#ifndef M3_I8_BIAS
+#define M3_I8_BIAS 1
+#endif
 template <int WF>
 __device__ __forceinline__ uint4 load_afrag(const uint8_t* p) {
   if constexpr (WF == WF_BF16) {
@@ -132,16 +132,29 @@ __device__ __forceinline__ uint4 load_afrag(const uint8_t* p) {
   } else {
     const uint2 q = *reinterpret_cast<const uint2*>(p);
     uint4 a;
-    s8x4_to_f16x2(q.x, a.x, a.y);
-    s8x4_to_f16x2(q.y, a.z, a.w);
+    u8x4_to_f16x2_biased(q.x, a.x, a.y);
+    u8x4_to_f16x2_biased(q.y, a.z, a.w);
+#if !M3_I8_BIAS
+    const __half2 bias = __half2half2(__ushort_as_half((unsigned short)0x6480));  // 1152
+    __half2* h = reinterpret_cast<__half2*>(&a);
+    h[0] = __hsub2(h[0], bias); h[1] = __hsub2(h[1], bias);
+    h[2] = __hsub2(h[2], bias); h[3] = __hsub2(h[3], bias);
+#endif
     return a;
   }
 }
 
 template <int WF>
 __device__ __forceinline__ void mma_w(float* c, uint4 a, uint2 b) {
-  if constexpr (WF == WF_BF16) mma_bf16(c, a, b.x, b.y);
-  else mma_f16(c, a, b.x, b.y);
+  if constexpr (WF == WF_BF16) {
+    mma_bf16(c, a, b.x, b.y);
+  } else {
+    constexpr uint32_t kMinus1152 = 0xE480E480u;  // f16 pair (-1152, -1152)
+    mma_f16(c, a, b.x, b.y);
+#if M3_I8_BIAS
+    mma_f16(c, make_uint4(kMinus1152, kMinus1152, kMinus1152, kMinus1152), b.x, b.y);
+#endif
+  }
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -220,15 +233,22 @@ __device__ __forceinline__ void rows_reduce(const float* vals, int n, int mr, in
 
 // The consumer threads' setup of one launch (nt threads, named barrier 1),
 // which also waits for the previous kernel (after fetching static gains):
-// RMSNorm statistics over the whole K (when a.gamma), the int8 scale
-// exponent, and the activations of tiles [kt0, kt0 + Tr) in B-fragment
-// order, xs[j][m][t] = {(k, k+1), (k+8, k+9)} with k = 16 (kt0 + j) + 2t,
-// normalised as out = bf16(gamma * bf16(x / rms)).
+// RMSNorm statistics over the whole K (when a.gamma) and the activations of
+// tiles [kt0, kt0 + Tr) in B-fragment order, xs[j][m][t] = {(k, k+1),
+// (k+8, k+9)} with k = 16 (kt0 + j) + 2t, normalised as
+// out = bf16(gamma * bf16(x / rms)).
 // The sum of squares comes from a.ssq_in when the previous kernel left
 // per-unit partials there ([mr][a.ssq_n], summed here in a fixed order),
 // else from a pass over x.  Each thread holds up to NB items (16 inputs of
 // one row) in registers, so with the partials the setup is one round trip
 // to L2.  `sq` is scratch of T * mr floats that may alias xs.
+// int8 weights take f16 activations scaled by 2^-e per row, e >= 0 the
+// smallest exponent that keeps the largest staged magnitude of the row below
+// 2^15 (rpow[m] = 2^e undoes it on the sums; the CTAs of a cluster stage
+// different K ranges, so each scales its own partial sums).  Every row is staged at scale 1
+// first; magnitudes >= 2^15 (normally none) are recorded, and only then are
+// the exponents set and the rows staged again.  rpow + 16 holds 17 words of
+// scratch (row maxima, an any-row flag).
 template <int WF, int NB, bool GAMMA>
 __device__ __forceinline__ void stage_activations(const GemvArgs& a, int mr, int kt0, int Tr,
                                                   float* rinv, float* rpow, float* sq, uint2* xs,
@@ -238,6 +258,7 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, int mr, int
   const __nv_bfloat16* __restrict__ x = a.x;
   const __nv_bfloat16* __restrict__ gm = GAMMA ? a.gamma : nullptr;
   const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+  unsigned* big = reinterpret_cast<unsigned*>(rpow + 16);  // [16] maxima >= 2^15, [16] flag
   auto set_rinv = [&](int m, float s) { rinv[m] = 1.0f / sqrtf(s / (float)K + a.eps); };
   auto normalise = [&](int m, const uint4& xl, const uint4& xh, const uint4& gl, const uint4& gh,
                        float* v) {
@@ -261,13 +282,14 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, int mr, int
       if (gm && i < Tr * mr) load16(gm + 16 * (kt0 + i / mr), gl[q], gh[q]);
     }
   };
+  if (WF == WF_I8ROW && tid < 17) {
+    big[tid] = 0u;
+    if (tid < 16) rpow[tid] = 1.0f;
+  }
   load_gamma(tid);
   pdl_wait();  // the activations come from the previous kernel
+  if constexpr (WF == WF_I8ROW) named_bar_sync(1, nt);  // the scratch words are zero
   const bool have_ss = gm && a.ssq_in;
-  // int8 with the whole K in one batch per thread: the row maxima come from
-  // the normalised values held in registers (no extra pass over x)
-  const bool fast8 = (WF == WF_I8ROW) && Tr == T && Tr * mr <= NB * nt;
-  if (fast8 && tid < 16) rpow[tid] = 0.0f;  // row maxima (as bits) until the scale
   if (gm && !have_ss) {  // sum of squares per (row, 16 inputs), then per row
     for (int i0 = tid; i0 < T * mr; i0 += NB * nt) {
       uint4 xl[NB], xh[NB];
@@ -293,42 +315,6 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, int mr, int
     rows_reduce<false>(sq, T, mr, warp, nwarps, lane, set_rinv);
     named_bar_sync(1, nt);
   }
-  if (WF == WF_I8ROW && !fast8) {  // largest normalised magnitude per row
-    if (have_ss) {
-      rows_reduce<false>(a.ssq_in, a.ssq_n, mr, warp, nwarps, lane, set_rinv);
-      named_bar_sync(1, nt);
-    }
-    for (int i0 = tid; i0 < T * mr; i0 += NB * nt) {
-      uint4 xl[NB], xh[NB], gl[NB], gh[NB];
-#pragma unroll
-      for (int q = 0; q < NB; ++q) {
-        const int i = i0 + q * nt;
-        xl[q] = xh[q] = gl[q] = gh[q] = z4;
-        if (i < T * mr) {
-          load16(x + (size_t)(i / T) * a.ldx + 16 * (i % T), xl[q], xh[q]);
-          if (gm) load16(gm + 16 * (i % T), gl[q], gh[q]);
-        }
-      }
-#pragma unroll
-      for (int q = 0; q < NB; ++q) {
-        const int i = i0 + q * nt;
-        if (i >= T * mr) continue;
-        float v[16];
-        normalise(i / T, xl[q], xh[q], gl[q], gh[q], v);
-        float mx = 0.0f;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) mx = fmaxf(mx, fabsf(v[e]));
-        sq[i] = mx;
-      }
-    }
-    named_bar_sync(1, nt);
-    rows_reduce<true>(sq, T, mr, warp, nwarps, lane, [&](int m, float s) {
-      int e = 0;  // largest magnitude below 2^15 after scaling by 2^-e
-      if (s >= 32768.0f) e = ilogbf(s) - 14;
-      rpow[m] = ldexpf(1.0f, e);
-    });
-    named_bar_sync(1, nt);
-  }
   // the slice in B-fragment order, NB items per thread per batch; item i is
   // (tile jj = i / mr, row m = i % mr), so a warp's stores are 32-byte
   // steps and its loads 32-byte sectors
@@ -340,7 +326,8 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, int mr, int
       if (i < Tr * mr) load16(x + (size_t)(i % mr) * a.ldx + 16 * (kt0 + i / mr), xl[q], xh[q]);
     }
   };
-  auto store_batch = [&](int i0) {
+  // first: the first pass (int8 at scale 1, recording large magnitudes)
+  auto store_batch = [&](int i0, bool first) {
 #pragma unroll
     for (int q = 0; q < NB; ++q) {
       const int i = i0 + q * nt;
@@ -368,28 +355,49 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, int mr, int
         dst[0] = make_uint4(w[0], w[4], w[1], w[5]);
         dst[1] = make_uint4(w[2], w[6], w[3], w[7]);
       } else {
-        float v[16];
-        normalise(m, xl[q], xh[q], gl[q], gh[q], v);
-        if (h_out) {
-          __nv_bfloat16* h = h_out + (size_t)m * K + 16 * (kt0 + jj);
+        if (gm) {
+          const uint32_t gw[8] = {gl[q].x, gl[q].y, gl[q].z, gl[q].w,
+                                  gh[q].x, gh[q].y, gh[q].z, gh[q].w};
+          const uint64_t r2 = pack_f32x2(rinv[m], rinv[m]);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) h[e] = __float2bfloat16_rn(v[e]);
+          for (int p = 0; p < 8; ++p) {
+            const uint32_t t1 = f32x2_to_bf16x2(fmul2(bf16x2_to_f32x2(w[p]), r2));
+            w[p] = f32x2_to_bf16x2(fmul2(bf16x2_to_f32x2(gw[p]), bf16x2_to_f32x2(t1)));
+          }
         }
-        const float sc = 1.0f / rpow[m];  // a power of two: exact
+        if (h_out) {
+          uint4* h = reinterpret_cast<uint4*>(h_out + (size_t)m * K + 16 * (kt0 + jj));
+          h[0] = make_uint4(w[0], w[1], w[2], w[3]);
+          h[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        }
+        if (first) {
+          // |bf16| bits as fp32 bits order like the magnitudes
+          uint32_t mx = 0u;
+#pragma unroll
+          for (int p = 0; p < 8; ++p)
+            mx = max(mx, max((w[p] << 16) & 0x7FFFFFFFu, w[p] & 0x7FFF0000u));
+          if (mx >= 0x47000000u) {  // 2^15
+            atomicMax(big + m, mx);
+            big[16] = 1u;
+          }
+        }
+        const uint64_t s2 = first ? pack_f32x2(1.0f, 1.0f)
+                                  : pack_f32x2(1.0f / rpow[m], 1.0f / rpow[m]);  // powers of two
         uint32_t f[8];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          f[2 * t] = pack_f16x2(v[2 * t] * sc, v[2 * t + 1] * sc);
-          f[2 * t + 1] = pack_f16x2(v[2 * t + 8] * sc, v[2 * t + 9] * sc);
+        for (int p = 0; p < 8; ++p) {
+          const float2 v = unpack_f32x2(fmul2(bf16x2_to_f32x2(w[p]), s2));
+          f[p] = pack_f16x2(v.x, v.y);
         }
+        // f[p] = inputs (2p, 2p+1): entry t = {pair t, pair t + 4}
         uint4* dst = reinterpret_cast<uint4*>(xs + ((size_t)jj * mr + m) * 4);
-        dst[0] = make_uint4(f[0], f[1], f[2], f[3]);
-        dst[1] = make_uint4(f[4], f[5], f[6], f[7]);
+        dst[0] = make_uint4(f[0], f[4], f[1], f[5]);
+        dst[1] = make_uint4(f[2], f[6], f[3], f[7]);
       }
     }
   };
   load_x(tid);
-  if ((WF != WF_I8ROW || fast8) && have_ss) {
+  if (have_ss) {
     // the row statistics from the previous kernel's partials, loaded while
     // this thread's first activations are in flight: one partial per thread
     // and row, a shuffle tree per warp, the warps in order
@@ -417,71 +425,28 @@ __device__ __forceinline__ void stage_activations(const GemvArgs& a, int mr, int
     }
     named_bar_sync(1, nt);
   }
-  if (fast8) {
-    named_bar_sync(1, nt);  // the maxima are zero
-    // normalised bf16 words of the thread's items, their row maxima
-    uint32_t ww[NB][8];
-#pragma unroll
-    for (int q = 0; q < NB; ++q) {
-      const int i = tid + q * nt;
-      const uint32_t wx[8] = {xl[q].x, xl[q].y, xl[q].z, xl[q].w, xh[q].x, xh[q].y, xh[q].z, xh[q].w};
-      const uint32_t gw[8] = {gl[q].x, gl[q].y, gl[q].z, gl[q].w, gh[q].x, gh[q].y, gh[q].z, gh[q].w};
-      const int m = i % mr;
-      const uint64_t r2 = gm ? pack_f32x2(rinv[m], rinv[m]) : 0ull;
-      uint32_t mx = 0u;
-#pragma unroll
-      for (int p = 0; p < 8; ++p) {
-        uint32_t w = wx[p];
-        if (gm) {
-          const uint32_t t1 = f32x2_to_bf16x2(fmul2(bf16x2_to_f32x2(w), r2));
-          w = f32x2_to_bf16x2(fmul2(bf16x2_to_f32x2(gw[p]), bf16x2_to_f32x2(t1)));
-        }
-        ww[q][p] = w;
-        // |bf16| bits as fp32 bits order like the magnitudes
-        mx = max(mx, max((w << 16) & 0x7FFFFFFFu, w & 0x7FFF0000u));
-      }
-      if (i < Tr * mr) atomicMax(reinterpret_cast<unsigned*>(rpow) + m, mx);
-    }
-    named_bar_sync(1, nt);
+  store_batch(tid, true);
+  for (int i0 = tid + NB * nt; i0 < Tr * mr; i0 += NB * nt) {
+    load_gamma(i0);
+    load_x(i0);
+    store_batch(i0, true);
+  }
+  named_bar_sync(1, nt);
+  if (WF == WF_I8ROW && big[16]) {  // some row reaches 2^15: its exponent, then again
     if (tid < mr) {
-      const float mxf = __uint_as_float(reinterpret_cast<unsigned*>(rpow)[tid]);
+      const float mxf = __uint_as_float(big[tid]);
       int e = 0;  // largest magnitude below 2^15 after scaling by 2^-e
       if (mxf >= 32768.0f) e = ilogbf(mxf) - 14;
       rpow[tid] = ldexpf(1.0f, e);
     }
     named_bar_sync(1, nt);
-#pragma unroll
-    for (int q = 0; q < NB; ++q) {
-      const int i = tid + q * nt;
-      if (i >= Tr * mr) continue;
-      const int m = i % mr, jj = i / mr;
-      if (h_out) {
-        uint4* h = reinterpret_cast<uint4*>(h_out + (size_t)m * K + 16 * (kt0 + jj));
-        h[0] = make_uint4(ww[q][0], ww[q][1], ww[q][2], ww[q][3]);
-        h[1] = make_uint4(ww[q][4], ww[q][5], ww[q][6], ww[q][7]);
-      }
-      const float sc = 1.0f / rpow[m];  // a power of two: exact
-      const uint64_t s2 = pack_f32x2(sc, sc);
-      uint32_t f[8];
-#pragma unroll
-      for (int p = 0; p < 8; ++p) {
-        const float2 v = unpack_f32x2(fmul2(bf16x2_to_f32x2(ww[q][p]), s2));
-        f[p] = pack_f16x2(v.x, v.y);
-      }
-      // f[p] = inputs (2p, 2p+1): entry t = {pair t, pair t + 4}
-      uint4* dst = reinterpret_cast<uint4*>(xs + ((size_t)jj * mr + m) * 4);
-      dst[0] = make_uint4(f[0], f[4], f[1], f[5]);
-      dst[1] = make_uint4(f[2], f[6], f[3], f[7]);
+    for (int i0 = tid; i0 < Tr * mr; i0 += NB * nt) {
+      load_gamma(i0);
+      load_x(i0);
+      store_batch(i0, false);
     }
-  } else {
-    store_batch(tid);
+    named_bar_sync(1, nt);
   }
-  for (int i0 = tid + NB * nt; i0 < Tr * mr; i0 += NB * nt) {
-    load_gamma(i0);
-    load_x(i0);
-    store_batch(i0);
-  }
-  named_bar_sync(1, nt);
 }
 
 // ------------------------------------------------------------ top-k draw --
@@ -709,6 +674,10 @@ __global__ void __launch_bounds__(kTThreads, 1) gemv_tile_kernel(const GemvArgs 
           float y = 0.0f;
 #pragma unroll
           for (int w = 0; w < kTW; ++w) y += pu[(size_t)w * WU + r];
+          // int8: this CTA's own power-of-two activation scale (a cluster's
+          // CTAs stage different K ranges and may scale them differently);
+          // exact in fp32
+          if constexpr (WF == WF_I8ROW) y *= rpow[r / kUnitRows];
           cpart[(size_t)ul * WU + r] = y;
         }
       }
@@ -745,7 +714,7 @@ __global__ void __launch_bounds__(kTThreads, 1) gemv_tile_kernel(const GemvArgs 
       float o2 = 0.0f;
       if (n < a.N) {
         float y = usum(ul, r);
-        if constexpr (WF == WF_I8ROW) y = y * rpow[m] * __ldg(a.scales + n);
+        if constexpr (WF == WF_I8ROW) y = y * __ldg(a.scales + n);  // rpow is in the unit sums
         __nv_bfloat16* o = a.out + (size_t)m * a.ldo + n;
         __nv_bfloat16 ob;
         if constexpr (EPI == EPI_STORE) ob = __float2bfloat16_rn(y);
@@ -769,8 +738,8 @@ __global__ void __launch_bounds__(kTThreads, 1) gemv_tile_kernel(const GemvArgs 
       if (n >= a.N) continue;
       float yg = usum(ul, m * kUnitRows + 2 * jj), yu = usum(ul, m * kUnitRows + 2 * jj + 1);
       if constexpr (WF == WF_I8ROW) {
-        yg = yg * rpow[m] * __ldg(a.scales + n);
-        yu = yu * rpow[m] * __ldg(a.scales + n + 1);
+        yg = yg * __ldg(a.scales + n);  // rpow is in the unit sums
+        yu = yu * __ldg(a.scales + n + 1);
       }
       const float gb = round_bf16(yg), ub = round_bf16(yu);
       const float act = round_bf16(round_bf16(silu_f(gb)) * ub);
@@ -792,8 +761,8 @@ __global__ void __launch_bounds__(kTThreads, 1) gemv_tile_kernel(const GemvArgs 
       float y1 = cfg ? usum(ul, (m0 + 1) * kUnitRows + nn) : 0.0f;
       if constexpr (WF == WF_I8ROW) {
         const float sc = __ldg(a.scales + n);
-        y0 = y0 * rpow[m0] * sc;
-        if (cfg) y1 = y1 * rpow[m0 + 1] * sc;
+        y0 = y0 * sc;  // rpow is in the unit sums
+        if (cfg) y1 = y1 * sc;
       }
       if (a.smp.logits) {
         a.smp.logits[(size_t)(a.row0 + m0) * a.smp.logits_ld + n] = y0;

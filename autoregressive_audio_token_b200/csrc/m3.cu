@@ -269,6 +269,10 @@ extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) 
   if (const char* e = getenv("M3_GEMV_STAGES_O")) c->tile_ns_o = atoi(e);
   if (const char* e = getenv("M3_GEMV_DYN")) c->tile_dyn = (e[0] == '1');
   if (const char* e = getenv("M3_GEMV_DYN_MASK")) c->tile_dyn_mask = atoi(e);
+  if (const char* e = getenv("M3_ATTN_MAX_SPLITS")) {
+    const int v = atoi(e);
+    if (v >= 1 && v <= kAttnMaxSplits) c->max_splits = v;
+  }
   if (const char* e = getenv("M3_ATTN_PF")) c->attn_pf = (e[0] == '1');
   if (const char* e = getenv("M3_GEMV_PF")) c->tile_pfa = atoi(e);
   if (const char* e = getenv("M3_GEMV_LAZY")) c->tile_lazy = atoi(e);
@@ -432,7 +436,8 @@ static int alloc_mat(m3_ctx* c, DMat& M, int N, int K, int wf) {
   // tiled: rows padded to whole 16-row units with zeros
   const size_t rows = M.tiled ? (size_t)(N + kUnitRows - 1) / kUnitRows * kUnitRows : (size_t)N;
   CKR(dalloc(c, &M.w, esz * rows * K));
-  if (M.tiled && rows != (size_t)N) CK(cudaMemset(M.w, 0, esz * rows * K));
+  // padding rows: zeros (int8 is stored biased: 0x80 is q = 0)
+  if (M.tiled && rows != (size_t)N) CK(cudaMemset(M.w, wf == WF_I8ROW ? 0x80 : 0, esz * rows * K));
   if (wf == WF_I8ROW) CKR(dalloc(c, &M.s, sizeof(float) * N));
   if (wf == WF_I8G128) CKR(dalloc(c, &M.s, sizeof(float) * (size_t)N * (K / 128)));
   return M3_OK;
@@ -602,6 +607,8 @@ extern "C" int m3_export_weight(m3_ctx* c, int which, int layer, void* q_host, f
       for (int k = 0; k < M->K; ++k)
         memcpy(q + (size_t)r * rb + k * esz,
                t.data() + tile_byte_offset(row0 + r * step, k, M->K, (int)esz), esz);
+    if (M->wf == WF_I8ROW)  // tiled int8 is stored biased (q + 128)
+      for (size_t i = 0; i < (size_t)rows * rb; ++i) q[i] ^= 0x80u;
   } else {
     CK(cudaMemcpy2D(q_host, rb, static_cast<const char*>(M->w) + (size_t)row0 * rb, rb * step, rb,
                     rows, cudaMemcpyDeviceToHost));

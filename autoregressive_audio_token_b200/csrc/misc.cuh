@@ -107,7 +107,8 @@ __global__ void quantize_g128_kernel(const __nv_bfloat16* __restrict__ w, int64_
 }
 
 // Row-major [rows][K] weights (bf16 or int8) -> the tiled layout of
-// gemv_tile.cuh, source row r going to matrix row dst_row0 + r * row_step.
+// gemv_tile.cuh, source row r going to matrix row dst_row0 + r * row_step;
+// int8 is stored biased, byte = q + 128 (the GEMV's f16 conversion).
 template <typename T>
 __global__ void tile_rows_kernel(const T* __restrict__ src, int rows, int K, uint8_t* dst,
                                  int dst_row0, int row_step) {
@@ -116,7 +117,9 @@ __global__ void tile_rows_kernel(const T* __restrict__ src, int rows, int K, uin
        i += (int64_t)gridDim.x * blockDim.x) {
     const int r = (int)(i / K), k = (int)(i % K);
     const int n = dst_row0 + r * row_step;
-    *reinterpret_cast<T*>(dst + tile_byte_offset(n, k, K, (int)sizeof(T))) = src[i];
+    T v = src[i];
+    if constexpr (sizeof(T) == 1) v = (T)((uint8_t)v ^ 0x80u);  // int8 stored biased: q + 128
+    *reinterpret_cast<T*>(dst + tile_byte_offset(n, k, K, (int)sizeof(T))) = v;
   }
 }
 

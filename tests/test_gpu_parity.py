@@ -100,6 +100,32 @@ def test_tiny_many_rows(ora, rows, cfg, wdtype):
         m.close()
 
 
+@pytest.mark.parametrize("rows", [2, 9])
+def test_int8_activation_beyond_f16_range(ora, rows):
+    # int8 weights take f16 activations; a norm gain of 4e5 on two inputs
+    # puts normalised activations far beyond 2^15, so those rows are staged
+    # again with a power-of-two scale (the QKV and gate/up launches)
+    s = synth.TINY
+    Ls = [synth.layer_weights(s, 13, 0)]
+    for name in ("attn_norm", "mlp_norm"):
+        g = Ls[0][name].clone()
+        g[3] = 4.0e5
+        g[200] = -4.0e5
+        Ls[0][name] = g
+    m = Model(s, seed=13, max_rows=16, wdtype=1, layers=Ls)
+    try:
+        kc, vc = m.kv_setup(rows=rows, n_prefill=20, max_pos=64)
+        pos = [20] * rows
+        x = synth.frame_input(s, rows, 13, 0)
+        codes, h, lg = m.decode(pos, seed=3, frame=1, x_in=x)
+        oc, oh, olg = m.ora.decode_frame(kc, vc, pos, 3, 1, bits(x))
+        assert np.all(np.isfinite(lg))
+        assert rel_err(lg, olg) <= TOL[1], rel_err(lg, olg)
+        check_codes_teacher_forced(m, h, codes, 3, 1)
+    finally:
+        m.close()
+
+
 def _guided(lg, p, cfg):
     # the kernel's guided logits, in the same fp32 operations
     if cfg > 0:
