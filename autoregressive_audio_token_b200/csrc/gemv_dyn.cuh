@@ -231,7 +231,7 @@ __global__ void __maxnreg__(128) gemv_dyn_kernel(const GemvArgs a) {
       stage_activations<WF, 4, true>(a, mr, 0, T, rinv, rpow, reinterpret_cast<float*>(xs), xs,
                                      nullptr, tid, NT);
     else
-      stage_activations<WF, 8, false>(a, mr, 0, T, rinv, rpow, reinterpret_cast<float*>(xs), xs,
+      stage_activations<WF, kStageItems<WF>, false>(a, mr, 0, T, rinv, rpow, reinterpret_cast<float*>(xs), xs,
                                       nullptr, tid, NT);
     const int g = lane >> 2, t = lane & 3;
     const uint2* xl = g < mr ? xs + g * 4 + t : zpad;  // B fragment stream of batch row g

@@ -122,9 +122,12 @@ __device__ __forceinline__ void u8x4_to_f16x2_biased(uint32_t w, uint32_t& b0, u
 }
 
 // One lane's A fragment of a weight tile in shared memory (int8: 1152 + q).
-#ifndef M3_I8_BIAS
-#define M3_I8_BIAS 1
-#endif
+// Items (16 inputs of one row) a thread stages per batch when there is no
+// norm: 8 for bf16; 4 for int8, whose conversion needs more registers (8
+// measured slower)
+template <int WF>
+constexpr int kStageItems = WF == WF_I8ROW ? 4 : 8;
+
 template <int WF>
 __device__ __forceinline__ uint4 load_afrag(const uint8_t* p) {
   if constexpr (WF == WF_BF16) {
@@ -134,12 +137,6 @@ __device__ __forceinline__ uint4 load_afrag(const uint8_t* p) {
     uint4 a;
     u8x4_to_f16x2_biased(q.x, a.x, a.y);
     u8x4_to_f16x2_biased(q.y, a.z, a.w);
-#if !M3_I8_BIAS
-    const __half2 bias = __half2half2(__ushort_as_half((unsigned short)0x6480));  // 1152
-    __half2* h = reinterpret_cast<__half2*>(&a);
-    h[0] = __hsub2(h[0], bias); h[1] = __hsub2(h[1], bias);
-    h[2] = __hsub2(h[2], bias); h[3] = __hsub2(h[3], bias);
-#endif
     return a;
   }
 }
@@ -151,9 +148,7 @@ __device__ __forceinline__ void mma_w(float* c, uint4 a, uint2 b) {
   } else {
     constexpr uint32_t kMinus1152 = 0xE480E480u;  // f16 pair (-1152, -1152)
     mma_f16(c, a, b.x, b.y);
-#if M3_I8_BIAS
     mma_f16(c, make_uint4(kMinus1152, kMinus1152, kMinus1152, kMinus1152), b.x, b.y);
-#endif
   }
 }
 
@@ -612,7 +607,7 @@ __global__ void __launch_bounds__(kTThreads, 1) gemv_tile_kernel(const GemvArgs 
       stage_activations<WF, 4, true>(a, mr, kt0, P.Tr, rinv, rpow, reinterpret_cast<float*>(xs),
                                      xs, h_out, tid, NT);
     else
-      stage_activations<WF, 8, false>(a, mr, kt0, P.Tr, rinv, rpow, reinterpret_cast<float*>(xs),
+      stage_activations<WF, kStageItems<WF>, false>(a, mr, kt0, P.Tr, rinv, rpow, reinterpret_cast<float*>(xs),
                                       xs, h_out, tid, NT);
 
     const int g = lane >> 2, t = lane & 3;

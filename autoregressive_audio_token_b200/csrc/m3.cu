@@ -124,13 +124,15 @@ struct m3_ctx {
   std::map<std::pair<int, int>, cudaGraphExec_t> dgraphs;
 
   // tiled GEMV: ring geometry and the launch plan per (N, K, rows, format, epilogue)
-  int tile_sb = 65536, tile_ns = 3;
-  int tile_ns_o = 3;  // ring stages of the O projection (2 would let it sit beside attention)
+  // ring stages (0: by weight format, measured: 3 for bf16, 2 for int8) and
+  // those of the O projection alone (0: the same)
+  int tile_sb = 65536, tile_ns = 0;
+  int tile_ns_o = 0;
   bool tile_dyn = true;  // dynamic unit claiming where it applies
-  // ... for the epilogues whose bit is set: the store (QKV) and SwiGLU
-  // (gate/up) launches; the residual projections (O, down) balance better
-  // split over clusters (measured)
-  int tile_dyn_mask = (1 << EPI_STORE) | (1 << EPI_SWIGLU);
+  // ... for the epilogues whose bit is set (-1: by weight format, measured:
+  // bf16 leaves the residual projections, O and down, to the cluster-split
+  // kernel, which balances them better; int8 claims everywhere)
+  int tile_dyn_mask = -1;
   int tile_pfa = 0;       // dynamic GEMV: L2 prefetch this many ring stages ahead
   int tile_lazy = 1;      // dynamic GEMV: claim ahead only once the consumers run
   std::map<std::tuple<int, int, int, int, int>, TileLaunch> tile_plans;
@@ -743,10 +745,19 @@ static int attn_splits(const m3_ctx* c, int rows, int nb) {
 // A GEMV over all `rows` batch rows: one launch of the tiled tensor-core
 // kernel, or launches of at most 4 rows of the CUDA-core kernel (int8 with
 // group-128 scales).
+static int ring_stages(const m3_ctx* c, int wf) {
+  return c->tile_ns > 0 ? c->tile_ns : (wf == WF_I8ROW ? 2 : 3);
+}
+
+static int dyn_mask(const m3_ctx* c, int wf) {
+  if (c->tile_dyn_mask >= 0) return c->tile_dyn_mask;
+  return wf == WF_I8ROW ? ~0 : (1 << EPI_STORE) | (1 << EPI_SWIGLU);
+}
+
 static int gemv_rows(m3_ctx* c, const DMat& M, int epi, int rows, const bf16* x, int ldx,
                      const bf16* gamma, bf16* out, int ldo, const SampleArgs* smp, bool& pdl,
                      const FrameParams* fp = nullptr, bool cache_plan = true, int ring_ns = 0) {
-  const int ns = ring_ns > 0 ? ring_ns : c->tile_ns;
+  const int ns = ring_ns > 0 ? ring_ns : ring_stages(c, M.wf);
   const int step = M.tiled ? rows : 4;
   for (int r0 = 0; r0 < rows; r0 += step) {
     GemvArgs a{};
@@ -773,7 +784,7 @@ static int gemv_rows(m3_ctx* c, const DMat& M, int epi, int rows, const bf16* x,
         L = it->second;
       } else {
         CK(plan_gemv_tile(M.N, M.K, a.mr, M.wf, epi, c->nsm, c->tile_sb, ns,
-                          c->tile_dyn && ((c->tile_dyn_mask >> epi) & 1) && a.ldx % 8 == 0,
+                          c->tile_dyn && ((dyn_mask(c, M.wf) >> epi) & 1) && a.ldx % 8 == 0,
                           &L));
         if (cache_plan) c->tile_plans.emplace(key, L);
       }
@@ -838,7 +849,8 @@ static int record_layer(m3_ctx* c, const DLayer& L, Acts& A, int rows, int H, in
     const size_t esz = L.o.wf == WF_BF16 ? 2 : 1;
     const size_t ob = esz * (size_t)(L.o.N + kUnitRows - 1) / kUnitRows * kUnitRows * L.o.K;
     // (a 3-stage ring does not fit beside attention: nothing is loaded before)
-    const size_t pre = c->tile_ns_o <= 2 ? (size_t)c->nsm * c->tile_sb * c->tile_ns_o : 0;
+    const int ns_o = c->tile_ns_o > 0 ? c->tile_ns_o : ring_stages(c, L.o.wf);
+    const size_t pre = ns_o <= 2 ? (size_t)c->nsm * c->tile_sb * ns_o : 0;
     if (ob > pre) {
       at.pf[0] = static_cast<const uint8_t*>(L.o.w) + pre;
       at.pf_bytes[0] = ob - pre;
