@@ -65,4 +65,8 @@ cudaError_t launch_gemv_tile(const GemvArgs& a, int wf, int epi, const TileLaunc
 cudaError_t launch_attn(const AttnArgs& a, int D, int kv_f16, int splits, int rows,
                         cudaStream_t st, bool pdl);
 
+struct DepthArgs;
+size_t depth_smem_bytes(const DepthArgs& a);
+cudaError_t launch_depth(const DepthArgs& a, int max_grid, cudaStream_t st);
+
 }  // namespace m3

@@ -18,6 +18,7 @@
 #include "launch.cuh"
 #include "misc.cuh"
 #include "gemv_tile.cuh"
+#include "depth.cuh"
 
 using namespace m3;
 typedef __nv_bfloat16 bf16;
@@ -119,6 +120,12 @@ struct m3_ctx {
   float* dlogits = nullptr;
   unsigned long long* d_dpages = nullptr;
   void* dkv = nullptr;
+  // the depth decoder as one persistent kernel (depth.cuh), opt-in
+  // (M3_DEPTH_FUSED=1): measured slower than its separate launches
+  bool depth_fused = false;
+  bf16 *dfx = nullptr, *dfqkv = nullptr, *dfatt = nullptr, *dfact = nullptr, *dfkv = nullptr;
+  unsigned long long* dfpart = nullptr;
+  unsigned* dfbar = nullptr;
 
   std::map<std::pair<int, int>, cudaGraphExec_t> graphs;
   std::map<std::pair<int, int>, cudaGraphExec_t> dgraphs;
@@ -325,6 +332,19 @@ extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) 
         (rc = dalloc(c, &c->dforced, sizeof(int) * R * NC)) ||
         (rc = dalloc(c, &c->dlogits, sizeof(float) * R * NC * g.depth_vocab)))
       return bail(rc);
+    // scratch of the persistent depth kernel
+    const size_t qn = (size_t)g.depth_heads * g.depth_head_dim;
+    if ((rc = dalloc(c, &c->dfx, sizeof(bf16) * R * Dh)) ||
+        (rc = dalloc(c, &c->dfqkv, sizeof(bf16) * R * 3 * qn)) ||
+        (rc = dalloc(c, &c->dfatt, sizeof(bf16) * R * qn)) ||
+        (rc = dalloc(c, &c->dfact, sizeof(bf16) * R * g.depth_ffn)) ||
+        (rc = dalloc(c, &c->dfkv, sizeof(bf16) * R * g.depth_layers * (NC + 1) * 2 * qn)) ||
+        (rc = dalloc(c, &c->dfpart, sizeof(unsigned long long) * c->nsm * kMaxRows)))
+      return bail(rc);
+    if ((rc = dzalloc(c, &p, sizeof(unsigned) * 4))) return bail(rc);
+    c->dfbar = static_cast<unsigned*>(p);
+    if (const char* e = getenv("M3_DEPTH_FUSED")) c->depth_fused = e[0] == '1';
+    if (g.depth_layers > kDepthMaxLayers || NC > kDepthMaxCB) c->depth_fused = false;
     // depth KV: one 32-position page per (row, layer), bf16
     const size_t page = (size_t)2 * g.depth_heads * 32 * g.depth_head_dim * 2;
     if ((rc = dzalloc(c, &c->dkv, page * R * g.depth_layers))) return bail(rc);
@@ -976,9 +996,64 @@ extern "C" int m3_decode_frame(m3_ctx* c, int rows, const int32_t* positions, ui
 }
 
 // --------------------------------------------------------- depth decoder ---
+// The persistent depth kernel (depth.cuh) over the same buffers.
+static int record_depth_fused(m3_ctx* c, int rows, bool forced, const bf16* hin) {
+  const m3_config& g = c->cfg;
+  DepthArgs a{};
+  auto dm = [](const DMat& M) { return DepthMat{static_cast<const int8_t*>(M.w), M.s}; };
+  for (int l = 0; l < g.depth_layers; ++l) {
+    const DLayer& L = c->DL[l];
+    a.L[l].qkv = dm(L.qkv);
+    a.L[l].o = dm(L.o);
+    a.L[l].gu = dm(L.gu);
+    a.L[l].d = dm(L.d);
+    a.L[l].attn_norm = L.attn_norm;
+    a.L[l].mlp_norm = L.mlp_norm;
+    a.L[l].q_norm = L.q_norm;
+    a.L[l].k_norm = L.k_norm;
+  }
+  a.proj = dm(c->dproj);
+  for (int j = 0; j < g.depth_codebooks; ++j) {
+    a.heads[j] = dm(c->dheads[j]);
+    a.emb[j] = c->demb[j];
+    a.emb_rows[j] = c->demb_rows[j];
+  }
+  a.final_norm = c->dfinal;
+  a.inv_freq = c->dinv_freq;
+  a.n_layers = g.depth_layers;
+  a.Dh = g.depth_hidden;
+  a.nh = g.depth_heads;
+  a.hd = g.depth_head_dim;
+  a.F = g.depth_ffn;
+  a.NC = g.depth_codebooks;
+  a.V = g.depth_vocab;
+  a.Hin = g.hidden;
+  a.rows = rows;
+  a.zero_code = g.has_end_token ? g.slice_len : INT_MIN;
+  a.eps = g.rms_eps;
+  a.fp = c->fp;
+  a.h_in = hin;
+  a.code0 = c->dprev;
+  a.forced = forced ? c->dforced : nullptr;
+  a.codes = c->dcodes;
+  a.logits = c->dlogits;
+  a.x = c->dfx;
+  a.qkv = c->dfqkv;
+  a.att = c->dfatt;
+  a.act = c->dfact;
+  a.kv = c->dfkv;
+  a.part = c->dfpart;
+  a.bar = c->dfbar;
+  a.err = c->err;
+  CK(cudaMemsetAsync(c->dfbar, 0, sizeof(unsigned) * 4, c->st));
+  CK(launch_depth(a, c->nsm, c->st));
+  return M3_OK;
+}
+
 // hin: the frame's final-normed hidden state [rows][hidden]; the semantic
 // code is in dprev.
 static int record_depth(m3_ctx* c, int rows, bool forced, const bf16* hin) {
+  if (c->depth_fused) return record_depth_fused(c, rows, forced, hin);
   const m3_config& g = c->cfg;
   const int Dh = g.depth_hidden, NC = g.depth_codebooks, V = g.depth_vocab;
   bool pdl = false;

@@ -333,8 +333,11 @@ def test_layer8b_vs_oracle(ora, wdtype, rows, kv_f16, ring, monkeypatch):
 
 # -------------------------------------------------------- depth decoder ----
 
+@pytest.mark.parametrize("fused", ["0", "1"])
 @pytest.mark.parametrize("rows,cfg", [(1, 0.0), (2, 1.5)])
-def test_depth_decoder_teacher_forced(ora, rows, cfg):
+def test_depth_decoder_teacher_forced(ora, rows, cfg, fused, monkeypatch):
+    # fused "1": the persistent one-kernel depth decoder (opt-in)
+    monkeypatch.setenv("M3_DEPTH_FUSED", fused)
     s = synth.TINY
     D = synth.DepthShape(hidden=256, n_layers=2, n_heads=4, head_dim=64, ffn=384, codebooks=7,
                          vocab=128, sem_vocab=s.slice_len, in_hidden=s.hidden)
