@@ -803,9 +803,17 @@ static int gemv_rows(m3_ctx* c, const DMat& M, int epi, int rows, const bf16* x,
       if (it != c->tile_plans.end()) {
         L = it->second;
       } else {
-        CK(plan_gemv_tile(M.N, M.K, a.mr, M.wf, epi, c->nsm, c->tile_sb, ns,
-                          c->tile_dyn && ((dyn_mask(c, M.wf) >> epi) & 1) && a.ldx % 8 == 0,
-                          &L));
+        // the preferred ring and kernel; when the activations of many rows
+        // leave no room for that ring, two stages, then dynamic claiming
+        const bool dyn_ok = c->tile_dyn && a.ldx % 8 == 0;
+        cudaError_t pe = plan_gemv_tile(M.N, M.K, a.mr, M.wf, epi, c->nsm, c->tile_sb, ns,
+                                        dyn_ok && ((dyn_mask(c, M.wf) >> epi) & 1), &L);
+        if (pe == cudaErrorInvalidConfiguration && ns > 2)
+          pe = plan_gemv_tile(M.N, M.K, a.mr, M.wf, epi, c->nsm, c->tile_sb, 2,
+                              dyn_ok && ((dyn_mask(c, M.wf) >> epi) & 1), &L);
+        if (pe == cudaErrorInvalidConfiguration)
+          pe = plan_gemv_tile(M.N, M.K, a.mr, M.wf, epi, c->nsm, c->tile_sb, 2, dyn_ok, &L);
+        CK(pe);
         if (cache_plan) c->tile_plans.emplace(key, L);
       }
       if (L.dyn) {

@@ -331,6 +331,26 @@ def test_layer8b_vs_oracle(ora, wdtype, rows, kv_f16, ring, monkeypatch):
         m.close()
 
 
+@pytest.mark.parametrize("rows,wdtype", [(8, 0), (16, 0), (8, 1)])
+def test_layer8b_many_rows(ora, rows, wdtype):
+    # the 8B layer at 8 and 16 rows: the down projection's activations
+    # (K = 12288) leave no room for the default ring, so the launch plans
+    # fall back to two stages or dynamic claiming
+    s = synth.LAYER8B
+    m = Model(s, seed=17, device="cuda", wdtype=wdtype, max_rows=16)
+    try:
+        kc, vc = m.kv_setup(rows=rows, n_prefill=64, max_pos=80)
+        x = synth.frame_input(s, rows, 17, 0)
+        pos = [64] * rows
+        cfg = 1.5 if rows % 2 == 0 else 0.0
+        codes, h, lg = m.decode(pos, 5, 0, x, cfg_scale=cfg)
+        oc, oh, olg = m.ora.decode_frame(kc, vc, pos, 5, 0, bits(x), cfg_scale=cfg)
+        assert rel_err(lg, olg) <= TOL[wdtype], rel_err(lg, olg)
+        check_codes_teacher_forced(m, h, codes, 5, 0, cfg_scale=cfg)
+    finally:
+        m.close()
+
+
 # -------------------------------------------------------- depth decoder ----
 
 @pytest.mark.parametrize("fused", ["0", "1"])
