@@ -61,6 +61,10 @@ struct AttnArgs {
   // while attention runs): up to two byte ranges, split evenly over the CTAs
   const uint8_t* pf[2];
   size_t pf_bytes[2];
+  // 0: decode (the new token's K/V are appended and attended from registers);
+  // 1: append only (prefill: every row's K/V of its position, then exit);
+  // 2: attend from the cache only, own position included (prefill, after 1)
+  int mode;
 };
 
 template <int D>
@@ -166,9 +170,10 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const Attn
   chunk = (chunk + kAttnTile - 1) / kAttnTile * kAttnTile;
   const int j0 = sidx * chunk;
   const int j1 = min(n, j0 + chunk);
-  const int jc1 = min(j1, pos);  // cached positions [j0, jc1)
-  const bool has_new = (j0 <= pos) && (pos < j1);
-  const int ntiles = jc1 > j0 ? (jc1 - j0 + kAttnTile - 1) / kAttnTile : 0;
+  const int mode = a.mode;
+  const int jc1 = mode == 2 ? j1 : min(j1, pos);  // cached positions [j0, jc1)
+  const bool has_new = mode == 0 && (j0 <= pos) && (pos < j1);
+  const int ntiles = (mode != 1 && jc1 > j0) ? (jc1 - j0 + kAttnTile - 1) / kAttnTile : 0;
   const unsigned long long* pt = a.pages + ((size_t)r * a.n_layers + a.layer) * a.max_pages;
 
   auto issue_tile = [&](int t) {
@@ -274,7 +279,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const Attn
       const uint16_t vb = f32_to_kv<KVF16>(vin[i]);
       k_s[dim] = kv_to_f32<KVF16>(kb);
       v_s[dim] = kv_to_f32<KVF16>(vb);
-      if (sidx == 0) {
+      if (sidx == 0 && mode != 2) {
         const int page = pos / a.page_size, off = pos % a.page_size;
         uint16_t* base = reinterpret_cast<uint16_t*>(pt[page]);
         base[kv_elem_offset(g, a.page_size, off, D, dim)] = kb;
@@ -283,6 +288,9 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const Attn
     }
   }
   __syncthreads();
+  // append only: the K/V are stored (no tile was issued, no cluster barrier
+  // is taken by any CTA of this launch)
+  if (mode == 1) return;
   if (w < grp) {  // score of the new token for head w
     float p = 0.0f;
 #pragma unroll

@@ -167,6 +167,7 @@ struct m3_ctx {
   std::vector<bf16*> fb_aud;       // depth_codebooks tables [depth_vocab][H]
   bf16** d_fb_aud = nullptr;       // device array of the fb_aud pointers
   LoopState* loop = nullptr;
+  unsigned long long* d_vpages = nullptr;  // prefill: every row -> one sequence's pages
   LoopState* h_loop = nullptr;     // pinned
   int* h_err = nullptr;            // pinned
   std::map<std::pair<int, int>, cudaGraphExec_t> lgraphs;
@@ -672,6 +673,12 @@ extern "C" int m3_kv_alloc(m3_ctx* c, int rows, int max_positions, int kvdtype, 
   }
   CKR(dalloc(c, &c->d_pages, sizeof(unsigned long long) * c->h_pages.size()));
   CK(cudaMemset(c->d_pages, 0, sizeof(unsigned long long) * c->h_pages.size()));
+  if (c->d_vpages) {  // the prefill table is sized by max_pages too
+    cudaFree(c->d_vpages);
+    for (auto it = c->allocs.begin(); it != c->allocs.end(); ++it)
+      if (*it == c->d_vpages) { c->allocs.erase(it); break; }
+    c->d_vpages = nullptr;
+  }
   return leave(c);
 }
 
@@ -846,10 +853,14 @@ static int gemv_rows(m3_ctx* c, const DMat& M, int epi, int rows, const bf16* x,
   return M3_OK;
 }
 
+// prefill: the rows are tokens of one sequence whose page-table rows all
+// point at its pages; the attention first appends every row's K/V, then
+// attends from the cache (causal through the positions).
 static int record_layer(m3_ctx* c, const DLayer& L, Acts& A, int rows, int H, int Hq, int Hkv,
                         int d, int ffn, const unsigned long long* pages, int layer, int n_layers,
                         int max_pages, int page_size, int kv_f16, int splits, int fixed_pos,
-                        const double* inv_freq, const float2* rope, bool& pdl) {
+                        const double* inv_freq, const float2* rope, bool& pdl,
+                        bool prefill = false) {
   const int ldqkv = (Hq + 2 * Hkv) * d;
   CKR(gemv_rows(c, L.qkv, EPI_STORE, rows, A.x, H, L.attn_norm, A.qkv, ldqkv, nullptr, pdl));
   AttnArgs at{};
@@ -887,7 +898,15 @@ static int record_layer(m3_ctx* c, const DLayer& L, Acts& A, int rows, int H, in
     at.pf[1] = static_cast<const uint8_t*>(L.gu.w);
     at.pf_bytes[1] = (c->attn_pf_bytes < gb ? c->attn_pf_bytes : gb) & ~(size_t)255;
   }
-  CK(launch_attn(at, d, kv_f16, splits, rows, c->st, true));
+  if (prefill) {
+    at.mode = 1;
+    CK(launch_attn(at, d, kv_f16, 1, rows, c->st, true));
+    // the cached tiles are fetched before a PDL wait: take a full dependency
+    at.mode = 2;
+    CK(launch_attn(at, d, kv_f16, splits, rows, c->st, false));
+  } else {
+    CK(launch_attn(at, d, kv_f16, splits, rows, c->st, true));
+  }
   // the projection after attention: a ring small enough for its CTAs to
   // sit beside the attention CTAs and stream while attention runs
   CKR(gemv_rows(c, L.o, EPI_RESID, rows, A.o, Hq * d, nullptr, A.x, H, nullptr, pdl, nullptr,
@@ -1127,6 +1146,67 @@ extern "C" int m3_depth_decode(m3_ctx* c, int rows, const void* h_frame, const i
   if (logits)
     CK(cudaMemcpyAsync(logits, c->dlogits, sizeof(float) * rows * NC * g.depth_vocab,
                        cudaMemcpyDeviceToDevice, c->st));
+  return leave(c);
+}
+
+// ----------------------------------------------------------- prefill ----
+extern "C" int m3_prefill(m3_ctx* c, int row, int start, int n_tokens, const void* x,
+                          void* h_last) {
+  if (!c || !x) return fail(M3_EINVAL, "null argument");
+  const m3_config& g = c->cfg;
+  if (!c->d_pages) return fail(M3_ESTATE, "m3_kv_alloc first");
+  for (int l = 0; l < g.n_layers; ++l)
+    if (!c->loaded[l]) return fail(M3_ESTATE, "layer " + std::to_string(l) + " not loaded");
+  if (h_last && !c->final_norm) return fail(M3_ESTATE, "final norm not loaded");
+  if (row < 0 || row >= c->kv_rows) return fail(M3_EINVAL, "row");
+  if (n_tokens < 1 || start < 0) return fail(M3_EINVAL, "start / n_tokens");
+  if ((long long)start + n_tokens > c->kv_max_pos)
+    return fail(M3_ECAPACITY, "start + n_tokens outside the KV capacity");
+  const int R = g.max_rows;
+  CKR(enter(c));
+  CKR(ensure_pages(c, start + n_tokens));
+  // every token row of a chunk reads and writes the sequence's pages
+  const size_t per_row = (size_t)g.n_layers * c->max_pages;
+  if (!c->d_vpages) CKR(dalloc(c, &c->d_vpages, sizeof(unsigned long long) * R * per_row));
+  std::vector<unsigned long long> vp((size_t)R * per_row);
+  for (int r = 0; r < R; ++r)
+    std::memcpy(&vp[(size_t)r * per_row], &c->h_pages[(size_t)row * per_row],
+                sizeof(unsigned long long) * per_row);
+  CK(cudaMemcpyAsync(c->d_vpages, vp.data(), sizeof(unsigned long long) * vp.size(),
+                     cudaMemcpyHostToDevice, c->st));
+  CK(cudaStreamSynchronize(c->st));  // the host staging of the page table
+  const bf16* xs = static_cast<const bf16*>(x);
+  for (int c0 = 0; c0 < n_tokens; c0 += R) {
+    const int cn = n_tokens - c0 < R ? n_tokens - c0 : R;
+    FrameParams fp{};
+    fp.rows = cn;
+    fp.temperature = 1.0f;
+    for (int r = 0; r < cn; ++r) fp.pos[r] = start + c0 + r;
+    CK(cudaMemcpyAsync(c->A.x, xs + (size_t)c0 * g.hidden, sizeof(bf16) * cn * g.hidden,
+                       cudaMemcpyDeviceToDevice, c->st));
+    set_frame_params_kernel<<<1, 32, 0, c->st>>>(c->fp, fp);
+    CK(cudaGetLastError());
+    rope_table_kernel<<<cn, 64, 0, c->st>>>(c->fp, c->inv_freq, g.head_dim / 2, c->rope);
+    CK(cudaGetLastError());
+    const int splits = attn_splits(c, cn, c->n_buckets);
+    bool pdl = false;
+    c->ssq_cur = nullptr;  // the chunk's input was copied in
+    c->ssq_track = true;
+    int rc = M3_OK;
+    for (int l = 0; l < g.n_layers && rc == M3_OK; ++l)
+      rc = record_layer(c, c->L[l], c->A, cn, g.hidden, g.n_q_heads, g.n_kv_heads, g.head_dim,
+                        g.ffn, c->d_vpages, l, g.n_layers, c->max_pages, c->bucket, c->kv_f16,
+                        splits, -1, c->inv_freq, c->rope, pdl, true);
+    c->ssq_track = false;
+    c->ssq_cur = nullptr;
+    if (rc != M3_OK) return rc;
+    if (h_last && c0 + cn == n_tokens) {
+      rmsnorm_rows_kernel<<<1, 256, 0, c->st>>>(c->A.x + (size_t)(cn - 1) * g.hidden,
+                                                c->final_norm, g.rms_eps, g.hidden,
+                                                static_cast<bf16*>(h_last));
+      CK(cudaGetLastError());
+    }
+  }
   return leave(c);
 }
 

@@ -193,6 +193,30 @@ __global__ void kv_get_kernel(uint16_t* k, uint16_t* v, const unsigned long long
   }
 }
 
+// One RMSNorm row per CTA (any blockDim multiple of 32, up to 1024):
+// out = bf16(gamma * bf16(x / rms)), the sum of squares in fp32.
+__global__ void rmsnorm_rows_kernel(const __nv_bfloat16* __restrict__ x,
+                                    const __nv_bfloat16* __restrict__ gamma, float eps, int n,
+                                    __nv_bfloat16* out) {
+  __shared__ float red[32];
+  const __nv_bfloat16* xr = x + (size_t)blockIdx.x * n;
+  float s = 0.0f;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const float f = __bfloat162float(xr[i]);
+    s = fmaf(f, f, s);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  float t = 0.0f;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w];
+  const float r = 1.0f / sqrtf(t / (float)n + eps);
+  for (int i = threadIdx.x; i < n; i += blockDim.x)
+    out[(size_t)blockIdx.x * n + i] =
+        __float2bfloat16_rn(__bfloat162float(gamma[i]) * round_bf16(__bfloat162float(xr[i]) * r));
+}
+
 // ------------------------------------------------------ generation loop --
 // Device state of a generation loop ("第二阶段" of the DiffSynth-Studio
 // article: each frame's codes are embedded back as the next input until the

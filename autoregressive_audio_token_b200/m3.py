@@ -26,7 +26,7 @@ M3_MEM_HOST, M3_MEM_DEVICE = 0, 1
 EXPORTED = ("m3_create", "m3_load_weights", "m3_load_depth_weights", "m3_kv_alloc", "m3_kv_set",
             "m3_kv_get", "m3_decode_frame", "m3_depth_decode", "m3_embed", "m3_quantize_int8",
             "m3_export_weight", "m3_frame_bytes", "m3_time_gemv", "m3_sample_noalloc", "m3_set_top_k",
-            "m3_load_feedback", "m3_generate", "m3_sync_status",
+            "m3_load_feedback", "m3_generate", "m3_prefill", "m3_sync_status",
             "m3_last_error", "m3_destroy")
 
 
@@ -91,6 +91,7 @@ def load_library() -> C.CDLL:
     L.m3_time_gemv.argtypes = [vp, i32, i32, i32, C.POINTER(C.c_float), C.POINTER(C.c_double)]
     L.m3_sample_noalloc.argtypes = [vp, i32, vp, u64, u64, f32, f32, vp, vp]
     L.m3_load_feedback.argtypes = [vp, vp, C.POINTER(vp), i32]
+    L.m3_prefill.argtypes = [vp, i32, i32, i32, vp, vp]
     L.m3_generate.argtypes = [vp, i32, vp, u64, u64, vp, f32, f32, i32, vp, vp, vp]
     L.m3_sync_status.argtypes = [vp]
     L.m3_last_error.restype = C.c_char_p
@@ -293,6 +294,12 @@ def m3_generate(ctx: int, positions, seed: int, frame0: int, x_in: torch.Tensor,
     if rc not in (M3_OK, M3_EEMPTY):
         _check(rc)
     return rc, [int(v) for v in nf]
+
+
+def m3_prefill(ctx: int, row: int, start: int, x: torch.Tensor,
+               h_last: torch.Tensor | None = None) -> None:
+    """Prompt prefill of cache row `row` (see m3.h): x bf16 [n_tokens, H] on the GPU."""
+    _check(lib.m3_prefill(ctx, row, start, x.shape[0], _ptr(x.contiguous()), _ptr(h_last)))
 
 
 def m3_sync_status(ctx: int) -> None:

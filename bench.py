@@ -56,6 +56,8 @@ def parse():
     p.add_argument("--generate", type=int, default=0, metavar="F",
                    help="time the GPU generation loop (m3_generate) over F frames of a song "
                         "after a 300-position prompt, against host-driven m3_decode_frame")
+    p.add_argument("--prefill", type=int, default=0, metavar="P",
+                   help="time the prompt prefill (m3_prefill) of P tokens into one row")
     p.add_argument("--sweep", action="store_true",
                    help="batched-variations sweep: rows 1..16 x context 1500/4500/9000, "
                         "bf16 and int8; one JSON line per point")
@@ -590,9 +592,46 @@ def run_generate(args):
     m3.m3_destroy(ctx)
 
 
+def run_prefill(args):
+    """Prompt prefill of P tokens (a prompt's worth, N(0, 0.02^2) embeddings)
+    into one cache row of the full 8B, in chunks of 16 tokens; timed with
+    CUDA events over 3 runs after one untimed run."""
+    import torch
+    from autoregressive_audio_token_b200 import m3
+    import synth
+    torch.cuda.set_device(0)
+    P = args.prefill
+    wdtype = m3.M3_W_INT8 if args.wdtype == "int8" else m3.M3_W_BF16
+    s, ctx = build_model(torch, m3, synth, 0, wdtype, args.layers, max_rows=16)
+    m3.m3_kv_alloc(ctx, 2, P + 1, m3.M3_KV_F16 if args.kv == "f16" else m3.M3_KV_BF16, 256)
+    x = synth.normal((P, s.hidden), 0, "bench/prompt", std=0.02, device="cuda")
+    h = torch.empty(s.hidden, dtype=torch.bfloat16, device="cuda")
+    m3.m3_prefill(ctx, 0, 0, x, h)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(3):
+        m3.m3_prefill(ctx, 1, 0, x, h)
+    e1.record()
+    torch.cuda.synchronize()
+    m3.m3_sync_status(ctx)
+    ms = e0.elapsed_time(e1) / 3
+    layer_w = m3.m3_frame_bytes(ctx, 0, -1)  # weights only (no KV)
+    flops = 2.0 * P * (layer_w / (1 if wdtype == m3.M3_W_INT8 else 2))
+    print(json.dumps({"metric": "prompt prefill tokens/s (8B, one row)", "value": 1000.0 * P / ms,
+                      "unit": "tokens/s", "ms": ms, "tokens": P, "chunk": 16,
+                      "dtype": args.wdtype, "approx_tflops": flops / ms / 1e9,
+                      "config": {"workload": f"qwen3-8b-{args.layers}L-{args.wdtype}-prefill{P}"}}))
+    m3.m3_destroy(ctx)
+
+
 def main():
     args = parse()
     rank, world, local = dist_env()
+    if args.prefill:
+        if rank == 0:
+            run_prefill(args)
+        return
     if args.generate:
         if rank == 0:
             run_generate(args)

@@ -174,7 +174,20 @@ M3_API int m3_kv_set(m3_ctx* ctx, int row, int n_positions, const void* k, const
  * raw cache-type bits (bf16 or f16).  Synchronises the stream. */
 M3_API int m3_kv_get(m3_ctx* ctx, int row, int n_positions, void* k_host, void* v_host);
 
-/* The end token.  With cfg.has_end_token the draw of m3_decode_frame chooses
+/* Prompt prefill of one cache row (the prompt embedder's tokens, DiffSynth-
+ * Studio article "第一阶段", ahead of the autoregressive frames): token t of
+ * x (dev bf16 [n_tokens, H]) runs through every layer at position start + t,
+ * attending to positions 0..start + t of the row (causal), and its K/V land
+ * in the row's cache -- the same result as decoding the tokens one by one.
+ * Tokens go in chunks of up to max_rows, each chunk one pass of the layers
+ * with the chunk's tokens as the batch rows of the tensor-core projections.
+ *  h_last (dev bf16 [H], nullable): the final-normed hidden state of the last
+ *    token.
+ * start + n_tokens must be <= max_positions (M3_ECAPACITY).  May allocate KV
+ * buckets; synchronises the stream once. */
+M3_API int m3_prefill(m3_ctx* ctx, int row, int start, int n_tokens, const void* x, void* h_last);
+
+/* The end token./* The end token.  With cfg.has_end_token the draw of m3_decode_frame chooses
  * among slice_len + 1 candidates: the code block and, as slice-relative code
  * slice_len, the end token (noise index end_token); the vocabulary mask of
  * "第二阶段" in the DiffSynth-Studio article, which leaves the audio codes and
