@@ -3,6 +3,8 @@
 // co-resident cluster capacity, shared-memory ring size.
 #include <cuda_runtime.h>
 
+#include <cstdlib>
+
 #include "gemv_dyn.cuh"
 #include "gemv_tile.cuh"
 #include "launch.cuh"
@@ -146,8 +148,12 @@ cudaError_t plan_gemv_tile(int N, int K, int mr, int wf, int epi, int nsm, int s
   }
   double best_cost = 0.0;
   bool found = false;
+  // M3_GEMV_CLUSTER: only this cluster size (tuning)
+  int force_c = 0;
+  if (const char* e = getenv("M3_GEMV_CLUSTER")) force_c = atoi(e);
   for (int C = 1; C <= 8; C *= 2) {
     if (T % C || C > nsm) continue;
+    if (force_c > 0 && C != force_c) continue;
     int ncl = nsm / C;
     if (ncl > U) ncl = U;
     TilePlan p = tile_plan(N, K, esz, C, ncl, sb, sb * ns);

@@ -796,17 +796,23 @@ __global__ void __launch_bounds__(kTThreads, 1) gemv_tile_kernel(const GemvArgs 
       if (tid == 0) *a.smp.counter = 0u;
     } else if (*flag) {  // the last CTA: argmax over the CTAs' winners
       __threadfence();
-      if (tid < np) {
-        float bz = -INFINITY;
-        int bi = 0x7fffffff;
-        for (int bb = 0; bb < (int)gridDim.x; ++bb) {
-          const float z = __ldcg(a.smp.part_z + bb * kMaxRows + tid);
-          const int i = __ldcg(a.smp.part_i + bb * kMaxRows + tid);
-          if (z > bz || (z == bz && i < bi)) {
-            bz = z;
-            bi = i;
-          }
+      // all threads at once (one CTA's winner each), the 64-bit key's max in
+      // shared memory: the largest z, the lowest index on equal z
+      if (tid < kMaxRows) best[tid] = 0ull;
+      __syncthreads();
+      for (int p = 0; p < np; ++p) {
+        unsigned long long kb = 0ull;
+        for (int bb = tid; bb < (int)gridDim.x; bb += kTThreads) {
+          const int i = __ldcg(a.smp.part_i + bb * kMaxRows + p);
+          if (i == 0x7fffffff) continue;  // a CTA without outputs
+          const unsigned long long k = argmax_key(__ldcg(a.smp.part_z + bb * kMaxRows + p), i);
+          kb = k > kb ? k : kb;
         }
+        if (kb) atomicMax(&best[p], kb);
+      }
+      __syncthreads();
+      if (tid < np) {
+        const int bi = best[tid] ? key_idx(best[tid]) : 0x7fffffff;
         const int nm = cfg ? 2 : 1;
         for (int q = 0; q < nm; ++q) {
           const int r = a.row0 + (cfg ? 2 * tid + q : tid);
