@@ -85,6 +85,24 @@ __device__ __forceinline__ unsigned long long smp_index(const SampleArgs& s, int
   return n == s.end_row1 - 1 ? s.end_index : s.index_base + (unsigned long long)n;
 }
 
+// Order-preserving key for the sampler's argmax: larger z first, then the
+// smaller index (-0.0 counts as +0.0, as in a float comparison).
+__device__ __forceinline__ unsigned long long argmax_key(float z, int idx) {
+  uint32_t b = __float_as_uint(z == 0.0f ? 0.0f : z);
+  b = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+  return ((unsigned long long)b << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)idx);
+}
+
+__device__ __forceinline__ float key_z(unsigned long long key) {
+  uint32_t b = (uint32_t)(key >> 32);
+  b = (b & 0x80000000u) ? (b & 0x7FFFFFFFu) : ~b;
+  return __uint_as_float(b);
+}
+
+__device__ __forceinline__ int key_idx(unsigned long long key) {
+  return (int)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull));
+}
+
 struct GemvArgs {
   const void* w;              // [N][K] row-major, bf16 or int8
   const float* scales;        // int8: [N] or [N][K/128]
@@ -392,24 +410,31 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvArgs a)
       last = __shfl_sync(0xffffffffu, last, 0);
       if (!last) return;
       __threadfence();
-      if (lane < np) {
-        float bz = -INFINITY;
-        int bi = 0x7fffffff;
-        for (int bb = 0; bb < (int)gridDim.x; ++bb) {
-          const float z = __ldcg(a.smp.part_z + bb * kMaxRows + lane);
-          const int i = __ldcg(a.smp.part_i + bb * kMaxRows + lane);
-          if (z > bz || (z == bz && i < bi)) {
-            bz = z;
-            bi = i;
-          }
+      // per key, the warp's lanes take every 32nd CTA's winner; the 64-bit
+      // key's max (largest z, lowest index on equal z) by a shuffle tree
+      const bool cfg = a.fp->cfg_on != 0;
+      for (int p = 0; p < np; ++p) {
+        unsigned long long kb = 0ull;
+        for (int bb = lane; bb < (int)gridDim.x; bb += 32) {
+          const int i = __ldcg(a.smp.part_i + bb * kMaxRows + p);
+          if (i == 0x7fffffff) continue;  // a CTA without outputs
+          const unsigned long long k = argmax_key(__ldcg(a.smp.part_z + bb * kMaxRows + p), i);
+          kb = k > kb ? k : kb;
         }
-        const bool cfg = a.fp->cfg_on != 0;
-        const int nm = cfg ? 2 : 1;
-        for (int q = 0; q < nm; ++q) {
-          const int r = a.row0 + (cfg ? 2 * lane + q : lane);
-          a.smp.codes[(size_t)r * a.smp.code_stride] = bi;
-          if (a.smp.prev)
-            a.smp.prev[r] = a.smp.forced ? a.smp.forced[(size_t)r * a.smp.forced_stride] : bi;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const unsigned long long y = __shfl_xor_sync(0xffffffffu, kb, o);
+          kb = y > kb ? y : kb;
+        }
+        if (lane == 0) {
+          const int bi = kb ? key_idx(kb) : 0x7fffffff;
+          const int nm = cfg ? 2 : 1;
+          for (int q = 0; q < nm; ++q) {
+            const int r = a.row0 + (cfg ? 2 * p + q : p);
+            a.smp.codes[(size_t)r * a.smp.code_stride] = bi;
+            if (a.smp.prev)
+              a.smp.prev[r] = a.smp.forced ? a.smp.forced[(size_t)r * a.smp.forced_stride] : bi;
+          }
         }
       }
       if (lane == 0) *a.smp.counter = 0u;

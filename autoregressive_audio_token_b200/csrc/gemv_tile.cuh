@@ -177,24 +177,6 @@ __device__ __forceinline__ void put_cfrag(float* pb, const float* c, int lane, i
   }
 }
 
-// Order-preserving key for the sampler's argmax: larger z first, then the
-// smaller index (-0.0 counts as +0.0, as in a float comparison).
-__device__ __forceinline__ unsigned long long argmax_key(float z, int idx) {
-  uint32_t b = __float_as_uint(z == 0.0f ? 0.0f : z);
-  b = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-  return ((unsigned long long)b << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)idx);
-}
-
-__device__ __forceinline__ float key_z(unsigned long long key) {
-  uint32_t b = (uint32_t)(key >> 32);
-  b = (b & 0x80000000u) ? (b & 0x7FFFFFFFu) : ~b;
-  return __uint_as_float(b);
-}
-
-__device__ __forceinline__ int key_idx(unsigned long long key) {
-  return (int)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull));
-}
-
 // ------------------------------------------------------------ activations --
 // 16 consecutive bf16 at p (16-byte aligned) -> fp32.
 __device__ __forceinline__ void load16(const __nv_bfloat16* p, uint4& lo, uint4& hi) {
