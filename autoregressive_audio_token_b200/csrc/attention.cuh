@@ -50,6 +50,7 @@ struct AttnArgs {
   float eps;
   const double* inv_freq;     // [D/2] theta^(-2i/D)
   const float2* rope;         // nullable: this frame's (cos, sin) [rows][D/2]
+  int rope_ld;                // row stride of `rope` in entries (0: one position for all rows)
   const unsigned long long* pages;  // [rows][n_layers][max_pages] page base addresses
   int layer, n_layers, max_pages, page_size;
   int Hq, Hkv;
@@ -223,7 +224,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const Attn
 #pragma unroll
     for (int i = 0; i < VPL / 2; ++i) {
       if (a.rope) {
-        const float2 cs = a.rope[(size_t)r * (D / 2) + lane + 32 * i];
+        const float2 cs = a.rope[(size_t)r * a.rope_ld + lane + 32 * i];
         rc[i] = cs.x;
         rs[i] = cs.y;
       } else {

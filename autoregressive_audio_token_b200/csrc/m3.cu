@@ -93,6 +93,7 @@ struct m3_ctx {
   std::vector<DMat> dheads;
   bf16* dfinal = nullptr;
   double* dinv_freq = nullptr;
+  float2* drope = nullptr;  // (cos, sin) of the depth decoder's positions [codebooks + 1][hd / 2]
 
   // KV cache
   int kv_rows = 0, kv_max_pos = 0, kv_f16 = 0, bucket = 256, max_pages = 0, n_buckets = 0;
@@ -325,6 +326,13 @@ extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) 
     c->DL.resize(g.depth_layers);
     c->dinv_freq = make_inv_freq(c, g.depth_head_dim, g.depth_rope_theta, &rc);
     if (rc) return bail(rc);
+    {
+      const int half = g.depth_head_dim / 2, npos = NC + 1;
+      if ((rc = dalloc(c, &c->drope, sizeof(float2) * npos * half))) return bail(rc);
+      rope_positions_kernel<<<1, 256>>>(c->dinv_freq, half, npos, c->drope);
+      if (cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
+        return bail(fail(M3_ECUDA, "depth RoPE table"));
+    }
     if ((rc = alloc_acts(c, c->DA, R, Dh, g.depth_heads, g.depth_heads, g.depth_head_dim,
                          g.depth_ffn)) ||
         (rc = dalloc(c, &c->dh, sizeof(bf16) * R * g.hidden)) ||
@@ -871,6 +879,7 @@ static int record_layer(m3_ctx* c, const DLayer& L, Acts& A, int rows, int H, in
   at.eps = c->cfg.rms_eps;
   at.inv_freq = inv_freq;
   at.rope = rope;
+  at.rope_ld = fixed_pos >= 0 ? 0 : d / 2;  // a fixed position: one row of the table
   at.pages = pages;
   at.layer = layer;
   at.n_layers = n_layers;
@@ -1096,7 +1105,7 @@ static int record_depth(m3_ctx* c, int rows, bool forced, const bf16* hin) {
     for (int l = 0; l < g.depth_layers; ++l)
       CKR(record_layer(c, c->DL[l], c->DA, rows, Dh, g.depth_heads, g.depth_heads,
                        g.depth_head_dim, g.depth_ffn, c->d_dpages, l, g.depth_layers, 1, 32, 0, 1,
-                       j, c->dinv_freq, nullptr, pdl));
+                       j, c->dinv_freq, c->drope + (size_t)j * (g.depth_head_dim / 2), pdl));
     if (j >= 1) {
       SampleArgs sa{};
       sa.logits = c->dlogits + (size_t)(j - 1) * V;
