@@ -56,7 +56,8 @@ struct AttnArgs {
   int Hq, Hkv;
   __nv_bfloat16* out;         // [rows][Hq*D]
   const FrameParams* fp;
-  int fixed_pos;              // >= 0: every row is at this position (depth decoder)
+  int fixed_pos;              // >= 0: row r is at fixed_pos + r * pos_stride
+  int pos_stride;             // 0: one position for all rows (depth decoder); 1: a prompt chunk
   int* err;
   // L2 prefetch of the weights the next kernels stream (HBM is nearly idle
   // while attention runs): up to two byte ranges, split evenly over the CTAs
@@ -165,7 +166,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const Attn
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int r = blockIdx.z, g = blockIdx.y, sidx = blockIdx.x, S = gridDim.x;
   const int grp = a.Hq / a.Hkv;
-  const int pos = a.fixed_pos >= 0 ? a.fixed_pos : a.fp->pos[r];
+  const int pos = a.fixed_pos >= 0 ? a.fixed_pos + r * a.pos_stride : a.fp->pos[r];
   const int n = pos + 1;
   int chunk = (n + S - 1) / S;
   chunk = (chunk + kAttnTile - 1) / kAttnTile * kAttnTile;

@@ -65,6 +65,21 @@ cudaError_t launch_gemv_tile(const GemvArgs& a, int wf, int epi, const TileLaunc
 cudaError_t launch_attn(const AttnArgs& a, int D, int kv_f16, int splits, int rows,
                         cudaStream_t st, bool pdl);
 
+// The prefill's tensor-core GEMM (gemm_tc.cu, tcgen05 with tensor-memory
+// accumulators): Y[t][o] = sum_k W[o][k] X[t][k] for T tokens, W in the tiled
+// layout of gemv_tile.cuh (bf16, or int8 with one scale per row).
+struct GemmTcArgs {
+  const uint8_t* w;        // tiled weights, rows padded to 16
+  const float* scales;     // int8: [N] row scales; else null
+  int N, K;                // output rows, inputs (K a multiple of 16)
+  const __nv_bfloat16* x;  // [T][ldx] activations (16-byte aligned rows)
+  int ldx, T;
+  __nv_bfloat16* out;      // STORE: out[t][o]; RESID: out[t][o] += y; SWIGLU: out[t][o / 2]
+  int ldo;
+  int* err;
+};
+cudaError_t launch_gemm_tc(const GemmTcArgs& a, int wf, int epi, cudaStream_t st);
+
 struct DepthArgs;
 size_t depth_smem_bytes(const DepthArgs& a);
 cudaError_t launch_depth(const DepthArgs& a, int max_grid, cudaStream_t st);

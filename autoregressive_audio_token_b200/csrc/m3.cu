@@ -169,6 +169,11 @@ struct m3_ctx {
   bf16** d_fb_aud = nullptr;       // device array of the fb_aud pointers
   LoopState* loop = nullptr;
   unsigned long long* d_vpages = nullptr;  // prefill: every row -> one sequence's pages
+  // prefill on the tensor-core GEMM: prompt chunks of pf_chunk tokens
+  bool prefill_tc = true;
+  int pf_chunk = 256;
+  bf16 *pf_x = nullptr, *pf_n = nullptr, *pf_qkv = nullptr, *pf_o = nullptr, *pf_act = nullptr;
+  float2* pf_rope = nullptr;       // [pf_chunk][head_dim / 2]
   LoopState* h_loop = nullptr;     // pinned
   int* h_err = nullptr;            // pinned
   std::map<std::pair<int, int>, cudaGraphExec_t> lgraphs;
@@ -285,6 +290,11 @@ extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) 
     if (v >= 1 && v <= kAttnMaxSplits) c->max_splits = v;
   }
   if (const char* e = getenv("M3_ATTN_PF")) c->attn_pf = (e[0] == '1');
+  if (const char* e = getenv("M3_PREFILL_TC")) c->prefill_tc = (e[0] == '1');
+  if (const char* e = getenv("M3_PREFILL_CHUNK")) {
+    const int v = atoi(e);
+    if (v >= 16 && v <= 4096) c->pf_chunk = v;
+  }
   if (const char* e = getenv("M3_GEMV_PF")) c->tile_pfa = atoi(e);
   if (const char* e = getenv("M3_GEMV_LAZY")) c->tile_lazy = atoi(e);
   if (const char* e = getenv("M3_ATTN_PF_MB")) c->attn_pf_bytes = (size_t)atoi(e) << 20;
@@ -329,7 +339,7 @@ extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) 
     {
       const int half = g.depth_head_dim / 2, npos = NC + 1;
       if ((rc = dalloc(c, &c->drope, sizeof(float2) * npos * half))) return bail(rc);
-      rope_positions_kernel<<<1, 256>>>(c->dinv_freq, half, npos, c->drope);
+      rope_positions_kernel<<<1, 256>>>(c->dinv_freq, half, 0, npos, c->drope);
       if (cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
         return bail(fail(M3_ECUDA, "depth RoPE table"));
     }
@@ -1159,6 +1169,77 @@ extern "C" int m3_depth_decode(m3_ctx* c, int rows, const void* h_frame, const i
 }
 
 // ----------------------------------------------------------- prefill ----
+// One layer over a prompt chunk of T tokens at positions p0 .. p0 + T - 1
+// with the tensor-core GEMM: the norms over all T rows, the four projections
+// as GEMMs, and the attention appending every token's K/V, then attending
+// from the cache (causal through the positions).
+static int record_prefill_layer(m3_ctx* c, const DLayer& L, int T, int p0, int layer) {
+  const m3_config& g = c->cfg;
+  const int H = g.hidden, d = g.head_dim, ldqkv = (g.n_q_heads + 2 * g.n_kv_heads) * d;
+  const int hq = g.n_q_heads * d;
+  auto gemm = [&](const DMat& M, int epi, const bf16* x, int ldx, bf16* out, int ldo) -> int {
+    GemmTcArgs a{};
+    a.w = static_cast<const uint8_t*>(M.w);
+    a.scales = M.s;
+    a.N = M.N;
+    a.K = M.K;
+    a.x = x;
+    a.ldx = ldx;
+    a.T = T;
+    a.out = out;
+    a.ldo = ldo;
+    a.err = c->err;
+    CK(launch_gemm_tc(a, M.wf, epi, c->st));
+    return M3_OK;
+  };
+  rmsnorm_rows_kernel<<<T, 256, 0, c->st>>>(c->pf_x, L.attn_norm, g.rms_eps, H, c->pf_n);
+  CK(cudaGetLastError());
+  CKR(gemm(L.qkv, EPI_STORE, c->pf_n, H, c->pf_qkv, ldqkv));
+  AttnArgs at{};
+  at.qkv = c->pf_qkv;
+  at.ldqkv = ldqkv;
+  at.q_norm = L.q_norm;
+  at.k_norm = L.k_norm;
+  at.eps = g.rms_eps;
+  at.inv_freq = c->inv_freq;
+  at.rope = c->pf_rope;
+  at.rope_ld = d / 2;
+  at.pages = c->d_vpages;
+  at.layer = layer;
+  at.n_layers = g.n_layers;
+  at.max_pages = c->max_pages;
+  at.page_size = c->bucket;
+  at.Hq = g.n_q_heads;
+  at.Hkv = g.n_kv_heads;
+  at.out = c->pf_o;
+  at.fp = c->fp;
+  at.fixed_pos = p0;
+  at.pos_stride = 1;
+  at.err = c->err;
+  at.mode = 1;
+  CK(launch_attn(at, d, c->kv_f16, 1, T, c->st, false));
+  at.mode = 2;
+  CK(launch_attn(at, d, c->kv_f16, attn_splits(c, T, c->n_buckets), T, c->st, false));
+  CKR(gemm(L.o, EPI_RESID, c->pf_o, hq, c->pf_x, H));
+  rmsnorm_rows_kernel<<<T, 256, 0, c->st>>>(c->pf_x, L.mlp_norm, g.rms_eps, H, c->pf_n);
+  CK(cudaGetLastError());
+  CKR(gemm(L.gu, EPI_SWIGLU, c->pf_n, H, c->pf_act, g.ffn));
+  CKR(gemm(L.d, EPI_RESID, c->pf_act, g.ffn, c->pf_x, H));
+  return M3_OK;
+}
+
+static bool prefill_tc_ok(const m3_ctx* c) {
+  if (!c->prefill_tc) return false;
+  const m3_config& g = c->cfg;
+  if (g.hidden % 16 || g.ffn % 16 || (g.n_q_heads * g.head_dim) % 16) return false;
+  for (int l = 0; l < g.n_layers; ++l) {
+    const DLayer& L = c->L[l];
+    for (const DMat* M : {&L.qkv, &L.o, &L.gu, &L.d})
+      if (!M->tiled || (M->wf != WF_BF16 && M->wf != WF_I8ROW)) return false;
+  }
+  return true;
+}
+
 extern "C" int m3_prefill(m3_ctx* c, int row, int start, int n_tokens, const void* x,
                           void* h_last) {
   if (!c || !x) return fail(M3_EINVAL, "null argument");
@@ -1172,19 +1253,49 @@ extern "C" int m3_prefill(m3_ctx* c, int row, int start, int n_tokens, const voi
   if ((long long)start + n_tokens > c->kv_max_pos)
     return fail(M3_ECAPACITY, "start + n_tokens outside the KV capacity");
   const int R = g.max_rows;
+  const bool tc = prefill_tc_ok(c);
+  const int P = c->pf_chunk;
+  const int Rv = tc && P > R ? P : R;  // rows of the page table that map to the sequence
   CKR(enter(c));
   CKR(ensure_pages(c, start + n_tokens));
   // every token row of a chunk reads and writes the sequence's pages
   const size_t per_row = (size_t)g.n_layers * c->max_pages;
-  if (!c->d_vpages) CKR(dalloc(c, &c->d_vpages, sizeof(unsigned long long) * R * per_row));
-  std::vector<unsigned long long> vp((size_t)R * per_row);
-  for (int r = 0; r < R; ++r)
+  if (!c->d_vpages) CKR(dalloc(c, &c->d_vpages, sizeof(unsigned long long) * (P > R ? P : R) * per_row));
+  std::vector<unsigned long long> vp((size_t)Rv * per_row);
+  for (int r = 0; r < Rv; ++r)
     std::memcpy(&vp[(size_t)r * per_row], &c->h_pages[(size_t)row * per_row],
                 sizeof(unsigned long long) * per_row);
   CK(cudaMemcpyAsync(c->d_vpages, vp.data(), sizeof(unsigned long long) * vp.size(),
                      cudaMemcpyHostToDevice, c->st));
   CK(cudaStreamSynchronize(c->st));  // the host staging of the page table
   const bf16* xs = static_cast<const bf16*>(x);
+  if (tc) {
+    const int H = g.hidden, d = g.head_dim, ldqkv = (g.n_q_heads + 2 * g.n_kv_heads) * d;
+    if (!c->pf_x) {
+      CKR(dalloc(c, &c->pf_x, sizeof(bf16) * P * H));
+      CKR(dalloc(c, &c->pf_n, sizeof(bf16) * P * H));
+      CKR(dalloc(c, &c->pf_qkv, sizeof(bf16) * P * ldqkv));
+      CKR(dalloc(c, &c->pf_o, sizeof(bf16) * P * g.n_q_heads * d));
+      CKR(dalloc(c, &c->pf_act, sizeof(bf16) * P * g.ffn));
+      CKR(dalloc(c, &c->pf_rope, sizeof(float2) * P * (d / 2)));
+    }
+    for (int c0 = 0; c0 < n_tokens; c0 += P) {
+      const int T = n_tokens - c0 < P ? n_tokens - c0 : P;
+      const int p0 = start + c0;
+      CK(cudaMemcpyAsync(c->pf_x, xs + (size_t)c0 * H, sizeof(bf16) * T * H,
+                         cudaMemcpyDeviceToDevice, c->st));
+      rope_positions_kernel<<<(T * (d / 2) + 255) / 256, 256, 0, c->st>>>(c->inv_freq, d / 2, p0,
+                                                                         T, c->pf_rope);
+      CK(cudaGetLastError());
+      for (int l = 0; l < g.n_layers; ++l) CKR(record_prefill_layer(c, c->L[l], T, p0, l));
+      if (h_last && c0 + T == n_tokens) {
+        rmsnorm_rows_kernel<<<1, 256, 0, c->st>>>(c->pf_x + (size_t)(T - 1) * H, c->final_norm,
+                                                  g.rms_eps, H, static_cast<bf16*>(h_last));
+        CK(cudaGetLastError());
+      }
+    }
+    return leave(c);
+  }
   for (int c0 = 0; c0 < n_tokens; c0 += R) {
     const int cn = n_tokens - c0 < R ? n_tokens - c0 : R;
     FrameParams fp{};

@@ -30,12 +30,13 @@ __global__ void rope_table_kernel(const FrameParams* __restrict__ fp,
   }
 }
 
-// (cos, sin) of p * inv_freq[i] (fp64, then fp32) for positions p < npos:
-// the depth decoder's frame-local positions, once.
-__global__ void rope_positions_kernel(const double* __restrict__ inv_freq, int half, int npos,
-                                      float2* table) {
+// (cos, sin) of p * inv_freq[i] (fp64, then fp32) for positions
+// p = p0 .. p0 + npos - 1: the depth decoder's frame-local positions (once),
+// a prompt chunk's positions.
+__global__ void rope_positions_kernel(const double* __restrict__ inv_freq, int half, int p0,
+                                      int npos, float2* table) {
   for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < npos * half; k += gridDim.x * blockDim.x) {
-    const double ang = (double)(k / half) * inv_freq[k % half];
+    const double ang = (double)(p0 + k / half) * inv_freq[k % half];
     table[k] = make_float2((float)cos(ang), (float)sin(ang));
   }
 }

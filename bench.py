@@ -594,8 +594,10 @@ def run_generate(args):
 
 def run_prefill(args):
     """Prompt prefill of P tokens (a prompt's worth, N(0, 0.02^2) embeddings)
-    into one cache row of the full 8B, in chunks of 16 tokens; timed with
-    CUDA events over 3 runs after one untimed run."""
+    into one cache row of the full 8B: chunks of M3_PREFILL_CHUNK tokens (256)
+    through the tcgen05 GEMMs, or with M3_PREFILL_TC=0 chunks of 16 through
+    the decode GEMVs; timed with CUDA events over 3 runs after one untimed
+    run."""
     import torch
     from autoregressive_audio_token_b200 import m3
     import synth
@@ -616,10 +618,13 @@ def run_prefill(args):
     torch.cuda.synchronize()
     m3.m3_sync_status(ctx)
     ms = e0.elapsed_time(e1) / 3
+    tc = os.environ.get("M3_PREFILL_TC", "1") == "1"
+    chunk = int(os.environ.get("M3_PREFILL_CHUNK", "256")) if tc else 16
+    path = "tcgen05 GEMM" if tc else "decode GEMV"
     layer_w = m3.m3_frame_bytes(ctx, 0, -1)  # weights only (no KV)
     flops = 2.0 * P * (layer_w / (1 if wdtype == m3.M3_W_INT8 else 2))
     print(json.dumps({"metric": "prompt prefill tokens/s (8B, one row)", "value": 1000.0 * P / ms,
-                      "unit": "tokens/s", "ms": ms, "tokens": P, "chunk": 16,
+                      "unit": "tokens/s", "ms": ms, "tokens": P, "chunk": chunk, "path": path,
                       "dtype": args.wdtype, "approx_tflops": flops / ms / 1e9,
                       "config": {"workload": f"qwen3-8b-{args.layers}L-{args.wdtype}-prefill{P}"}}))
     m3.m3_destroy(ctx)

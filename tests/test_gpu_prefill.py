@@ -3,9 +3,10 @@
 Prefilling tokens at positions start .. start + n - 1 is defined as decoding
 them one by one (each token attends to every earlier position of its row and
 to itself); the oracle runs exactly that, token by token, through its
-single-row layers.  The GPU runs the tokens in chunks of up to max_rows as
-the batch rows of the tensor-core projections, with a causal attention over
-the row's cache.  Compared:
+single-row layers.  The GPU runs the prompt in chunks (256 tokens by default)
+whose projections are tcgen05 GEMMs, with a causal attention over the row's
+cache; M3_PREFILL_TC=0 selects the decode GEMV kernels over chunks of up to
+max_rows tokens instead.  Compared:
   * the K/V the prefill leaves in the row's cache (every layer, position);
   * the final-normed hidden state of the last token;
   * the other rows' caches, untouched;
@@ -33,12 +34,20 @@ def _cuda():
     torch.cuda.init()
 
 
-@pytest.mark.parametrize("start,n,max_rows,wdtype", [(3, 37, 16, 0), (0, 1, 2, 0), (5, 20, 8, 1)])
-def test_prefill_matches_sequential_decode(ora, start, n, max_rows, wdtype):
+@pytest.mark.parametrize("start,n,max_rows,wdtype,tc,chunk", [
+    (3, 37, 16, 0, "1", 256), (0, 1, 2, 0, "1", 256), (5, 20, 8, 1, "1", 256),
+    (2, 70, 4, 0, "1", 32),     # three chunks, the last one ragged
+    (0, 200, 16, 0, "1", 256),  # two token tiles of the GEMM, the second ragged
+    (1, 150, 4, 1, "1", 64),    # int8, chunks of 64
+    (3, 37, 16, 0, "0", 256), (5, 20, 8, 1, "0", 256)])  # the GEMV prefill
+def test_prefill_matches_sequential_decode(ora, start, n, max_rows, wdtype, tc, chunk,
+                                           monkeypatch):
+    monkeypatch.setenv("M3_PREFILL_TC", tc)
+    monkeypatch.setenv("M3_PREFILL_CHUNK", str(chunk))
     s = TWO_LAYERS
     m = Model(s, seed=21, max_rows=max_rows, wdtype=wdtype)
     try:
-        kc, vc = m.kv_setup(rows=2, n_prefill=start, max_pos=80, bucket=32)
+        kc, vc = m.kv_setup(rows=2, n_prefill=start, max_pos=start + n + 8, bucket=32)
         xs = synth.normal((n, s.hidden), 21, "prompt", std=0.02)
         h_last = torch.empty(s.hidden, dtype=torch.bfloat16, device="cuda")
         m.m3.m3_prefill(m.ctx, 1, start, xs.cuda(), h_last)
@@ -71,6 +80,35 @@ def test_prefill_matches_sequential_decode(ora, start, n, max_rows, wdtype):
         oc, oh, olg = m.ora.decode_frame(kc, vc, pos, 4, 7, bits(x))
         assert rel_err(lg, olg) <= (2e-2 if wdtype == 0 else 5e-2)
         check_codes_teacher_forced(m, h, codes, 4, 7)
+    finally:
+        m.close()
+
+
+@pytest.mark.parametrize("wdtype", [0, 1])
+def test_prefill_8b_layer(ora, wdtype):
+    # one Qwen3-8B layer, 160 prompt tokens: the GEMMs at full width (K up to
+    # 12288, 48 to 192 weight blocks), two token tiles with a ragged second
+    s = synth.LAYER8B
+    m = Model(s, seed=23, device="cuda", wdtype=wdtype, max_rows=2)
+    try:
+        start, n = 8, 160
+        kc, vc = m.kv_setup(rows=1, n_prefill=start, max_pos=start + n + 4, bucket=64)
+        xs = synth.normal((n, s.hidden), 23, "prompt8b", std=0.02)
+        h_last = torch.empty(s.hidden, dtype=torch.bfloat16, device="cuda")
+        m.m3.m3_prefill(m.ctx, 0, start, xs.cuda(), h_last)
+        torch.cuda.synchronize()
+        m.m3.m3_sync_status(m.ctx)
+        xb = bits(xs)
+        x_out = None
+        for t in range(n):
+            x_out = m.ora.body(kc, vc, [start + t], xb[t:t + 1].copy())
+        npos = start + n
+        gk, gv = m.m3.m3_kv_get(m.ctx, 0, s.n_layers, npos, s.n_kv_heads, s.head_dim)
+        tol = 2e-2 if wdtype == 0 else 5e-2
+        assert rel_err(f32(gk.numpy().view(np.uint16)[0]), f32(kc[0, 0, :npos])) <= tol
+        assert rel_err(f32(gv.numpy().view(np.uint16)[0]), f32(vc[0, 0, :npos])) <= tol
+        href = ora.rmsnorm(f32(x_out[0]), bits(m.final_norm), s.rms_eps)
+        assert rel_err(f32(bits(h_last)), href) <= tol
     finally:
         m.close()
 
