@@ -9,31 +9,29 @@
 //   * A = a 128-row block of W (the MMA's M = 128 accumulator lanes),
 //     B = 128 tokens of X (N = 128 fp32 columns of tensor memory), K in
 //     stages of 64, four tcgen05.mma of K = 16 per stage;
-//   * the MMAs read both operands from shared memory in the canonical
-//     K-major layout without swizzle: "core matrices" of 8 rows x 16 bytes
-//     (128 contiguous bytes), K-adjacent core matrices 128 bytes apart (the
-//     descriptor's leading byte offset), 8-row groups 1024 bytes apart (its
-//     stride byte offset);
-//   * a producer warp streams each stage with bulk copies (TMA) into a raw
-//     4-stage ring: per 16-row tile of W its 4 K-tiles (contiguous in the
-//     decode path's tiled layout, gemv_tile.cuh), per token its 64 inputs
-//     (rows padded to 144 bytes so the reads below are free of bank
-//     conflicts);
-//   * four warps rewrite each raw stage into one of two canonical buffers:
-//     one lane's 16 bytes of a W tile are four 4-byte (row, k-pair) words
-//     that land in the same slot of four core matrices, so each warp store
-//     is 128 contiguous bytes; int8 weights (stored q + 128) become bf16 q
-//     exactly on the way (the row scale is applied in the epilogue,
-//     y = s * sum q x, as the int8 definition states); out-of-range rows,
-//     tokens and inputs become zeros.  They fence their generic-proxy writes
-//     for the async proxy, synchronise, and one thread issues the MMAs and
-//     commits them to the buffer's "empty" mbarrier;
+//   * both operands sit in shared memory in the canonical K-major layout
+//     without swizzle: "core matrices" of 8 rows x 16 bytes (128 contiguous
+//     bytes), K-adjacent core matrices 128 bytes apart (the descriptor's
+//     leading byte offset), 8-row groups 1024 bytes apart (its stride byte
+//     offset);
+//   * W stays in the decode path's tiled fragment layout (gemv_tile.cuh):
+//     one lane's 16 bytes of a 16x16 tile are four 4-byte pairs that land in
+//     the same (row, word) slot of four core matrices, so a warp stores each
+//     core matrix as 128 contiguous bytes.  int8 weights (stored q + 128)
+//     become bf16 q exactly on the way in; the row scale is applied in the
+//     epilogue, y = s * sum q x, as the int8 definition states;
+//   * bf16: a 6-stage ring filled by cp.async (4-byte copies of W straight
+//     into their core-matrix slots, 16-byte copies of X), five stages in
+//     flight; int8: a 4-stage ring staged through registers (the bytes are
+//     converted on the way).  Every thread fences its generic-proxy writes for
+//     the async proxy before the CTA barrier; one thread then issues the
+//     MMAs and commits them to the stage's "empty" mbarrier;
 //   * the epilogue reads the accumulator with tcgen05.ld (warp w owns lanes
 //     32w..32w+31, one output row per thread) and applies the projection's
 //     rounding: store bf16(y); residual x = bf16(x + bf16(y)); SwiGLU on the
 //     interleaved (gate, up) row pairs.
-// Every wait is bounded; a timeout records kErrTimeout, and the kernel still
-// waits for its MMAs (bounded) and frees its tensor memory.
+// Every wait is bounded; a timeout records kErrTimeout and the kernel still
+// frees its tensor memory.
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -45,32 +43,24 @@ namespace m3 {
 
 namespace {
 
-constexpr int kBM = 128;      // weight rows per CTA (MMA M, TMEM lanes)
-constexpr int kBN = 128;      // tokens per CTA (MMA N, TMEM columns)
-constexpr int kBK = 64;       // K per stage
-constexpr int kMmaK = 16;     // K per tcgen05.mma (bf16)
-constexpr int kRawStages = 4; // bulk-copy ring
-constexpr int kCanon = 2;     // canonical buffers the MMAs read
-constexpr int kConsumers = 128;             // warps 0-3: rewrite + epilogue
-constexpr int kThreads = kConsumers + 32;   // + the producer warp
-constexpr int kOpBytes = kBM * kBK * 2;     // one canonical operand: 16 KB
-constexpr int kCanonBytes = 2 * kOpBytes;
-constexpr int kXPitch = 144;                // raw token row: 128 bytes + 16 of padding
-constexpr int kRawW = kBM * kBK * 2;        // raw W stage (bf16 size; int8 uses half)
-constexpr int kRawBytes = kRawW + kBN * kXPitch;
-constexpr int kCoreBytes = 128;             // 8 rows x 16 bytes
-constexpr int kLBO = kCoreBytes;            // K-adjacent core matrices
-constexpr int kSBO = (kBK / 8) * kCoreBytes;  // 8-row groups: 1024 bytes
-constexpr int kBarBytes = 256;
-constexpr size_t kSmemBytes =
-    (size_t)kCanon * kCanonBytes + (size_t)kRawStages * kRawBytes + kBarBytes + 1024;
-constexpr int kTmemCols = kBN;              // fp32 accumulator, one column per token
-constexpr int kBarConsumers = 1;            // named barrier of the 128 consumer threads
+constexpr int kBM = 128;     // weight rows per CTA (MMA M, TMEM lanes)
+constexpr int kBN = 128;     // tokens per CTA (MMA N, TMEM columns)
+constexpr int kBK = 64;      // K per stage
+constexpr int kMmaK = 16;    // K per tcgen05.mma (bf16)
+constexpr int kStagesBF16 = 6;   // cp.async ring: 5 stages of loads in flight
+constexpr int kStagesI8 = 4;     // register-staged ring (the int8 -> bf16 conversion)
+constexpr int kMaxStages = 6;
+constexpr int kThreads = 128;
+constexpr int kOpBytes = kBM * kBK * 2;          // one operand of one stage: 16 KB
+constexpr int kStageBytes = 2 * kOpBytes;
+constexpr int kCoreBytes = 128;                  // 8 rows x 16 bytes
+constexpr int kLBO = kCoreBytes;                 // K-adjacent core matrices
+constexpr int kSBO = (kBK / 8) * kCoreBytes;     // 8-row groups: 1024 bytes
+constexpr size_t smem_bytes(int stages) { return (size_t)stages * kStageBytes + 1024 + 256; }
+constexpr int kTmemCols = kBN;                   // fp32 accumulator, one column per token
 
 static_assert(kBM == 128 && kBN % 16 == 0 && kBN >= 16 && kBN <= 256, "tcgen05 M=128 shape");
-static_assert(kConsumers == kBM, "one epilogue thread per accumulator lane");
-static_assert(kRawBytes % 128 == 0, "raw stages stay 128-byte aligned");
-static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+static_assert(kThreads == kBM, "one epilogue thread per accumulator lane");
 
 // Instruction descriptor of kind::f16: D fp32 (bits 4-5 = 1), A and B bf16
 // (bits 7-9, 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bit 17,
@@ -127,13 +117,61 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// A bounded wait (no early exit on other launches' error words: shared and
-// tensor memory stay in use until this kernel's own copies and MMAs end).
+// A bounded wait on the kernel's own MMAs (no early exit on other launches'
+// error words: tensor memory and shared memory stay in use until they end).
 __device__ __forceinline__ bool own_wait(uint64_t* bar, uint32_t parity, int* err) {
   for (long long i = 0; i < kSpinLimit; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   record_error(err, kErrTimeout);
   return false;
+}
+
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, bool ok) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src),
+               "r"(ok ? 4 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool ok) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(ok ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// One bf16 stage by cp.async: each lane's 16-byte fragment of a W tile as
+// four 4-byte copies into its four core matrices; X as in store_stage.  An
+// operand outside the matrix copies zero bytes (the slot is zero-filled).
+__device__ __forceinline__ void issue_stage_bf16(const GemmTcArgs& a, int m0, int n0, int k0,
+                                                 uint32_t sa, uint32_t sb) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int Kt = a.K >> 4, rt_valid = (a.N + 15) >> 4;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int tl = warp * 8 + i;
+    const int rt = tl >> 2, kt = tl & 3;
+    const int grt = (m0 >> 4) + rt, gkt = (k0 >> 4) + kt;
+    const bool ok = grt < rt_valid && gkt < Kt;
+    const uint8_t* src = ok ? a.w + ((size_t)grt * Kt + gkt) * 512 + lane * 16 : a.w;
+    const uint32_t d = sa + (2 * rt) * kSBO + (2 * kt) * kLBO + lane * 4;
+    cp_async4(d, src, ok);
+    cp_async4(d + kSBO, ok ? src + 4 : src, ok);
+    cp_async4(d + kLBO, ok ? src + 8 : src, ok);
+    cp_async4(d + kSBO + kLBO, ok ? src + 12 : src, ok);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int c = i * kThreads + tid;
+    const int tok = n0 + (c >> 6) * 8 + (c & 7);
+    const int k = k0 + ((c >> 3) & 7) * 8;
+    const bool ok = tok < a.T && k < a.K;
+    cp_async16(sb + (uint32_t)c * 16, ok ? a.x + (size_t)tok * a.ldx + k : a.x, ok);
+  }
 }
 
 // bf16 pair of two biased int8 bytes (q + 128), exact.
@@ -143,104 +181,90 @@ __device__ __forceinline__ uint32_t i8pair_to_bf16x2(uint32_t b0, uint32_t b1) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// Producer: stage kb of the raw ring by bulk copies, all completing on
-// `full`.  W: per 16-row tile its (up to) 4 K-tiles, one copy; X: per token
-// its inputs k0 .. k0 + 63 (fewer at the end of K), one copy.
-template <int WF>
-__device__ __forceinline__ void produce_stage(const GemmTcArgs& a, int m0, int n0, int kb,
-                                              uint8_t* raw, uint64_t* full, int lane) {
-  constexpr int TB = WF == WF_BF16 ? 512 : 256;  // bytes of one 16x16 tile
-  const int Kt = a.K >> 4, rt_valid = (a.N + 15) >> 4;
-  const int gkt0 = kb * (kBK / 16);
-  const int nkt = Kt - gkt0 < 4 ? Kt - gkt0 : 4;
-  const int nrt = rt_valid - (m0 >> 4) < 8 ? rt_valid - (m0 >> 4) : 8;
-  const int ntok = a.T - n0 < kBN ? a.T - n0 : kBN;
-  const uint32_t xbytes = (uint32_t)nkt * 32;   // 16 inputs of 2 bytes per K-tile
-  const uint32_t bytes = (uint32_t)(nrt * nkt * TB) + (uint32_t)ntok * xbytes;
-  if (lane == 0) mbar_arrive_expect_tx(full, bytes);
-  __syncwarp();
-  if (lane < nrt) {
-    const int grt = (m0 >> 4) + lane;
-    bulk_g2s_nohint(raw + lane * 4 * TB, a.w + ((size_t)grt * Kt + gkt0) * TB,
-                    (uint32_t)(nkt * TB), full);
-  }
-  uint8_t* rx = raw + kRawW;
-  for (int t = lane; t < ntok; t += 32)
-    bulk_g2s_nohint(rx + t * kXPitch, a.x + (size_t)(n0 + t) * a.ldx + (size_t)kb * kBK, xbytes,
-                    full);
-}
+// One stage's operands in registers: 8 fragment tiles of W per warp (one
+// 16-byte fragment per lane each) and 8 16-byte chunks of X per thread.
+struct StageRegs {
+  uint4 w[8];
+  uint4 x[8];
+};
 
-// Consumers: raw stage -> canonical buffer (zeros outside the matrices).
 template <int WF>
-__device__ __forceinline__ void rewrite_stage(const GemmTcArgs& a, int m0, int n0, int kb,
-                                              const uint8_t* raw, uint8_t* ca, int tid) {
-  constexpr int TB = WF == WF_BF16 ? 512 : 256;
-  const int warp = tid >> 5, lane = tid & 31;
-  const int Kt = a.K >> 4, rt_valid = (a.N + 15) >> 4;
-  const int gkt0 = kb * (kBK / 16);
+__device__ __forceinline__ void load_stage(const GemmTcArgs& a, int m0, int n0, int k0,
+                                           StageRegs& R) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int Kt = a.K >> 4;                   // 16-wide K tiles per row tile
+  const int rt_valid = (a.N + 15) >> 4;      // stored row tiles
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const int tl = warp * 8 + i;  // tile (rt, kt) of the 8 x 4 block
+    const int tl = warp * 8 + i;             // tile of the 8 x 4 block: (rt, kt)
     const int rt = tl >> 2, kt = tl & 3;
+    const int grt = (m0 >> 4) + rt, gkt = (k0 >> 4) + kt;
     uint4 v = make_uint4(0, 0, 0, 0);
-    if ((m0 >> 4) + rt < rt_valid && gkt0 + kt < Kt) {
-      const uint8_t* src = raw + (rt * 4 + kt) * TB;
+    if (grt < rt_valid && gkt < Kt) {
+      const size_t tile = (size_t)grt * Kt + gkt;
       if constexpr (WF == WF_BF16) {
-        v = *reinterpret_cast<const uint4*>(src + lane * 16);
+        v = __ldg(reinterpret_cast<const uint4*>(a.w + tile * 512) + lane);
       } else {
-        const uint2 q = *reinterpret_cast<const uint2*>(src + lane * 8);
+        const uint2 q = __ldg(reinterpret_cast<const uint2*>(a.w + tile * 256) + lane);
         v.x = i8pair_to_bf16x2(q.x & 0xFF, (q.x >> 8) & 0xFF);
         v.y = i8pair_to_bf16x2((q.x >> 16) & 0xFF, q.x >> 24);
         v.z = i8pair_to_bf16x2(q.y & 0xFF, (q.y >> 8) & 0xFF);
         v.w = i8pair_to_bf16x2((q.y >> 16) & 0xFF, q.y >> 24);
       }
     }
+    R.w[i] = v;
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int c = i * kThreads + tid;        // chunk = (token group, k group, token in group)
+    const int tok = n0 + (c >> 6) * 8 + (c & 7);
+    const int k = k0 + ((c >> 3) & 7) * 8;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (tok < a.T && k < a.K)
+      v = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)tok * a.ldx + k));
+    R.x[i] = v;
+  }
+}
+
+__device__ __forceinline__ void store_stage(uint8_t* sa, uint8_t* sb, const StageRegs& R) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int tl = warp * 8 + i;
+    const int rt = tl >> 2, kt = tl & 3;
     // fragment words: (row g, k 2t), (row g+8, k 2t), (row g, k 2t+8),
     // (row g+8, k 2t+8) with g = lane / 4, t = lane % 4 -> word `lane` of
     // core matrices (2rt, 2kt), (2rt+1, 2kt), (2rt, 2kt+1), (2rt+1, 2kt+1)
-    uint8_t* d = ca + (2 * rt) * kSBO + (2 * kt) * kLBO + lane * 4;
-    *reinterpret_cast<uint32_t*>(d) = v.x;
-    *reinterpret_cast<uint32_t*>(d + kSBO) = v.y;
-    *reinterpret_cast<uint32_t*>(d + kLBO) = v.z;
-    *reinterpret_cast<uint32_t*>(d + kSBO + kLBO) = v.w;
+    uint8_t* base = sa + (2 * rt) * kSBO + (2 * kt) * kLBO + lane * 4;
+    *reinterpret_cast<uint32_t*>(base) = R.w[i].x;
+    *reinterpret_cast<uint32_t*>(base + kSBO) = R.w[i].y;
+    *reinterpret_cast<uint32_t*>(base + kLBO) = R.w[i].z;
+    *reinterpret_cast<uint32_t*>(base + kSBO + kLBO) = R.w[i].w;
   }
-  const uint8_t* rx = raw + kRawW;
-  uint8_t* cb = ca + kOpBytes;
-  const int kin = a.K - kb * kBK;  // inputs of this stage (>= 16)
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    // chunk c = (token group c / 64, k group (c / 8) % 8, token c % 8) -> byte 16 c
-    const int c = i * kConsumers + tid;
-    const int t = (c >> 6) * 8 + (c & 7), kk = (c >> 3) & 7;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (n0 + t < a.T && kk * 8 < kin) v = *reinterpret_cast<const uint4*>(rx + t * kXPitch + kk * 16);
-    *reinterpret_cast<uint4*>(cb + (size_t)c * 16) = v;
+    const int c = i * kThreads + tid;
+    // (token group c / 64, k group (c / 8) % 8, token c % 8) -> byte 16 c
+    *reinterpret_cast<uint4*>(sb + (size_t)c * 16) = R.x[i];
   }
 }
 
 template <int WF, int EPI>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const GemmTcArgs a) {
+  constexpr int S = WF == WF_BF16 ? kStagesBF16 : kStagesI8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* canon = smem;                                   // [kCanon][A | B]
-  uint8_t* raw = smem + kCanon * kCanonBytes;              // [kRawStages][W | X]
-  uint64_t* full = reinterpret_cast<uint64_t*>(raw + kRawStages * kRawBytes);
-  uint64_t* rempty = full + kRawStages;
-  uint64_t* cempty = rempty + kRawStages;
-  uint64_t* done = cempty + kCanon;
+  uint8_t* ops = smem;                                             // [stage][A | B]
+  uint64_t* empty = reinterpret_cast<uint64_t*>(smem + S * kStageBytes);
+  uint64_t* done = empty + S;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n0 = blockIdx.x * kBN;  // tokens: fastest, so the CTAs of one W block share it in L2
   const int m0 = blockIdx.y * kBM;
-  const int KB = (a.K + kBK - 1) / kBK;
 
   if (tid == 0) {
-    for (int s = 0; s < kRawStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&rempty[s], 1);
-    }
-    for (int c = 0; c < kCanon; ++c) mbar_init(&cempty[c], 1);
+    for (int s = 0; s < S; ++s) mbar_init(&empty[s], 1);
     mbar_init(done, 1);
     fence_barrier_init();
   }
@@ -252,38 +276,60 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const GemmTcArgs a
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   tc_fence_before();
-  __syncthreads();  // the last barrier of all 160 threads
+  __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kConsumers / 32) {  // producer warp
-    bool ok = true;
-    for (int kb = 0; kb < KB && ok; ++kb) {
-      const int s = kb % kRawStages;
-      if (kb >= kRawStages) ok = own_wait(&rempty[s], (uint32_t)((kb / kRawStages) - 1) & 1u, a.err);
-      if (ok) produce_stage<WF>(a, m0, n0, kb, raw + (size_t)s * kRawBytes, &full[s], lane);
-    }
-    return;
-  }
-
-  bool ok = true;
-  for (int kb = 0; kb < KB; ++kb) {
-    const int s = kb % kRawStages, c = kb % kCanon;
-    if (ok) ok = own_wait(&full[s], (uint32_t)(kb / kRawStages) & 1u, a.err);
-    if (kb >= kCanon && ok) ok = own_wait(&cempty[c], (uint32_t)((kb / kCanon) - 1) & 1u, a.err);
-    uint8_t* ca = canon + (size_t)c * kCanonBytes;
-    rewrite_stage<WF>(a, m0, n0, kb, raw + (size_t)s * kRawBytes, ca, tid);
-    fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
-    named_bar_sync(kBarConsumers, kConsumers);
-    if (tid == 0) {
-      mbar_arrive(&rempty[s]);  // the raw stage is free for the producer
-      tc_fence_after();
-      const uint32_t a0 = smem_u32(ca), b0 = a0 + kOpBytes;
+  const int KB = (a.K + kBK - 1) / kBK;
+  auto issue_mma = [&](int kb) {
+    const int s = kb % S;
+    tc_fence_after();
+    const uint32_t a0 = smem_u32(ops + (size_t)s * kStageBytes), b0 = a0 + kOpBytes;
 #pragma unroll
-      for (int ks = 0; ks < kBK / kMmaK; ++ks)  // K = 16: two core matrices along K
-        tc_mma(tmem, smem_desc(a0 + ks * 2 * kLBO), smem_desc(b0 + ks * 2 * kLBO),
-               (kb > 0 || ks > 0) ? 1u : 0u);
-      tc_commit(&cempty[c]);
+    for (int ks = 0; ks < kBK / kMmaK; ++ks)  // K = 16: two core matrices along K
+      tc_mma(tmem, smem_desc(a0 + ks * 2 * kLBO), smem_desc(b0 + ks * 2 * kLBO),
+             (kb > 0 || ks > 0) ? 1u : 0u);
+    tc_commit(&empty[s]);
+  };
+  if constexpr (WF == WF_BF16) {
+    const uint32_t ops0 = smem_u32(ops);
+#pragma unroll 1
+    for (int s = 0; s < S - 1; ++s) {
+      if (s < KB) issue_stage_bf16(a, m0, n0, s * kBK, ops0 + s * kStageBytes,
+                                   ops0 + s * kStageBytes + kOpBytes);
+      cp_async_commit();
+    }
+    bool ok = true;
+#pragma unroll 1
+    for (int kb = 0; kb < KB; ++kb) {
+      cp_async_wait<S - 2>();    // this thread's copies of stage kb have landed
+      fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+      __syncthreads();
+      if (tid == 0) issue_mma(kb);
+      const int nk = kb + S - 1;  // refill the slot the MMAs of kb - 1 read
+      if (nk < KB) {
+        const int s = nk % S;
+        if (kb >= 1 && ok) ok = own_wait(&empty[s], (uint32_t)((kb - 1) / S) & 1u, a.err);
+        issue_stage_bf16(a, m0, n0, nk * kBK, ops0 + s * kStageBytes,
+                         ops0 + s * kStageBytes + kOpBytes);
+      }
+      cp_async_commit();
+    }
+  } else {
+    StageRegs R;
+    load_stage<WF>(a, m0, n0, 0, R);
+    bool ok = true;
+#pragma unroll 1
+    for (int kb = 0; kb < KB; ++kb) {
+      const int s = kb % S;
+      uint8_t* sa = ops + (size_t)s * kStageBytes;
+      uint8_t* sb = sa + kOpBytes;
+      if (kb >= S && ok) ok = own_wait(&empty[s], (uint32_t)((kb / S) - 1) & 1u, a.err);
+      store_stage(sa, sb, R);
+      fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor core
+      __syncthreads();
+      if (kb + 1 < KB) load_stage<WF>(a, m0, n0, (kb + 1) * kBK, R);
+      if (tid == 0) issue_mma(kb);
     }
   }
   if (tid == 0) tc_commit(done);
@@ -321,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const GemmTcArgs a
   }
 
   tc_fence_before();
-  named_bar_sync(kBarConsumers, kConsumers);
+  __syncthreads();
   if (warp == 0) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
@@ -333,11 +379,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const GemmTcArgs a
 template <int WF, int EPI>
 cudaError_t launch_gemm_tc_t(const GemmTcArgs& a, cudaStream_t st) {
   auto kern = gemm_tc_kernel<WF, EPI>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kSmemBytes);
+  const size_t smem = smem_bytes(WF == WF_BF16 ? kStagesBF16 : kStagesI8);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const dim3 grid((a.T + kBN - 1) / kBN, (a.N + kBM - 1) / kBM);
-  kern<<<grid, kThreads, kSmemBytes, st>>>(a);
+  kern<<<grid, kThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
 
