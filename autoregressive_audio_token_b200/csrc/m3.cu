@@ -169,8 +169,10 @@ struct m3_ctx {
   bf16** d_fb_aud = nullptr;       // device array of the fb_aud pointers
   LoopState* loop = nullptr;
   unsigned long long* d_vpages = nullptr;  // prefill: every row -> one sequence's pages
-  // prefill on the tensor-core GEMM: prompt chunks of pf_chunk tokens
-  bool prefill_tc = true;
+  // prefill on the tensor-core GEMM, prompt chunks of pf_chunk tokens:
+  // 1 always, 0 never, -1 for bf16 weights only (int8 streams faster through
+  // the decode GEMVs, whose tiles convert in registers without a ring)
+  int prefill_tc = -1;
   int pf_chunk = 256;
   bf16 *pf_x = nullptr, *pf_n = nullptr, *pf_qkv = nullptr, *pf_o = nullptr, *pf_act = nullptr;
   float2* pf_rope = nullptr;       // [pf_chunk][head_dim / 2]
@@ -290,7 +292,7 @@ extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) 
     if (v >= 1 && v <= kAttnMaxSplits) c->max_splits = v;
   }
   if (const char* e = getenv("M3_ATTN_PF")) c->attn_pf = (e[0] == '1');
-  if (const char* e = getenv("M3_PREFILL_TC")) c->prefill_tc = (e[0] == '1');
+  if (const char* e = getenv("M3_PREFILL_TC")) c->prefill_tc = (e[0] == '1') ? 1 : 0;
   if (const char* e = getenv("M3_PREFILL_CHUNK")) {
     const int v = atoi(e);
     if (v >= 16 && v <= 4096) c->pf_chunk = v;
@@ -1229,13 +1231,15 @@ static int record_prefill_layer(m3_ctx* c, const DLayer& L, int T, int p0, int l
 }
 
 static bool prefill_tc_ok(const m3_ctx* c) {
-  if (!c->prefill_tc) return false;
+  if (c->prefill_tc == 0) return false;
   const m3_config& g = c->cfg;
   if (g.hidden % 16 || g.ffn % 16 || (g.n_q_heads * g.head_dim) % 16) return false;
   for (int l = 0; l < g.n_layers; ++l) {
     const DLayer& L = c->L[l];
     for (const DMat* M : {&L.qkv, &L.o, &L.gu, &L.d})
-      if (!M->tiled || (M->wf != WF_BF16 && M->wf != WF_I8ROW)) return false;
+      if (!M->tiled || (M->wf != WF_BF16 && M->wf != WF_I8ROW) ||
+          (c->prefill_tc < 0 && M->wf != WF_BF16))
+        return false;
   }
   return true;
 }

@@ -3,10 +3,11 @@
 Prefilling tokens at positions start .. start + n - 1 is defined as decoding
 them one by one (each token attends to every earlier position of its row and
 to itself); the oracle runs exactly that, token by token, through its
-single-row layers.  The GPU runs the prompt in chunks (256 tokens by default)
-whose projections are tcgen05 GEMMs, with a causal attention over the row's
-cache; M3_PREFILL_TC=0 selects the decode GEMV kernels over chunks of up to
-max_rows tokens instead.  Compared:
+single-row layers.  With M3_PREFILL_TC=1 (the default for bf16 weights) the
+GPU runs the prompt in chunks (256 tokens by default) whose projections are
+tcgen05 GEMMs, with a causal attention over the row's cache; M3_PREFILL_TC=0
+(the default for int8) selects the decode GEMV kernels over chunks of up to
+max_rows tokens.  Compared:
   * the K/V the prefill leaves in the row's cache (every layer, position);
   * the final-normed hidden state of the last token;
   * the other rows' caches, untouched;
@@ -85,9 +86,10 @@ def test_prefill_matches_sequential_decode(ora, start, n, max_rows, wdtype, tc, 
 
 
 @pytest.mark.parametrize("wdtype", [0, 1])
-def test_prefill_8b_layer(ora, wdtype):
+def test_prefill_8b_layer(ora, wdtype, monkeypatch):
     # one Qwen3-8B layer, 160 prompt tokens: the GEMMs at full width (K up to
     # 12288, 48 to 192 weight blocks), two token tiles with a ragged second
+    monkeypatch.setenv("M3_PREFILL_TC", "1")
     s = synth.LAYER8B
     m = Model(s, seed=23, device="cuda", wdtype=wdtype, max_rows=2)
     try:
