@@ -49,7 +49,6 @@ constexpr int kBK = 64;      // K per stage
 constexpr int kMmaK = 16;    // K per tcgen05.mma (bf16)
 constexpr int kStagesBF16 = 6;   // cp.async ring: 5 stages of loads in flight
 constexpr int kStagesI8 = 4;     // register-staged ring (the int8 -> bf16 conversion)
-constexpr int kMaxStages = 6;
 constexpr int kThreads = 128;
 constexpr int kOpBytes = kBM * kBK * 2;          // one operand of one stage: 16 KB
 constexpr int kStageBytes = 2 * kOpBytes;
