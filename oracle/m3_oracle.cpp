@@ -147,6 +147,13 @@ float ora_gumbel(uint64_t seed, uint64_t frame, uint64_t row, uint64_t index) {
   return (float)g;
 }
 
+// G(seed, frame, row, index0 + i) for i < n.
+void ora_gumbel_fill(uint64_t seed, uint64_t frame, uint64_t row, uint64_t index0, int64_t n,
+                     float* out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < n; ++i) out[i] = ora_gumbel(seed, frame, row, index0 + (uint64_t)i);
+}
+
 // ---------------------------------------------------- int8 quantiser -------
 // One symmetric scale per group of `group` consecutive elements of a row
 // (group == cols gives one scale per row):
@@ -187,7 +194,42 @@ struct OraMat {
   int wfmt;
 };
 
+// The summation-order comparator: with g_acc64 set, every GEMV sum runs in
+// fp64 (each product exact, one rounding to fp32 at the end) instead of the
+// sequential fp32 loop.  It is the same definition computed with a different
+// (more accurate) summation, used by the tests to measure how far two
+// correct summation orders of the same frame drift apart after many layers.
+static int g_acc64 = 0;
+
+static void gemv64(const OraMat& m, int64_t rows, int64_t cols, const float* x, float* y) {
+#pragma omp parallel for schedule(static)
+  for (int64_t o = 0; o < rows; ++o) {
+    double tot = 0.0;
+    if (m.wfmt == 0) {
+      const bf16_t* wr = m.w + o * cols;
+      for (int64_t i = 0; i < cols; ++i) tot += (double)bf2f(wr[i]) * (double)x[i];
+    } else if (m.wfmt == 1) {
+      const int8_t* qr = m.q + o * cols;
+      for (int64_t i = 0; i < cols; ++i) tot += (double)qr[i] * (double)x[i];
+      tot *= (double)m.s[o];
+    } else {
+      const int8_t* qr = m.q + o * cols;
+      int64_t ng = cols / 128;
+      for (int64_t g = 0; g < ng; ++g) {
+        double acc = 0.0;
+        for (int64_t i = g * 128; i < g * 128 + 128; ++i) acc += (double)qr[i] * (double)x[i];
+        tot += (double)m.s[o * ng + g] * acc;
+      }
+    }
+    y[o] = (float)tot;
+  }
+}
+
 static void gemv(const OraMat& m, int64_t rows, int64_t cols, const float* x, float* y) {
+  if (g_acc64) {
+    gemv64(m, rows, cols, x, y);
+    return;
+  }
 #pragma omp parallel for schedule(static)
   for (int64_t o = 0; o < rows; ++o) {
     if (m.wfmt == 0) {
@@ -219,6 +261,9 @@ void ora_gemv(const bf16_t* w, const int8_t* q, const float* s, int wfmt, int64_
   OraMat m{w, q, s, wfmt};
   gemv(m, rows, cols, x, y);
 }
+
+// 0: sequential fp32 GEMV sums (the oracle's definition); 1: fp64 sums.
+void ora_set_accum64(int on) { g_acc64 = on ? 1 : 0; }
 
 // ------------------------------------------------------------ norms --------
 // RMSNorm as torch's Qwen3RMSNorm computes it on a bf16 tensor:
@@ -442,6 +487,41 @@ void ora_topk_draws(const float* logits, int64_t n, int64_t k, float temperature
   for (int64_t t = 0; t < ndraws; ++t)
     out[t] = (int32_t)topk_gumbel_argmax(logits, n, k, temperature, seed, frame0 + (uint64_t)t, 0,
                                          NoiseIndex{0, -1, 0}, nullptr);
+}
+
+// The draw on given per-row logits [rows, n] (another implementation's
+// logits): with cfg_scale > 0 the rows are (cond, uncond) pairs and
+// g = l_u + c (l_c - l_u) is drawn once per pair with key_row = pair index
+// (both rows get the code); else g = l with key_row = row.  Candidate i has
+// noise index index_base + i, except candidate end_i (>= 0), whose index is
+// end_index.  margin (nullable): per row the gap between the best and the
+// second-best z.  Returns -1 when cfg_scale > 0 and rows is odd.
+int ora_draw(const float* logits, int rows, int64_t n, float cfg_scale, float temperature,
+             int top_k, uint64_t seed, uint64_t frame, uint64_t index_base, int64_t end_i,
+             uint64_t end_index, int32_t* codes, float* margin) {
+  if (cfg_scale > 0.0f && (rows % 2)) return -1;
+  const NoiseIndex ni{index_base, end_i, end_index};
+  const int npick = cfg_scale > 0.0f ? rows / 2 : rows;
+  std::vector<float> g(n);
+  for (int p = 0; p < npick; ++p) {
+    if (cfg_scale > 0.0f) {
+      const float* lc = logits + (size_t)(2 * p) * n;
+      const float* lu = logits + (size_t)(2 * p + 1) * n;
+      for (int64_t i = 0; i < n; ++i) g[i] = lu[i] + cfg_scale * (lc[i] - lu[i]);
+    } else {
+      std::memcpy(g.data(), logits + (size_t)p * n, sizeof(float) * n);
+    }
+    float mg = 0.0f;
+    const int64_t best = topk_gumbel_argmax(g.data(), n, top_k, temperature, seed, frame,
+                                            (uint64_t)p, ni, &mg);
+    const int rr[2] = {cfg_scale > 0.0f ? 2 * p : p, cfg_scale > 0.0f ? 2 * p + 1 : -1};
+    for (int q = 0; q < 2; ++q) {
+      if (rr[q] < 0) continue;
+      codes[rr[q]] = (int32_t)best;
+      if (margin) margin[rr[q]] = mg;
+    }
+  }
+  return 0;
 }
 
 // Repeated draws from fixed logits: draw t uses frame = frame0 + t and

@@ -102,6 +102,13 @@ def lib():
         L.ora_topk_draw.argtypes = [vp, i64, i64, f32, u64, u64, u64, u64]
         L.ora_topk_draws.restype = None
         L.ora_topk_draws.argtypes = [vp, i64, i64, f32, u64, u64, i64, vp]
+        L.ora_set_accum64.restype = None
+        L.ora_set_accum64.argtypes = [C.c_int]
+        L.ora_gumbel_fill.restype = None
+        L.ora_gumbel_fill.argtypes = [u64, u64, u64, u64, i64, vp]
+        L.ora_draw.restype = C.c_int
+        L.ora_draw.argtypes = [vp, C.c_int, i64, f32, f32, C.c_int, u64, u64, u64, i64, u64, vp,
+                               vp]
         L.ora_num_threads.restype = C.c_int
         L.ora_set_num_threads.argtypes = [C.c_int]
         _lib = L
@@ -200,6 +207,41 @@ def topk_draws(logits, k, temperature, seed, frame0, ndraws) -> np.ndarray:
     out = np.empty(ndraws, np.int32)
     lib().ora_topk_draws(_p(lg), lg.size, k, temperature, seed, frame0, ndraws, _p(out))
     return out
+
+
+def gumbel_fill(seed, frame, row, index0, n) -> np.ndarray:
+    """G(seed, frame, row, index0 + i) for i < n, fp32."""
+    out = np.empty(n, np.float32)
+    lib().ora_gumbel_fill(seed, frame, row, index0, n, _p(out))
+    return out
+
+
+def draw(logits, seed, frame, cfg_scale=0.0, temperature=1.0, top_k=0, index_base=0,
+         end_i=-1, end_index=0):
+    """The oracle's draw on given per-row logits [rows, n] (CFG pairs when
+    cfg_scale > 0): (codes [rows], margins [rows])."""
+    lg = np.ascontiguousarray(logits, np.float32)
+    rows, n = lg.shape
+    codes = np.empty(rows, np.int32)
+    mg = np.empty(rows, np.float32)
+    rc = lib().ora_draw(_p(lg), rows, n, cfg_scale, temperature, top_k, seed, frame, index_base,
+                        end_i, end_index, _p(codes), _p(mg))
+    if rc != 0:
+        raise RuntimeError(f"ora_draw: {rc}")
+    return codes, mg
+
+
+class accum64:
+    """Context manager: the oracle's GEMV sums in fp64 (the summation-order
+    comparator) inside the block, the fp32 definition outside."""
+
+    def __enter__(self):
+        lib().ora_set_accum64(1)
+        return self
+
+    def __exit__(self, *exc):
+        lib().ora_set_accum64(0)
+        return False
 
 
 def set_threads(n: int) -> None:

@@ -268,3 +268,115 @@ def test_depth_noise_index_per_codebook(ora):
     for j in range(D.codebooks):
         z = [L.ora_gumbel(9, 0, 0, ((j + 1) << 32) | i) for i in range(D.vocab)]
         assert codes[0, j] == int(np.argmax(z))
+
+
+# ------------------------------------------------ the q/k norm -> RoPE chain --
+
+def _rbf(x):
+    """fp64 -> fp32 -> bf16 (round to nearest even) -> fp64, in numpy."""
+    b = np.asarray(x, np.float64).astype(np.float32).view(np.uint32).astype(np.uint64)
+    b = ((b + 0x7FFF + ((b >> 16) & 1)) >> 16) << 16
+    return b.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def _to_bits(x):
+    return (np.asarray(_rbf(x), np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def _head_chain(v, gamma, pos, theta, eps):
+    """The reading of the head step (DiffSynth-Studio article, "各子模型的结构要点":
+    Qwen3 q/k RMSNorm, then rope_theta 1e6 rotary embedding, half rotation):
+    bf16(RoPE_pos(bf16(gamma * bf16(v / rms(v))))), here in fp64."""
+    d = v.size
+    n = _rbf(v / np.sqrt(np.mean(v * v) + eps))
+    n = _rbf(gamma * n)
+    i = np.arange(d // 2)
+    ang = pos * theta ** (-2.0 * i / d)
+    c, s = np.cos(ang), np.sin(ang)
+    a, b = n[: d // 2], n[d // 2:]
+    return _rbf(np.concatenate([a * c - b * s, b * c + a * s]))
+
+
+def test_qk_norm_rope_chain_and_score(ora):
+    """Pins the order of the head step inside the layer, which the function
+    pins of RMSNorm and RoPE alone cannot: x = e_a makes the normalised input
+    16 e_a exactly, so q, k and v are 16 x (column a of Wq, Wk, Wv), chosen
+    bf16 values.  The key stored at `pos` must be the rotated, normalised,
+    gained key of the closed form; a norm after the rotation, an unrotated
+    key, the angle of pos + 1 or the q gain on k each move it by far more
+    than one bf16 step.  The attention output (Wo = I) then exposes the two
+    softmax weights of a two-position context, whose log ratio must be the
+    fp64 score difference q'.(k'_1 - k_0)/sqrt(d) of the same closed form."""
+    s = synth.TINY
+    d, Hq, Hkv, H = s.head_dim, s.n_q_heads, s.n_kv_heads, s.hidden
+    grp = Hq // Hkv
+    rng = np.random.default_rng(11)
+    a = 5                                     # the one non-zero input column
+    bq, bk = 7, 9                             # value dims that carry p0 and p1
+
+    def bf(x):
+        return torch.from_numpy(_to_bits(x).view(np.int16)).view(torch.bfloat16)
+
+    Lw = synth.layer_weights(s, 0, 0)
+    wq = np.zeros((Hq * d, H)); wq[:, a] = rng.standard_normal(Hq * d) * 0.25
+    wk = np.zeros((Hkv * d, H)); wk[:, a] = rng.standard_normal(Hkv * d) * 0.25
+    wv = np.zeros((Hkv * d, H))
+    for g in range(Hkv):
+        wv[g * d + bk, a] = 1.0 / 16.0       # v_1 = e_bk in every KV head
+    Lw.update(wq=bf(wq), wk=bf(wk), wv=bf(wv), wo=torch.eye(H, dtype=torch.bfloat16),
+              wd=torch.zeros_like(Lw["wd"]), attn_norm=bf(np.ones(H)),
+              q_norm=bf(1.0 + 0.5 * np.sign(np.sin(np.arange(d) * 1.7))),
+              k_norm=bf(np.where(np.arange(d) < d // 2, 1.75, 0.375)))
+    body = ora.Body(s, [Lw], synth.final_norm(s, 0), synth.lm_head_slice(s, 0))
+    gq = _f(_bits(Lw["q_norm"])).astype(np.float64)
+    gk = _f(_bits(Lw["k_norm"])).astype(np.float64)
+    theta, eps = s.rope_theta, s.rms_eps
+
+    rows, maxp = 2, 64
+    positions = [1, 37]
+    kc, vc = body.new_cache(rows, maxp)
+    k0 = rng.standard_normal((Hkv, d)) * 1.5
+    kc[0, 0, 0] = _to_bits(k0)
+    v0 = np.zeros((Hkv, d)); v0[:, bq] = 1.0  # v_0 = e_bq
+    vc[0, 0, 0] = _to_bits(v0)
+    K, V = synth.kv_prefill(s, 1, 37, 3)
+    kc[1, 0, :37] = _bits(K[0])
+    vc[1, 0, :37] = _bits(V[0])
+    x = np.zeros((rows, H), np.uint16)
+    x[:, a] = 0x3F80                          # 1.0
+    out = body.body(kc, vc, positions, x)
+
+    q = _f(_bits(Lw["wq"]))[:, a].astype(np.float64) * 16.0
+    k = _f(_bits(Lw["wk"]))[:, a].astype(np.float64) * 16.0
+    ulp = 2.0 ** -7                           # one bf16 step, relative
+    for r, pos in enumerate(positions):
+        got = _f(kc[r, 0, pos]).astype(np.float64)
+        for g in range(Hkv):
+            ref = _head_chain(k[g * d:(g + 1) * d], gk, pos, theta, eps)
+            dev = np.abs(got[g] - ref)
+            assert np.all(dev <= ulp * np.abs(ref) + 1e-30), (r, g, dev.max())
+            assert np.mean(dev == 0) >= 0.95
+            # the plausible misreadings all land far away
+            n = _rbf(k[g * d:(g + 1) * d] / np.sqrt(np.mean(k[g * d:(g + 1) * d] ** 2) + eps))
+            wrong = {
+                "unrotated": _rbf(gk * n),
+                "pos+1": _head_chain(k[g * d:(g + 1) * d], gk, pos + 1, theta, eps),
+                "q gain": _head_chain(k[g * d:(g + 1) * d], gq, pos, theta, eps),
+                "rope first": _rbf(gk * _rbf(_head_chain(k[g * d:(g + 1) * d], np.ones(d), pos,
+                                                         theta, eps))),
+            }
+            for name, w in wrong.items():
+                assert np.max(np.abs(got[g] - w)) > 0.05, name
+        assert (_f(vc[r, 0, pos]).reshape(Hkv, d)[:, bk] == 1.0).all()
+
+    # row 0: context {0, 1}; o_h = p0 e_bq + p1 e_bk, and Wo = I puts o_h at x[h d + .]
+    xo = _f(out[0]).astype(np.float64)
+    for h in range(Hq):
+        g = h // grp
+        qh = _head_chain(q[h * d:(h + 1) * d], gq, 1, theta, eps)
+        k1 = _f(kc[0, 0, 1, g]).astype(np.float64)
+        ds = qh @ (k1 - _f(kc[0, 0, 0, g]).astype(np.float64)) / np.sqrt(d)
+        p0, p1 = xo[h * d + bq], xo[h * d + bk]
+        assert abs(p0 + p1 - 1.0) < 2e-2
+        # p0, p1 are bf16 values: ln(p1/p0) holds them to about 2 x 2^-8
+        assert abs(np.log(p1 / p0) - ds) < 2e-2 + 0.01 * abs(ds), (h, np.log(p1 / p0), ds)

@@ -128,3 +128,13 @@ def test_gumbel_range_bound(ora):
     for i in range(20000):
         g = L.ora_gumbel(5, 5, 5, i)
         assert lo - 1e-5 <= g <= hi + 1e-5
+
+
+def test_gumbel_fill_is_the_generator(ora):
+    """The bulk fill returns the generator's values, including the depth
+    decoder's indices (j << 32) | i and the end token's vocab row."""
+    for seed, frame, row, base in [(0, 0, 0, 0), (7, 123, 3, 151675), (1, 2, 1, 5 << 32),
+                                   (9, 9, 0, 151670)]:
+        got = ora.gumbel_fill(seed, frame, row, base, 64)
+        ref = np.array([ora.gumbel(seed, frame, row, base + i) for i in range(64)], np.float32)
+        assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))

@@ -216,3 +216,33 @@ def test_attention_special_cases(ora):
     assert np.array_equal(ora.attention(q, k, v[:1]), v[0])  # one position -> v_0
     kk = np.repeat(k, 5, 0)  # equal keys -> mean of V
     assert np.allclose(ora.attention(q, kk, v), v.astype(np.float64).mean(0), atol=1e-6)
+
+
+def test_gemv_fp64_comparator(ora):
+    """The summation-order comparator of the oracle's GEMV: with fp64 sums the
+    result is the fp64 dot product rounded once to fp32 (numpy's fp64 matmul,
+    within one fp32 step), in every weight format; outside the block the
+    sequential fp32 definition is back."""
+    rng = np.random.default_rng(5)
+    rows, cols = 64, 4096
+    w = (rng.standard_normal((rows, cols)).astype(np.float32) * 0.02)
+    wb = (w.view(np.uint32) >> 16).astype(np.uint16)
+    wf = (wb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    x = rng.standard_normal(cols).astype(np.float32)
+    y32 = ora.gemv(w=wb, wfmt=0, x=x)
+    with ora.accum64():
+        y64 = ora.gemv(w=wb, wfmt=0, x=x)
+        q, s = ora.quantize(wb, None)
+        yq = ora.gemv(q=q, s=s, wfmt=1, x=x)
+        qg, sg = ora.quantize(wb, 128)
+        yg = ora.gemv(q=qg, s=sg, wfmt=2, x=x)
+    ref = (wf @ x.astype(np.float64)).astype(np.float32)
+    step = np.spacing(np.abs(ref))
+    assert np.all(np.abs(y64 - ref) <= step)
+    refq = (q.astype(np.float64) @ x.astype(np.float64) * s.astype(np.float64)).astype(np.float32)
+    assert np.all(np.abs(yq - refq) <= np.spacing(np.abs(refq)))
+    refg = sum((qg[:, g * 128:(g + 1) * 128].astype(np.float64) @ x[g * 128:(g + 1) * 128]
+                .astype(np.float64)) * sg[:, g] for g in range(cols // 128)).astype(np.float32)
+    assert np.all(np.abs(yg - refg) <= 2 * np.spacing(np.abs(refg)))
+    assert np.array_equal(ora.gemv(w=wb, wfmt=0, x=x), y32)
+    assert not np.array_equal(y32, y64)  # the two orders do differ

@@ -86,3 +86,34 @@ def test_sampler_topk_draws_within_the_kept_set(ora):
         codes, _ = body.sample(h, seed=1, frame=f, cfg_scale=1.5)
         outside += int(codes[0]) not in keep
     assert outside > 0
+
+
+def test_draw_on_given_logits(ora):
+    """ora_draw, the sampler applied to another implementation's logits: its
+    code is the argmax of g/T + G over the noise the pinned generator gives
+    (computed here with numpy's argmax), its margin the gap to the runner-up;
+    guidance c = 1 reproduces the cond row, and the pair shares one draw keyed
+    by the pair index.  Depth-style noise indices (j << 32) | i and an end
+    candidate with its own vocab row as index are honoured."""
+    rng = np.random.default_rng(4)
+    n = 300
+    for trial in range(6):
+        lg = rng.standard_normal((4, n)).astype(np.float32) * 2
+        base = (3 << 32) if trial % 2 else 151675
+        codes, mg = ora.draw(lg, seed=trial, frame=9, index_base=base, temperature=0.8)
+        for r in range(4):
+            z = lg[r] / np.float32(0.8) + ora.gumbel_fill(trial, 9, r, base, n)
+            order = np.argsort(-z, kind="stable")
+            assert codes[r] == order[0]
+            assert mg[r] == np.float32(z[order[0]] - z[order[1]])
+        # c = 1: g = l_u + 1 (l_c - l_u) = l_c for exactly representable logits
+        q = np.round(lg * 8) / 8
+        pc, _ = ora.draw(q, seed=trial, frame=9, cfg_scale=1.0, index_base=base)
+        cc, _ = ora.draw(q[0::2].copy(), seed=trial, frame=9, index_base=base)
+        assert np.array_equal(pc[0::2], cc) and np.array_equal(pc[1::2], cc)
+    # an end candidate: index 0 carries noise index 151670 instead of base + 0
+    lg = np.zeros((1, 8), np.float32)
+    c, _ = ora.draw(lg, seed=2, frame=3, index_base=1000, end_i=0, end_index=151670)
+    z = ora.gumbel_fill(2, 3, 0, 1000, 8)
+    z[0] = ora.gumbel(2, 3, 0, 151670)
+    assert c[0] == int(np.argmax(z))
