@@ -59,10 +59,6 @@ struct AttnArgs {
   int fixed_pos;              // >= 0: row r is at fixed_pos + r * pos_stride
   int pos_stride;             // 0: one position for all rows (depth decoder); 1: a prompt chunk
   int* err;
-  // L2 prefetch of the weights the next kernels stream (HBM is nearly idle
-  // while attention runs): up to two byte ranges, split evenly over the CTAs
-  const uint8_t* pf[2];
-  size_t pf_bytes[2];
   // 0: decode (the new token's K/V are appended and attended from registers);
   // 1: append only (prefill: every row's K/V of its position, then exit);
   // 2: attend from the cache only, own position included (prefill, after 1)
@@ -196,17 +192,6 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_decode_kernel(const Attn
     for (int b = 0; b < kAttnBuf; ++b) mbar_init(&bars[b], 1);
     fence_barrier_init();
     for (int t = 0; t < min(kAttnBuf, ntiles); ++t) issue_tile(t);
-  } else if (tid == 32) {
-    const size_t nb = (size_t)gridDim.x * gridDim.y * gridDim.z;
-    const size_t b = ((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      if (!a.pf_bytes[q]) continue;
-      const size_t per = (a.pf_bytes[q] / nb + 255) & ~(size_t)255;
-      const size_t lo = b * per, hi = min(lo + per, a.pf_bytes[q]);
-      for (size_t o = lo; o < hi; o += 65536)
-        bulk_prefetch_l2(a.pf[q] + o, (uint32_t)min((size_t)65536, hi - o));
-    }
   }
   __syncthreads();
   pdl_launch_dependents();

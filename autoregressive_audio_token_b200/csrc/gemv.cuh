@@ -121,7 +121,6 @@ struct GemvArgs {
   // tiled kernels (gemv_tile.cuh, gemv_dyn.cuh) only: CTAs per cluster,
   // stage bytes, stages; the dynamic kernel's {claim, done} counter pair
   int tc, tsb, tns;
-  int pfa;  // dynamic GEMV: L2 prefetch this many ring stages ahead (0: none)
   int lazy_claim;  // dynamic GEMV: claim ahead only once the consumers run
   unsigned* ctr;
   // RMSNorm partials: a residual-add launch writes sum(x_new^2) per (row m,

@@ -110,7 +110,6 @@ __global__ void __maxnreg__(128) gemv_dyn_kernel(const GemvArgs a) {
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
       const uint8_t* wb = static_cast<const uint8_t*>(a.w);
-      const int pfa = a.pfa < ppr ? a.pfa : ppr;  // at most into the next unit
       // Before the consumers run, a CTA claims only its first unit: claiming
       // ahead that early would let the CTAs that launch first take two units
       // each before the others start, which unbalances launches of about two
@@ -143,20 +142,6 @@ __global__ void __maxnreg__(128) gemv_dyn_kernel(const GemvArgs a) {
         mbar_arrive_expect_tx(&full[slot], bytes);
         bulk_g2s(ring + (size_t)slot * D.stage, wb + ((size_t)u * T + t0) * TB, bytes,
                  &full[slot], pol);
-        // keep HBM busy past the ring: the part pfa stages later in this
-        // CTA's sequence (in this unit or the one claimed next) goes to L2,
-        // so that the ring's refill of it hits L2
-        if (pfa > 0) {
-          int q = p + pfa, uq = u;
-          if (q >= ppr) {
-            q -= ppr;
-            uq = un;
-          }
-          if (uq >= 0 && uq < U && q < ppr) {
-            const int q0 = q * pt, q1 = min(T, q0 + pt);
-            bulk_prefetch_l2(wb + ((size_t)uq * T + q0) * TB, (uint32_t)((q1 - q0) * TB));
-          }
-        }
         if (++p == ppr) u = -1;
       }
       // this CTA claims no more; the last CTA to stop resets the pair

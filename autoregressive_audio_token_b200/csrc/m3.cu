@@ -9,7 +9,6 @@
 #include <cstdio>
 #include <cstring>
 #include <map>
-#include <mutex>
 #include <string>
 #include <tuple>
 #include <vector>
@@ -18,7 +17,6 @@
 #include "launch.cuh"
 #include "misc.cuh"
 #include "gemv_tile.cuh"
-#include "depth.cuh"
 
 using namespace m3;
 typedef __nv_bfloat16 bf16;
@@ -121,12 +119,6 @@ struct m3_ctx {
   float* dlogits = nullptr;
   unsigned long long* d_dpages = nullptr;
   void* dkv = nullptr;
-  // the depth decoder as one persistent kernel (depth.cuh), opt-in
-  // (M3_DEPTH_FUSED=1): measured slower than its separate launches
-  bool depth_fused = false;
-  bf16 *dfx = nullptr, *dfqkv = nullptr, *dfatt = nullptr, *dfact = nullptr, *dfkv = nullptr;
-  unsigned long long* dfpart = nullptr;
-  unsigned* dfbar = nullptr;
 
   std::map<std::pair<int, int>, cudaGraphExec_t> graphs;
   std::map<std::pair<int, int>, cudaGraphExec_t> dgraphs;
@@ -141,7 +133,6 @@ struct m3_ctx {
   // bf16 leaves the residual projections, O and down, to the cluster-split
   // kernel, which balances them better; int8 claims everywhere)
   int tile_dyn_mask = -1;
-  int tile_pfa = 0;       // dynamic GEMV: L2 prefetch this many ring stages ahead
   int tile_lazy = 1;      // dynamic GEMV: claim ahead only once the consumers run
   std::map<std::tuple<int, int, int, int, int>, TileLaunch> tile_plans;
   // {claim, done} counter pairs of the dynamically scheduled GEMV, one per
@@ -159,10 +150,6 @@ struct m3_ctx {
   bool ssq_track = false;
   float2* rope = nullptr;  // this frame's RoPE (cos, sin) [max_rows][head_dim / 2]
   int top_k = 0;           // the frame draw keeps the top_k guided logits (0: all)
-  // L2 prefetch from the attention kernel: the O projection's tail and the
-  // first attn_pf_bytes of gate/up
-  bool attn_pf = false;
-  size_t attn_pf_bytes = (size_t)16 << 20;
   // generation loop: feedback tables, device state, its host copy, graphs
   bf16* fb_tok = nullptr;          // [slice_len][H]
   std::vector<bf16*> fb_aud;       // depth_codebooks tables [depth_vocab][H]
@@ -180,11 +167,28 @@ struct m3_ctx {
   int* h_err = nullptr;            // pinned
   std::map<std::pair<int, int>, cudaGraphExec_t> lgraphs;
   float* gbuf = nullptr;   // the guided logits of the top-k draw [max_rows][candidates]
+  // host-side fault injection (m3_inject_fault, environment M3_FAULT): the
+  // fault_left-th next call of kind fault_kind fails as its CUDA call would
+  int fault_kind = 0;
+  long long fault_left = 0;
+  // device address of the allocation-free sampler's static scratch on this
+  // context's device (looked up once, at m3_create)
+  unsigned char* noalloc_scratch = nullptr;
 };
+
+// Is this call of `kind` the one scheduled to fail?  (Counts down, then
+// clears the schedule: one injected failure per m3_inject_fault.)
+static bool fault_due(m3_ctx* c, int kind) {
+  if (!c || c->fault_kind != kind) return false;
+  if (--c->fault_left > 0) return false;
+  c->fault_kind = M3_FAULT_NONE;
+  return true;
+}
 
 template <typename T>
 static int dalloc(m3_ctx* c, T** p, size_t bytes) {
   void* q = nullptr;
+  if (fault_due(c, M3_FAULT_ALLOC)) return fail(M3_ENOMEM, "injected device allocation failure");
   CK(cudaMalloc(&q, bytes < 256 ? 256 : bytes));
   c->allocs.push_back(q);
   *p = static_cast<T*>(q);
@@ -269,6 +273,23 @@ static bool valid_cfg(const m3_config* g, std::string& why) {
   return true;
 }
 
+// ------------------------------------------- allocation-free sampler -------
+// Scratch of m3_sample_noalloc: the frame-parameter block, the cross-CTA
+// argmax ticket and the per-CTA partial argmaxes live in this file-scope
+// device array instead of context-owned buffers.  Every GPU that loads the
+// library holds it (about 129 KB) until the process exits.
+namespace {
+constexpr int kNoAllocMaxCtas = 1024;
+constexpr size_t kNoAllocParamsOff = 0;
+constexpr size_t kNoAllocCounterOff = 256;
+constexpr size_t kNoAllocPartZOff = 512;
+constexpr size_t kNoAllocPartIOff = kNoAllocPartZOff + sizeof(float) * kNoAllocMaxCtas * kMaxRows;
+constexpr size_t kNoAllocBytes = kNoAllocPartIOff + sizeof(int) * kNoAllocMaxCtas * kMaxRows;
+static_assert(sizeof(FrameParams) <= 256, "frame params fit their slot");
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
 // ------------------------------------------------------------------ create --
 extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) {
   if (!cfg || !out) return fail(M3_EINVAL, "null argument");
@@ -281,6 +302,31 @@ extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) 
   if (cudaGetDevice(&c->dev) != cudaSuccess) return bail(fail(M3_ECUDA, "cudaGetDevice"));
   if (cudaDeviceGetAttribute(&c->nsm, cudaDevAttrMultiProcessorCount, c->dev) != cudaSuccess)
     return bail(fail(M3_ECUDA, "SM count"));
+  {
+    // the host-side name of the static scratch is not a device address: look
+    // the address up on this device now, before any stream capture
+    void* sp = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&sp, g_noalloc_scratch);
+    if (e != cudaSuccess)
+      return bail(fail(M3_ECUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e)));
+    c->noalloc_scratch = static_cast<unsigned char*>(sp);
+  }
+  if (const char* e = getenv("M3_FAULT")) {
+    // "alloc:N", "h2d:N" or "graph:N": the N-th such call from here on fails
+    const char* colon = strchr(e, ':');
+    const long long n = colon ? atoll(colon + 1) : 0;
+    const size_t len = colon ? (size_t)(colon - e) : 0;
+    const int kind = (len == 5 && !strncmp(e, "alloc", 5)) ? M3_FAULT_ALLOC
+                   : (len == 3 && !strncmp(e, "h2d", 3))   ? M3_FAULT_H2D
+                   : (len == 5 && !strncmp(e, "graph", 5)) ? M3_FAULT_GRAPH
+                                                           : M3_FAULT_NONE;
+    if (kind == M3_FAULT_NONE || n < 1) {
+      delete c;
+      return fail(M3_EINVAL, "M3_FAULT must be alloc:N, h2d:N or graph:N with N >= 1");
+    }
+    c->fault_kind = kind;
+    c->fault_left = n;
+  }
   if (const char* e = getenv("M3_NO_GRAPH")) c->use_graphs = (e[0] == '0');
   if (const char* e = getenv("M3_GEMV_STAGE_KB")) c->tile_sb = atoi(e) * 1024;
   if (const char* e = getenv("M3_GEMV_STAGES")) c->tile_ns = atoi(e);
@@ -291,15 +337,12 @@ extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) 
     const int v = atoi(e);
     if (v >= 1 && v <= kAttnMaxSplits) c->max_splits = v;
   }
-  if (const char* e = getenv("M3_ATTN_PF")) c->attn_pf = (e[0] == '1');
   if (const char* e = getenv("M3_PREFILL_TC")) c->prefill_tc = (e[0] == '1') ? 1 : 0;
   if (const char* e = getenv("M3_PREFILL_CHUNK")) {
     const int v = atoi(e);
     if (v >= 16 && v <= 4096) c->pf_chunk = v;
   }
-  if (const char* e = getenv("M3_GEMV_PF")) c->tile_pfa = atoi(e);
   if (const char* e = getenv("M3_GEMV_LAZY")) c->tile_lazy = atoi(e);
-  if (const char* e = getenv("M3_ATTN_PF_MB")) c->attn_pf_bytes = (size_t)atoi(e) << 20;
   if (cudaStreamCreateWithFlags(&c->st, cudaStreamNonBlocking) != cudaSuccess ||
       cudaEventCreateWithFlags(&c->ev_in, cudaEventDisableTiming) != cudaSuccess ||
       cudaEventCreateWithFlags(&c->ev_out, cudaEventDisableTiming) != cudaSuccess)
@@ -353,19 +396,6 @@ extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) 
         (rc = dalloc(c, &c->dforced, sizeof(int) * R * NC)) ||
         (rc = dalloc(c, &c->dlogits, sizeof(float) * R * NC * g.depth_vocab)))
       return bail(rc);
-    // scratch of the persistent depth kernel
-    const size_t qn = (size_t)g.depth_heads * g.depth_head_dim;
-    if ((rc = dalloc(c, &c->dfx, sizeof(bf16) * R * Dh)) ||
-        (rc = dalloc(c, &c->dfqkv, sizeof(bf16) * R * 3 * qn)) ||
-        (rc = dalloc(c, &c->dfatt, sizeof(bf16) * R * qn)) ||
-        (rc = dalloc(c, &c->dfact, sizeof(bf16) * R * g.depth_ffn)) ||
-        (rc = dalloc(c, &c->dfkv, sizeof(bf16) * R * g.depth_layers * (NC + 1) * 2 * qn)) ||
-        (rc = dalloc(c, &c->dfpart, sizeof(unsigned long long) * c->nsm * kMaxRows)))
-      return bail(rc);
-    if ((rc = dzalloc(c, &p, sizeof(unsigned) * 4))) return bail(rc);
-    c->dfbar = static_cast<unsigned*>(p);
-    if (const char* e = getenv("M3_DEPTH_FUSED")) c->depth_fused = e[0] == '1';
-    if (g.depth_layers > kDepthMaxLayers || NC > kDepthMaxCB) c->depth_fused = false;
     // depth KV: one 32-position page per (row, layer), bf16
     const size_t page = (size_t)2 * g.depth_heads * 32 * g.depth_head_dim * 2;
     if ((rc = dzalloc(c, &c->dkv, page * R * g.depth_layers))) return bail(rc);
@@ -414,8 +444,17 @@ static int stage_src(m3_ctx* c, const void* src, size_t bytes, int mem, const vo
     *dev = src;
     return M3_OK;
   }
+  if (fault_due(c, M3_FAULT_ALLOC)) return fail(M3_ENOMEM, "injected device allocation failure");
   CK(cudaMallocAsync(owned, bytes, c->st));
-  CK(cudaMemcpyAsync(*owned, src, bytes, cudaMemcpyHostToDevice, c->st));
+  const cudaError_t e = fault_due(c, M3_FAULT_H2D)
+                            ? cudaErrorUnknown
+                            : cudaMemcpyAsync(*owned, src, bytes, cudaMemcpyHostToDevice, c->st);
+  if (e != cudaSuccess) {
+    cudaFreeAsync(*owned, c->st);
+    *owned = nullptr;
+    return fail(M3_ECUDA, std::string("host-to-device copy of a source: ") +
+                              (e == cudaErrorUnknown ? "injected failure" : cudaGetErrorString(e)));
+  }
   *dev = *owned;
   return M3_OK;
 }
@@ -713,9 +752,10 @@ static int ensure_pages(m3_ctx* c, int npos) {
   const size_t page_bytes = (size_t)2 * g.n_kv_heads * c->bucket * g.head_dim * 2;
   for (int b = c->n_buckets; b < need; ++b) {
     void* p = nullptr;
+    if (fault_due(c, M3_FAULT_ALLOC)) return fail(M3_ENOMEM, "injected KV bucket allocation failure");
     CK(cudaMalloc(&p, c->bucket_bytes));
+    c->buckets.push_back(p);  // owned from here on, even if what follows fails
     CK(cudaMemset(p, 0, c->bucket_bytes));
-    c->buckets.push_back(p);
     for (int r = 0; r < c->kv_rows; ++r)
       for (int l = 0; l < g.n_layers; ++l)
         c->h_pages[((size_t)r * g.n_layers + l) * c->max_pages + b] =
@@ -741,7 +781,10 @@ extern "C" int m3_kv_set(m3_ctx* c, int row, int n_positions, const void* k, con
   const void *dk = nullptr, *dv = nullptr;
   void *ok = nullptr, *ov = nullptr;
   CKR(stage_src(c, k, bytes, mem, &dk, &ok));
-  CKR(stage_src(c, v, bytes, mem, &dv, &ov));
+  if (const int rc = stage_src(c, v, bytes, mem, &dv, &ov)) {
+    if (ok) cudaFreeAsync(ok, c->st);
+    return rc;
+  }
   kv_set_kernel<<<c->nsm * 4, 256, 0, c->st>>>(
       static_cast<const bf16*>(dk), static_cast<const bf16*>(dv),
       c->d_pages + (size_t)row * g.n_layers * c->max_pages, g.n_layers, c->max_pages, c->bucket,
@@ -803,7 +846,8 @@ static int dyn_mask(const m3_ctx* c, int wf) {
 
 static int gemv_rows(m3_ctx* c, const DMat& M, int epi, int rows, const bf16* x, int ldx,
                      const bf16* gamma, bf16* out, int ldo, const SampleArgs* smp, bool& pdl,
-                     const FrameParams* fp = nullptr, bool cache_plan = true, int ring_ns = 0) {
+                     const FrameParams* fp = nullptr, bool cache_plan = true, int ring_ns = 0,
+                     int max_grid = 0) {
   const int ns = ring_ns > 0 ? ring_ns : ring_stages(c, M.wf);
   const int step = M.tiled ? rows : 4;
   for (int r0 = 0; r0 < rows; r0 += step) {
@@ -843,9 +887,11 @@ static int gemv_rows(m3_ctx* c, const DMat& M, int epi, int rows, const bf16* x,
         CK(pe);
         if (cache_plan) c->tile_plans.emplace(key, L);
       }
+      // a caller's fixed-size scratch (part_z / part_i) bounds the CTAs
+      if (max_grid > 0 && L.grid > max_grid)
+        return fail(M3_EINVAL, "the launch needs more CTAs than the static scratch holds");
       if (L.dyn) {
         a.ctr = c->tile_ctrs + 2 * (c->tile_ctr_next % kTileCtrPairs);
-        a.pfa = c->tile_pfa;
         a.lazy_claim = c->tile_lazy;
         ++c->tile_ctr_next;
       }
@@ -866,6 +912,7 @@ static int gemv_rows(m3_ctx* c, const DMat& M, int epi, int rows, const bf16* x,
         c->ssq_n = (M.N + kUnitRows - 1) / kUnitRows;
       }
     } else {
+      if (max_grid > 0) return fail(M3_EINVAL, "static scratch needs the tiled GEMV");
       CK(launch_gemv(a, M.wf, epi, c->st, pdl, c->nsm));
     }
     pdl = true;
@@ -903,22 +950,6 @@ static int record_layer(m3_ctx* c, const DLayer& L, Acts& A, int rows, int H, in
   at.fp = c->fp;
   at.fixed_pos = fixed_pos;
   at.err = c->err;
-  if (fixed_pos < 0 && c->attn_pf) {
-    // the O projection past what its CTAs load before their wait, and the
-    // first attn_pf_bytes of gate/up
-    const size_t esz = L.o.wf == WF_BF16 ? 2 : 1;
-    const size_t ob = esz * (size_t)(L.o.N + kUnitRows - 1) / kUnitRows * kUnitRows * L.o.K;
-    // (a 3-stage ring does not fit beside attention: nothing is loaded before)
-    const int ns_o = c->tile_ns_o > 0 ? c->tile_ns_o : ring_stages(c, L.o.wf);
-    const size_t pre = ns_o <= 2 ? (size_t)c->nsm * c->tile_sb * ns_o : 0;
-    if (ob > pre) {
-      at.pf[0] = static_cast<const uint8_t*>(L.o.w) + pre;
-      at.pf_bytes[0] = ob - pre;
-    }
-    const size_t gb = esz * (size_t)(L.gu.N + kUnitRows - 1) / kUnitRows * kUnitRows * L.gu.K;
-    at.pf[1] = static_cast<const uint8_t*>(L.gu.w);
-    at.pf_bytes[1] = (c->attn_pf_bytes < gb ? c->attn_pf_bytes : gb) & ~(size_t)255;
-  }
   if (prefill) {
     at.mode = 1;
     CK(launch_attn(at, d, kv_f16, 1, rows, c->st, true));
@@ -980,6 +1011,7 @@ static int run_graph(m3_ctx* c, std::map<std::pair<int, int>, cudaGraphExec_t>& 
   auto it = cache.find(key);
   if (it == cache.end()) {
     cudaGraph_t graph = nullptr;
+    if (fault_due(c, M3_FAULT_GRAPH)) return fail(M3_ECUDA, "injected graph capture failure");
     CK(cudaStreamBeginCapture(c->st, cudaStreamCaptureModeThreadLocal));
     int rc = record();
     cudaError_t e = cudaStreamEndCapture(c->st, &graph);
@@ -1044,64 +1076,10 @@ extern "C" int m3_decode_frame(m3_ctx* c, int rows, const int32_t* positions, ui
 }
 
 // --------------------------------------------------------- depth decoder ---
-// The persistent depth kernel (depth.cuh) over the same buffers.
-static int record_depth_fused(m3_ctx* c, int rows, bool forced, const bf16* hin) {
-  const m3_config& g = c->cfg;
-  DepthArgs a{};
-  auto dm = [](const DMat& M) { return DepthMat{static_cast<const int8_t*>(M.w), M.s}; };
-  for (int l = 0; l < g.depth_layers; ++l) {
-    const DLayer& L = c->DL[l];
-    a.L[l].qkv = dm(L.qkv);
-    a.L[l].o = dm(L.o);
-    a.L[l].gu = dm(L.gu);
-    a.L[l].d = dm(L.d);
-    a.L[l].attn_norm = L.attn_norm;
-    a.L[l].mlp_norm = L.mlp_norm;
-    a.L[l].q_norm = L.q_norm;
-    a.L[l].k_norm = L.k_norm;
-  }
-  a.proj = dm(c->dproj);
-  for (int j = 0; j < g.depth_codebooks; ++j) {
-    a.heads[j] = dm(c->dheads[j]);
-    a.emb[j] = c->demb[j];
-    a.emb_rows[j] = c->demb_rows[j];
-  }
-  a.final_norm = c->dfinal;
-  a.inv_freq = c->dinv_freq;
-  a.n_layers = g.depth_layers;
-  a.Dh = g.depth_hidden;
-  a.nh = g.depth_heads;
-  a.hd = g.depth_head_dim;
-  a.F = g.depth_ffn;
-  a.NC = g.depth_codebooks;
-  a.V = g.depth_vocab;
-  a.Hin = g.hidden;
-  a.rows = rows;
-  a.zero_code = g.has_end_token ? g.slice_len : INT_MIN;
-  a.eps = g.rms_eps;
-  a.fp = c->fp;
-  a.h_in = hin;
-  a.code0 = c->dprev;
-  a.forced = forced ? c->dforced : nullptr;
-  a.codes = c->dcodes;
-  a.logits = c->dlogits;
-  a.x = c->dfx;
-  a.qkv = c->dfqkv;
-  a.att = c->dfatt;
-  a.act = c->dfact;
-  a.kv = c->dfkv;
-  a.part = c->dfpart;
-  a.bar = c->dfbar;
-  a.err = c->err;
-  CK(cudaMemsetAsync(c->dfbar, 0, sizeof(unsigned) * 4, c->st));
-  CK(launch_depth(a, c->nsm, c->st));
-  return M3_OK;
-}
 
 // hin: the frame's final-normed hidden state [rows][hidden]; the semantic
 // code is in dprev.
 static int record_depth(m3_ctx* c, int rows, bool forced, const bf16* hin) {
-  if (c->depth_fused) return record_depth_fused(c, rows, forced, hin);
   const m3_config& g = c->cfg;
   const int Dh = g.depth_hidden, NC = g.depth_codebooks, V = g.depth_vocab;
   bool pdl = false;
@@ -1571,6 +1549,42 @@ extern "C" int m3_time_gemv(m3_ctx* c, int which, int rows, int iters, float* av
   return leave(c);
 }
 
+// ------------------------------------------------------ checking hooks -----
+extern "C" int m3_gumbel_fill(uint64_t seed, uint64_t frame, uint64_t row, uint64_t index0,
+                              int64_t n, float* out, void* cuda_stream) {
+  if (n < 0 || (n > 0 && !out)) return fail(M3_EINVAL, "n < 0 or null output");
+  if (n == 0) return M3_OK;
+  const long long blocks = (n + 255) / 256;
+  gumbel_fill_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0,
+                       static_cast<cudaStream_t>(cuda_stream)>>>(seed, frame, row, index0,
+                                                                 (long long)n, out);
+  CK(cudaGetLastError());
+  return M3_OK;
+}
+
+extern "C" int m3_inject_fault(m3_ctx* c, int kind, int64_t nth) {
+  if (!c) return fail(M3_EINVAL, "null ctx");
+  if (kind == M3_FAULT_NONE) {
+    c->fault_kind = M3_FAULT_NONE;
+    c->fault_left = 0;
+    return M3_OK;
+  }
+  if (kind < M3_FAULT_ALLOC || kind > M3_FAULT_GRAPH || nth < 1)
+    return fail(M3_EINVAL, "kind must be M3_FAULT_ALLOC / _H2D / _GRAPH and nth >= 1");
+  c->fault_kind = kind;
+  c->fault_left = nth;
+  return M3_OK;
+}
+
+extern "C" int m3_stalled_wait(m3_ctx* c, int64_t polls) {
+  if (!c) return fail(M3_EINVAL, "null ctx");
+  if (polls < 1 || polls > kSpinLimit) return fail(M3_EINVAL, "polls out of 1..2^22");
+  CKR(enter(c));
+  stalled_wait_kernel<<<1, 32, 0, c->st>>>(c->err, (long long)polls);
+  CK(cudaGetLastError());
+  return leave(c);
+}
+
 extern "C" int m3_sync_status(m3_ctx* c) {
   if (!c) return fail(M3_EINVAL, "null ctx");
   CK(cudaSetDevice(c->dev));
@@ -1588,42 +1602,6 @@ extern "C" int m3_sync_status(m3_ctx* c) {
   return M3_OK;
 }
 
-// ------------------------------------------- allocation-free sampler -------
-// Scratch of m3_sample_noalloc: the frame-parameter block, the cross-CTA
-// argmax ticket and the per-CTA partial argmaxes live in this file-scope
-// device array instead of context-owned buffers.  Every GPU that loads the
-// library holds it (about 129 KB) until the process exits.
-namespace {
-constexpr int kNoAllocMaxCtas = 1024;
-constexpr size_t kNoAllocParamsOff = 0;
-constexpr size_t kNoAllocCounterOff = 256;
-constexpr size_t kNoAllocPartZOff = 512;
-constexpr size_t kNoAllocPartIOff = kNoAllocPartZOff + sizeof(float) * kNoAllocMaxCtas * kMaxRows;
-constexpr size_t kNoAllocBytes = kNoAllocPartIOff + sizeof(int) * kNoAllocMaxCtas * kMaxRows;
-static_assert(sizeof(FrameParams) <= 256, "frame params fit their slot");
-}  // namespace
-
-static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
-
-// Device address of g_noalloc_scratch per device, looked up once per device
-// (the host-side name of the array is not a device address).
-static std::mutex g_noalloc_mu;
-static void* g_noalloc_ptr[64] = {};
-
-static int noalloc_scratch(int dev, unsigned char** out) {
-  if (dev < 0 || dev >= 64) return fail(M3_EINVAL, "device index beyond 63");
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess)
-      return fail(M3_ECUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
-    g_noalloc_ptr[dev] = p;
-  }
-  *out = static_cast<unsigned char*>(g_noalloc_ptr[dev]);
-  return M3_OK;
-}
-
 extern "C" int m3_sample_noalloc(m3_ctx* c, int rows, const void* h, uint64_t seed,
                                  uint64_t frame, float cfg_scale, float temperature,
                                  int32_t* codes, float* logits) {
@@ -1634,11 +1612,7 @@ extern "C" int m3_sample_noalloc(m3_ctx* c, int rows, const void* h, uint64_t se
     return fail(M3_EINVAL, "rows must be in 1..min(16, max_rows)");
   if (!(cfg_scale >= 0.0f) || !(temperature > 0.0f)) return fail(M3_EINVAL, "cfg_scale / temperature");
   if (cfg_scale > 0.0f && rows % 2) return fail(M3_EINVAL, "cfg_scale > 0 needs (cond, uncond) row pairs");
-  const int grid = n_cand(g) < c->nsm ? n_cand(g) : c->nsm;
-  if (grid > kNoAllocMaxCtas) return fail(M3_EINVAL, "more CTAs than the static scratch holds");
-  CK(cudaSetDevice(c->dev));
-  unsigned char* scratch = nullptr;
-  CKR(noalloc_scratch(c->dev, &scratch));
+  unsigned char* scratch = c->noalloc_scratch;
   CKR(enter(c));
   FrameParams fp{};
   fp.rows = rows;
@@ -1667,6 +1641,6 @@ extern "C" int m3_sample_noalloc(m3_ctx* c, int rows, const void* h, uint64_t se
   // h is already the final-normed hidden state: no gain; launch plans are
   // looked up, not cached, so this call allocates nothing on the host either
   CKR(gemv_rows(c, c->lm, EPI_SAMPLE, rows, static_cast<const bf16*>(h), g.hidden, nullptr,
-                nullptr, 0, &sa, pdl, dfp, false));
+                nullptr, 0, &sa, pdl, dfp, false, 0, kNoAllocMaxCtas));
   return leave(c);
 }

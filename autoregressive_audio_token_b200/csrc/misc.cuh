@@ -5,6 +5,7 @@
 #include "common.cuh"
 #include "gemv.cuh"
 #include "gemv_tile.cuh"
+#include "noise.cuh"
 
 namespace m3 {
 
@@ -350,6 +351,37 @@ __global__ void loop_advance_kernel(LoopArgs a) {
   if (t == 0) {
     ls->step += 1;
     fp->frame += 1ull;
+  }
+}
+
+// ------------------------------------------------------------ noise export --
+// G(seed, frame, row, index0 + i) for i < n, by the same device function the
+// samplers draw with (noise.cuh): the noise made visible for a bit-for-bit
+// comparison with any other implementation of its definition.
+__global__ void gumbel_fill_kernel(unsigned long long seed, unsigned long long frame,
+                                   unsigned long long row, unsigned long long index0, long long n,
+                                   float* __restrict__ out) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x)
+    out[i] = gumbel_noise(seed, frame, row, index0 + (unsigned long long)i);
+}
+
+// ------------------------------------------------------- bounded-wait check --
+// One mbarrier that nothing ever arrives on, waited for with at most `polls`
+// try_wait polls: the wait gives up, records kErrTimeout and the kernel
+// returns -- the path every bounded wait of the library takes when its
+// producer never comes, exercised without hanging or faulting the GPU.
+__global__ void stalled_wait_kernel(int* err, long long polls) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    bool done = false;
+    for (long long i = 0; i < polls && !done; ++i) done = mbar_try_wait(&bar, 0);
+    if (!done) record_error(err, kErrTimeout);
   }
 }
 

@@ -22,12 +22,13 @@ M3_EEMPTY = -8
 M3_W_BF16, M3_W_INT8 = 0, 1
 M3_KV_BF16, M3_KV_F16 = 0, 1
 M3_MEM_HOST, M3_MEM_DEVICE = 0, 1
+M3_FAULT_NONE, M3_FAULT_ALLOC, M3_FAULT_H2D, M3_FAULT_GRAPH = 0, 1, 2, 3
 
 EXPORTED = ("m3_create", "m3_load_weights", "m3_load_depth_weights", "m3_kv_alloc", "m3_kv_set",
             "m3_kv_get", "m3_decode_frame", "m3_depth_decode", "m3_embed", "m3_quantize_int8",
             "m3_export_weight", "m3_frame_bytes", "m3_time_gemv", "m3_sample_noalloc", "m3_set_top_k",
-            "m3_load_feedback", "m3_generate", "m3_prefill", "m3_sync_status",
-            "m3_last_error", "m3_destroy")
+            "m3_load_feedback", "m3_generate", "m3_prefill", "m3_gumbel_fill", "m3_inject_fault",
+            "m3_stalled_wait", "m3_sync_status", "m3_last_error", "m3_destroy")
 
 
 class M3Error(RuntimeError):
@@ -93,6 +94,9 @@ def load_library() -> C.CDLL:
     L.m3_load_feedback.argtypes = [vp, vp, C.POINTER(vp), i32]
     L.m3_prefill.argtypes = [vp, i32, i32, i32, vp, vp]
     L.m3_generate.argtypes = [vp, i32, vp, u64, u64, vp, f32, f32, i32, vp, vp, vp]
+    L.m3_gumbel_fill.argtypes = [u64, u64, u64, u64, i64, vp, vp]
+    L.m3_inject_fault.argtypes = [vp, i32, i64]
+    L.m3_stalled_wait.argtypes = [vp, i64]
     L.m3_sync_status.argtypes = [vp]
     L.m3_last_error.restype = C.c_char_p
     L.m3_destroy.argtypes = [vp]
@@ -300,6 +304,25 @@ def m3_prefill(ctx: int, row: int, start: int, x: torch.Tensor,
                h_last: torch.Tensor | None = None) -> None:
     """Prompt prefill of cache row `row` (see m3.h): x bf16 [n_tokens, H] on the GPU."""
     _check(lib.m3_prefill(ctx, row, start, x.shape[0], _ptr(x.contiguous()), _ptr(h_last)))
+
+
+def m3_gumbel_fill(seed: int, frame: int, row: int, index0: int, n: int,
+                   stream=None) -> torch.Tensor:
+    """The device's Gumbel noise G(seed, frame, row, index0 + i), i < n (see m3.h)."""
+    out = torch.empty(n, dtype=torch.float32, device="cuda")
+    _check(lib.m3_gumbel_fill(seed, frame, row, index0, n, _ptr(out), _stream(stream)))
+    return out
+
+
+def m3_inject_fault(ctx: int, kind: int, nth: int = 1) -> None:
+    """Make the nth next call of `kind` fail on the host (see m3.h)."""
+    _check(lib.m3_inject_fault(ctx, kind, nth))
+
+
+def m3_stalled_wait(ctx: int, polls: int) -> None:
+    """A kernel whose bounded wait is never satisfied (see m3.h); the next
+    m3_sync_status raises M3_ETIMEOUT."""
+    _check(lib.m3_stalled_wait(ctx, polls))
 
 
 def m3_sync_status(ctx: int) -> None:

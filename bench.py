@@ -58,6 +58,14 @@ def parse():
                         "after a 300-position prompt, against host-driven m3_decode_frame")
     p.add_argument("--prefill", type=int, default=0, metavar="P",
                    help="time the prompt prefill (m3_prefill) of P tokens into one row")
+    p.add_argument("--rows", type=int, default=ROWS,
+                   help="batch rows (even: CFG pairs); 2 = the workload")
+    p.add_argument("--ctx", type=int, default=0,
+                   help="every timed frame at this context (prefilled) instead of the "
+                        "1500-frame song's spread of positions; for profiling cases")
+    p.add_argument("--depth-only", action="store_true",
+                   help="time the RVQ depth decoder (m3_depth_decode) alone, int8 group-128, "
+                        "on a frame's hidden state")
     p.add_argument("--sweep", action="store_true",
                    help="batched-variations sweep: rows 1..16 x context 1500/4500/9000, "
                         "bf16 and int8; one JSON line per point")
@@ -242,34 +250,42 @@ def run_ours(args, rank, world, local):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     seed = replica_seed(rank)
+    rows = args.rows
+    song = args.ctx if args.ctx > 0 else SONG_FRAMES
     wdtype = m3.M3_W_INT8 if args.wdtype == "int8" else m3.M3_W_BF16
-    s, ctx = build_model(torch, m3, synth, seed, wdtype, args.layers, depth=args.depth)
+    s, ctx = build_model(torch, m3, synth, seed, wdtype, args.layers, depth=args.depth,
+                         max_rows=rows)
     m3.m3_set_top_k(ctx, args.top_k)
-    prefill_kv(torch, m3, synth, s, ctx, ROWS, SONG_FRAMES, seed, args.kv == "f16")
-    xs = synth.normal((64, ROWS, s.hidden), seed, "bench/x_in", std=0.02, device="cuda")
-    codes = torch.empty(ROWS, dtype=torch.int32, device="cuda")
-    h_dev = torch.empty((ROWS, s.hidden), dtype=torch.bfloat16, device="cuda")
-    dcodes = torch.empty((ROWS, synth.DEPTH.codebooks), dtype=torch.int32, device="cuda")
+    prefill_kv(torch, m3, synth, s, ctx, rows, song, seed, args.kv == "f16")
+    xs = synth.normal((64, rows, s.hidden), seed, "bench/x_in", std=0.02, device="cuda")
+    codes = torch.empty(rows, dtype=torch.int32, device="cuda")
+    h_dev = torch.empty((rows, s.hidden), dtype=torch.bfloat16, device="cuda")
+    dcodes = torch.empty((rows, synth.DEPTH.codebooks), dtype=torch.int32, device="cuda")
     stream = torch.cuda.current_stream()
+    cfg = CFG_SCALE if rows % 2 == 0 else 0.0
+
+    def frame_positions(k):
+        # the song's evenly spaced positions, or every frame at the given context
+        return [song - 1] * k if args.ctx > 0 else song_positions(k)
 
     def frame(i, pos):
         if args.depth:
-            m3.m3_decode_frame(ctx, [pos] * ROWS, seed, i, xs[i % 64], CFG_SCALE, 1.0, codes, h_dev)
-            m3.m3_depth_decode(ctx, h_dev, codes, seed, i, CFG_SCALE, 1.0, dcodes)
+            m3.m3_decode_frame(ctx, [pos] * rows, seed, i, xs[i % 64], cfg, 1.0, codes, h_dev)
+            m3.m3_depth_decode(ctx, h_dev, codes, seed, i, cfg, 1.0, dcodes)
         else:
-            m3.m3_decode_frame(ctx, [pos] * ROWS, seed, i, xs[i % 64], CFG_SCALE, 1.0, codes)
+            m3.m3_decode_frame(ctx, [pos] * rows, seed, i, xs[i % 64], cfg, 1.0, codes)
 
     # capture every bucket's graph before timing, then warm up
-    for b in range(0, SONG_FRAMES, 256):
+    for b in range(0, song, 256):
         frame(0, b)
-    warm = song_positions(max(args.warmup, 3))
+    warm = frame_positions(max(args.warmup, 3))
     for i, p in enumerate(warm):
         frame(i, p)
     torch.cuda.synchronize()
     m3.m3_sync_status(ctx)
 
     # ---- device-timed region: inputs resident in HBM -----------------------
-    positions = song_positions(args.steps)
+    positions = frame_positions(args.steps)
     clocks = ClockSampler(local, f"/tmp/m3_clocks_rank{rank}.csv")
     barrier(world)
     torch.cuda.synchronize()
@@ -289,15 +305,15 @@ def run_ours(args, rank, world, local):
 
     # ---- end to end through the C ABI with host buffers ---------------------
     x_host = xs[:64].cpu().pin_memory()
-    codes_host = torch.empty((args.steps, ROWS), dtype=torch.int32).pin_memory()
-    x_dev = torch.empty((ROWS, s.hidden), dtype=torch.bfloat16, device="cuda")
+    codes_host = torch.empty((args.steps, rows), dtype=torch.int32).pin_memory()
+    x_dev = torch.empty((rows, s.hidden), dtype=torch.bfloat16, device="cuda")
     barrier(world)
     torch.cuda.synchronize()
     e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2.record(stream)
     for i, p in enumerate(positions):
         x_dev.copy_(x_host[i % 64], non_blocking=True)
-        m3.m3_decode_frame(ctx, [p] * ROWS, seed, i, x_dev, CFG_SCALE, 1.0, codes)
+        m3.m3_decode_frame(ctx, [p] * rows, seed, i, x_dev, cfg, 1.0, codes)
         codes_host[i].copy_(codes, non_blocking=True)
     e3.record(stream)
     torch.cuda.synchronize()
@@ -308,11 +324,11 @@ def run_ours(args, rank, world, local):
     kernels = {}
     for which, name in [(2, "gate_up_swiglu"), (3, "down"), (0, "qkv"), (1, "o_proj"),
                         (4, "lm_head_sample")]:
-        kms, kbytes = m3.m3_time_gemv(ctx, which, ROWS, 72 if which != 4 else 20)
+        kms, kbytes = m3.m3_time_gemv(ctx, which, rows, 72 if which != 4 else 20)
         kernels[name] = {"ms": kms, "bytes": kbytes, "gbs": kbytes / kms / 1e6}
 
     mean_ctx = sum(positions) / len(positions)
-    frame_bytes = m3.m3_frame_bytes(ctx, ROWS, int(round(mean_ctx)))
+    frame_bytes = m3.m3_frame_bytes(ctx, rows, int(round(mean_ctx)))
     peaks = {}
     try:
         peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
@@ -346,8 +362,8 @@ def run_ours(args, rank, world, local):
         "dtype": args.wdtype,
         "data": "synthetic (seeded N(0,0.02^2) weights, N(0,1) KV prefill, random-init 8B shape)",
         "config": {"workload": variant,
-                   "rows": ROWS, "song_frames": SONG_FRAMES, "mean_ctx": mean_ctx,
-                   "cfg_scale": CFG_SCALE, "temperature": 1.0, "kv": f"{args.kv} pages of 256",
+                   "rows": rows, "song_frames": song, "mean_ctx": mean_ctx,
+                   "cfg_scale": cfg, "temperature": 1.0, "kv": f"{args.kv} pages of 256",
                    "depth_decoder": bool(args.depth), "top_k": args.top_k,
                    "l2": "no flush: 14 GB of weights per frame >> 126 MB L2",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
@@ -356,14 +372,14 @@ def run_ours(args, rank, world, local):
                   "frac_of_measured_hbm": frame_bytes / ms_per_step / 1e6 / hbm_peak,
                   "frac_of_8tbs": frame_bytes / ms_per_step / 1e6 / 8000.0},
         "roofline": {"bound": "hbm",
-                     "kernel": f"gemv_dyn_kernel gate/up + SwiGLU ({args.wdtype}, {ROWS} rows)",
+                     "kernel": f"gemv_dyn_kernel gate/up + SwiGLU ({args.wdtype}, {rows} rows)",
                      "achieved": dom["gbs"], "peak": hbm_peak, "unit": "GB/s",
                      "frac": dom["gbs"] / hbm_peak, "peak_source": peak_src,
                      "traffic": traffic, "algorithmic_bytes_per_launch": dom["bytes"]},
         "kernels": kernels,
         "e2e": {"value": 1000.0 / e2e_ms * world, "unit": "frames/s",
-                "h2d_bytes_per_step": ROWS * s.hidden * 2 + 4 * ROWS,
-                "d2h_bytes_per_step": 4 * ROWS},
+                "h2d_bytes_per_step": rows * s.hidden * 2 + 4 * rows,
+                "d2h_bytes_per_step": 4 * rows},
         "clocks": clk,
     }
     # per frame: parameter block + RoPE table + 5 kernels per layer (qkv,
@@ -376,7 +392,7 @@ def run_ours(args, rank, world, local):
     del xs
     torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(steps=1)
+        out["cpu_baseline"] = cpu_baseline()
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -398,59 +414,121 @@ def kernel_source_hash() -> str:
 SAMPLE_LAYERS = 2
 
 
-def cpu_baseline(steps: int = 1) -> dict:
-    """The CPU oracle as it stands on this host's cores: a bounded sample of the
-    frame (SAMPLE_LAYERS of the 36 body layers at the song's mean context, plus
-    the final norm + sliced lm_head + CFG + Gumbel-argmax), scaled to a full
-    frame as 36/SAMPLE_LAYERS x body-sample time + head time."""
-    import numpy as np
-    import torch
+class OracleSample:
+    """A bounded sample of the frame on the CPU oracle (as it stands): the
+    first SAMPLE_LAYERS of the 36 body layers for the 2 rows at the song's
+    mean context, then the final norm + sliced lm_head + CFG + Gumbel-argmax.
+    One step = one such sample, scaled to a full frame as
+    36 / SAMPLE_LAYERS x body time + head time."""
+
+    def __init__(self):
+        import dataclasses
+        import synth
+        from oracle import oracle as O
+        self.O = O
+        s = synth.FULL8B
+        sub = dataclasses.replace(s, n_layers=SAMPLE_LAYERS)
+        layers = [synth.layer_weights(s, 0, l) for l in range(SAMPLE_LAYERS)]
+        self.body = O.Body(sub, layers, synth.final_norm(s, 0), synth.lm_head_slice(s, 0))
+        self.ctx = SONG_FRAMES // 2
+        self.kc, self.vc = self.body.new_cache(ROWS, self.ctx + 1)
+        K, V = synth.kv_prefill(sub, ROWS, self.ctx, 7)
+        self.kc[:, :, :self.ctx] = O.bits(K)
+        self.vc[:, :, :self.ctx] = O.bits(V)
+        self.x = O.bits(synth.frame_input(s, ROWS, 7, 0))
+        self.n_layers = s.n_layers
+
+    def frame_seconds(self, i: int) -> float:
+        t0 = time.perf_counter()
+        hx = self.body.body(self.kc, self.vc, [self.ctx] * ROWS, self.x)
+        t1 = time.perf_counter()
+        self.body.sample(hx, 7, i, cfg_scale=CFG_SCALE)
+        t2 = time.perf_counter()
+        return (t1 - t0) * self.n_layers / SAMPLE_LAYERS + (t2 - t1)
+
+    def describe(self, frames: int) -> str:
+        return (f"{frames} frame(s), each {SAMPLE_LAYERS} of 36 layers at ctx {self.ctx} for "
+                f"{ROWS} rows + lm_head/CFG/draw, scaled to a full frame as "
+                f"36/{SAMPLE_LAYERS} x body + head")
+
+
+def tiny_oracle_frames() -> dict:
+    """The oracle on the tiny 1-layer model: 16 consecutive frames, each
+    frame's code fed back through the token embedding (the tiny workload the
+    GPU parity tests run), all host cores."""
     import synth
     from oracle import oracle as O
+    s = synth.TINY
+    body = O.Body(s, [synth.layer_weights(s, 0, 0)], synth.final_norm(s, 0),
+                  synth.lm_head_slice(s, 0))
+    kc, vc = body.new_cache(1, 128)
+    K, V = synth.kv_prefill(s, 1, 64, 0)
+    kc[:, :, :64] = O.bits(K)
+    vc[:, :, :64] = O.bits(V)
+    E = O.bits(synth.embedding(s, 0))
+    x = O.bits(synth.frame_input(s, 1, 0, 0))
+    t0 = time.perf_counter()
+    for f in range(16):
+        codes, _, _ = body.decode_frame(kc, vc, [64 + f], 0, f, x)
+        x = E[s.slice_start + codes].copy()
+    return {"ms_per_frame": (time.perf_counter() - t0) * 1000.0 / 16, "frames": 16}
 
-    s = synth.FULL8B
-    import dataclasses
-    sub = dataclasses.replace(s, n_layers=SAMPLE_LAYERS)
-    layers = [synth.layer_weights(s, 0, l) for l in range(SAMPLE_LAYERS)]
-    body = O.Body(sub, layers, synth.final_norm(s, 0), synth.lm_head_slice(s, 0))
-    ctx = SONG_FRAMES // 2
-    kc, vc = body.new_cache(ROWS, ctx + 1)
-    K, V = synth.kv_prefill(sub, ROWS, ctx, 7)
-    kc[:, :, :ctx] = O.bits(K)
-    vc[:, :, :ctx] = O.bits(V)
-    x = O.bits(synth.frame_input(s, ROWS, 7, 0))
-    t_body, t_head = [], []
-    for i in range(steps):
-        t0 = time.perf_counter()
-        hx = body.body(kc, vc, [ctx] * ROWS, x)
-        t1 = time.perf_counter()
-        body.sample(hx, 7, i, cfg_scale=CFG_SCALE)
-        t2 = time.perf_counter()
-        t_body.append(t1 - t0)
-        t_head.append(t2 - t1)
-    frame_s = statistics.mean(t_body) * s.n_layers / SAMPLE_LAYERS + statistics.mean(t_head)
-    return {"value": 1.0 / frame_s, "unit": "frames/s", "cores": O.num_threads(),
+
+def cpu_baseline(frames: int = 2) -> dict:
+    """The CPU oracle as it stands on this host's cores (OracleSample), plus
+    the same sample on one core and the tiny model's 16-frame run."""
+    O = __import__("oracle.oracle", fromlist=["oracle"])
+    smp = OracleSample()
+    cores = O.num_threads()
+    t = [smp.frame_seconds(i) for i in range(frames)]
+    O.set_threads(1)
+    try:
+        t1 = smp.frame_seconds(0)
+    finally:
+        O.set_threads(cores)
+    frame_s = statistics.mean(t)
+    return {"value": 1.0 / frame_s, "unit": "frames/s", "cores": cores,
             "kind": "oracle", "ms_per_frame": frame_s * 1000.0,
-            "sample": f"{SAMPLE_LAYERS} of 36 layers at ctx {ctx} for 2 rows + lm_head/CFG/draw, "
-                      f"{steps} frame(s); full frame = 36/{SAMPLE_LAYERS} x body + head"}
+            "sample": smp.describe(frames),
+            "one_core": {"ms_per_frame": t1 * 1000.0, "frames_per_s": 1.0 / t1, "cores": 1},
+            "tiny_1layer_16frames": tiny_oracle_frames()}
 
 
 def run_reference(args, rank, world):
+    """The oracle arm: W untimed warm-up samples, then exactly K timed steps,
+    each one OracleSample frame; rank 0 only."""
     if rank != 0:
         return None
-    cb = cpu_baseline(steps=max(1, args.steps if args.steps <= 3 else 3))
-    return {"metric": METRIC, "value": cb["value"], "unit": "frames/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": cb["ms_per_frame"],
+    O = __import__("oracle.oracle", fromlist=["oracle"])
+    smp = OracleSample()
+    for i in range(args.warmup):
+        smp.frame_seconds(i)
+    t = [smp.frame_seconds(args.warmup + i) for i in range(args.steps)]
+    frame_s = statistics.mean(t)
+    value = 1.0 / frame_s
+    cb = {"value": value, "unit": "frames/s", "cores": O.num_threads(), "kind": "oracle",
+          "ms_per_frame": frame_s * 1000.0, "sample": smp.describe(args.steps)}
+    return {"metric": METRIC, "value": value, "unit": "frames/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": frame_s * 1000.0,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": WORKLOAD, "rows": ROWS, "song_frames": SONG_FRAMES},
+            "config": {"workload": WORKLOAD, "rows": ROWS, "song_frames": SONG_FRAMES,
+                       "sample": smp.describe(args.steps)},
             "cpu_baseline": cb,
-            "e2e": {"value": cb["value"], "unit": "frames/s", "h2d_bytes_per_step": 0,
+            "e2e": {"value": value, "unit": "frames/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
 
 def workload_name(args) -> str:
     name = WORKLOAD.replace("bf16", args.wdtype)
+    if args.rows != ROWS:
+        name = name.replace("2rows", f"{args.rows}rows")
+    if args.ctx > 0:
+        name = name.replace("song1500", f"ctx{args.ctx}")
+    if args.rows % 2:
+        name = name.replace("-cfg1.5", "")
+    if args.layers != 36:
+        name = name.replace("36L", f"{args.layers}L")
     if args.kv != "bf16":
         name += f"-{args.kv}kv"
     if args.depth:
@@ -592,6 +670,41 @@ def run_generate(args):
     m3.m3_destroy(ctx)
 
 
+def run_depth_only(args):
+    """The RVQ depth decoder alone (int8 weights, one scale per group of 128):
+    m3_depth_decode on a fixed final hidden state and semantic code, 2 rows
+    (one CFG pair), timed with CUDA events over --steps calls after --warmup.
+    The body is a single layer, loaded only because the context needs one."""
+    import torch
+    from autoregressive_audio_token_b200 import m3
+    import synth
+    torch.cuda.set_device(0)
+    s, ctx = build_model(torch, m3, synth, 0, m3.M3_W_INT8, 1, depth=True)
+    h = synth.normal((ROWS, s.hidden), 0, "bench/depth_h", std=1.0, device="cuda")
+    code0 = torch.tensor([5, 5], dtype=torch.int32, device="cuda")
+    dcodes = torch.empty((ROWS, synth.DEPTH.codebooks), dtype=torch.int32, device="cuda")
+    for i in range(max(args.warmup, 3)):
+        m3.m3_depth_decode(ctx, h, code0, 1, i, CFG_SCALE, 1.0, dcodes)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        m3.m3_depth_decode(ctx, h, code0, 1, i, CFG_SCALE, 1.0, dcodes)
+    e1.record()
+    torch.cuda.synchronize()
+    m3.m3_sync_status(ctx)
+    ms = e0.elapsed_time(e1) / args.steps
+    D = synth.DEPTH
+    wbytes = (D.n_layers * (4 * D.hidden * D.n_heads * D.head_dim + 3 * D.hidden * D.ffn) *
+              (D.codebooks + 1) + D.hidden * D.in_hidden + D.codebooks * D.vocab * D.hidden)
+    print(json.dumps({"metric": "depth decoder calls/s (7 residual codes, 2 rows)",
+                      "value": 1000.0 / ms, "unit": "calls/s", "ms_per_call": ms,
+                      "steps": args.steps, "dtype": "int8 g128",
+                      "weight_bytes_per_call": wbytes, "achieved_gbs": wbytes / ms / 1e6,
+                      "config": {"workload": "depth-decoder-4L-1024-int8g128-2rows-cfg1.5"}}))
+    m3.m3_destroy(ctx)
+
+
 def run_prefill(args):
     """Prompt prefill of P tokens (a prompt's worth, N(0, 0.02^2) embeddings)
     into one cache row of the full 8B: chunks of M3_PREFILL_CHUNK tokens (256)
@@ -637,6 +750,10 @@ def main():
     if args.prefill:
         if rank == 0:
             run_prefill(args)
+        return
+    if args.depth_only:
+        if rank == 0:
+            run_depth_only(args)
         return
     if args.generate:
         if rank == 0:

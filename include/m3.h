@@ -332,13 +332,46 @@ M3_API int m3_time_gemv(m3_ctx* ctx, int which, int rows, int iters, float* avg_
  *  temperature, codes, logits as in m3_decode_frame (logits nullable).
  * Its scratch (parameter block, argmax partials, ticket; about 129 KB) is a
  * file-scope __device__ array that every GPU loading the library holds
- * until exit.  The first call on a device looks up that array's device
- * address, so make the first call before any stream capture.  All calls
+ * until exit.  m3_create looks up that array's device address on the
+ * context's device (so this call does no lookup and takes no lock); a
+ * cudaDeviceReset invalidates it together with the context.  All calls
  * share the array and keep the last call's contents (the ticket is cleared
  * by each call): calls that overlap on the GPU -- on different streams or
- * contexts of one device -- race and must be ordered by the caller. */
+ * contexts of one device -- race and must be ordered by the caller.  A
+ * launch plan needing more than 1024 CTAs is rejected with M3_EINVAL. */
 M3_API int m3_sample_noalloc(m3_ctx* ctx, int rows, const void* h, uint64_t seed, uint64_t frame,
                              float cfg_scale, float temperature, int32_t* codes, float* logits);
+
+/* The Gumbel noise of the draws, written out: out[i] (dev fp32 [n]) =
+ * G(seed, frame, row, index0 + i), computed by the same device function the
+ * samplers use, so that the noise can be compared bit for bit with another
+ * implementation of its definition (the diffusers issue "MiniMax Music 3
+ * modular pipeline", finding 3: Gumbel-argmax in place of softmax +
+ * multinomial; definition: SplitMix64 counters, u = ((b >> 40) + 0.5) 2^-24,
+ * G = -ln(-ln u) in fp64 with a series ln, rounded to fp32).  Stateless;
+ * asynchronous on cuda_stream.  M3_EINVAL for n < 0 or a null output. */
+M3_API int m3_gumbel_fill(uint64_t seed, uint64_t frame, uint64_t row, uint64_t index0,
+                          int64_t n, float* out, void* cuda_stream);
+
+/* Host-side fault injection, for testing the error paths: the nth (>= 1) next
+ * device allocation (M3_FAULT_ALLOC, the call then returns M3_ENOMEM), host-
+ * to-device copy of a host source (M3_FAULT_H2D, M3_ECUDA) or CUDA-graph
+ * capture (M3_FAULT_GRAPH, M3_ECUDA) made by this context fails as if the
+ * CUDA call had; the context stays usable, and the same call made again
+ * succeeds.  One failure per injection; M3_FAULT_NONE cancels.  The
+ * environment variable M3_FAULT = alloc:N | h2d:N | graph:N, read by
+ * m3_create, schedules the same from the context's creation on.  No GPU
+ * fault is involved: the CUDA call is simply not made. */
+enum { M3_FAULT_NONE = 0, M3_FAULT_ALLOC = 1, M3_FAULT_H2D = 2, M3_FAULT_GRAPH = 3 };
+M3_API int m3_inject_fault(m3_ctx* ctx, int kind, int64_t nth);
+
+/* Launch, on the context's stream, one kernel that waits on an mbarrier no
+ * thread ever arrives on, with at most `polls` (1..2^22) polls: the bounded
+ * wait gives up and records the timeout error word, which the next
+ * m3_sync_status returns as M3_ETIMEOUT (and clears).  This is the path every
+ * device-side wait of the library takes when the copy or the CTA it waits
+ * for never comes; the kernel returns normally and the context stays usable. */
+M3_API int m3_stalled_wait(m3_ctx* ctx, int64_t polls);
 
 /* Synchronise the stream and return the first error a kernel recorded on
  * the device (M3_ETIMEOUT / M3_EDEVICE), clearing it, or M3_OK. */

@@ -48,3 +48,12 @@ def test_null_arguments_are_einval():
     from autoregressive_audio_token_b200 import m3
     assert m3.lib.m3_decode_frame(None, 1, None, 0, 0, None, 0.0, 1.0, None, None, None) == m3.M3_EINVAL
     assert m3.lib.m3_quantize_int8(None, 1, 1, 1, None, None, None) == m3.M3_EINVAL
+
+
+def test_checking_hooks_validate_before_any_cuda_call():
+    from autoregressive_audio_token_b200 import m3
+    assert m3.lib.m3_inject_fault(None, m3.M3_FAULT_ALLOC, 1) == m3.M3_EINVAL
+    assert m3.lib.m3_stalled_wait(None, 10) == m3.M3_EINVAL
+    assert m3.lib.m3_gumbel_fill(1, 2, 3, 4, -1, None, None) == m3.M3_EINVAL
+    assert m3.lib.m3_gumbel_fill(1, 2, 3, 4, 5, None, None) == m3.M3_EINVAL
+    assert m3.lib.m3_gumbel_fill(1, 2, 3, 4, 0, None, None) == m3.M3_OK  # nothing to do

@@ -8,22 +8,25 @@ so one frame per variant is checked: codes teacher-forced (the oracle's
 sampler on the GPU's own final hidden state), KV written at the frame's
 position, the quantised weights bit-exact, and the logits.
 
-Logits: a 36-layer stack of random N(0, 0.02^2) weights amplifies rounding.
-The oracle's own logits move by ~4.5-4.8% (relative to the largest logit)
-when one input element changes by one bf16 ulp, so no two correct
-implementations with different fp32 summation orders can agree to 2e-2 at
-full depth.  The test therefore measures that one-ulp sensitivity of the
-oracle in the same run and requires the GPU's deviation to be within
-max(tolerance, 1.5 x sensitivity); the 2e-2 / 5e-2 bounds themselves are
-enforced at one layer of every shape (test_gpu_parity), where nothing
-amplifies.
+Logits: a 36-layer stack of random N(0, 0.02^2) weights amplifies rounding
+(the oracle's own logits move by several per cent when one input element
+changes by one bf16 step), so two correct implementations that sum in
+different orders drift apart at full depth.  The comparator is the oracle
+against itself: the same frame with every GEMV summed in fp64 instead of
+the sequential fp32 loop.  Its distance from the fp32 definition is the
+summation-order spread; the GPU's distance from the fp64-summed frame must
+be within max(tolerance, 1.5 x spread), i.e. the GPU sits no farther from
+the more exact sum than the definition itself does, with a margin.  The
+2e-2 / 5e-2 bounds themselves hold at one layer of every shape
+(test_gpu_parity), where nothing amplifies.  The measured numbers are
+printed (run with -s to see them).
 """
 import numpy as np
 import pytest
 import torch
 
 import synth
-from gpu_util import bits, f32, rel_err
+from gpu_util import bits, check_depth_draws, check_draws, f32, rel_err
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -82,19 +85,30 @@ def test_full_frame_vs_oracle(ora, variant):
         m3.m3_sync_status(ctx)
         hb = bits(h)
         kc2, vc2 = kc.copy(), vc.copy()
+        kc3, vc3 = kc.copy(), vc.copy()
         oc, oh, olg = body.decode_frame(kc, vc, pos, 99, 7, bits(x), cfg_scale=1.5)
-        # the oracle's own sensitivity: one input element one bf16 ulp up
+        # the summation-order comparator: the same frame with fp64 GEMV sums
+        with ora.accum64():
+            _, _, olg64 = body.decode_frame(kc2, vc2, pos, 99, 7, bits(x), cfg_scale=1.5)
+        # for the record: the oracle's response to one input element one bf16 step up
         xp = bits(x).copy()
         xp[0, 0] += 1
-        _, _, olg_p = body.decode_frame(kc2, vc2, pos, 99, 7, xp, cfg_scale=1.5)
+        _, _, olg_p = body.decode_frame(kc3, vc3, pos, 99, 7, xp, cfg_scale=1.5)
+        del kc2, vc2, kc3, vc3
         sens = rel_err(olg_p, olg)
+        spread = rel_err(olg, olg64)
         tol = 2e-2 if wdtype == 0 else 5e-2
-        err = rel_err(lg.cpu().numpy(), olg)
-        assert err <= max(tol, 1.5 * sens), (err, sens)
+        glg = lg.cpu().numpy()
+        err = rel_err(glg, olg)
+        err64 = rel_err(glg, olg64)
+        print(f"\n[{variant}] logits rel err: GPU vs oracle {err:.4f}, GPU vs fp64-summed "
+              f"oracle {err64:.4f}, oracle fp32 vs fp64 sums (spread) {spread:.4f}, "
+              f"one-step input sensitivity {sens:.4f}")
+        assert err64 <= max(tol, 1.5 * spread), (err64, spread, err, sens)
         # teacher-forced draw on the GPU's own hidden state
         tc, _, margin = body.sample(hb, 99, 7, cfg_scale=1.5, with_margin=True)
         gc = codes.cpu().numpy()
-        assert np.all((tc == gc) | (margin < 1e-3)), (tc, gc, margin)
+        check_draws(tc, margin, gc)
         assert gc[0] == gc[1]  # the pair shares its code
         # the frame's KV slot in the last layer
         k, v = m3.m3_kv_get(ctx, 0, s.n_layers, CTX, s.n_kv_heads, s.head_dim)
@@ -122,9 +136,11 @@ def test_full_frame_vs_oracle(ora, variant):
                                  "heads": [hh.cpu() for hh in dw["heads"]]})
             gdc = dcodes.cpu().numpy()
             odc, odl = dora.decode(hb, code0.cpu().numpy(), 99, 7, cfg_scale=1.5, forced=gdc)
-            glg = dlg.cpu().numpy()
+            dglg = dlg.cpu().numpy()
             for j in range(D.codebooks):
-                assert rel_err(glg[:, j], odl[:, j]) <= 5e-2, (j, rel_err(glg[:, j], odl[:, j]))
+                assert rel_err(dglg[:, j], odl[:, j]) <= 5e-2, (j, rel_err(dglg[:, j], odl[:, j]))
             assert np.array_equal(gdc[0], gdc[1])
+            # every residual draw against the oracle's sampler on the GPU's depth logits
+            check_depth_draws(dglg, gdc, 99, 7, cfg_scale=1.5)
     finally:
         m3.m3_destroy(ctx)
