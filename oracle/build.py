@@ -9,14 +9,16 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "m3_oracle.cpp")
+SRCS = [SRC, os.path.join(HERE, "dit_oracle.cpp")]
 OUT = os.path.join(HERE, "liboracle.so")
 
 
 def build(force: bool = False) -> str:
-    if not force and os.path.exists(OUT) and os.path.getmtime(OUT) >= os.path.getmtime(SRC):
+    if not force and os.path.exists(OUT) and \
+            os.path.getmtime(OUT) >= max(os.path.getmtime(f) for f in SRCS):
         return OUT
     cmd = ["g++", "-O2", "-std=c++17", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
-           "-fPIC", "-shared", SRC, "-o", OUT + ".tmp"]
+           "-fPIC", "-shared", *SRCS, "-o", OUT + ".tmp"]
     subprocess.check_call(cmd)
     os.replace(OUT + ".tmp", OUT)
     return OUT

@@ -434,3 +434,155 @@ class Depth:
         if rc != 0:
             raise RuntimeError(f"ora_depth_decode: {rc}")
         return codes, lg
+
+
+# ------------------------------------------------------------------- DiT ----
+# The chunk-denoise DiT (oracle/dit_oracle.cpp); fp16 values cross as uint16 bits.
+
+class OraDitCfg(C.Structure):
+    _fields_ = [("width", C.c_int), ("n_layers", C.c_int), ("n_heads", C.c_int),
+                ("head_dim", C.c_int), ("ffn", C.c_int), ("latent", C.c_int), ("cond", C.c_int),
+                ("temb", C.c_int), ("rope_dims", C.c_int), ("rope_theta", C.c_double),
+                ("ln_eps", C.c_float)]
+
+
+DIT_LAYER_FIELDS = ("ln1_g", "ln1_b", "wqkv", "wo", "ln2_g", "ln2_b", "wg", "wu", "wd")
+
+
+class OraDitLayer(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in DIT_LAYER_FIELDS]
+
+
+class OraDitWeights(C.Structure):
+    _fields_ = [("w_in", C.c_void_p), ("w_t1", C.c_void_p), ("w_t2", C.c_void_p),
+                ("layers", C.POINTER(OraDitLayer)), ("lnf_g", C.c_void_p), ("lnf_b", C.c_void_p),
+                ("w_out", C.c_void_p)]
+
+
+def _dit_lib():
+    L = lib()
+    if not getattr(L, "_dit_ready", False):
+        vp, i64, f32, f64 = C.c_void_p, C.c_int64, C.c_float, C.c_double
+        L.ora_dit_layernorm.restype = None
+        L.ora_dit_layernorm.argtypes = [vp, vp, vp, i64, f32, vp]
+        L.ora_dit_rope.restype = None
+        L.ora_dit_rope.argtypes = [vp, C.c_int, i64, f64]
+        L.ora_dit_attention.restype = None
+        L.ora_dit_attention.argtypes = [vp, vp, vp, i64, C.c_int, vp]
+        L.ora_dit_time_features.restype = None
+        L.ora_dit_time_features.argtypes = [f32, C.c_int, vp]
+        L.ora_dit_layers.restype = C.c_int
+        L.ora_dit_layers.argtypes = [C.POINTER(OraDitCfg), C.POINTER(OraDitLayer), C.c_int,
+                                     C.c_int, C.c_int, vp]
+        L.ora_dit_forward.restype = C.c_int
+        L.ora_dit_forward.argtypes = [C.POINTER(OraDitCfg), C.POINTER(OraDitWeights), C.c_int,
+                                      C.c_int, vp, f32, vp, vp]
+        L.ora_dit_guide_step.restype = None
+        L.ora_dit_guide_step.argtypes = [i64, vp, vp, vp, f32, f32, f32, vp, vp]
+        L.ora_dit_step.restype = C.c_int
+        L.ora_dit_step.argtypes = [C.POINTER(OraDitCfg), C.POINTER(OraDitWeights), C.c_int, vp,
+                                   vp, vp, f32, f32, f32, vp, vp, vp]
+        L._dit_ready = True
+    return L
+
+
+def h16(t) -> np.ndarray:
+    """fp16 tensor / array as C-contiguous uint16 bits."""
+    return bits(t)
+
+
+def f16_to_f32(u16: np.ndarray) -> np.ndarray:
+    return np.ascontiguousarray(u16, np.uint16).view(np.float16).astype(np.float32)
+
+
+def dit_layernorm(x, g_bits, b_bits, eps) -> np.ndarray:
+    x = np.ascontiguousarray(x, np.float32)
+    out = np.empty_like(x)
+    _dit_lib().ora_dit_layernorm(_p(x), _p(np.ascontiguousarray(g_bits, np.uint16)),
+                                 _p(np.ascontiguousarray(b_bits, np.uint16)), x.size, eps, _p(out))
+    return out
+
+
+def dit_rope(v, rot, pos, theta) -> np.ndarray:
+    v = np.array(v, np.float32, copy=True)
+    _dit_lib().ora_dit_rope(_p(v), rot, pos, theta)
+    return v
+
+
+def dit_attention(q, k, v) -> np.ndarray:
+    q, k, v = (np.ascontiguousarray(a, np.float32) for a in (q, k, v))
+    T, d = q.shape
+    out = np.empty((T, d), np.float32)
+    _dit_lib().ora_dit_attention(_p(q), _p(k), _p(v), T, d, _p(out))
+    return out
+
+
+def dit_time_features(t, temb) -> np.ndarray:
+    out = np.empty(temb, np.float32)
+    _dit_lib().ora_dit_time_features(t, temb, _p(out))
+    return out
+
+
+def dit_guide_step(x, vc_bits, vu_bits, cfg_scale, sigma, sigma_next):
+    x = np.ascontiguousarray(x, np.float32)
+    xn = np.empty_like(x)
+    vg = np.empty_like(x)
+    _dit_lib().ora_dit_guide_step(x.size, _p(x), _p(np.ascontiguousarray(vc_bits, np.uint16)),
+                                  _p(np.ascontiguousarray(vu_bits, np.uint16)), cfg_scale, sigma,
+                                  sigma_next, _p(xn), _p(vg))
+    return xn, vg
+
+
+class Dit:
+    """The oracle's DiT: fp16 weights (synth.dit_weights) as raw bits."""
+
+    def __init__(self, shape, w: dict):
+        self.shape = shape
+        self.keep = _Keep()
+        k = self.keep
+        self.cfg = OraDitCfg(shape.width, shape.n_layers, shape.n_heads, shape.head_dim,
+                             shape.ffn, shape.latent, shape.cond, shape.temb, shape.rope_dims,
+                             shape.rope_theta, shape.ln_eps)
+        arr = (OraDitLayer * max(1, len(w["layers"])))()
+        for i, Lw in enumerate(w["layers"]):
+            arr[i] = OraDitLayer(*[k(h16(Lw[n])) for n in DIT_LAYER_FIELDS])
+        self.layers = arr
+        self.W = OraDitWeights(k(h16(w["w_in"])), k(h16(w["w_t1"])), k(h16(w["w_t2"])), arr,
+                               k(h16(w["lnf_g"])), k(h16(w["lnf_b"])), k(h16(w["w_out"])))
+
+    def layers_forward(self, h_bits, B, T, first=0, n=None):
+        """Blocks first..first+n on h [B, T, W] (fp16 bits); returns the new bits."""
+        h = np.ascontiguousarray(h_bits, np.uint16).copy()
+        n = self.shape.n_layers - first if n is None else n
+        sub = C.cast(C.byref(self.layers, first * C.sizeof(OraDitLayer)), C.POINTER(OraDitLayer))
+        rc = _dit_lib().ora_dit_layers(C.byref(self.cfg), sub, n, B, T, _p(h))
+        if rc:
+            raise RuntimeError(f"ora_dit_layers: {rc}")
+        return h
+
+    def forward(self, h_in_bits, B, T, t, with_h=False):
+        s = self.shape
+        hin = np.ascontiguousarray(h_in_bits, np.uint16)
+        v = np.empty((B, T, s.latent), np.uint16)
+        hl = np.empty((B, T, s.width), np.uint16) if with_h else None
+        rc = _dit_lib().ora_dit_forward(C.byref(self.cfg), C.byref(self.W), B, T, _p(hin), t,
+                                        _p(v), _p(hl) if with_h else None)
+        if rc:
+            raise RuntimeError(f"ora_dit_forward: {rc}")
+        return (v, hl) if with_h else v
+
+    def step(self, x, ctx_bits, cond_bits, sigma, sigma_next, cfg_scale):
+        """One denoising step: (x_next fp32 [T, latent], guided v fp32, v_pair f16 bits)."""
+        s = self.shape
+        x = np.ascontiguousarray(x, np.float32)
+        T = x.shape[0]
+        xn = np.empty_like(x)
+        vg = np.empty_like(x)
+        vp = np.empty((2, T, s.latent), np.uint16)
+        rc = _dit_lib().ora_dit_step(C.byref(self.cfg), C.byref(self.W), T, _p(x),
+                                     _p(np.ascontiguousarray(ctx_bits, np.uint16)),
+                                     _p(np.ascontiguousarray(cond_bits, np.uint16)), sigma,
+                                     sigma_next, cfg_scale, _p(xn), _p(vg), _p(vp))
+        if rc:
+            raise RuntimeError(f"ora_dit_step: {rc}")
+        return xn, vg, vp

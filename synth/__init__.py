@@ -201,3 +201,79 @@ def depth_weights(d: DepthShape, seed: int, device="cpu") -> dict:
     out["heads"] = [normal((d.vocab, d.hidden), seed, f"depth/head{j}", std=0.02, device=device)
                     for j in range(d.codebooks)]
     return out
+
+
+# ------------------------------------------------------------------- DiT ----
+
+@dataclasses.dataclass(frozen=True)
+class DitShape:
+    """Shape of the chunk-denoise DiT (DiffSynth-Studio article, "各子模型的结构要点")."""
+    width: int = 2048        # 32 heads x 64
+    n_layers: int = 36
+    n_heads: int = 32
+    head_dim: int = 64
+    ffn: int = 8192
+    latent: int = 128        # Flow-VAE latent channels
+    cond: int = 2048         # condition channels
+    temb: int = 256          # Fourier timestep features
+    rope_dims: int = 32      # rotated dims per head (partial rotary embedding)
+    rope_theta: float = 1.0e4
+    ln_eps: float = 1.0e-5
+
+
+DIT = DitShape()
+# A 200-frame chunk at the latent rate 44100 / 512 Hz: int(200 * 44100 / 512 / 25)
+DIT_CHUNK_T = 689
+DIT_TINY = DitShape(width=128, n_layers=2, n_heads=2, head_dim=64, ffn=256, latent=16, cond=96,
+                    temb=32, rope_dims=32)
+
+DIT_LAYER_TENSORS = ("ln1_g", "ln1_b", "wqkv", "wo", "ln2_g", "ln2_b", "wg", "wu", "wd")
+
+
+def dit_layer_weights(s: DitShape, seed: int, layer: int, device="cpu") -> dict:
+    """One DiT block's fp16 tensors: weights N(0, .02^2), LayerNorm gains
+    1 + N(0, .01^2) and biases N(0, .01^2)."""
+    W, F = s.width, s.ffn
+    shapes = {"ln1_g": (W,), "ln1_b": (W,), "wqkv": (3 * W, W), "wo": (W, W), "ln2_g": (W,),
+              "ln2_b": (W,), "wg": (F, W), "wu": (F, W), "wd": (W, F)}
+    out = {}
+    for name, shape in shapes.items():
+        tag = f"dit/L{layer}/{name}"
+        if name.endswith("_g"):
+            out[name] = normal(shape, seed, tag, std=0.01, mean=1.0, device=device,
+                               dtype=torch.float16)
+        elif name.endswith("_b"):
+            out[name] = normal(shape, seed, tag, std=0.01, device=device, dtype=torch.float16)
+        else:
+            out[name] = normal(shape, seed, tag, std=0.02, device=device, dtype=torch.float16)
+    return out
+
+
+def dit_weights(s: DitShape, seed: int, device="cpu", layers=None) -> dict:
+    """The DiT's fp16 tensors outside the blocks, plus the blocks (all of them,
+    or the given list)."""
+    W, Cin = s.width, 2 * s.latent + s.cond
+    f16 = torch.float16
+    return {
+        "w_in": normal((W, Cin), seed, "dit/w_in", std=0.02, device=device, dtype=f16),
+        "w_t1": normal((W, s.temb), seed, "dit/w_t1", std=0.02, device=device, dtype=f16),
+        "w_t2": normal((W, W), seed, "dit/w_t2", std=0.02, device=device, dtype=f16),
+        "layers": layers if layers is not None else
+        [dit_layer_weights(s, seed, l, device) for l in range(s.n_layers)],
+        "lnf_g": normal((W,), seed, "dit/lnf_g", std=0.01, mean=1.0, device=device, dtype=f16),
+        "lnf_b": normal((W,), seed, "dit/lnf_b", std=0.01, device=device, dtype=f16),
+        "w_out": normal((s.latent, W), seed, "dit/w_out", std=0.02, device=device, dtype=f16),
+    }
+
+
+def dit_inputs(s: DitShape, T: int, seed: int, device="cpu"):
+    """A chunk's step inputs: x_t [T, latent] fp32 N(0, 1) (the noisy latent),
+    the context latent [T, latent] fp16 N(0, 1) over the first overlap frames
+    (172 of a full chunk, proportionally fewer for short T) and zeros after,
+    and the condition [T, cond] fp16 N(0, 1)."""
+    x = normal((T, s.latent), seed, "dit/x_t", device=device, dtype=torch.float32)
+    ctx = normal((T, s.latent), seed, "dit/ctx", device=device, dtype=torch.float16)
+    n_ov = min(T, max(1, (172 * T) // DIT_CHUNK_T))
+    ctx[n_ov:] = 0
+    cond = normal((T, s.cond), seed, "dit/cond", device=device, dtype=torch.float16)
+    return x, ctx, cond
