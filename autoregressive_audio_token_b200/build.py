@@ -24,12 +24,12 @@ FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", 
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]
 
 SOURCES = ["m3.cu", "attention.cu", "gemv_tile.cu", "gemv_bf16.cu", "gemv_i8row.cu",
-           "gemv_i8g128.cu", "gemm_tc.cu"]
+           "gemv_i8g128.cu", "gemm_tc.cu", "dit.cu", "dit_gemm.cu"]
 
 
 def _deps_mtime() -> float:
-    files = [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [os.path.join(INCLUDE, "m3.h"),
-                                                                  os.path.abspath(__file__)]
+    files = ([os.path.join(CSRC, f) for f in os.listdir(CSRC)] +
+             [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE)] + [os.path.abspath(__file__)])
     return max(os.path.getmtime(f) for f in files)
 
 

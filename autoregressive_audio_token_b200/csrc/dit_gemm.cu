@@ -1,0 +1,394 @@
+// dit_gemm.cu -- persistent tcgen05 GEMM of the DiT (see dit_gemm.cuh).
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "dit_gemm.cuh"
+
+namespace m3 {
+
+namespace {
+
+constexpr int kGM = 128;                         // tokens per tile (MMA M = TMEM lanes)
+constexpr int kGN = 256;                         // outputs per tile (MMA N = TMEM columns)
+constexpr int kGK = 64;                          // K per stage: 64 fp16 = 128 bytes
+constexpr int kGStages = 4;
+constexpr int kGThreads = 192;                   // TMA warp, MMA warp, 4 epilogue warps
+constexpr uint32_t kABytes = kGM * kGK * 2;      // 16 KB
+constexpr uint32_t kBBytes = kGN * kGK * 2;      // 32 KB
+constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr uint32_t kAccCols = kGN;               // fp32 columns of one accumulator
+constexpr uint32_t kTmemCols = 2 * kAccCols;     // two accumulators: all 512 columns
+constexpr size_t kGSmem = (size_t)kGStages * kStageBytes + 1024 /* align */ + 256 /* bars */;
+
+// kind::f16 instruction descriptor: D fp32 (bits 4-5 = 1), A and B fp16
+// (bits 7-9, 10-12 = 0), both K-major (bits 15, 16 = 0), N >> 3 at bit 17,
+// M >> 4 at bit 24.
+constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(kGN >> 3) << 17) | ((uint32_t)(kGM >> 4) << 24);
+
+// Shared-memory matrix descriptor of a K-major operand in the 128-byte swizzle:
+// start address >> 4 (bits 0-13), leading byte offset (unused by swizzled
+// K-major layouts: 16 bytes) at bit 16, stride byte offset 1024 (8 rows of
+// 128 bytes) >> 4 at bit 32, version 1 at bit 46, swizzle mode 2 (128 B) at
+// bit 61.  The tile bases are 1024-byte aligned, so the base offset is 0.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         (1ull << 46) | (2ull << 61);
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_mma_f16(uint32_t tmem_d, uint64_t a, uint64_t b,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+      ::"r"(tmem_d), "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u),
+        "r"(0u)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's accumulator lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 2-D tiled tensor-map copy global -> this CTA's shared memory (no multicast).
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, "
+      "{%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* tm) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm)) : "memory");
+}
+
+__device__ __forceinline__ uint32_t h2pack(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+__device__ __forceinline__ float rh(float v) { return __half2float(__float2half_rn(v)); }
+
+// The epilogue of 32 accumulator columns o0..o0+31 of token row t.
+template <int EPI>
+__device__ __forceinline__ void epilogue_chunk(const DitGemmArgs& a, int t, int o0,
+                                               float (&v)[32]) {
+  if (t >= a.M) return;
+  if constexpr (EPI == DIT_EPI_GLU) {
+    // columns (2j, 2j+1) are (gate, up) of GLU output o0/2 + j
+    float y[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float g = rh(v[2 * j]), u = rh(v[2 * j + 1]);
+      const float s = rh(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))));
+      y[j] = __fmul_rn(s, u);
+    }
+    uint4* q = reinterpret_cast<uint4*>(a.out + (size_t)t * a.ldo + (o0 >> 1));
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+      q[c] = make_uint4(h2pack(y[8 * c], y[8 * c + 1]), h2pack(y[8 * c + 2], y[8 * c + 3]),
+                        h2pack(y[8 * c + 4], y[8 * c + 5]), h2pack(y[8 * c + 6], y[8 * c + 7]));
+  } else {
+  float y[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) y[j] = rh(v[j]);
+  __half* p = a.out + (size_t)t * a.ldo + o0;  // N is a multiple of 32: whole chunks only
+  if constexpr (EPI == DIT_EPI_TEMB) {
+    const uint4* q = reinterpret_cast<const uint4*>(a.vec + o0);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint4 w = q[c];
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws[k]));
+        y[8 * c + 2 * k] = __fadd_rn(y[8 * c + 2 * k], f.x);
+        y[8 * c + 2 * k + 1] = __fadd_rn(y[8 * c + 2 * k + 1], f.y);
+      }
+    }
+  } else if constexpr (EPI == DIT_EPI_ROPE) {
+    // the first 2 * rope_half dims of every q / k head: pairs (i, i + rope_half)
+    if (o0 < a.rope_cols && (o0 % a.head_dim) == 0 && a.rope_half == 16) {
+      const float2* cs = a.rope + (size_t)(t % a.rope_T) * 16;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float2 r = cs[i];
+        const float x0 = y[i], x1 = y[i + 16];
+        y[i] = __fsub_rn(__fmul_rn(x0, r.x), __fmul_rn(x1, r.y));
+        y[i + 16] = __fadd_rn(__fmul_rn(x1, r.x), __fmul_rn(x0, r.y));
+      }
+    }
+  } else if constexpr (EPI == DIT_EPI_RESID) {
+    const uint4* q = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint4 w = q[c];
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws[k]));
+        y[8 * c + 2 * k] = __fadd_rn(f.x, y[8 * c + 2 * k]);
+        y[8 * c + 2 * k + 1] = __fadd_rn(f.y, y[8 * c + 2 * k + 1]);
+      }
+    }
+  }
+  uint4* q = reinterpret_cast<uint4*>(p);
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    q[c] = make_uint4(h2pack(y[8 * c], y[8 * c + 1]), h2pack(y[8 * c + 2], y[8 * c + 3]),
+                      h2pack(y[8 * c + 4], y[8 * c + 5]), h2pack(y[8 * c + 6], y[8 * c + 7]));
+  }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kGThreads, 1)
+    dit_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const DitGemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGStages * kStageBytes);
+  uint64_t* empty = full + kGStages;
+  uint64_t* tfull = empty + kGStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  int* counts = reinterpret_cast<int*>(tmem_slot + 1);  // [0] issued, [1] consumed
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int num_m = (a.M + kGM - 1) / kGM, num_n = (a.N + kGN - 1) / kGN;
+  const int ntiles = num_m * num_n;
+  const int KB = a.K / kGK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kGStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 4);  // one arrival per epilogue warp
+    }
+    mbar_init(drain, 1);
+    counts[0] = counts[1] = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA --
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const int m0 = (tile % num_m) * kGM, n0 = (tile / num_m) * kGN;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % kGStages, use = it / kGStages;
+          if (use > 0 && !(ok = mbar_wait(&empty[s], (uint32_t)(use - 1) & 1u, a.err))) break;
+          uint8_t* sa = smem + (size_t)s * kStageBytes;
+          mbar_arrive_expect_tx(&full[s], kStageBytes);
+          tma_load_2d(sa, &tmA, kb * kGK, m0, &full[s]);
+          tma_load_2d(sa + kABytes, &tmB, kb * kGK, n0, &full[s]);
+        }
+      }
+      counts[0] = it;
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA --
+    if (lane == 0) {
+      int it = 0, lt = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++lt) {
+        const int acc = lt & 1, use_a = lt >> 1;
+        if (use_a > 0 && !(ok = mbar_wait(&tempty[acc], (uint32_t)(use_a - 1) & 1u, a.err))) break;
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)acc * kAccCols;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % kGStages, use = it / kGStages;
+          if (!(ok = mbar_wait(&full[s], (uint32_t)use & 1u, a.err))) break;
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + (size_t)s * kStageBytes), sb = sa + kABytes;
+#pragma unroll
+          for (int ks = 0; ks < kGK / 16; ++ks)
+            tc_mma_f16(d, sw128_desc(sa + ks * 32), sw128_desc(sb + ks * 32),
+                       (kb > 0 || ks > 0) ? 1u : 0u);
+          tc_commit(&empty[s]);
+        }
+        if (ok) tc_commit(&tfull[acc]);
+      }
+      counts[1] = it;
+      if (!ok) {  // let this thread's MMAs finish before the memory goes away
+        tc_commit(drain);
+        for (long long i = 0; i < kSpinLimit && !mbar_try_wait(drain, 0); ++i) {
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------- epilogue --
+    const int q = warp & 3;  // TMEM lanes 32q..32q+31 (the warp's access window)
+    int lt = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++lt) {
+      const int acc = lt & 1, use_a = lt >> 1;
+      if (!mbar_wait(&tfull[acc], (uint32_t)use_a & 1u, a.err)) break;
+      tc_fence_after();
+      const int m0 = (tile % num_m) * kGM, n0 = (tile / num_m) * kGN;
+      const int t = m0 + q * 32 + lane;
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * kAccCols;
+#pragma unroll 1
+      for (int c = 0; c < kGN / 32; ++c) {
+        if (n0 + c * 32 >= a.N) break;  // the last output block may be narrower (uniform)
+        float v[32];
+        tmem_ld32(taddr + (uint32_t)(c * 32), v);
+        epilogue_chunk<EPI>(a, t, n0 + c * 32, v);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // copies issued but never consumed (only after a failed wait): let them land
+    for (int it = counts[1]; it < counts[0]; ++it) {
+      const int s = it % kGStages;
+      for (long long i = 0; i < kSpinLimit && !mbar_try_wait(&full[s], (uint32_t)(it / kGStages) & 1u);
+           ++i) {
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// A [rows][ld] fp16 row-major matrix as a tensor map of (box_rows x 64) boxes
+// in the 128-byte swizzle.
+cudaError_t make_map(CUtensorMap* tm, const __half* base, int rows, int cols, int ld,
+                     int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {(cuuint32_t)kGK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int EPI>
+cudaError_t set_attr() {
+  return cudaFuncSetAttribute(dit_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)kGSmem);
+}
+
+template <int EPI>
+cudaError_t launch_t(const CUtensorMap& ta, const CUtensorMap& tb, const DitGemmArgs& a, int nsm,
+                     cudaStream_t st) {
+  const int ntiles = ((a.M + kGM - 1) / kGM) * ((a.N + kGN - 1) / kGN);
+  const int grid = ntiles < nsm ? ntiles : nsm;
+  dit_gemm_kernel<EPI><<<grid, kGThreads, kGSmem, st>>>(ta, tb, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t prepare_dit_gemm() {
+  if (!encode_fn()) return cudaErrorNotSupported;
+  cudaError_t e = set_attr<DIT_EPI_STORE>();
+  if (e == cudaSuccess) e = set_attr<DIT_EPI_TEMB>();
+  if (e == cudaSuccess) e = set_attr<DIT_EPI_ROPE>();
+  if (e == cudaSuccess) e = set_attr<DIT_EPI_RESID>();
+  if (e == cudaSuccess) e = set_attr<DIT_EPI_GLU>();
+  return e;
+}
+
+cudaError_t launch_dit_gemm(const __half* X, int ldx, const __half* W, const DitGemmArgs& a,
+                            int epi, int nsm, cudaStream_t st) {
+  if (!X || !W || !a.out || a.M < 1 || a.N < 1 || a.K < kGK || a.K % kGK || ldx < a.K ||
+      ldx % 8 || (reinterpret_cast<uintptr_t>(X) & 15) || (reinterpret_cast<uintptr_t>(W) & 15) ||
+      (reinterpret_cast<uintptr_t>(a.out) & 15) || a.ldo % 8 || nsm < 1)
+    return cudaErrorInvalidValue;
+  // whole 32-column chunks in the epilogue; 16-byte aligned vector accesses
+  if (a.N % 32 || (epi == DIT_EPI_GLU ? a.ldo < a.N / 2 : a.ldo < a.N)) return cudaErrorInvalidValue;
+  if (epi == DIT_EPI_TEMB && (reinterpret_cast<uintptr_t>(a.vec) & 15)) return cudaErrorInvalidValue;
+  if (epi == DIT_EPI_TEMB && !a.vec) return cudaErrorInvalidValue;
+  if (epi == DIT_EPI_ROPE && (!a.rope || a.rope_T < 1 || a.head_dim % 32 || a.rope_half != 16))
+    return cudaErrorInvalidValue;
+  CUtensorMap ta, tb;
+  cudaError_t e = make_map(&ta, X, a.M, a.K, ldx, kGM);
+  if (e == cudaSuccess) e = make_map(&tb, W, a.N, a.K, a.K, kGN);
+  if (e != cudaSuccess) return e;
+  switch (epi) {
+    case DIT_EPI_STORE: return launch_t<DIT_EPI_STORE>(ta, tb, a, nsm, st);
+    case DIT_EPI_TEMB: return launch_t<DIT_EPI_TEMB>(ta, tb, a, nsm, st);
+    case DIT_EPI_ROPE: return launch_t<DIT_EPI_ROPE>(ta, tb, a, nsm, st);
+    case DIT_EPI_RESID: return launch_t<DIT_EPI_RESID>(ta, tb, a, nsm, st);
+    case DIT_EPI_GLU: return launch_t<DIT_EPI_GLU>(ta, tb, a, nsm, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace m3

@@ -29,6 +29,11 @@ static int fail(int code, const std::string& msg) {
   return code;
 }
 
+namespace m3 {
+// The same thread-local message for the library's other translation units.
+int set_error(int code, const std::string& msg) { return fail(code, msg); }
+}  // namespace m3
+
 #define CK(call)                                                                        \
   do {                                                                                  \
     cudaError_t e_ = (call);                                                            \

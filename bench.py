@@ -66,6 +66,10 @@ def parse():
     p.add_argument("--depth-only", action="store_true",
                    help="time the RVQ depth decoder (m3_depth_decode) alone, int8 group-128, "
                         "on a frame's hidden state")
+    p.add_argument("--dit", action="store_true",
+                   help="the DiT chunk-denoise workload: full-size DiT (36 blocks, width 2048, "
+                        "FFN 8192), one 200-frame chunk = 689 latent frames, cond + uncond as "
+                        "one batch-2 forward; a step is one denoising step")
     p.add_argument("--sweep", action="store_true",
                    help="batched-variations sweep: rows 1..16 x context 1500/4500/9000, "
                         "bf16 and int8; one JSON line per point")
@@ -670,6 +674,111 @@ def run_generate(args):
     m3.m3_destroy(ctx)
 
 
+DIT_CFG = 1.7
+
+
+def dit_step_flops(s, T: int) -> float:
+    """FLOPs of one denoising step (batch 2 x T tokens): every projection as
+    2 M N K plus attention's Q K^T and P V (4 B T^2 W per block)."""
+    M = 2 * T
+    W, F, Cin = s.width, s.ffn, 2 * s.latent + s.cond
+    per_block = 3 * W * W + W * W + 2 * F * W + F * W
+    gemm = 2.0 * M * (Cin * W + s.n_layers * per_block + W * s.latent)
+    attn = 4.0 * 2 * T * T * W * s.n_layers
+    return gemm + attn
+
+
+def run_dit(args):
+    """The DiT chunk-denoise step on one GPU: the full-size DiT, one 200-frame
+    chunk (689 latent frames), cond + uncond as one batch-2 forward, CFG 1.7.
+    W untimed steps, then K steps in one m3_dit_denoise call between CUDA
+    events; every step streams 4.8 GB of fp16 weights and 1378 tokens'
+    activations (far beyond L2), so no flush is needed."""
+    import torch
+    from autoregressive_audio_token_b200 import dit as D
+    import synth
+    torch.cuda.set_device(0)
+    s, T = synth.DIT, synth.DIT_CHUNK_T
+    h = D.m3_dit_create(D.config_from_shape(s, T))
+    for l in range(s.n_layers):  # generate on the GPU, load block by block
+        D.m3_dit_load(h, {"layers": [synth.dit_layer_weights(s, 0, l, device="cuda")]},
+                      first_layer=l, outer=False)
+    w = synth.dit_weights(s, 0, device="cuda", layers=[])
+    D.m3_dit_load(h, w)
+    x, ctx, cond = synth.dit_inputs(s, T, 1, device="cuda")
+    K, Wm = args.steps, max(args.warmup, 3)
+    sig = [1.0 - i / K for i in range(K + 1)]
+    xw = x.clone()
+    D.m3_dit_denoise(h, xw, ctx, cond, [1.0 - i / Wm for i in range(Wm + 1)], DIT_CFG)
+    torch.cuda.synchronize()
+    D.m3_dit_sync_status(h)
+    clocks = ClockSampler(0, "/tmp/m3_clocks_dit.csv")
+    xt = x.clone()
+    torch.cuda.synchronize()
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    D.m3_dit_denoise(h, xt, ctx, cond, sig, DIT_CFG)
+    e1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    D.m3_dit_sync_status(h)
+    ms = e0.elapsed_time(e1) / K
+    # end to end: inputs from pinned host memory and the latent back, per step
+    xh, ch, dh = x.cpu().pin_memory(), ctx.cpu().pin_memory(), cond.cpu().pin_memory()
+    xo = torch.empty_like(xh).pin_memory()
+    xd, cd, dd = torch.empty_like(x), torch.empty_like(ctx), torch.empty_like(cond)
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record()
+    for i in range(K):
+        xd.copy_(xh, non_blocking=True)
+        cd.copy_(ch, non_blocking=True)
+        dd.copy_(dh, non_blocking=True)
+        D.m3_dit_step(h, xd, cd, dd, sig[i], sig[i + 1], DIT_CFG)
+        xo.copy_(xd, non_blocking=True)
+    e3.record()
+    torch.cuda.synchronize()
+    D.m3_dit_sync_status(h)
+    e2e_ms = e2.elapsed_time(e3) / K
+    kernels = {}
+    for which, name in [(2, "gate_up_glu"), (3, "down"), (0, "qkv_rope"), (1, "o_proj")]:
+        kms, kfl = D.m3_dit_time_gemm(h, which, T, 36)
+        kernels[name] = {"ms": kms, "flops": kfl, "tflops": kfl / kms / 1e9}
+    D.m3_dit_destroy(h)
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except Exception:
+        pass
+    # a kernel timed alone takes the burst peak; fp16 and bf16 share the rate
+    peak = peaks.get("bf16_tflops", 1590.0)
+    flops = dit_step_flops(s, T)
+    dom = kernels["gate_up_glu"]
+    out = {
+        "metric": "DiT chunk-denoise steps/s (36 blocks, 2 x 689 tokens, fp16)",
+        "value": 1000.0 / ms, "unit": "steps/s", "n_gpus": 1, "steps": K, "warmup": Wm,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16", "data": "synthetic (seeded N(0,0.02^2) fp16 weights, N(0,1) latents and "
+                                "condition)",
+        "config": {"workload": "dit-36L-2048-ffn8192-chunk200-T689-batch2-cfg1.7",
+                   "tokens": 2 * T, "cfg_scale": DIT_CFG,
+                   "l2": "no flush: 4.8 GB of weights per step >> 126 MB L2"},
+        "achieved_tflops": flops / ms / 1e9, "flops_per_step": flops,
+        "roofline": {"bound": "tensor", "kernel": "dit_gemm_kernel gate/up + GLU (f16)",
+                     "achieved": dom["tflops"], "peak": peak, "unit": "TFLOP/s",
+                     "frac": dom["tflops"] / peak,
+                     "peak_source": "measured" if "bf16_tflops" in peaks else "fallback",
+                     "traffic": None, "flops_per_launch": dom["flops"]},
+        "kernels": kernels,
+        "e2e": {"value": 1000.0 / e2e_ms, "unit": "steps/s",
+                "h2d_bytes_per_step": x.numel() * 4 + ctx.numel() * 2 + cond.numel() * 2,
+                "d2h_bytes_per_step": x.numel() * 4},
+        "gpu_launches": (1 + 3 + 1 + 7 * s.n_layers + 2 + 1) * K,
+        "clocks": clk,
+    }
+    print(json.dumps(out))
+
+
 def run_depth_only(args):
     """The RVQ depth decoder alone (int8 weights, one scale per group of 128):
     m3_depth_decode on a fixed final hidden state and semantic code, 2 rows
@@ -754,6 +863,10 @@ def main():
     if args.depth_only:
         if rank == 0:
             run_depth_only(args)
+        return
+    if args.dit:
+        if rank == 0:
+            run_dit(args)
         return
     if args.generate:
         if rank == 0:

@@ -224,7 +224,7 @@ class DitShape:
 DIT = DitShape()
 # A 200-frame chunk at the latent rate 44100 / 512 Hz: int(200 * 44100 / 512 / 25)
 DIT_CHUNK_T = 689
-DIT_TINY = DitShape(width=128, n_layers=2, n_heads=2, head_dim=64, ffn=256, latent=16, cond=96,
+DIT_TINY = DitShape(width=256, n_layers=2, n_heads=4, head_dim=64, ffn=512, latent=32, cond=192,
                     temb=32, rope_dims=32)
 
 DIT_LAYER_TENSORS = ("ln1_g", "ln1_b", "wqkv", "wo", "ln2_g", "ln2_b", "wg", "wu", "wd")

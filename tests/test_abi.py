@@ -8,9 +8,15 @@ import re
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _declared():
-    src = open(os.path.join(ROOT, "include", "m3.h")).read()
-    return sorted(set(re.findall(r"^M3_API\s+[\w\s\*]+?\b(m3_\w+)\s*\(", src, re.M)))
+def _declared(header=None):
+    """The functions include/*.h declare (or one header's)."""
+    inc = os.path.join(ROOT, "include")
+    names = set()
+    for h in sorted(os.listdir(inc)):
+        if header is None or h == header:
+            src = open(os.path.join(inc, h)).read()
+            names |= set(re.findall(r"^M3_API\s+[\w\s\*]+?\b(m3_\w+)\s*\(", src, re.M))
+    return sorted(names)
 
 
 def test_header_declares_the_abi():
@@ -28,10 +34,27 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_binding_covers_the_abi():
-    from autoregressive_audio_token_b200 import m3
-    assert sorted(m3.EXPORTED) == _declared()
-    for n in _declared():
+    from autoregressive_audio_token_b200 import dit, m3
+    assert sorted(m3.EXPORTED) == _declared("m3.h")
+    assert sorted(dit.EXPORTED) == _declared("m3_dit.h")
+    for n in _declared("m3.h"):
         assert hasattr(m3, n), n
+    for n in _declared("m3_dit.h"):
+        assert hasattr(dit, n), n
+
+
+def test_dit_create_rejects_unsupported_shapes_without_gpu():
+    import synth
+    from autoregressive_audio_token_b200 import dit, m3
+    for bad in ({"head_dim": 128}, {"rope_dims": 16}, {"width": 384, "n_heads": 6},
+                {"ffn": 100}, {"temb": 12}, {"latent": 12}):
+        import dataclasses
+        s = dataclasses.replace(synth.DIT, **bad)
+        d = C.c_void_p()
+        rc = m3.lib.m3_dit_create(C.byref(dit.config_from_shape(s, 689)), None, C.byref(d))
+        assert rc == m3.M3_EINVAL, bad
+        assert b"m3_dit_config" in m3.lib.m3_last_error()
+    assert m3.lib.m3_dit_step(None, 1, None, None, None, 1.0, 0.9, 1.7, None, None) == m3.M3_EINVAL
 
 
 def test_create_rejects_bad_config_without_gpu():

@@ -159,24 +159,28 @@ def _loop_case(ora, rows, cfg, k, with_depth, F, bucket, end_logit, n_prefill=20
             V = DEPTH.vocab
             all_o, all_m, all_g = [], [], []
             for f in range(F):
-                if not np.all(gc[f, :, 1] >= 0):
+                live = gc[f, :, 1] >= 0  # rows whose key drew residual codes this frame
+                if not live.any():
                     continue
+                # rows are independent in the depth decoder (CFG pairs stop together),
+                # so stopped rows ride along on any valid code
+                c0 = torch.from_numpy(np.where(gc[f, :, 0] < 0, 0, gc[f, :, 0]).astype(np.int32))
                 dc = torch.empty((rows, nc), dtype=torch.int32, device="cuda")
                 dl = torch.empty((rows, nc, V), dtype=torch.float32, device="cuda")
-                m.m3.m3_depth_decode(m.ctx, hh[f].contiguous(), codes[f, :, 0].contiguous(),
-                                     21, 500 + f, cfg, 1.0, dc, logits=dl)
+                m.m3.m3_depth_decode(m.ctx, hh[f].contiguous(), c0.cuda(), 21, 500 + f, cfg, 1.0,
+                                     dc, logits=dl)
                 torch.cuda.synchronize()
                 m.m3.m3_sync_status(m.ctx)
                 dcn = dc.cpu().numpy()
-                assert np.array_equal(dcn, gc[f, :, 1:]), f
+                assert np.array_equal(dcn[live], gc[f, live, 1:]), f
                 glg = dl.cpu().numpy()
                 for j in range(nc):
                     o, mg = ora.draw(np.ascontiguousarray(glg[:, j]), 21, 500 + f,
                                      cfg_scale=cfg, index_base=(j + 1) << 32)
-                    all_o.append(o)
-                    all_m.append(mg)
-                    all_g.append(dcn[:, j])
-            assert all_o, "no frame with every row running"
+                    all_o.append(o[live])
+                    all_m.append(mg[live])
+                    all_g.append(dcn[live, j])
+            assert all_o, "no frame drew residual codes"
             check_draws(np.concatenate(all_o), np.concatenate(all_m), np.concatenate(all_g))
         return nf
     finally:

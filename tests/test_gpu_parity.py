@@ -388,7 +388,7 @@ def test_depth_decoder_teacher_forced(ora, rows, cfg):
     s = synth.TINY
     D = synth.DepthShape(hidden=256, n_layers=2, n_heads=4, head_dim=64, ffn=384, codebooks=7,
                          vocab=128, sem_vocab=s.slice_len, in_hidden=s.hidden)
-    m = Model(s, seed=6, depth=D, max_rows=2)
+    m = Model(s, seed=6, depth=D, max_rows=max(2, rows))
     try:
         h = synth.normal((rows, s.hidden), 6, "hframe").cuda()
         code0 = torch.tensor([3, 77, 5, 400][:rows], dtype=torch.int32, device="cuda")
