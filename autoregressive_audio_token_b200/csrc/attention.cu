@@ -33,6 +33,27 @@ static cudaError_t launch_attn_t(const AttnArgs& a, int splits, int rows, cudaSt
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
+template <int D, int KVF16>
+static int attn_resident_t() {
+  constexpr size_t smem = attn_smem_bytes<D>();
+  auto kern = attn_decode_kernel<D, KVF16>;
+  int n = 0;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kAttnWarps * 32, smem) !=
+          cudaSuccess)
+    return 0;
+  return n;
+}
+
+int attn_ctas_per_sm(int D, int kv_f16) {
+  if (D == 128) return kv_f16 ? attn_resident_t<128, 1>() : attn_resident_t<128, 0>();
+  if (D == 64) return kv_f16 ? attn_resident_t<64, 1>() : attn_resident_t<64, 0>();
+  return 0;
+}
+
 cudaError_t launch_attn(const AttnArgs& a, int D, int kv_f16, int splits, int rows,
                         cudaStream_t st, bool pdl) {
   if (D == 128) return kv_f16 ? launch_attn_t<128, 1>(a, splits, rows, st, pdl)

@@ -164,8 +164,8 @@ __global__ void dit_rope_table_kernel(int T, int rot, double theta, float2* __re
 // Bidirectional attention of one (batch element, head) over its T tokens,
 // heads of 64: a CTA of 4 warps takes 64 queries (16 per warp) and walks the
 // keys in tiles of 64 with warp-level tensor-core MMA (m16n8k16, fp16 in,
-// fp32 accumulation): S = Q K^T / 8, online softmax in fp32, P rounded to
-// fp16 for O += P V, O / l at the end.  K / V tiles double-buffered in
+// fp32 accumulation): S = Q K^T / 8, online softmax in fp32 (in log2 units,
+// exp2), P rounded to fp16 for O += P V, O / l at the end.  K / V tiles double-buffered in
 // shared memory by cp.async.
 constexpr int kDaWarps = 4;
 constexpr int kDaQ = 16 * kDaWarps;  // queries per CTA
@@ -221,7 +221,8 @@ __global__ void __launch_bounds__(kDaWarps * 32)
 #pragma unroll
   for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
   float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
-  const float scale = 0.125f;  // 1 / sqrt(64)
+  // scores in log2 units: exp(s - m) = exp2(s log2e - m log2e), one MUFU op
+  const float scale = 0.125f * 1.4426950408889634f;  // 1 / sqrt(64) * log2(e)
 
   for (int kt = 0; kt < nkt; ++kt) {
     if (kt + 1 < nkt) load_kv(kt + 1, (kt + 1) & 1);
@@ -267,15 +268,15 @@ __global__ void __launch_bounds__(kDaWarps * 32)
       mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
       mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
       const float mn = fmaxf(m_run[h], mx[h]);
-      alpha[h] = expf(m_run[h] - mn);  // 0 at the first tile (m_run = -inf)
+      alpha[h] = exp2f(m_run[h] - mn);  // 0 at the first tile (m_run = -inf)
       m_run[h] = mn;
     }
     float ls[2] = {0.0f, 0.0f};
     uint32_t pa[4][4];  // P as the A operand of P V: 4 k-steps of 16 keys
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt) {
-      const float e0 = expf(s[nt][0] - m_run[0]), e1 = expf(s[nt][1] - m_run[0]);
-      const float e2 = expf(s[nt][2] - m_run[1]), e3 = expf(s[nt][3] - m_run[1]);
+      const float e0 = exp2f(s[nt][0] - m_run[0]), e1 = exp2f(s[nt][1] - m_run[0]);
+      const float e2 = exp2f(s[nt][2] - m_run[1]), e3 = exp2f(s[nt][3] - m_run[1]);
       ls[0] += e0 + e1;
       ls[1] += e2 + e3;
       const __half2 h01 = __floats2half2_rn(e0, e1), h23 = __floats2half2_rn(e2, e3);

@@ -62,6 +62,8 @@ cudaError_t plan_gemv_tile(int N, int K, int mr, int wf, int epi, int nsm, int s
 cudaError_t launch_gemv_tile(const GemvArgs& a, int wf, int epi, const TileLaunch& L,
                              cudaStream_t st, bool pdl);
 
+// Attention CTAs one SM holds at once (0 if the query fails).
+int attn_ctas_per_sm(int D, int kv_f16);
 cudaError_t launch_attn(const AttnArgs& a, int D, int kv_f16, int splits, int rows,
                         cudaStream_t st, bool pdl);
 

@@ -116,6 +116,7 @@ struct m3_ctx {
   FrameParams* fp = nullptr;
   int* err = nullptr;
   int max_splits = kAttnMaxSplits;
+  int attn_per_sm[2] = {0, 0};  // attention CTAs an SM holds (bf16 / f16 cache)
   // depth buffers
   bf16* dh = nullptr;
   int* dcodes = nullptr;
@@ -354,6 +355,8 @@ extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) 
     return bail(fail(M3_ECUDA, "stream/event creation"));
   const m3_config& g = c->cfg;
   const int R = g.max_rows;
+  c->attn_per_sm[0] = attn_ctas_per_sm(g.head_dim, 0);
+  c->attn_per_sm[1] = attn_ctas_per_sm(g.head_dim, 1);
   c->L.resize(g.n_layers);
   c->loaded.assign(g.n_layers, 0);
   int rc = M3_OK;
@@ -829,8 +832,11 @@ extern "C" int m3_kv_get(m3_ctx* c, int row, int n_positions, void* k_host, void
 
 // ------------------------------------------------------------ the frame ----
 static int attn_splits(const m3_ctx* c, int rows, int nb) {
+  // as many splits as keep every (row, KV head) pair's CTAs resident at
+  // once: a second, partial wave of CTAs would run at a fraction of the SMs
   const int pairs = rows * c->cfg.n_kv_heads;
-  int s = (2 * c->nsm + pairs - 1) / pairs;
+  const int per_sm = c->attn_per_sm[c->kv_f16 ? 1 : 0];
+  int s = (c->nsm * (per_sm > 0 ? per_sm : 2)) / pairs;
   const int tiles = nb * c->bucket / kAttnTile;
   if (s > tiles) s = tiles;
   if (s > c->max_splits) s = c->max_splits;

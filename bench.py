@@ -698,7 +698,10 @@ def run_dit(args):
     from autoregressive_audio_token_b200 import dit as D
     import synth
     torch.cuda.set_device(0)
+    import dataclasses
     s, T = synth.DIT, synth.DIT_CHUNK_T
+    if args.layers != 36:  # fewer blocks only for profiling small cases
+        s = dataclasses.replace(s, n_layers=args.layers)
     h = D.m3_dit_create(D.config_from_shape(s, T))
     for l in range(s.n_layers):  # generate on the GPU, load block by block
         D.m3_dit_load(h, {"layers": [synth.dit_layer_weights(s, 0, l, device="cuda")]},
@@ -742,7 +745,7 @@ def run_dit(args):
     e2e_ms = e2.elapsed_time(e3) / K
     kernels = {}
     for which, name in [(2, "gate_up_glu"), (3, "down"), (0, "qkv_rope"), (1, "o_proj")]:
-        kms, kfl = D.m3_dit_time_gemm(h, which, T, 36)
+        kms, kfl = D.m3_dit_time_gemm(h, which, T, max(36, s.n_layers))
         kernels[name] = {"ms": kms, "flops": kfl, "tflops": kfl / kms / 1e9}
     D.m3_dit_destroy(h)
     peaks = {}
@@ -760,7 +763,7 @@ def run_dit(args):
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f16", "data": "synthetic (seeded N(0,0.02^2) fp16 weights, N(0,1) latents and "
                                 "condition)",
-        "config": {"workload": "dit-36L-2048-ffn8192-chunk200-T689-batch2-cfg1.7",
+        "config": {"workload": f"dit-{s.n_layers}L-2048-ffn8192-chunk200-T689-batch2-cfg1.7",
                    "tokens": 2 * T, "cfg_scale": DIT_CFG,
                    "l2": "no flush: 4.8 GB of weights per step >> 126 MB L2"},
         "achieved_tflops": flops / ms / 1e9, "flops_per_step": flops,
