@@ -23,9 +23,13 @@ constexpr uint32_t kTmemCols = 2 * kAccCols;     // two accumulators: all 512 co
 constexpr size_t kGSmem = (size_t)kGStages * kStageBytes + 1024 /* align */ + 256 /* bars */;
 
 // kind::f16 instruction descriptor: D fp32 (bits 4-5 = 1), A and B fp16
-// (bits 7-9, 10-12 = 0), both K-major (bits 15, 16 = 0), N >> 3 at bit 17,
-// M >> 4 at bit 24.
-constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(kGN >> 3) << 17) | ((uint32_t)(kGM >> 4) << 24);
+// (bits 7-9, 10-12 = 0) or both bf16 (= 1), both K-major (bits 15, 16 = 0),
+// N >> 3 at bit 17, M >> 4 at bit 24.
+template <int BF>
+constexpr uint32_t idesc_1() {
+  return (1u << 4) | ((uint32_t)BF << 7) | ((uint32_t)BF << 10) | ((uint32_t)(kGN >> 3) << 17) |
+         ((uint32_t)(kGM >> 4) << 24);
+}
 
 // Shared-memory matrix descriptor of a K-major operand in the 128-byte swizzle:
 // start address >> 4 (bits 0-13), leading byte offset (unused by swizzled
@@ -44,14 +48,15 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
+template <int BF>
 __device__ __forceinline__ void tc_mma_f16(uint32_t tmem_d, uint64_t a, uint64_t b,
                                            uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
-      ::"r"(tmem_d), "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u),
-        "r"(0u)
+      ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc_1<BF>()), "r"(accumulate), "r"(0u), "r"(0u),
+        "r"(0u), "r"(0u)
       : "memory");
 }
 
@@ -93,37 +98,57 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* tm) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm)) : "memory");
 }
 
+// Two fp32 -> the output type's packed pair (round to nearest even); one fp32
+// through the output type; a packed pair of the output type -> fp32.
+template <int BF>
 __device__ __forceinline__ uint32_t h2pack(float lo, float hi) {
-  const __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
+  if constexpr (BF) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  } else {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  }
 }
 
-__device__ __forceinline__ float rh(float v) { return __half2float(__float2half_rn(v)); }
+template <int BF>
+__device__ __forceinline__ float rh(float v) {
+  if constexpr (BF) return __bfloat162float(__float2bfloat16_rn(v));
+  else return __half2float(__float2half_rn(v));
+}
+
+template <int BF>
+__device__ __forceinline__ float2 unpack2(uint32_t w) {
+  if constexpr (BF) return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
+  else return __half22float2(*reinterpret_cast<const __half2*>(&w));
+}
 
 // The epilogue of 32 accumulator columns o0..o0+31 of token row t.
-template <int EPI>
+template <int EPI, int BF>
 __device__ __forceinline__ void epilogue_chunk(const DitGemmArgs& a, int t, int o0,
                                                float (&v)[32]) {
+  typedef uint16_t elem_t;  // the output type's bits (fp16 or bf16)
+  elem_t* const out = static_cast<elem_t*>(a.out);
   if (t >= a.M) return;
   if constexpr (EPI == DIT_EPI_GLU) {
     // columns (2j, 2j+1) are (gate, up) of GLU output o0/2 + j
     float y[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
-      const float g = rh(v[2 * j]), u = rh(v[2 * j + 1]);
-      const float s = rh(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))));
+      const float g = rh<BF>(v[2 * j]), u = rh<BF>(v[2 * j + 1]);
+      const float s = rh<BF>(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))));
       y[j] = __fmul_rn(s, u);
     }
-    uint4* q = reinterpret_cast<uint4*>(a.out + (size_t)t * a.ldo + (o0 >> 1));
+    uint4* q = reinterpret_cast<uint4*>(out + (size_t)t * a.ldo + (o0 >> 1));
 #pragma unroll
     for (int c = 0; c < 2; ++c)
-      q[c] = make_uint4(h2pack(y[8 * c], y[8 * c + 1]), h2pack(y[8 * c + 2], y[8 * c + 3]),
-                        h2pack(y[8 * c + 4], y[8 * c + 5]), h2pack(y[8 * c + 6], y[8 * c + 7]));
+      q[c] = make_uint4(h2pack<BF>(y[8 * c], y[8 * c + 1]), h2pack<BF>(y[8 * c + 2], y[8 * c + 3]),
+                        h2pack<BF>(y[8 * c + 4], y[8 * c + 5]), h2pack<BF>(y[8 * c + 6], y[8 * c + 7]));
   } else {
   float y[32];
 #pragma unroll
-  for (int j = 0; j < 32; ++j) y[j] = rh(v[j]);
-  __half* p = a.out + (size_t)t * a.ldo + o0;  // N is a multiple of 32: whole chunks only
+  for (int j = 0; j < 32; ++j) y[j] = rh<BF>(v[j]);
+  elem_t* p = out + (size_t)t * a.ldo + o0;  // N is a multiple of 32: whole chunks only
   if constexpr (EPI == DIT_EPI_TEMB) {
     const uint4* q = reinterpret_cast<const uint4*>(a.vec + o0);
 #pragma unroll
@@ -132,7 +157,7 @@ __device__ __forceinline__ void epilogue_chunk(const DitGemmArgs& a, int t, int 
       const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws[k]));
+        const float2 f = unpack2<BF>(ws[k]);
         y[8 * c + 2 * k] = __fadd_rn(y[8 * c + 2 * k], f.x);
         y[8 * c + 2 * k + 1] = __fadd_rn(y[8 * c + 2 * k + 1], f.y);
       }
@@ -157,7 +182,7 @@ __device__ __forceinline__ void epilogue_chunk(const DitGemmArgs& a, int t, int 
       const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws[k]));
+        const float2 f = unpack2<BF>(ws[k]);
         y[8 * c + 2 * k] = __fadd_rn(f.x, y[8 * c + 2 * k]);
         y[8 * c + 2 * k + 1] = __fadd_rn(f.y, y[8 * c + 2 * k + 1]);
       }
@@ -166,12 +191,12 @@ __device__ __forceinline__ void epilogue_chunk(const DitGemmArgs& a, int t, int 
   uint4* q = reinterpret_cast<uint4*>(p);
 #pragma unroll
   for (int c = 0; c < 4; ++c)
-    q[c] = make_uint4(h2pack(y[8 * c], y[8 * c + 1]), h2pack(y[8 * c + 2], y[8 * c + 3]),
-                      h2pack(y[8 * c + 4], y[8 * c + 5]), h2pack(y[8 * c + 6], y[8 * c + 7]));
+    q[c] = make_uint4(h2pack<BF>(y[8 * c], y[8 * c + 1]), h2pack<BF>(y[8 * c + 2], y[8 * c + 3]),
+                      h2pack<BF>(y[8 * c + 4], y[8 * c + 5]), h2pack<BF>(y[8 * c + 6], y[8 * c + 7]));
   }
 }
 
-template <int EPI>
+template <int EPI, int BF>
 __global__ void __launch_bounds__(kGThreads, 1)
     dit_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const DitGemmArgs a) {
@@ -252,7 +277,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
           const uint32_t sa = smem_u32(smem + (size_t)s * kStageBytes), sb = sa + kABytes;
 #pragma unroll
           for (int ks = 0; ks < kGK / 16; ++ks)
-            tc_mma_f16(d, sw128_desc(sa + ks * 32), sw128_desc(sb + ks * 32),
+            tc_mma_f16<BF>(d, sw128_desc(sa + ks * 32), sw128_desc(sb + ks * 32),
                        (kb > 0 || ks > 0) ? 1u : 0u);
           tc_commit(&empty[s]);
         }
@@ -281,7 +306,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
         if (n0 + c * 32 >= a.N) break;  // the last output block may be narrower (uniform)
         float v[32];
         tmem_ld32(taddr + (uint32_t)(c * 32), v);
-        epilogue_chunk<EPI>(a, t, n0 + c * 32, v);
+        epilogue_chunk<EPI, BF>(a, t, n0 + c * 32, v);
       }
       tc_fence_before();
       __syncwarp();
@@ -325,7 +350,11 @@ constexpr uint32_t kPHalfBytes = 128 * kGK * 2;  // 16 KB: one operand half of a
 constexpr uint32_t kPStageBytes = 2 * kPHalfBytes;
 constexpr size_t kPSmem = (size_t)kPStages * kPStageBytes + 1024 + 256;
 // M = 256 (the pair), N = 256
-constexpr uint32_t kIdesc2 = (1u << 4) | ((uint32_t)(kGN >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+template <int BF>
+constexpr uint32_t idesc_2() {
+  return (1u << 4) | ((uint32_t)BF << 7) | ((uint32_t)BF << 10) | ((uint32_t)(kGN >> 3) << 17) |
+         ((uint32_t)(256 >> 4) << 24);
+}
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -350,6 +379,7 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
                : "memory");
 }
 
+template <int BF>
 __device__ __forceinline__ void tc_mma_f16_pair(uint32_t tmem_d, uint64_t a, uint64_t b,
                                                 uint32_t accumulate) {
   asm volatile(
@@ -357,7 +387,7 @@ __device__ __forceinline__ void tc_mma_f16_pair(uint32_t tmem_d, uint64_t a, uin
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8, %9, %10, %11, %12}, "
       "p;\n\t}" ::"r"(tmem_d),
-      "l"(a), "l"(b), "r"(kIdesc2), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u), "r"(0u),
+      "l"(a), "l"(b), "r"(idesc_2<BF>()), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u), "r"(0u),
       "r"(0u), "r"(0u), "r"(0u)
       : "memory");
 }
@@ -382,7 +412,7 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* t
       : "memory");
 }
 
-template <int EPI>
+template <int EPI, int BF>
 __global__ void __launch_bounds__(kGThreads, 1)
     dit_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmB, const DitGemmArgs a) {
@@ -468,7 +498,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
           const uint32_t sa = smem_u32(smem + (size_t)s * kPStageBytes), sb = sa + kPHalfBytes;
 #pragma unroll
           for (int ks = 0; ks < kGK / 16; ++ks)
-            tc_mma_f16_pair(d, sw128_desc(sa + ks * 32), sw128_desc(sb + ks * 32),
+            tc_mma_f16_pair<BF>(d, sw128_desc(sa + ks * 32), sw128_desc(sb + ks * 32),
                             (kb > 0 || ks > 0) ? 1u : 0u);
           tc_commit_pair(&empty[s]);
         }
@@ -498,7 +528,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
         if (n0 + c * 32 >= a.N) break;  // the last output block may be narrower (uniform)
         float v[32];
         tmem_ld32(taddr + (uint32_t)(c * 32), v);
-        epilogue_chunk<EPI>(a, t, n0 + c * 32, v);
+        epilogue_chunk<EPI, BF>(a, t, n0 + c * 32, v);
       }
       tc_fence_before();
       __syncwarp();
@@ -540,32 +570,33 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// A [rows][ld] fp16 row-major matrix as a tensor map of (box_rows x 64) boxes
-// in the 128-byte swizzle.
-cudaError_t make_map(CUtensorMap* tm, const __half* base, int rows, int cols, int ld,
-                     int box_rows) {
+// A [rows][ld] fp16 or bf16 row-major matrix as a tensor map of
+// (box_rows x 64) boxes in the 128-byte swizzle.
+cudaError_t make_map(CUtensorMap* tm, const void* base, int rows, int cols, int ld,
+                     int box_rows, bool bf16) {
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
   cuuint32_t box[2] = {(cuuint32_t)kGK, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(base), dims,
+  const CUresult r = fn(tm, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                        2, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int EPI>
+template <int EPI, int BF>
 cudaError_t set_attr() {
   const cudaError_t e = cudaFuncSetAttribute(
-      dit_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGSmem);
+      dit_gemm_kernel<EPI, BF>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGSmem);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(dit_gemm_pair_kernel<EPI>,
+  return cudaFuncSetAttribute(dit_gemm_pair_kernel<EPI, BF>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPSmem);
 }
 
-template <int EPI>
+template <int EPI, int BF>
 cudaError_t launch_pair_t(const CUtensorMap& ta, const CUtensorMap& tb, const DitGemmArgs& a,
                           int nsm, cudaStream_t st) {
   const int ntiles = ((a.M + 255) / 256) * ((a.N + kGN - 1) / kGN);
@@ -582,15 +613,15 @@ cudaError_t launch_pair_t(const CUtensorMap& ta, const CUtensorMap& tb, const Di
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, dit_gemm_pair_kernel<EPI>, ta, tb, a);
+  return cudaLaunchKernelEx(&cfg, dit_gemm_pair_kernel<EPI, BF>, ta, tb, a);
 }
 
-template <int EPI>
+template <int EPI, int BF>
 cudaError_t launch_t(const CUtensorMap& ta, const CUtensorMap& tb, const DitGemmArgs& a, int nsm,
                      cudaStream_t st) {
   const int ntiles = ((a.M + kGM - 1) / kGM) * ((a.N + kGN - 1) / kGN);
   const int grid = ntiles < nsm ? ntiles : nsm;
-  dit_gemm_kernel<EPI><<<grid, kGThreads, kGSmem, st>>>(ta, tb, a);
+  dit_gemm_kernel<EPI, BF><<<grid, kGThreads, kGSmem, st>>>(ta, tb, a);
   return cudaGetLastError();
 }
 
@@ -598,16 +629,19 @@ cudaError_t launch_t(const CUtensorMap& ta, const CUtensorMap& tb, const DitGemm
 
 cudaError_t prepare_dit_gemm() {
   if (!encode_fn()) return cudaErrorNotSupported;
-  cudaError_t e = set_attr<DIT_EPI_STORE>();
-  if (e == cudaSuccess) e = set_attr<DIT_EPI_TEMB>();
-  if (e == cudaSuccess) e = set_attr<DIT_EPI_ROPE>();
-  if (e == cudaSuccess) e = set_attr<DIT_EPI_RESID>();
-  if (e == cudaSuccess) e = set_attr<DIT_EPI_GLU>();
+  cudaError_t e = set_attr<DIT_EPI_STORE, 0>();
+  if (e == cudaSuccess) e = set_attr<DIT_EPI_TEMB, 0>();
+  if (e == cudaSuccess) e = set_attr<DIT_EPI_ROPE, 0>();
+  if (e == cudaSuccess) e = set_attr<DIT_EPI_RESID, 0>();
+  if (e == cudaSuccess) e = set_attr<DIT_EPI_GLU, 0>();
+  if (e == cudaSuccess) e = set_attr<DIT_EPI_STORE, 1>();
+  if (e == cudaSuccess) e = set_attr<DIT_EPI_RESID, 1>();
+  if (e == cudaSuccess) e = set_attr<DIT_EPI_GLU, 1>();
   return e;
 }
 
-cudaError_t launch_dit_gemm(const __half* X, int ldx, const __half* W, const DitGemmArgs& a,
-                            int epi, int nsm, cudaStream_t st) {
+cudaError_t launch_dit_gemm(const void* X, int ldx, const void* W, const DitGemmArgs& a,
+                            int epi, int nsm, cudaStream_t st, bool bf16) {
   if (!X || !W || !a.out || a.M < 1 || a.N < 1 || a.K < kGK || a.K % kGK || ldx < a.K ||
       ldx % 8 || (reinterpret_cast<uintptr_t>(X) & 15) || (reinterpret_cast<uintptr_t>(W) & 15) ||
       (reinterpret_cast<uintptr_t>(a.out) & 15) || a.ldo % 8 || nsm < 1)
@@ -617,6 +651,9 @@ cudaError_t launch_dit_gemm(const __half* X, int ldx, const __half* W, const Dit
   if (epi == DIT_EPI_TEMB && (reinterpret_cast<uintptr_t>(a.vec) & 15)) return cudaErrorInvalidValue;
   if (epi == DIT_EPI_TEMB && !a.vec) return cudaErrorInvalidValue;
   if (epi == DIT_EPI_ROPE && (!a.rope || a.rope_T < 1 || a.head_dim % 32 || a.rope_half != 16))
+    return cudaErrorInvalidValue;
+  // bf16 operands: the epilogues of the prompt prefill (store, residual, GLU)
+  if (bf16 && epi != DIT_EPI_STORE && epi != DIT_EPI_RESID && epi != DIT_EPI_GLU)
     return cudaErrorInvalidValue;
   // CTA pairs or single CTAs: a pair tile streams about 12 % faster per SM
   // (32 instead of 48 KB of operands per stage, measured on the chunk's
@@ -628,25 +665,39 @@ cudaError_t launch_dit_gemm(const __half* X, int ldx, const __half* W, const Dit
   const long long rounds2 = nsm >= 2 ? ((a.M + 255) / 256 * n_blk + nsm / 2 - 1) / (nsm / 2) : 0;
   const bool pair = a.M >= 256 && nsm >= 2 && rounds2 * 88 < rounds1 * 100;
   CUtensorMap ta, tb;
-  cudaError_t e = make_map(&ta, X, a.M, a.K, ldx, kGM);
-  if (e == cudaSuccess) e = make_map(&tb, W, a.N, a.K, a.K, pair ? 128 : kGN);
+  cudaError_t e = make_map(&ta, X, a.M, a.K, ldx, kGM, bf16);
+  if (e == cudaSuccess) e = make_map(&tb, W, a.N, a.K, a.K, pair ? 128 : kGN, bf16);
   if (e != cudaSuccess) return e;
+  if (bf16) {
+    if (pair) {
+      switch (epi) {
+        case DIT_EPI_STORE: return launch_pair_t<DIT_EPI_STORE, 1>(ta, tb, a, nsm, st);
+        case DIT_EPI_RESID: return launch_pair_t<DIT_EPI_RESID, 1>(ta, tb, a, nsm, st);
+        default: return launch_pair_t<DIT_EPI_GLU, 1>(ta, tb, a, nsm, st);
+      }
+    }
+    switch (epi) {
+      case DIT_EPI_STORE: return launch_t<DIT_EPI_STORE, 1>(ta, tb, a, nsm, st);
+      case DIT_EPI_RESID: return launch_t<DIT_EPI_RESID, 1>(ta, tb, a, nsm, st);
+      default: return launch_t<DIT_EPI_GLU, 1>(ta, tb, a, nsm, st);
+    }
+  }
   if (pair) {
     switch (epi) {
-      case DIT_EPI_STORE: return launch_pair_t<DIT_EPI_STORE>(ta, tb, a, nsm, st);
-      case DIT_EPI_TEMB: return launch_pair_t<DIT_EPI_TEMB>(ta, tb, a, nsm, st);
-      case DIT_EPI_ROPE: return launch_pair_t<DIT_EPI_ROPE>(ta, tb, a, nsm, st);
-      case DIT_EPI_RESID: return launch_pair_t<DIT_EPI_RESID>(ta, tb, a, nsm, st);
-      case DIT_EPI_GLU: return launch_pair_t<DIT_EPI_GLU>(ta, tb, a, nsm, st);
+      case DIT_EPI_STORE: return launch_pair_t<DIT_EPI_STORE, 0>(ta, tb, a, nsm, st);
+      case DIT_EPI_TEMB: return launch_pair_t<DIT_EPI_TEMB, 0>(ta, tb, a, nsm, st);
+      case DIT_EPI_ROPE: return launch_pair_t<DIT_EPI_ROPE, 0>(ta, tb, a, nsm, st);
+      case DIT_EPI_RESID: return launch_pair_t<DIT_EPI_RESID, 0>(ta, tb, a, nsm, st);
+      case DIT_EPI_GLU: return launch_pair_t<DIT_EPI_GLU, 0>(ta, tb, a, nsm, st);
       default: return cudaErrorInvalidValue;
     }
   }
   switch (epi) {
-    case DIT_EPI_STORE: return launch_t<DIT_EPI_STORE>(ta, tb, a, nsm, st);
-    case DIT_EPI_TEMB: return launch_t<DIT_EPI_TEMB>(ta, tb, a, nsm, st);
-    case DIT_EPI_ROPE: return launch_t<DIT_EPI_ROPE>(ta, tb, a, nsm, st);
-    case DIT_EPI_RESID: return launch_t<DIT_EPI_RESID>(ta, tb, a, nsm, st);
-    case DIT_EPI_GLU: return launch_t<DIT_EPI_GLU>(ta, tb, a, nsm, st);
+    case DIT_EPI_STORE: return launch_t<DIT_EPI_STORE, 0>(ta, tb, a, nsm, st);
+    case DIT_EPI_TEMB: return launch_t<DIT_EPI_TEMB, 0>(ta, tb, a, nsm, st);
+    case DIT_EPI_ROPE: return launch_t<DIT_EPI_ROPE, 0>(ta, tb, a, nsm, st);
+    case DIT_EPI_RESID: return launch_t<DIT_EPI_RESID, 0>(ta, tb, a, nsm, st);
+    case DIT_EPI_GLU: return launch_t<DIT_EPI_GLU, 0>(ta, tb, a, nsm, st);
     default: return cudaErrorInvalidValue;
   }
 }

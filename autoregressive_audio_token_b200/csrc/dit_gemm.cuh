@@ -25,6 +25,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -41,7 +42,7 @@ enum : int {
 
 struct DitGemmArgs {
   int M, N, K;           // tokens, outputs, inputs
-  __half* out;           // [M][ldo]; for the GLU [M][N/2]
+  void* out;             // [M][ldo] of the operand type; for the GLU [M][N/2]
   int ldo;
   const __half* vec;     // DIT_EPI_TEMB: [N]
   const float2* rope;    // DIT_EPI_ROPE: (cos, sin) [rope_T][rope_half]
@@ -56,9 +57,11 @@ struct DitGemmArgs {
 // the kernels' shared-memory limit and the tensor-map encoder.
 cudaError_t prepare_dit_gemm();
 
-// One GEMM on the stream: X [M][ldx] fp16 and W [N][K] fp16 (ldx >= K, both
-// 16-byte aligned, K a multiple of 64, ldx a multiple of 8).
-cudaError_t launch_dit_gemm(const __half* X, int ldx, const __half* W, const DitGemmArgs& a,
-                            int epi, int nsm, cudaStream_t st);
+// One GEMM on the stream: X [M][ldx] and W [N][K], both fp16 or (bf16 =
+// true, the prompt prefill of the decode body: store, residual and GLU
+// epilogues with bf16 roundings) both bf16 (ldx >= K, both 16-byte aligned,
+// K a multiple of 64, ldx a multiple of 8).
+cudaError_t launch_dit_gemm(const void* X, int ldx, const void* W, const DitGemmArgs& a,
+                            int epi, int nsm, cudaStream_t st, bool bf16 = false);
 
 }  // namespace m3

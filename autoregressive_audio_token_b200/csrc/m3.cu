@@ -17,6 +17,7 @@
 #include "launch.cuh"
 #include "misc.cuh"
 #include "gemv_tile.cuh"
+#include "dit_gemm.cuh"
 
 using namespace m3;
 typedef __nv_bfloat16 bf16;
@@ -166,9 +167,17 @@ struct m3_ctx {
   // 1 always, 0 never, -1 for bf16 weights only (int8 streams faster through
   // the decode GEMVs, whose tiles convert in registers without a ring)
   int prefill_tc = -1;
-  int pf_chunk = 256;
+  // 0 until the first GEMM prefill: then 2048 on the TMA-fed GEMM (bf16
+  // weights; a large M keeps its tiles' rounds full and reads the weights
+  // once per 2048 tokens), else 256
+  int pf_chunk = 0;
   bf16 *pf_x = nullptr, *pf_n = nullptr, *pf_qkv = nullptr, *pf_o = nullptr, *pf_act = nullptr;
   float2* pf_rope = nullptr;       // [pf_chunk][head_dim / 2]
+  // the prefill GEMM's operands: a row-major copy of each bf16 layer's
+  // projections (qkv | o | gate/up interleaved | down), made at the first
+  // GEMM prefill from the tiled weights; stale once the layer is reloaded
+  std::vector<bf16*> pf_rm;
+  std::vector<char> pf_rm_ok;
   LoopState* h_loop = nullptr;     // pinned
   int* h_err = nullptr;            // pinned
   std::map<std::pair<int, int>, cudaGraphExec_t> lgraphs;
@@ -581,6 +590,7 @@ extern "C" int m3_load_weights(m3_ctx* c, const m3_weight_src* src, int wdtype) 
     CKR(load_layer(c, c->L[l], src->layers[i], src->mem, wf, g.hidden, g.n_q_heads, g.n_kv_heads,
                    g.head_dim, g.ffn));
     c->loaded[l] = 1;
+    if ((size_t)l < c->pf_rm_ok.size()) c->pf_rm_ok[l] = 0;  // the prefill copy is stale
   }
   if (src->final_norm) CKR(put_vec(c, &c->final_norm, src->final_norm, g.hidden, src->mem));
   if (src->lm_head) {
@@ -1164,11 +1174,70 @@ extern "C" int m3_depth_decode(m3_ctx* c, int rows, const void* h_frame, const i
 // with the tensor-core GEMM: the norms over all T rows, the four projections
 // as GEMMs, and the attention appending every token's K/V, then attending
 // from the cache (causal through the positions).
+// Elements of each projection in a layer's row-major prefill copy, in order.
+static void pf_rm_sizes(const m3_config& g, size_t (&n)[4]) {
+  const size_t H = g.hidden, q = (size_t)(g.n_q_heads + 2 * g.n_kv_heads) * g.head_dim;
+  const size_t hq = (size_t)g.n_q_heads * g.head_dim, F = g.ffn;
+  n[0] = q * H;       // qkv
+  n[1] = H * hq;      // o
+  n[2] = 2 * F * H;   // gate/up, interleaved rows
+  n[3] = H * F;       // down
+}
+
+// The row-major bf16 copies the prefill GEMM reads, for every layer whose
+// copy is missing or stale (untiled on the GPU from the decode layout).
+static int ensure_prefill_copies(m3_ctx* c) {
+  const m3_config& g = c->cfg;
+  if (c->pf_rm.size() != (size_t)g.n_layers) {
+    c->pf_rm.assign(g.n_layers, nullptr);
+    c->pf_rm_ok.assign(g.n_layers, 0);
+  }
+  size_t n[4];
+  pf_rm_sizes(g, n);
+  CK(prepare_dit_gemm());  // the GEMM kernels' shared-memory limit, the tensor-map encoder
+  for (int l = 0; l < g.n_layers; ++l) {
+    if (c->pf_rm_ok[l]) continue;
+    if (!c->pf_rm[l]) CKR(dalloc(c, &c->pf_rm[l], sizeof(bf16) * (n[0] + n[1] + n[2] + n[3])));
+    const DLayer& L = c->L[l];
+    bf16* dst = c->pf_rm[l];
+    const DMat* mats[4] = {&L.qkv, &L.o, &L.gu, &L.d};
+    for (int m = 0; m < 4; ++m) {
+      untile_rows_kernel<<<c->nsm * 8, 256, 0, c->st>>>(static_cast<const uint8_t*>(mats[m]->w),
+                                                          mats[m]->N, mats[m]->K, dst);
+      CK(cudaGetLastError());
+      dst += n[m];
+    }
+    c->pf_rm_ok[l] = 1;
+  }
+  return M3_OK;
+}
+
 static int record_prefill_layer(m3_ctx* c, const DLayer& L, int T, int p0, int layer) {
   const m3_config& g = c->cfg;
   const int H = g.hidden, d = g.head_dim, ldqkv = (g.n_q_heads + 2 * g.n_kv_heads) * d;
   const int hq = g.n_q_heads * d;
+  // bf16 weights with their row-major copy: the TMA-fed tcgen05 GEMM
+  const bf16* rm = (size_t)layer < c->pf_rm_ok.size() && c->pf_rm_ok[layer] ? c->pf_rm[layer]
+                                                                           : nullptr;
+  size_t nrm[4];
+  pf_rm_sizes(g, nrm);
   auto gemm = [&](const DMat& M, int epi, const bf16* x, int ldx, bf16* out, int ldo) -> int {
+    if (rm) {
+      const bf16* w = rm + (&M == &L.qkv ? 0 : &M == &L.o ? nrm[0]
+                                           : &M == &L.gu ? nrm[0] + nrm[1]
+                                                         : nrm[0] + nrm[1] + nrm[2]);
+      DitGemmArgs a{};
+      a.M = T;
+      a.N = M.N;
+      a.K = M.K;
+      a.out = out;
+      a.ldo = ldo;
+      a.err = c->err;
+      const int de = epi == EPI_STORE ? DIT_EPI_STORE : epi == EPI_RESID ? DIT_EPI_RESID
+                                                                         : DIT_EPI_GLU;
+      CK(launch_dit_gemm(x, ldx, w, a, de, c->nsm, c->st, true));
+      return M3_OK;
+    }
     GemmTcArgs a{};
     a.w = static_cast<const uint8_t*>(M.w);
     a.scales = M.s;
@@ -1219,6 +1288,12 @@ static int record_prefill_layer(m3_ctx* c, const DLayer& L, int T, int p0, int l
   return M3_OK;
 }
 
+// Shapes the TMA GEMM takes: every K a multiple of 64, every N of 32.
+static bool prefill_gemm_shapes_ok(const m3_config& g) {
+  const int q = (g.n_q_heads + 2 * g.n_kv_heads) * g.head_dim, hq = g.n_q_heads * g.head_dim;
+  return g.hidden % 64 == 0 && hq % 64 == 0 && g.ffn % 64 == 0 && q % 32 == 0;
+}
+
 static bool prefill_tc_ok(const m3_ctx* c) {
   if (c->prefill_tc == 0) return false;
   const m3_config& g = c->cfg;
@@ -1247,6 +1322,8 @@ extern "C" int m3_prefill(m3_ctx* c, int row, int start, int n_tokens, const voi
     return fail(M3_ECAPACITY, "start + n_tokens outside the KV capacity");
   const int R = g.max_rows;
   const bool tc = prefill_tc_ok(c);
+  if (c->pf_chunk == 0)
+    c->pf_chunk = c->wdtype == M3_W_BF16 && prefill_gemm_shapes_ok(g) ? 2048 : 256;
   const int P = c->pf_chunk;
   const int Rv = tc && P > R ? P : R;  // rows of the page table that map to the sequence
   CKR(enter(c));
@@ -1272,6 +1349,7 @@ extern "C" int m3_prefill(m3_ctx* c, int row, int start, int n_tokens, const voi
       CKR(dalloc(c, &c->pf_act, sizeof(bf16) * P * g.ffn));
       CKR(dalloc(c, &c->pf_rope, sizeof(float2) * P * (d / 2)));
     }
+    if (c->wdtype == M3_W_BF16 && prefill_gemm_shapes_ok(g)) CKR(ensure_prefill_copies(c));
     for (int c0 = 0; c0 < n_tokens; c0 += P) {
       const int T = n_tokens - c0 < P ? n_tokens - c0 : P;
       const int p0 = start + c0;

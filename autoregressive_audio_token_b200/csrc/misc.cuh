@@ -135,6 +135,18 @@ __global__ void tile_rows_kernel(const T* __restrict__ src, int rows, int K, uin
   }
 }
 
+// The inverse of tile_rows_kernel for bf16: a tiled [N][K] matrix back to
+// row-major out[n][k] (rows N..pad of the tiling are not written).
+__global__ void untile_rows_kernel(const uint8_t* __restrict__ src, int N, int K,
+                                   __nv_bfloat16* __restrict__ out) {
+  const int64_t total = (int64_t)N * K;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int n = (int)(i / K), k = (int)(i % K);
+    out[i] = *reinterpret_cast<const __nv_bfloat16*>(src + tile_byte_offset(n, k, K, 2));
+  }
+}
+
 // x_out[r] = table[offset + codes[r]] for r < rows; an out-of-range code
 // records kErrBounds and yields a zero row.
 // A code equal to zero_code (the end token's code, at the depth decoder's

@@ -819,11 +819,11 @@ def run_depth_only(args):
 
 def run_prefill(args):
     """Prompt prefill of P tokens (a prompt's worth, N(0, 0.02^2) embeddings)
-    into one cache row of the full 8B: chunks of M3_PREFILL_CHUNK tokens (256)
-    through the tcgen05 GEMMs (the default for bf16 weights, M3_PREFILL_TC=1
-    for int8), or chunks of 16 through the decode GEMVs (the default for int8,
-    M3_PREFILL_TC=0 for bf16); timed with CUDA events over 3 runs after one
-    untimed run."""
+    into one cache row of the full 8B: chunks of M3_PREFILL_CHUNK tokens
+    (2048 for bf16, 256 for int8) through the tcgen05 GEMMs (the default for
+    bf16 weights, M3_PREFILL_TC=1 for int8), or chunks of 16 through the
+    decode GEMVs (the default for int8, M3_PREFILL_TC=0 for bf16); timed with
+    CUDA events over 3 runs after one untimed run."""
     import torch
     from autoregressive_audio_token_b200 import m3
     import synth
@@ -845,7 +845,8 @@ def run_prefill(args):
     m3.m3_sync_status(ctx)
     ms = e0.elapsed_time(e1) / 3
     tc = os.environ.get("M3_PREFILL_TC", "1" if args.wdtype == "bf16" else "0") == "1"
-    chunk = int(os.environ.get("M3_PREFILL_CHUNK", "256")) if tc else 16
+    chunk = (int(os.environ.get("M3_PREFILL_CHUNK", "2048" if args.wdtype == "bf16" else "256"))
+             if tc else 16)
     path = "tcgen05 GEMM" if tc else "decode GEMV"
     layer_w = m3.m3_frame_bytes(ctx, 0, -1)  # weights only (no KV)
     flops = 2.0 * P * (layer_w / (1 if wdtype == m3.M3_W_INT8 else 2))

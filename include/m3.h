@@ -179,16 +179,22 @@ M3_API int m3_kv_get(m3_ctx* ctx, int row, int n_positions, void* k_host, void* 
  * x (dev bf16 [n_tokens, H]) runs through every layer at position start + t,
  * attending to positions 0..start + t of the row (causal), and its K/V land
  * in the row's cache -- the same result as decoding the tokens one by one.
- * With bf16 weights the tokens go in chunks of 256 (environment
+ * With bf16 weights the tokens go in chunks of 2048 (environment
  * M3_PREFILL_CHUNK, 16..4096), each chunk one pass of the layers whose
- * projections are tcgen05 GEMMs over the chunk's tokens; with int8 weights
- * (or M3_PREFILL_TC=0) in chunks of up to max_rows as the batch rows of the
- * decode projections.  M3_PREFILL_TC=1 takes the GEMMs for int8 too.
+ * projections are tcgen05 GEMMs over the chunk's tokens, both operands
+ * brought in by TMA tensor maps: the weights from a row-major bf16 copy of
+ * every layer's projections (about 0.39 GB per 8B layer, 14 GB for 36),
+ * made on the device at the first prefill and again for a layer that
+ * m3_load_weights has replaced since.  With int8 weights (or
+ * M3_PREFILL_TC=0) the tokens go in chunks of up to max_rows as the batch
+ * rows of the decode projections; M3_PREFILL_TC=1 takes a GEMM over the
+ * tiled int8 weights (chunks of 256) instead.
  *  h_last (dev bf16 [H], nullable): the final-normed hidden state of the last
  *    token.
  * start + n_tokens must be <= max_positions (M3_ECAPACITY).  May allocate KV
- * buckets and, at the first GEMM prefill, chunk-sized activation buffers;
- * synchronises the stream once. */
+ * buckets and, at the first GEMM prefill, the weight copies and chunk-sized
+ * activation buffers (M3_ENOMEM when they do not fit); synchronises the
+ * stream once. */
 M3_API int m3_prefill(m3_ctx* ctx, int row, int start, int n_tokens, const void* x, void* h_last);
 
 /* The end token.  With cfg.has_end_token the draw of m3_decode_frame chooses

@@ -331,7 +331,7 @@ def test_layer8b_vs_oracle(ora, wdtype, rows, kv_f16, ring, monkeypatch):
         m.close()
 
 
-@pytest.mark.parametrize("rows,wdtype", [(8, 0), (16, 0), (8, 1)])
+@pytest.mark.parametrize("rows,wdtype", [(8, 0), (16, 0), (8, 1), (12, 0), (16, 1)])
 def test_layer8b_many_rows(ora, rows, wdtype):
     # the 8B layer at 8 and 16 rows: the down projection's activations
     # (K = 12288) leave no room for the default ring, so the launch plans

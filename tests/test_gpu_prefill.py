@@ -4,10 +4,12 @@ Prefilling tokens at positions start .. start + n - 1 is defined as decoding
 them one by one (each token attends to every earlier position of its row and
 to itself); the oracle runs exactly that, token by token, through its
 single-row layers.  With M3_PREFILL_TC=1 (the default for bf16 weights) the
-GPU runs the prompt in chunks (256 tokens by default) whose projections are
-tcgen05 GEMMs, with a causal attention over the row's cache; M3_PREFILL_TC=0
-(the default for int8) selects the decode GEMV kernels over chunks of up to
-max_rows tokens.  Compared:
+GPU runs the prompt in chunks (2048 tokens by default for bf16 weights, 256
+for int8) whose projections are tcgen05 GEMMs -- for bf16 the TMA-fed kernel
+over a row-major copy of the weights, single CTAs or CTA pairs by shape --
+with a causal attention over the row's cache; M3_PREFILL_TC=0 (the default
+for int8) selects the decode GEMV kernels over chunks of up to max_rows
+tokens.  Compared:
   * the K/V the prefill leaves in the row's cache (every layer, position);
   * the final-normed hidden state of the last token;
   * the other rows' caches, untouched;
@@ -39,6 +41,7 @@ def _cuda():
     (3, 37, 16, 0, "1", 256), (0, 1, 2, 0, "1", 256), (5, 20, 8, 1, "1", 256),
     (2, 70, 4, 0, "1", 32),     # three chunks, the last one ragged
     (0, 200, 16, 0, "1", 256),  # two token tiles of the GEMM, the second ragged
+    (0, 600, 16, 0, "1", 2048),  # one chunk on CTA pairs: 256-token tiles, the last ragged
     (1, 150, 4, 1, "1", 64),    # int8, chunks of 64
     (3, 37, 16, 0, "0", 256), (5, 20, 8, 1, "0", 256)])  # the GEMV prefill
 def test_prefill_matches_sequential_decode(ora, start, n, max_rows, wdtype, tc, chunk,
@@ -132,5 +135,33 @@ def test_prefill_argument_errors(ora):
             m3.m3_prefill(m.ctx, 1, 0, x)  # row 1 of a one-row cache
         assert e.value.code == m3.M3_EINVAL
         m3.m3_sync_status(m.ctx)
+    finally:
+        m.close()
+
+
+def test_prefill_after_reloading_a_layer(ora):
+    # the GEMM prefill reads a row-major copy of the bf16 weights made at the
+    # first prefill; reloading a layer must retire that layer's copy
+    s = TWO_LAYERS
+    m = Model(s, seed=31, max_rows=2)
+    try:
+        m.m3.m3_kv_alloc(m.ctx, 1, 64, 0, 32)
+        xs = synth.normal((24, s.hidden), 31, "prompt", std=0.02)
+        h1 = torch.empty(s.hidden, dtype=torch.bfloat16, device="cuda")
+        m.m3.m3_prefill(m.ctx, 0, 0, xs.cuda(), h1)
+        new = synth.layer_weights(s, 32, 1)
+        m.m3.m3_load_weights(m.ctx, [{k: v.cuda() for k, v in new.items()}], first_layer=1)
+        h2 = torch.empty_like(h1)
+        m.m3.m3_prefill(m.ctx, 0, 0, xs.cuda(), h2)
+        torch.cuda.synchronize()
+        m.m3.m3_sync_status(m.ctx)
+        body = ora.Body(s, [m.layers[0], new], m.final_norm, m.lm)
+        kc, vc = body.new_cache(1, 64)
+        xb = bits(xs)
+        for t in range(24):
+            x_out = body.body(kc, vc, [t], xb[t:t + 1].copy())
+        href = ora.rmsnorm(f32(x_out[0]), bits(m.final_norm), s.rms_eps)
+        assert rel_err(f32(bits(h2)), href) <= 2e-2
+        assert not np.array_equal(bits(h1), bits(h2))
     finally:
         m.close()
