@@ -1554,6 +1554,18 @@ extern "C" int m3_embed(m3_ctx* c, int rows, const int32_t* codes, const void* t
   return leave(c);
 }
 
+extern "C" int m3_frame_kernels(const m3_ctx* c, int rows) {
+  if (!c || rows < 1 || rows > c->cfg.max_rows) return fail(M3_EINVAL, "rows");
+  if (c->L.empty() || !c->loaded[0]) return fail(M3_ESTATE, "weights not loaded");
+  int n = 2 + 1;  // parameter block, RoPE table; the sampler
+  for (int l = 0; l < c->cfg.n_layers; ++l) {
+    n += 1;  // attention
+    for (const DMat* M : {&c->L[l].qkv, &c->L[l].o, &c->L[l].gu, &c->L[l].d})
+      n += M->tiled ? 1 : (rows + 3) / 4;
+  }
+  return n;
+}
+
 extern "C" double m3_frame_bytes(const m3_ctx* c, int rows, int ctx_len) {
   if (!c) return 0.0;
   const m3_config& g = c->cfg;

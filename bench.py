@@ -387,11 +387,12 @@ def run_ours(args, rank, world, local):
         "clocks": clk,
     }
     # per frame: parameter block + RoPE table + 5 kernels per layer (qkv,
-    # attention, o, gate/up, down) + lm_head sampler; the depth decoder adds
+    # attention, o, gate/up, down) + lm_head sampler, as the library counts
+    # them; the depth decoder adds
     # its parameter block, projection, 7 embeddings, 8 positions x layers x 5
     # kernels and 7 heads
     depth_launches = (2 + 7 + 8 * synth.DEPTH.n_layers * 5 + 7) if args.depth else 0
-    out["gpu_launches"] = (5 * s.n_layers + 1 + 2 + depth_launches) * args.steps
+    out["gpu_launches"] = (m3.m3_frame_kernels(ctx, rows) + depth_launches) * args.steps
     m3.m3_destroy(ctx)
     del xs
     torch.cuda.empty_cache()

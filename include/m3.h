@@ -312,6 +312,13 @@ M3_API int m3_quantize_int8(const void* w, int64_t rows, int64_t cols, int64_t g
  * q_host gets the bf16 bits and s_host is ignored. */
 M3_API int m3_export_weight(m3_ctx* ctx, int which, int layer, void* q_host, float* s_host);
 
+/* Kernels one m3_decode_frame of `rows` rows launches, for launch
+ * accounting: the parameter block, the RoPE table, QKV, attention, O,
+ * gate/up and down per layer (the int8 group-128 projections in launches of
+ * 4 rows) and the sampler.  A negative m3_status on bad arguments or before
+ * the weights are loaded. */
+M3_API int m3_frame_kernels(const m3_ctx* ctx, int rows);
+
 /* Algorithmic HBM bytes of one frame: weights read once per frame plus the
  * KV cache read for `rows` rows at context length ctx (positions 0..ctx). */
 M3_API double m3_frame_bytes(const m3_ctx* ctx, int rows, int ctx_len);
