@@ -284,6 +284,11 @@ def test_errors_are_status_codes(ora):
         # the context is still usable
         m3.m3_decode_frame(m.ctx, [0], 1, 0, x, 0.0, 1.0, codes)
         m3.m3_sync_status(m.ctx)
+        # launch accounting: parameter block, RoPE table, 5 per layer, sampler
+        assert m3.m3_frame_kernels(m.ctx, 1) == 2 + 5 * s.n_layers + 1
+        with pytest.raises(m3.M3Error) as e:
+            m3.m3_frame_kernels(m.ctx, 0)
+        assert e.value.code == m3.M3_EINVAL
     finally:
         m.close()
 
@@ -382,6 +387,31 @@ def test_layer8b_16rows_long_context(ora, n_ctx):
 
 
 # -------------------------------------------------------- depth decoder ----
+
+def test_depth_decoder_full_size(ora):
+    # the 8B model's depth decoder (16 heads of 64, hidden 1024, 4 layers,
+    # SwiGLU 2816, 7 codebooks of 1024, input 4096), one cluster of 16 CTAs,
+    # a CFG pair: logits against the oracle, every draw by the draw rule
+    s, D, rows, cfg = synth.LAYER8B, synth.DEPTH, 2, 1.5
+    m = Model(s, seed=9, depth=D, max_rows=2)
+    try:
+        h = synth.normal((rows, s.hidden), 9, "hframe", std=1.0).cuda()
+        code0 = torch.tensor([11, 16383], dtype=torch.int32, device="cuda")
+        codes = torch.empty((rows, D.codebooks), dtype=torch.int32, device="cuda")
+        lg = torch.empty((rows, D.codebooks, D.vocab), dtype=torch.float32, device="cuda")
+        m.m3.m3_depth_decode(m.ctx, h, code0, 5, 2, cfg, 1.0, codes, logits=lg)
+        torch.cuda.synchronize()
+        m.m3.m3_sync_status(m.ctx)
+        gc = codes.cpu().numpy()
+        oc, olg = m.ora_depth.decode(bits(h), code0.cpu().numpy(), 5, 2, cfg_scale=cfg,
+                                     forced=gc)
+        glg = lg.cpu().numpy()
+        for j in range(D.codebooks):
+            assert rel_err(glg[:, j], olg[:, j]) <= TOL[1], (j, rel_err(glg[:, j], olg[:, j]))
+        check_depth_draws(glg, gc, 5, 2, cfg_scale=cfg)
+    finally:
+        m.close()
+
 
 @pytest.mark.parametrize("rows,cfg", [(1, 0.0), (2, 1.5), (4, 1.5)])
 def test_depth_decoder_teacher_forced(ora, rows, cfg):
