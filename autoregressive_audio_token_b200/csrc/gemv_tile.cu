@@ -146,45 +146,64 @@ cudaError_t plan_gemv_tile(int N, int K, int mr, int wf, int epi, int nsm, int s
       return cudaSuccess;
     }
   }
-  double best_cost = 0.0;
-  bool found = false;
-  // M3_GEMV_CLUSTER: only this cluster size (tuning)
-  int force_c = 0;
-  if (const char* e = getenv("M3_GEMV_CLUSTER")) force_c = atoi(e);
-  for (int C = 1; C <= 8; C *= 2) {
-    if (T % C || C > nsm) continue;
-    if (force_c > 0 && C != force_c) continue;
-    int ncl = nsm / C;
-    if (ncl > U) ncl = U;
-    TilePlan p = tile_plan(N, K, esz, C, ncl, sb, sb * ns);
-    if (p.slots < 2) continue;
-    size_t smem = tile_smem_bytes(p, mr);
-    if (smem > 227 * 1024) continue;
-    int cap = 0;
-    cudaError_t e = max_clusters(wf, epi, C, smem, &cap);
-    if (e != cudaSuccess) return e;
-    if (cap < 1) continue;
-    if (ncl > cap) {
-      ncl = cap;
-      p = tile_plan(N, K, esz, C, ncl, sb, sb * ns);
-      smem = tile_smem_bytes(p, mr);
+  // the static partition: the cluster size (K split) whose busiest CTA
+  // streams the fewest tiles, for stage bytes sbt
+  auto search = [&](int sbt, TileLaunch* best, double* best_cost) -> cudaError_t {
+    bool found = false;
+    // M3_GEMV_CLUSTER: only this cluster size (tuning)
+    int force_c = 0;
+    if (const char* e = getenv("M3_GEMV_CLUSTER")) force_c = atoi(e);
+    for (int C = 1; C <= 8; C *= 2) {
+      if (T % C || C > nsm) continue;
+      if (force_c > 0 && C != force_c) continue;
+      int ncl = nsm / C;
+      if (ncl > U) ncl = U;
+      TilePlan p = tile_plan(N, K, esz, C, ncl, sbt, sbt * ns);
+      if (p.slots < 2) continue;
+      size_t smem = tile_smem_bytes(p, mr);
+      if (smem > 227 * 1024) continue;
+      int cap = 0;
+      cudaError_t e = max_clusters(wf, epi, C, smem, &cap);
+      if (e != cudaSuccess) return e;
+      if (cap < 1) continue;
+      if (ncl > cap) {
+        ncl = cap;
+        p = tile_plan(N, K, esz, C, ncl, sbt, sbt * ns);
+        smem = tile_smem_bytes(p, mr);
+      }
+      // time ~ the busiest CTA's tiles; a cluster reduction and a footprint
+      // that rules out co-residency cost a little extra
+      double cost = (double)p.nu_max * p.Tr * (1.0 + (C > 1 ? 0.01 : 0.0));
+      if (smem > kTCoresidentSmem) cost *= 1.05;
+      if (!found || cost < *best_cost) {
+        found = true;
+        *best_cost = cost;
+        best->C = C;
+        best->grid = ncl * C;
+        best->sb = sbt;
+        best->ns = ns;
+        best->smem = smem;
+        best->dyn = false;
+      }
     }
-    // time ~ the busiest CTA's tiles; a cluster reduction and a footprint
-    // that rules out co-residency cost a little extra
-    double cost = (double)p.nu_max * p.Tr * (1.0 + (C > 1 ? 0.01 : 0.0));
-    if (smem > kTCoresidentSmem) cost *= 1.05;
-    if (!found || cost < best_cost) {
-      found = true;
-      best_cost = cost;
-      out->C = C;
-      out->grid = ncl * C;
-      out->sb = sb;
-      out->ns = ns;
-      out->smem = smem;
-      out->dyn = false;
-    }
+    return found ? cudaSuccess : cudaErrorInvalidConfiguration;
+  };
+  double cost = 0.0;
+  cudaError_t e = search(sb, out, &cost);
+  if (e != cudaSuccess && e != cudaErrorInvalidConfiguration) return e;
+  // more than 8 rows: their activations crowd the shared memory, and half
+  // stages can admit a smaller cluster that runs on more SMs (16 rows of
+  // gate/up: 74 clusters of 2 instead of 33 of 4); taken when the busiest
+  // CTA's share drops by more than 5 % (where the full stages fit no ring at
+  // all, the caller's next try is fewer full stages, measured better)
+  if (e == cudaSuccess && mr > 8 && sb / 2 >= 4096 && (sb / 2) % (256 * esz) == 0) {
+    TileLaunch h;
+    double hc = 0.0;
+    const cudaError_t eh = search(sb / 2, &h, &hc);
+    if (eh != cudaSuccess && eh != cudaErrorInvalidConfiguration) return eh;
+    if (eh == cudaSuccess && hc < 0.95 * cost) *out = h;
   }
-  return found ? cudaSuccess : cudaErrorInvalidConfiguration;
+  return e;
 }
 
 cudaError_t launch_gemv_tile(const GemvArgs& a, int wf, int epi, const TileLaunch& L,

@@ -66,6 +66,10 @@ cudaError_t launch_gemv_tile(const GemvArgs& a, int wf, int epi, const TileLaunc
 int attn_ctas_per_sm(int D, int kv_f16);
 cudaError_t launch_attn(const AttnArgs& a, int D, int kv_f16, int splits, int rows,
                         cudaStream_t st, bool pdl);
+// The causal attention of a prompt chunk of T tokens at positions
+// a.fixed_pos .. + T - 1 (attn_prefill.cuh): their K/V appended to the row's
+// cache, then the tiled attention.
+cudaError_t launch_attn_prefill(const AttnArgs& a, int D, int kv_f16, int T, cudaStream_t st);
 
 // The prefill's tensor-core GEMM (gemm_tc.cu, tcgen05 with tensor-memory
 // accumulators): Y[t][o] = sum_k W[o][k] X[t][k] for T tokens, W in the tiled

@@ -1276,10 +1276,17 @@ static int record_prefill_layer(m3_ctx* c, const DLayer& L, int T, int p0, int l
   at.fixed_pos = p0;
   at.pos_stride = 1;
   at.err = c->err;
-  at.mode = 1;
-  CK(launch_attn(at, d, c->kv_f16, 1, T, c->st, false));
-  at.mode = 2;
-  CK(launch_attn(at, d, c->kv_f16, attn_splits(c, T, c->n_buckets), T, c->st, false));
+  const int grp = g.n_q_heads / g.n_kv_heads;
+  if ((d == 64 || d == 128) && 16 % grp == 0 && c->bucket % 32 == 0) {
+    // the chunk's K/V appended, then the tiled causal attention in which the
+    // chunk's tokens share every K/V tile
+    CK(launch_attn_prefill(at, d, c->kv_f16, T, c->st));
+  } else {
+    at.mode = 1;
+    CK(launch_attn(at, d, c->kv_f16, 1, T, c->st, false));
+    at.mode = 2;
+    CK(launch_attn(at, d, c->kv_f16, attn_splits(c, T, c->n_buckets), T, c->st, false));
+  }
   CKR(gemm(L.o, EPI_RESID, c->pf_o, hq, c->pf_x, H));
   rmsnorm_rows_kernel<<<T, 256, 0, c->st>>>(c->pf_x, L.mlp_norm, g.rms_eps, H, c->pf_n);
   CK(cudaGetLastError());

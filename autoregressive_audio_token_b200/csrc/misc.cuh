@@ -218,16 +218,36 @@ __global__ void kv_get_kernel(uint16_t* k, uint16_t* v, const unsigned long long
 }
 
 // One RMSNorm row per CTA (any blockDim multiple of 32, up to 1024):
-// out = bf16(gamma * bf16(x / rms)), the sum of squares in fp32.
+// out = bf16(gamma * bf16(x / rms)), the sum of squares in fp32.  Rows of a
+// multiple of 8 elements (16-byte aligned) go 16 bytes at a time (a thread's
+// 8 consecutive elements, then the threads, then the warps, in that order).
 __global__ void rmsnorm_rows_kernel(const __nv_bfloat16* __restrict__ x,
                                     const __nv_bfloat16* __restrict__ gamma, float eps, int n,
                                     __nv_bfloat16* out) {
   __shared__ float red[32];
   const __nv_bfloat16* xr = x + (size_t)blockIdx.x * n;
+  __nv_bfloat16* orow = out + (size_t)blockIdx.x * n;
+  const bool vec = n % 8 == 0 &&
+                   ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(gamma) |
+                     reinterpret_cast<uintptr_t>(out)) & 15) == 0;
   float s = 0.0f;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    const float f = __bfloat162float(xr[i]);
-    s = fmaf(f, f, s);
+  if (vec) {
+    for (int c = threadIdx.x; c < n / 8; c += blockDim.x) {
+      const uint4 w = *reinterpret_cast<const uint4*>(xr + 8 * c);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float lo, hi;
+        bf16x2_to_f32(ws[k], lo, hi);
+        s = fmaf(lo, lo, s);
+        s = fmaf(hi, hi, s);
+      }
+    }
+  } else {
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const float f = __bfloat162float(xr[i]);
+      s = fmaf(f, f, s);
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
@@ -236,9 +256,26 @@ __global__ void rmsnorm_rows_kernel(const __nv_bfloat16* __restrict__ x,
   float t = 0.0f;
   for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w];
   const float r = 1.0f / sqrtf(t / (float)n + eps);
-  for (int i = threadIdx.x; i < n; i += blockDim.x)
-    out[(size_t)blockIdx.x * n + i] =
-        __float2bfloat16_rn(__bfloat162float(gamma[i]) * round_bf16(__bfloat162float(xr[i]) * r));
+  if (vec) {
+    for (int c = threadIdx.x; c < n / 8; c += blockDim.x) {
+      const uint4 w = *reinterpret_cast<const uint4*>(xr + 8 * c);
+      const uint4 gv = *reinterpret_cast<const uint4*>(gamma + 8 * c);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w}, gs[4] = {gv.x, gv.y, gv.z, gv.w};
+      uint32_t os[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float lo, hi, glo, ghi;
+        bf16x2_to_f32(ws[k], lo, hi);
+        bf16x2_to_f32(gs[k], glo, ghi);
+        const __nv_bfloat162 o2 = __floats2bfloat162_rn(glo * round_bf16(lo * r), ghi * round_bf16(hi * r));
+        os[k] = *reinterpret_cast<const uint32_t*>(&o2);
+      }
+      *reinterpret_cast<uint4*>(orow + 8 * c) = make_uint4(os[0], os[1], os[2], os[3]);
+    }
+  } else {
+    for (int i = threadIdx.x; i < n; i += blockDim.x)
+      orow[i] = __float2bfloat16_rn(__bfloat162float(gamma[i]) * round_bf16(__bfloat162float(xr[i]) * r));
+  }
 }
 
 // ------------------------------------------------------ generation loop --
