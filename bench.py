@@ -310,6 +310,8 @@ def run_ours(args, rank, world, local):
     # ---- end to end through the C ABI with host buffers ---------------------
     x_host = xs[:64].cpu().pin_memory()
     codes_host = torch.empty((args.steps, rows), dtype=torch.int32).pin_memory()
+    nc = synth.DEPTH.codebooks if args.depth else 0
+    dcodes_host = torch.empty((args.steps, rows, max(nc, 1)), dtype=torch.int32).pin_memory()
     x_dev = torch.empty((rows, s.hidden), dtype=torch.bfloat16, device="cuda")
     barrier(world)
     torch.cuda.synchronize()
@@ -317,7 +319,12 @@ def run_ours(args, rank, world, local):
     e2.record(stream)
     for i, p in enumerate(positions):
         x_dev.copy_(x_host[i % 64], non_blocking=True)
-        m3.m3_decode_frame(ctx, [p] * rows, seed, i, x_dev, cfg, 1.0, codes)
+        if args.depth:  # the frame and its residual codes, both read back
+            m3.m3_decode_frame(ctx, [p] * rows, seed, i, x_dev, cfg, 1.0, codes, h_dev)
+            m3.m3_depth_decode(ctx, h_dev, codes, seed, i, cfg, 1.0, dcodes)
+            dcodes_host[i].copy_(dcodes, non_blocking=True)
+        else:
+            m3.m3_decode_frame(ctx, [p] * rows, seed, i, x_dev, cfg, 1.0, codes)
         codes_host[i].copy_(codes, non_blocking=True)
     e3.record(stream)
     torch.cuda.synchronize()
@@ -383,7 +390,7 @@ def run_ours(args, rank, world, local):
         "kernels": kernels,
         "e2e": {"value": 1000.0 / e2e_ms * world, "unit": "frames/s",
                 "h2d_bytes_per_step": rows * s.hidden * 2 + 4 * rows,
-                "d2h_bytes_per_step": 4 * rows},
+                "d2h_bytes_per_step": 4 * rows * (1 + nc)},
         "clocks": clk,
     }
     # per frame: parameter block + RoPE table + 5 kernels per layer (qkv,
