@@ -55,10 +55,10 @@ int attn_ctas_per_sm(int D, int kv_f16) {
   return 0;
 }
 
-template <int D, int KVF16, int KT>
+template <int D, int KVF16>
 static cudaError_t launch_attn_prefill_t(const AttnArgs& a, int T, cudaStream_t st) {
-  constexpr size_t smem = attn_prefill_smem<D, KT>();
-  auto kern = attn_prefill_kernel<D, KVF16, KT>;
+  constexpr size_t smem = attn_prefill_smem<D>();
+  auto kern = attn_prefill_kernel<D, KVF16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int tpw = 16 / (a.Hq / a.Hkv);
@@ -69,9 +69,8 @@ static cudaError_t launch_attn_prefill_t(const AttnArgs& a, int T, cudaStream_t 
 
 cudaError_t launch_attn_prefill(const AttnArgs& a, int D, int kv_f16, int T, cudaStream_t st) {
   if (T < 1 || a.Hkv < 1 || a.Hq % a.Hkv || 16 % (a.Hq / a.Hkv) || a.fixed_pos < 0 ||
-      a.page_size % 32)
+      a.page_size % kApKT)
     return cudaErrorInvalidValue;
-  const bool kt64 = a.page_size % 64 == 0;
   {  // the chunk's K/V first
     const dim3 grid((unsigned)((T * a.Hkv + 7) / 8));
     if (D == 128) {
@@ -84,18 +83,10 @@ cudaError_t launch_attn_prefill(const AttnArgs& a, int D, int kv_f16, int T, cud
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  if (D == 128) {
-    if (kt64) return kv_f16 ? launch_attn_prefill_t<128, 1, 64>(a, T, st)
-                            : launch_attn_prefill_t<128, 0, 64>(a, T, st);
-    return kv_f16 ? launch_attn_prefill_t<128, 1, 32>(a, T, st)
-                  : launch_attn_prefill_t<128, 0, 32>(a, T, st);
-  }
-  if (D == 64) {
-    if (kt64) return kv_f16 ? launch_attn_prefill_t<64, 1, 64>(a, T, st)
-                            : launch_attn_prefill_t<64, 0, 64>(a, T, st);
-    return kv_f16 ? launch_attn_prefill_t<64, 1, 32>(a, T, st)
-                  : launch_attn_prefill_t<64, 0, 32>(a, T, st);
-  }
+  if (D == 128) return kv_f16 ? launch_attn_prefill_t<128, 1>(a, T, st)
+                              : launch_attn_prefill_t<128, 0>(a, T, st);
+  if (D == 64) return kv_f16 ? launch_attn_prefill_t<64, 1>(a, T, st)
+                             : launch_attn_prefill_t<64, 0>(a, T, st);
   return cudaErrorInvalidValue;
 }
 

@@ -12,7 +12,7 @@
 //     16 / group tokens; it normalises and rotates its q rows itself (per-head
 //     RMSNorm with its gain, half-rotation RoPE at the token's position, bf16
 //     like the decode path) into shared memory, then A fragments;
-//   * K/V tiles of 32 or 64 positions come by bulk copies (the cache's chunk
+//   * K/V tiles of 32 positions come by bulk copies (the cache's chunk
 //     swizzle lands them conflict-free for ldmatrix) into a 3-deep ring,
 //     up to the CTA's last position; S = Q K^T (m16n8k16, fp32), the causal
 //     mask per row, online softmax in fp32, O += P V with P in two 16-bit
@@ -26,24 +26,22 @@
 namespace m3 {
 
 constexpr int kApWarps = 4;
+constexpr int kApKT = 32;    // positions per K/V tile
 constexpr int kApBuf = 3;    // K/V tiles in flight
 
-// KT: positions per K/V tile (32, or 64 where pages hold a multiple of 64)
-template <int D, int KT>
+template <int D>
 __host__ __device__ constexpr size_t attn_prefill_smem() {
-  return (size_t)kApWarps * 16 * D * 2       // q rows
-         + (size_t)kApBuf * 2 * KT * D * 2  // K, V tiles
+  return (size_t)kApWarps * 16 * D * 2          // q rows
+         + (size_t)kApBuf * 2 * kApKT * D * 2  // K, V tiles
          + kApBuf * sizeof(uint64_t);
 }
 
 // Query rows a CTA covers: 16 per warp.
 __host__ __device__ constexpr int attn_prefill_rows() { return kApWarps * 16; }
 
-template <int D, int KVF16, int KT>
+template <int D, int KVF16>
 __global__ void __launch_bounds__(kApWarps * 32)
     attn_prefill_kernel(const AttnArgs a, int T) {
-  constexpr int kApKT = KT;
-  constexpr int NJ = KT / 8;         // n-tiles of S
   constexpr int ROWB = D * 2;        // bytes per position (or q) row
   constexpr int KS = D / 16;         // k-steps of Q K^T
   constexpr int NTO = D / 8;         // n-tiles of O
@@ -163,10 +161,10 @@ __global__ void __launch_bounds__(kApWarps * 32)
     }
     if (js <= warp_last) {
       const uint32_t kb = smem_u32(kt + b * TILE_ELEMS), vb = smem_u32(vt + b * TILE_ELEMS);
-      // S = Q K^T: NJ n-tiles of 8 positions
-      float s[NJ][4];
+      // S = Q K^T: 4 n-tiles of 8 positions
+      float s[4][4];
 #pragma unroll
-      for (int j = 0; j < NJ; ++j) {
+      for (int j = 0; j < 4; ++j) {
         s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.0f;
         const int prow = 8 * j + (lane & 7);
 #pragma unroll
@@ -181,7 +179,7 @@ __global__ void __launch_bounds__(kApWarps * 32)
       // causal mask per row (positions past the row's own, or past the tile)
       float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-      for (int j = 0; j < NJ; ++j)
+      for (int j = 0; j < 4; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int p = js + 8 * j + 2 * tig + (e & 1);
@@ -200,7 +198,7 @@ __global__ void __launch_bounds__(kApWarps * 32)
       }
       float ls[2] = {0.0f, 0.0f};
 #pragma unroll
-      for (int j = 0; j < NJ; ++j)
+      for (int j = 0; j < 4; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float mm = m_run[e >> 1];
@@ -221,9 +219,9 @@ __global__ void __launch_bounds__(kApWarps * 32)
         o[j][2] *= corr[1];
         o[j][3] *= corr[1];
       }
-      // O += P V over k-steps of 16 positions, P = P_hi + P_lo
+      // O += P V over two k-steps of 16 positions, P = P_hi + P_lo
 #pragma unroll
-      for (int kk = 0; kk < KT / 16; ++kk) {
+      for (int kk = 0; kk < 2; ++kk) {
         const uint32_t h0 = pack2<KVF16>(s[2 * kk][0], s[2 * kk][1]);
         const uint32_t h1 = pack2<KVF16>(s[2 * kk][2], s[2 * kk][3]);
         const uint32_t h2 = pack2<KVF16>(s[2 * kk + 1][0], s[2 * kk + 1][1]);
