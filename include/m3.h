@@ -145,11 +145,15 @@ typedef struct {
 
 /* Create a context bound to the current CUDA device and `cuda_stream`
  * (cudaStream_t, may be 0 for the legacy default stream).  Allocates only
- * the small per-frame activation buffers (sized by cfg->max_rows). */
+ * the small per-frame activation buffers (sized by cfg->max_rows: the 2K
+ * rows of K lockstep variations, "MiniMax Music 3 modular pipeline",
+ * finding 4; the model shape of "MiniMax-Music3 ... DiffSynth-Studio",
+ * "各子模型的结构要点"). */
 M3_API int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out);
 
-/* Copy (and, for M3_W_INT8, quantise on the GPU) body weights into
- * library-owned device memory.  The first call fixes wdtype; the source
+/* Copy (and, for M3_W_INT8, quantise on the GPU: one fp32 scale per row,
+ * "MiniMax Music 3 on Metal", "Precision is the reference's") body weights
+ * into library-owned device memory.  The first call fixes wdtype; the source
  * may be freed once the call returns (host sources are copied
  * synchronously; device sources in stream order before the call returns). */
 M3_API int m3_load_weights(m3_ctx* ctx, const m3_weight_src* src, int wdtype);
@@ -157,8 +161,11 @@ M3_API int m3_load_weights(m3_ctx* ctx, const m3_weight_src* src, int wdtype);
 /* Copy and quantise (int8, one fp32 scale per 128 inputs) the depth decoder. */
 M3_API int m3_load_depth_weights(m3_ctx* ctx, const m3_depth_src* src);
 
-/* Set up the paged KV cache: `rows` independent rows, each with
- * capacity `max_positions` (<= 9000 for the 8B; any value fits memory).
+/* Set up the paged KV cache ("MiniMax Music 3, local", "Where the time
+ * went": the cache grows in buckets; an f16 cache option; the 9000-frame
+ * cap of "MiniMax-Music3 ... DiffSynth-Studio", "推理参数详解"): `rows`
+ * independent rows, each with capacity `max_positions` (<= 9000 for the
+ * 8B; any value fits memory).
  * Pages of `bucket` positions (a multiple of 32; 256 recommended) are
  * allocated lazily, one bucket for all rows and layers at a time, as frames
  * reach them -- the cache grows without copying.  kvdtype M3_KV_BF16 or
@@ -214,7 +221,11 @@ M3_API int m3_prefill(m3_ctx* ctx, int row, int start, int n_tokens, const void*
  * Returns M3_EINVAL for top_k < 0. */
 M3_API int m3_set_top_k(m3_ctx* ctx, int top_k);
 
-/* Decode one frame for rows 0..rows-1 (rows <= cache rows and <= max_rows).
+/* Decode one frame for rows 0..rows-1 (rows <= cache rows and <= max_rows):
+ * the per-frame step of "MiniMax-Music3 ... DiffSynth-Studio", "第二阶段"
+ * (the Global LLM's forward, the guided draw over the audio-code rows), with
+ * the static graph inputs, sliced lm_head and Gumbel-argmax draw of
+ * "MiniMax Music 3 modular pipeline", findings 2-3.
  *  positions (HOST, [rows]): the position each row writes this frame; the
  *    row attends to positions 0..positions[r] inclusive.  Every position must
  *    be < max_positions or the call returns M3_ECAPACITY before any launch.
