@@ -24,7 +24,7 @@ FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", 
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]
 
 SOURCES = ["m3.cu", "attention.cu", "gemv_tile.cu", "gemv_bf16.cu", "gemv_i8row.cu",
-           "gemv_i8g128.cu", "gemm_tc.cu", "dit.cu", "dit_gemm.cu"]
+           "gemv_i8g128.cu", "gemm_tc.cu", "dit.cu", "dit_gemm.cu", "depth.cu"]
 
 
 def _deps_mtime() -> float:

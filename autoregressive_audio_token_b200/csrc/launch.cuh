@@ -86,8 +86,5 @@ struct GemmTcArgs {
 };
 cudaError_t launch_gemm_tc(const GemmTcArgs& a, int wf, int epi, cudaStream_t st);
 
-struct DepthArgs;
-size_t depth_smem_bytes(const DepthArgs& a);
-cudaError_t launch_depth(const DepthArgs& a, int max_grid, cudaStream_t st);
 
 }  // namespace m3

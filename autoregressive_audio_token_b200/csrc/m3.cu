@@ -18,6 +18,7 @@
 #include "misc.cuh"
 #include "gemv_tile.cuh"
 #include "dit_gemm.cuh"
+#include "depth.cuh"
 
 using namespace m3;
 typedef __nv_bfloat16 bf16;
@@ -126,6 +127,12 @@ struct m3_ctx {
   float* dlogits = nullptr;
   unsigned long long* d_dpages = nullptr;
   void* dkv = nullptr;
+  // the persistent depth kernel: its tagged-word buffers (residual stream,
+  // qkv, attention output, SwiGLU output, frame-local K/V), argmax partials
+  // (one per SM) and launch count
+  uint32_t* dwords = nullptr;
+  unsigned long long* dpart = nullptr;
+  unsigned* dseq = nullptr;
 
   std::map<std::pair<int, int>, cudaGraphExec_t> graphs;
   std::map<std::pair<int, int>, cudaGraphExec_t> dgraphs;
@@ -423,6 +430,14 @@ extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) 
     if (cudaMemcpy(c->d_dpages, hp.data(), sizeof(unsigned long long) * hp.size(),
                    cudaMemcpyHostToDevice) != cudaSuccess)
       return bail(fail(M3_ECUDA, "depth page table"));
+    const size_t qn = (size_t)g.depth_heads * g.depth_head_dim;
+    const size_t words = (size_t)R * (Dh + 3 * qn + qn + g.depth_ffn) +
+                         (size_t)R * g.depth_layers * (NC + 1) * 2 * qn;
+    if ((rc = dzalloc(c, reinterpret_cast<void**>(&c->dwords), sizeof(uint32_t) * words)) ||
+        (rc = dzalloc(c, reinterpret_cast<void**>(&c->dpart),
+                      sizeof(unsigned long long) * c->nsm * kMaxRows)) ||
+        (rc = dzalloc(c, reinterpret_cast<void**>(&c->dseq), sizeof(unsigned))))
+      return bail(rc);
   }
   *out = c;
   return M3_OK;
@@ -1098,11 +1113,89 @@ extern "C" int m3_decode_frame(m3_ctx* c, int rows, const int32_t* positions, ui
 
 // --------------------------------------------------------- depth decoder ---
 
+// Arguments of the persistent depth kernel (depth.cu) for `rows` rows.
+static void fill_depth_args(const m3_ctx* c, int rows, bool forced, const bf16* hin, DepthArgs* a) {
+  const m3_config& g = c->cfg;
+  *a = DepthArgs{};
+  a->rows = rows;
+  a->Dh = g.depth_hidden;
+  a->nh = g.depth_heads;
+  a->hd = g.depth_head_dim;
+  a->F = g.depth_ffn;
+  a->NC = g.depth_codebooks;
+  a->V = g.depth_vocab;
+  a->Hin = g.hidden;
+  a->n_layers = g.depth_layers;
+  a->eps = g.rms_eps;
+  auto mat = [](const DMat& M) { return DepthMat{static_cast<const int8_t*>(M.w), M.s}; };
+  for (int l = 0; l < g.depth_layers && l < kDepthMaxLayers; ++l) {
+    const DLayer& L = c->DL[l];
+    a->L[l] = DepthLayerW{mat(L.qkv), mat(L.o), mat(L.gu), mat(L.d),
+                          L.attn_norm, L.mlp_norm, L.q_norm, L.k_norm};
+  }
+  a->proj = mat(c->dproj);
+  for (int j = 0; j < g.depth_codebooks && j < kDepthMaxCodebooks; ++j) {
+    if (j < (int)c->dheads.size()) a->heads[j] = mat(c->dheads[j]);
+    if (j < (int)c->demb.size()) {
+      a->emb[j] = c->demb[j];
+      a->emb_rows[j] = c->demb_rows[j];
+    }
+  }
+  a->final_norm = c->dfinal;
+  a->rope = c->drope;
+  a->h_in = hin;
+  a->code0 = c->dprev;
+  a->forced = forced ? c->dforced : nullptr;
+  // the end token's code (slice_len) has no semantic embedding: a zero input
+  a->zero_code = g.has_end_token ? g.slice_len : INT_MIN;
+  a->codes = c->dcodes;
+  a->prev = c->dprev;
+  a->logits = c->dlogits;
+  a->fp = c->fp;
+  const size_t R = g.max_rows, qn = (size_t)g.depth_heads * g.depth_head_dim;
+  a->xw = c->dwords;
+  a->qkvw = a->xw + R * g.depth_hidden;
+  a->attw = a->qkvw + R * 3 * qn;
+  a->actw = a->attw + R * qn;
+  a->kvw = a->actw + R * g.depth_ffn;
+  a->part = c->dpart;
+  a->seq = c->dseq;
+  a->err = c->err;
+}
+
+// Whether the persistent kernel takes `rows` rows of this decoder (its
+// shape limits and shared memory): then *smem its shared memory.
+static int depth_persistent_plan(const m3_ctx* c, DepthArgs* a, size_t* smem, bool* ok) {
+  const m3_config& g = c->cfg;
+  *ok = false;
+  if (g.depth_layers > kDepthMaxLayers || g.depth_codebooks > kDepthMaxCodebooks) return M3_OK;
+  const cudaError_t e = depth_plan(a, c->nsm, smem);
+  if (e == cudaErrorInvalidConfiguration) {
+    (void)cudaGetLastError();
+    return M3_OK;
+  }
+  CK(e);
+  *ok = true;
+  return M3_OK;
+}
+
 // hin: the frame's final-normed hidden state [rows][hidden]; the semantic
 // code is in dprev.
 static int record_depth(m3_ctx* c, int rows, bool forced, const bf16* hin) {
   const m3_config& g = c->cfg;
   const int Dh = g.depth_hidden, NC = g.depth_codebooks, V = g.depth_vocab;
+  {  // the whole decoder as one persistent launch where its shape allows
+    DepthArgs a;
+    fill_depth_args(c, rows, forced, hin, &a);
+    size_t smem = 0;
+    bool ok = false;
+    CKR(depth_persistent_plan(c, &a, &smem, &ok));
+    if (ok) {
+      CK(launch_depth(a, c->nsm, smem, c->st));
+      return M3_OK;
+    }
+  }
+  // separate launches per position and layer
   bool pdl = false;
   CKR(gemv_rows(c, c->dproj, EPI_STORE, rows, hin, g.hidden, nullptr, c->DA.x, Dh, nullptr, pdl));
   for (int j = 0; j <= NC; ++j) {
@@ -1571,6 +1664,23 @@ extern "C" int m3_frame_kernels(const m3_ctx* c, int rows) {
       n += M->tiled ? 1 : (rows + 3) / 4;
   }
   return n;
+}
+
+extern "C" int m3_depth_kernels(const m3_ctx* c, int rows) {
+  if (!c || rows < 1 || rows > c->cfg.max_rows) return fail(M3_EINVAL, "rows");
+  if (!c->depth_loaded) return fail(M3_ESTATE, "depth decoder not loaded");
+  const m3_config& g = c->cfg;
+  DepthArgs a;
+  fill_depth_args(c, rows, false, c->dh, &a);
+  size_t smem = 0;
+  bool ok = false;
+  CKR(depth_persistent_plan(c, &a, &smem, &ok));
+  if (ok) return 1;
+  // separate launches: the projections in launches of 4 rows (the CUDA-core
+  // group-128 GEMV), embeddings, attention per position and layer
+  const int P = g.depth_codebooks + 1, per4 = (rows + 3) / 4;
+  return (1 + P * g.depth_layers * 4 + g.depth_codebooks) * per4 + g.depth_codebooks +
+         P * g.depth_layers;
 }
 
 extern "C" double m3_frame_bytes(const m3_ctx* c, int rows, int ctx_len) {

@@ -26,7 +26,7 @@ M3_FAULT_NONE, M3_FAULT_ALLOC, M3_FAULT_H2D, M3_FAULT_GRAPH = 0, 1, 2, 3
 
 EXPORTED = ("m3_create", "m3_load_weights", "m3_load_depth_weights", "m3_kv_alloc", "m3_kv_set",
             "m3_kv_get", "m3_decode_frame", "m3_depth_decode", "m3_embed", "m3_quantize_int8",
-            "m3_export_weight", "m3_frame_bytes", "m3_frame_kernels", "m3_time_gemv", "m3_sample_noalloc", "m3_set_top_k",
+            "m3_export_weight", "m3_frame_bytes", "m3_frame_kernels", "m3_depth_kernels", "m3_time_gemv", "m3_sample_noalloc", "m3_set_top_k",
             "m3_load_feedback", "m3_generate", "m3_prefill", "m3_gumbel_fill", "m3_inject_fault",
             "m3_stalled_wait", "m3_sync_status", "m3_last_error", "m3_destroy")
 
@@ -90,6 +90,7 @@ def load_library() -> C.CDLL:
     L.m3_frame_bytes.argtypes = [vp, i32, i32]
     L.m3_frame_bytes.restype = C.c_double
     L.m3_frame_kernels.argtypes = [vp, i32]
+    L.m3_depth_kernels.argtypes = [vp, i32]
     L.m3_time_gemv.argtypes = [vp, i32, i32, i32, C.POINTER(C.c_float), C.POINTER(C.c_double)]
     L.m3_sample_noalloc.argtypes = [vp, i32, vp, u64, u64, f32, f32, vp, vp]
     L.m3_load_feedback.argtypes = [vp, vp, C.POINTER(vp), i32]
@@ -255,6 +256,13 @@ def m3_frame_bytes(ctx: int, rows: int, ctx_len: int) -> float:
 
 def m3_frame_kernels(ctx: int, rows: int) -> int:
     n = lib.m3_frame_kernels(ctx, rows)
+    if n < 0:
+        _check(n)
+    return n
+
+
+def m3_depth_kernels(ctx: int, rows: int) -> int:
+    n = lib.m3_depth_kernels(ctx, rows)
     if n < 0:
         _check(n)
     return n

@@ -398,7 +398,7 @@ def run_ours(args, rank, world, local):
     # them; the depth decoder adds
     # its parameter block, projection, 7 embeddings, 8 positions x layers x 5
     # kernels and 7 heads
-    depth_launches = (2 + 7 + 8 * synth.DEPTH.n_layers * 5 + 7) if args.depth else 0
+    depth_launches = m3.m3_depth_kernels(ctx, rows) if args.depth else 0
     out["gpu_launches"] = (m3.m3_frame_kernels(ctx, rows) + depth_launches) * args.steps
     m3.m3_destroy(ctx)
     del xs
@@ -792,17 +792,19 @@ def run_dit(args):
 
 def run_depth_only(args):
     """The RVQ depth decoder alone (int8 weights, one scale per group of 128):
-    m3_depth_decode on a fixed final hidden state and semantic code, 2 rows
-    (one CFG pair), timed with CUDA events over --steps calls after --warmup.
-    The body is a single layer, loaded only because the context needs one."""
+    m3_depth_decode on a fixed final hidden state and semantic code, --rows
+    rows (2 = one CFG pair, the workload), timed with CUDA events over
+    --steps calls after --warmup. The body is a single layer, loaded only
+    because the context needs one."""
     import torch
     from autoregressive_audio_token_b200 import m3
     import synth
     torch.cuda.set_device(0)
-    s, ctx = build_model(torch, m3, synth, 0, m3.M3_W_INT8, 1, depth=True)
-    h = synth.normal((ROWS, s.hidden), 0, "bench/depth_h", std=1.0, device="cuda")
-    code0 = torch.tensor([5, 5], dtype=torch.int32, device="cuda")
-    dcodes = torch.empty((ROWS, synth.DEPTH.codebooks), dtype=torch.int32, device="cuda")
+    rows = args.rows
+    s, ctx = build_model(torch, m3, synth, 0, m3.M3_W_INT8, 1, depth=True, max_rows=max(2, rows))
+    h = synth.normal((rows, s.hidden), 0, "bench/depth_h", std=1.0, device="cuda")
+    code0 = torch.tensor([5 + 7 * (r // 2) for r in range(rows)], dtype=torch.int32, device="cuda")
+    dcodes = torch.empty((rows, synth.DEPTH.codebooks), dtype=torch.int32, device="cuda")
     for i in range(max(args.warmup, 3)):
         m3.m3_depth_decode(ctx, h, code0, 1, i, CFG_SCALE, 1.0, dcodes)
     torch.cuda.synchronize()
@@ -817,11 +819,12 @@ def run_depth_only(args):
     D = synth.DEPTH
     wbytes = (D.n_layers * (4 * D.hidden * D.n_heads * D.head_dim + 3 * D.hidden * D.ffn) *
               (D.codebooks + 1) + D.hidden * D.in_hidden + D.codebooks * D.vocab * D.hidden)
-    print(json.dumps({"metric": "depth decoder calls/s (7 residual codes, 2 rows)",
+    print(json.dumps({"metric": f"depth decoder calls/s (7 residual codes, {rows} rows)",
                       "value": 1000.0 / ms, "unit": "calls/s", "ms_per_call": ms,
                       "steps": args.steps, "dtype": "int8 g128",
+                      "kernels_per_call": m3.m3_depth_kernels(ctx, rows),
                       "weight_bytes_per_call": wbytes, "achieved_gbs": wbytes / ms / 1e6,
-                      "config": {"workload": "depth-decoder-4L-1024-int8g128-2rows-cfg1.5"}}))
+                      "config": {"workload": f"depth-decoder-4L-1024-int8g128-{rows}rows-cfg1.5"}}))
     m3.m3_destroy(ctx)
 
 

@@ -330,6 +330,12 @@ M3_API int m3_export_weight(m3_ctx* ctx, int which, int layer, void* q_host, flo
  * the weights are loaded. */
 M3_API int m3_frame_kernels(const m3_ctx* ctx, int rows);
 
+/* Kernels one m3_depth_decode of `rows` rows launches, for launch
+ * accounting: 1 where the decoder runs as one persistent kernel (its shape
+ * and shared memory allow), else its separate launches.  A negative
+ * m3_status on bad arguments or before the depth weights are loaded. */
+M3_API int m3_depth_kernels(const m3_ctx* ctx, int rows);
+
 /* Algorithmic HBM bytes of one frame: weights read once per frame plus the
  * KV cache read for `rows` rows at context length ctx (positions 0..ctx). */
 M3_API double m3_frame_bytes(const m3_ctx* ctx, int rows, int ctx_len);

@@ -289,6 +289,9 @@ def test_errors_are_status_codes(ora):
         with pytest.raises(m3.M3Error) as e:
             m3.m3_frame_kernels(m.ctx, 0)
         assert e.value.code == m3.M3_EINVAL
+        with pytest.raises(m3.M3Error) as e:  # no depth decoder in this config
+            m3.m3_depth_kernels(m.ctx, 1)
+        assert e.value.code == m3.M3_ESTATE
     finally:
         m.close()
 
@@ -388,15 +391,20 @@ def test_layer8b_16rows_long_context(ora, n_ctx):
 
 # -------------------------------------------------------- depth decoder ----
 
-def test_depth_decoder_full_size(ora):
+@pytest.mark.parametrize("rows", [2, 16])
+def test_depth_decoder_full_size(ora, rows):
     # the 8B model's depth decoder (16 heads of 64, hidden 1024, 4 layers,
-    # SwiGLU 2816, 7 codebooks of 1024, input 4096), one cluster of 16 CTAs,
-    # a CFG pair: logits against the oracle, every draw by the draw rule
-    s, D, rows, cfg = synth.LAYER8B, synth.DEPTH, 2, 1.5
-    m = Model(s, seed=9, depth=D, max_rows=2)
+    # SwiGLU 2816, 7 codebooks of 1024, input 4096): one CFG pair (the
+    # attention inside the O projection's step) and 8 pairs (the attention
+    # as its own step, two 8-row MMA blocks, the input projection's rows in
+    # two passes): logits against the oracle, every draw by the draw rule
+    s, D, cfg = synth.LAYER8B, synth.DEPTH, 1.5
+    m = Model(s, seed=9, depth=D, max_rows=rows)
     try:
+        assert m.m3.m3_depth_kernels(m.ctx, rows) == 1  # the persistent kernel
         h = synth.normal((rows, s.hidden), 9, "hframe", std=1.0).cuda()
-        code0 = torch.tensor([11, 16383], dtype=torch.int32, device="cuda")
+        code0 = torch.tensor(([11, 16383] + [(977 * r) % 16384 for r in range(2, rows)])[:rows],
+                             dtype=torch.int32, device="cuda")
         codes = torch.empty((rows, D.codebooks), dtype=torch.int32, device="cuda")
         lg = torch.empty((rows, D.codebooks, D.vocab), dtype=torch.float32, device="cuda")
         m.m3.m3_depth_decode(m.ctx, h, code0, 5, 2, cfg, 1.0, codes, logits=lg)
@@ -413,15 +421,19 @@ def test_depth_decoder_full_size(ora):
         m.close()
 
 
-@pytest.mark.parametrize("rows,cfg", [(1, 0.0), (2, 1.5), (4, 1.5)])
+@pytest.mark.parametrize("rows,cfg", [(1, 0.0), (2, 1.5), (4, 1.5), (12, 1.5), (16, 0.0)])
 def test_depth_decoder_teacher_forced(ora, rows, cfg):
+    # 1..8 rows of 4 heads: the attention inside the O projection's step;
+    # 12 and 16 rows: as its own step, two 8-row MMA blocks
     s = synth.TINY
     D = synth.DepthShape(hidden=256, n_layers=2, n_heads=4, head_dim=64, ffn=384, codebooks=7,
                          vocab=128, sem_vocab=s.slice_len, in_hidden=s.hidden)
     m = Model(s, seed=6, depth=D, max_rows=max(2, rows))
     try:
+        assert m.m3.m3_depth_kernels(m.ctx, rows) == 1  # the persistent kernel
         h = synth.normal((rows, s.hidden), 6, "hframe").cuda()
-        code0 = torch.tensor([3, 77, 5, 400][:rows], dtype=torch.int32, device="cuda")
+        code0 = torch.tensor(([3, 77, 5, 400] + [(37 * r) % s.slice_len for r in range(4, rows)])[:rows],
+                             dtype=torch.int32, device="cuda")
         codes = torch.empty((rows, D.codebooks), dtype=torch.int32, device="cuda")
         lg = torch.empty((rows, D.codebooks, D.vocab), dtype=torch.float32, device="cuda")
         m.m3.m3_depth_decode(m.ctx, h, code0, 31, 4, cfg, 1.0, codes, logits=lg)
