@@ -421,6 +421,34 @@ def test_depth_decoder_full_size(ora, rows):
         m.close()
 
 
+def test_depth_decoder_separate_launches(ora):
+    # codebooks of 120 entries (not whole 16-row tiles): the persistent kernel
+    # does not take the shape and the decoder runs as separate launches
+    s = synth.TINY
+    D = synth.DepthShape(hidden=256, n_layers=2, n_heads=4, head_dim=64, ffn=384, codebooks=7,
+                         vocab=120, sem_vocab=s.slice_len, in_hidden=s.hidden)
+    rows, cfg = 2, 1.5
+    m = Model(s, seed=6, depth=D, max_rows=rows)
+    try:
+        assert m.m3.m3_depth_kernels(m.ctx, rows) > 1
+        h = synth.normal((rows, s.hidden), 6, "hframe").cuda()
+        code0 = torch.tensor([3, 77], dtype=torch.int32, device="cuda")
+        codes = torch.empty((rows, D.codebooks), dtype=torch.int32, device="cuda")
+        lg = torch.empty((rows, D.codebooks, D.vocab), dtype=torch.float32, device="cuda")
+        m.m3.m3_depth_decode(m.ctx, h, code0, 31, 4, cfg, 1.0, codes, logits=lg)
+        torch.cuda.synchronize()
+        m.m3.m3_sync_status(m.ctx)
+        gc = codes.cpu().numpy()
+        oc, olg = m.ora_depth.decode(bits(h), code0.cpu().numpy(), 31, 4, cfg_scale=cfg,
+                                     forced=gc)
+        glg = lg.cpu().numpy()
+        for j in range(D.codebooks):
+            assert rel_err(glg[:, j], olg[:, j]) <= TOL[1], (j, rel_err(glg[:, j], olg[:, j]))
+        check_depth_draws(glg, gc, 31, 4, cfg_scale=cfg)
+    finally:
+        m.close()
+
+
 @pytest.mark.parametrize("rows,cfg", [(1, 0.0), (2, 1.5), (4, 1.5), (12, 1.5), (16, 0.0)])
 def test_depth_decoder_teacher_forced(ora, rows, cfg):
     # 1..8 rows of 4 heads: the attention inside the O projection's step;
