@@ -10,7 +10,8 @@
 //
 // What keeps a step short:
 //   * no grid barrier: every value another CTA reads is written as a tagged
-//     32-bit word (bf16 value, 16-bit tag of the writing step) and the reader
+//     32-bit word (bf16 value, 16-bit tag = 1 + the writing step's number;
+//     the buffers are cleared to tag 0 before each launch) and the reader
 //     polls exactly the words it needs until they carry the expected tag --
 //     a step waits only for its own inputs, one L2 round trip after they
 //     land. It is sound because every reader of a buffer is upstream of the
@@ -103,14 +104,11 @@ __device__ __forceinline__ void wait_words4(const uint32_t* p, uint32_t tag, uin
   }
 }
 
-// Tag of step ph of this launch: 1 + (seq * P + ph) mod 65535 (never 0, the
-// value of a word no step has written; two launches in a row never share one).
+// Tag of step ph: 1 + ph (never 0, the value of every word when the launch
+// starts; a launch has at most 1 + 32 * 8 * 5 + 31 steps).
 struct Sched {
-  uint32_t base;  // (seq * P) mod 65535
   int L, S, merge;
-  __device__ __forceinline__ uint32_t tag(int ph) const {
-    return 1u + (base + (uint32_t)ph) % 65535u;
-  }
+  __device__ __forceinline__ uint32_t tag(int ph) const { return 1u + (uint32_t)ph; }
   // step ids: 0 the input projection; per position j, per layer l: QKV,
   // [attention,] O, gate/up, down; for j >= 1 then the head of codebook j
   __device__ __forceinline__ int pos0(int j) const { return 1 + j * L * S + (j > 0 ? j - 1 : 0); }
@@ -704,12 +702,10 @@ __global__ void __launch_bounds__(kDepthThreads, 1) depth_kernel(const DepthArgs
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int rows = a.rows, Dh = a.Dh, QN = a.nh * HD, F = a.F;
-  const unsigned seq = *reinterpret_cast<volatile const unsigned*>(a.seq);
   Sched sc;
   sc.L = a.n_layers;
   sc.S = a.merge_attn ? 4 : 5;
   sc.merge = a.merge_attn;
-  sc.base = (uint32_t)(((unsigned long long)seq * (unsigned long long)(1 + (a.NC + 1) * sc.L * sc.S + a.NC)) % 65535ull);
   if (tid == 0) {
     mbar_init(&wbar[0], 1);
     mbar_init(&wbar[1], 1);
@@ -959,11 +955,8 @@ __global__ void __launch_bounds__(kDepthThreads, 1) depth_kernel(const DepthArgs
     __syncthreads();
     ++gi;
   }
-  // the last codebook's draw: CTA 0 writes it, then counts the launch
-  if (blockIdx.x == 0) {
-    take_codes(a, a.NC, sc.tag(sc.head(a.NC)), pcode);
-    if (tid == 0) *reinterpret_cast<volatile unsigned*>(a.seq) = seq + 1;
-  }
+  // the last codebook's draw: CTA 0 writes it
+  if (blockIdx.x == 0) take_codes(a, a.NC, sc.tag(sc.head(a.NC)), pcode);
 }
 
 template <int NB>
@@ -1039,9 +1032,14 @@ cudaError_t depth_plan(DepthArgs* a, int grid, size_t* smem) {
   return cudaSuccess;
 }
 
-// One cooperative launch (every CTA resident at once: a step waits for
-// other CTAs' outputs).
+// The tagged buffers cleared to tag 0 (so that a word carries a step's tag
+// only once that step of this launch has written it), then one cooperative
+// launch (every CTA resident at once: a step waits for other CTAs' outputs).
 cudaError_t launch_depth(const DepthArgs& a, int grid, size_t smem, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(a.words, 0, a.words_bytes, st);
+  if (e == cudaSuccess)
+    e = cudaMemsetAsync(a.part, 0, sizeof(unsigned long long) * grid * kMaxRows, st);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kDepthThreads);

@@ -61,14 +61,16 @@ struct DepthArgs {
   // value in the low half, the tag of the step that wrote it in the high
   // half; a reader polls each word until it carries the tag it expects, so
   // no grid-wide barrier is needed (every reader of a buffer is upstream of
-  // the buffer's next writer).
+  // the buffer's next writer). All of them lie in [words, words +
+  // words_bytes), cleared before each launch.
+  uint32_t* words;
+  size_t words_bytes;
   uint32_t* xw;    // [rows][Dh] residual stream
   uint32_t* qkvw;  // [rows][3 nh hd]
   uint32_t* attw;  // [rows][nh hd]
   uint32_t* actw;  // [rows][F]
   uint32_t* kvw;   // [rows][n_layers][NC + 1][2][nh hd] normed/rotated keys, values
   unsigned long long* part;  // [grid][kMaxRows] per-CTA argmax keys, tag in the low 16 bits
-  unsigned* seq;             // launches so far (tags differ from launch to launch)
   int* err;
 };
 

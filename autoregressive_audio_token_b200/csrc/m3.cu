@@ -128,11 +128,11 @@ struct m3_ctx {
   unsigned long long* d_dpages = nullptr;
   void* dkv = nullptr;
   // the persistent depth kernel: its tagged-word buffers (residual stream,
-  // qkv, attention output, SwiGLU output, frame-local K/V), argmax partials
-  // (one per SM) and launch count
+  // qkv, attention output, SwiGLU output, frame-local K/V) and argmax
+  // partials (one per SM)
   uint32_t* dwords = nullptr;
+  size_t dwords_bytes = 0;
   unsigned long long* dpart = nullptr;
-  unsigned* dseq = nullptr;
 
   std::map<std::pair<int, int>, cudaGraphExec_t> graphs;
   std::map<std::pair<int, int>, cudaGraphExec_t> dgraphs;
@@ -433,10 +433,10 @@ extern "C" int m3_create(const m3_config* cfg, void* cuda_stream, m3_ctx** out) 
     const size_t qn = (size_t)g.depth_heads * g.depth_head_dim;
     const size_t words = (size_t)R * (Dh + 3 * qn + qn + g.depth_ffn) +
                          (size_t)R * g.depth_layers * (NC + 1) * 2 * qn;
-    if ((rc = dzalloc(c, reinterpret_cast<void**>(&c->dwords), sizeof(uint32_t) * words)) ||
+    c->dwords_bytes = sizeof(uint32_t) * words;
+    if ((rc = dzalloc(c, reinterpret_cast<void**>(&c->dwords), c->dwords_bytes)) ||
         (rc = dzalloc(c, reinterpret_cast<void**>(&c->dpart),
-                      sizeof(unsigned long long) * c->nsm * kMaxRows)) ||
-        (rc = dzalloc(c, reinterpret_cast<void**>(&c->dseq), sizeof(unsigned))))
+                      sizeof(unsigned long long) * c->nsm * kMaxRows)))
       return bail(rc);
   }
   *out = c;
@@ -1153,13 +1153,14 @@ static void fill_depth_args(const m3_ctx* c, int rows, bool forced, const bf16* 
   a->logits = c->dlogits;
   a->fp = c->fp;
   const size_t R = g.max_rows, qn = (size_t)g.depth_heads * g.depth_head_dim;
+  a->words = c->dwords;
+  a->words_bytes = c->dwords_bytes;
   a->xw = c->dwords;
   a->qkvw = a->xw + R * g.depth_hidden;
   a->attw = a->qkvw + R * 3 * qn;
   a->actw = a->attw + R * qn;
   a->kvw = a->actw + R * g.depth_ffn;
   a->part = c->dpart;
-  a->seq = c->dseq;
   a->err = c->err;
 }
 

@@ -421,6 +421,33 @@ def test_depth_decoder_full_size(ora, rows):
         m.close()
 
 
+def test_depth_decoder_row_counts_interleaved(ora):
+    # one context, calls of 16, 2 and again 16 rows (the persistent kernel's
+    # two attention modes): the repeated call is bit-identical to the first
+    s = synth.TINY
+    D = synth.DepthShape(hidden=256, n_layers=2, n_heads=4, head_dim=64, ffn=384, codebooks=7,
+                         vocab=128, sem_vocab=s.slice_len, in_hidden=s.hidden)
+    m = Model(s, seed=7, depth=D, max_rows=16, oracle=False)
+    try:
+        def call(rows, seed):
+            h = synth.normal((rows, s.hidden), seed, "hframe").cuda()
+            code0 = torch.tensor([(53 * r + seed) % s.slice_len for r in range(rows)],
+                                 dtype=torch.int32, device="cuda")
+            codes = torch.empty((rows, D.codebooks), dtype=torch.int32, device="cuda")
+            lg = torch.empty((rows, D.codebooks, D.vocab), dtype=torch.float32, device="cuda")
+            m.m3.m3_depth_decode(m.ctx, h, code0, 3, seed, 1.5, 1.0, codes, logits=lg)
+            torch.cuda.synchronize()
+            m.m3.m3_sync_status(m.ctx)
+            return codes.cpu().numpy(), lg.cpu().numpy()
+        c1, l1 = call(16, 1)
+        for i in range(3):
+            call(2, 2 + i)
+        c2, l2 = call(16, 1)
+        assert np.array_equal(c1, c2) and np.array_equal(l1, l2)
+    finally:
+        m.close()
+
+
 def test_depth_decoder_separate_launches(ora):
     # codebooks of 120 entries (not whole 16-row tiles): the persistent kernel
     # does not take the shape and the decoder runs as separate launches
