@@ -7,7 +7,8 @@
 // weights (53 MB of int8 with group-128 scales, "MiniMax Music 3 on Metal",
 // "Precision is the reference's") stay in L2 across the positions. As
 // separate launches it is bound by launch latency; this kernel runs the whole
-// chain with one CTA per SM and a grid barrier between steps.
+// chain with one CTA per SM, each step waiting only for the tagged words of
+// its own inputs.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -83,9 +84,9 @@ __host__ __device__ __forceinline__ int depth_slice_bytes(int nt, int K, int sid
 }
 
 // Shape checks and the shared-memory carve for `grid` CTAs; fills
-// a->wb_bytes, xs_bytes, max_tiles, merge_attn.  cudaErrorInvalidConfiguration
-// when the shape does not suit the kernel (the caller then takes the
-// per-launch path).
+// a->wb_bytes, xs_bytes, max_tiles, side_bytes, own_tiles, merge_attn.
+// cudaErrorInvalidConfiguration when the shape does not suit the kernel (the
+// caller then takes the per-launch path).
 cudaError_t depth_plan(DepthArgs* a, int grid, size_t* smem);
 cudaError_t launch_depth(const DepthArgs& a, int grid, size_t smem, cudaStream_t st);
 
