@@ -71,6 +71,10 @@ def test_null_arguments_are_einval():
     from autoregressive_audio_token_b200 import m3
     assert m3.lib.m3_decode_frame(None, 1, None, 0, 0, None, 0.0, 1.0, None, None, None) == m3.M3_EINVAL
     assert m3.lib.m3_quantize_int8(None, 1, 1, 1, None, None, None) == m3.M3_EINVAL
+    assert m3.lib.m3_depth_decode(None, 2, None, None, 0, 0, 1.5, 1.0, None, None, None) == m3.M3_EINVAL
+    # launch accounting answers without a context only with an error
+    assert m3.lib.m3_frame_kernels(None, 1) == m3.M3_EINVAL
+    assert m3.lib.m3_depth_kernels(None, 1) == m3.M3_EINVAL
 
 
 def test_checking_hooks_validate_before_any_cuda_call():
